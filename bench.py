@@ -1,0 +1,354 @@
+"""Benchmark of the CARVE recurrence library on B200.
+
+Default workload: the 1.3B-layer training step (B=8, H=16, T=4096, d=128, chunk 64, rank 32,
+bf16 q/k/v/o, fp32 gates) -- one step = carve_fwd (saving what the backward needs) + carve_bwd
+against a seeded upstream gradient.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl carve|reference]
+                  [--workload train|fwd|long|decode] [--no-e2e] [--no-cpu-baseline]
+
+Timing: CUDA events on the launch stream, W untimed warm-up steps, then K timed steps
+bracketed by a barrier and a device synchronize, max over ranks.  The working set of a step
+(about 3 GB) is far larger than the 126 MB L2, so no explicit flush is needed between steps.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from chunk_gated_delta_b200 import inputs as I  # noqa: E402
+
+METRIC = "fwd+bwd tokens/s per layer (B200, 16 heads, d=128) & % bf16 tensor peak"
+
+# Algorithmic HBM bytes per (token, head) at d = 128 with bf16 q/k/v/o and fp32 gates:
+#   forward : q,k,v 768 + g_logit,bx 1024 + w 4 + o 256                      = 2052
+#             + chunk-boundary state saved for the backward, 4 d^2 / L          (1024 at L=64)
+#   backward: inputs 1796 + dO 256 + boundary state 4 d^2 / L + dq,dk,dv 768
+#             + dg_logit,dbx 1024 + dw 4                                        = 3848 + 4 d^2 / L
+# FLOPs per (token, head), triangular halves only (forward exact for the WY algorithm,
+# backward counted from its GEMM list):
+#   forward : 5 L d + 6 d^2 + L^2/3 + (2 d^2 + 4 r d)/L
+#   backward: 14 L d + 14 d^2 + L^2
+def fwd_bytes(d, L):
+    return 2052 + 4 * d * d / L
+
+
+def bwd_bytes(d, L):
+    return 3848 + 4 * d * d / L
+
+
+def fwd_flops(d, L, r):
+    return 5 * L * d + 6 * d * d + L * L / 3 + (2 * d * d + 4 * r * d) / L
+
+
+def bwd_flops(d, L, r):
+    return 14 * L * d + 14 * d * d + L * L
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm=j["hbm_gbs"], bf16=j["bf16_tflops"], bf16_sustained=j.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows)}
+
+
+# ---------------------------------------------------------------------------------------
+def dist_setup():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier_sync(ws):
+    import torch
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(w, d, dO, target_s=12.0, max_T=None):
+    """Time the fp64 oracle (fwd + bwd) on batch element 0 (all heads) over a prefix of the
+    sequence, doubling the prefix until the run takes at least target_s / 2 seconds.
+    Returns (tokens/s of the whole layer, cores used, sample description)."""
+    import oracle
+    T = 128
+    max_T = w.T if max_T is None else max_T
+    while True:
+        sub = {k: (v[:1, :T] if v.ndim >= 3 and k not in ("A", "B") else v) for k, v in d.items()}
+        t0 = time.perf_counter()
+        oracle.fwd(sub, L=w.L, mc_mode=w.mc_mode)
+        oracle.bwd(sub, w.L, dO[:1, :T], mc_mode=w.mc_mode)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 2 or T >= max_T:
+            break
+        T = min(max_T, T * 2)
+    return T / dt, oracle.threads(), f"oracle fwd+bwd, batch 0 (all {w.H} heads), first {T} of {w.T} tokens"
+
+
+# ---------------------------------------------------------------------------------------
+def run_reference(args, w):
+    """The reference arm: the fp64 oracle on the host cores, bounded sample per step."""
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if ws > 1 and rank != 0:
+        return
+    import oracle
+    Tp = 256
+    d = I.make_inputs(w, T=Tp)
+    dO = I.make_grad_out(w, T=Tp)
+    sub = {k: (v[:1] if v.ndim >= 3 and k not in ("A", "B") else v) for k, v in d.items()}
+    for _ in range(args.warmup):
+        oracle.fwd(sub, L=w.L)
+        oracle.bwd(sub, w.L, dO[:1])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.fwd(sub, L=w.L)
+        oracle.bwd(sub, w.L, dO[:1])
+    dt = (time.perf_counter() - t0) / args.steps
+    v = Tp / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "sample": f"batch 0, all {w.H} heads, first {Tp} tokens per step"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                             "sample": f"oracle fwd+bwd on batch 0 (all {w.H} heads), {Tp} tokens per step"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_train(args, w):
+    import torch
+    import chunk_gated_delta_b200 as carve
+    ws, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    seed = w.seed + 7919 * rank      # each rank holds its own batch shard (weak scaling)
+    d = I.make_inputs(w, seed=seed)
+    dO = I.make_grad_out(w, seed=seed)
+    bf = torch.bfloat16 if w.io == "bf16" else torch.float32
+    host = {}
+    for k, v in dict(d, dO=dO).items():
+        t = torch.from_numpy(v)
+        if k in ("q", "k", "v", "dO"):
+            t = t.to(bf)
+        host[k] = t.pin_memory()
+    dv_ = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    torch.cuda.synchronize()
+    L, mode = w.L, w.mc_mode
+    fwd_out = carve.carve_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
+                              dv_["B"], chunk=L, mc_mode=mode)
+    bwd_out = carve.carve_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
+                              dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode)
+    workspace = torch.empty(carve.bwd_workspace_bytes(carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode)),
+                            dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(x, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        carve.carve_fwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"], chunk=L,
+                        mc_mode=mode, out=fwd_out)
+        if ev is not None:
+            ev[1].record(stream)
+        carve.carve_bwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"],
+                        fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace)
+        if ev is not None:
+            ev[2].record(stream)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.all_reduce(bwd_out["dA"])
+            dist.all_reduce(bwd_out["dB"])
+
+    for _ in range(args.warmup):
+        step(dv_)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier_sync(ws)
+        start.record(stream)
+        for j in range(args.steps):
+            step(dv_, evs[j])
+        end.record(stream)
+        barrier_sync(ws)
+    ms = max_over_ranks(start.elapsed_time(end), ws) / args.steps
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    tokens = w.B * w.T * ws
+    value = tokens / (ms * 1e-3)
+
+    th = w.B * w.T * w.H          # token-heads of one rank's launch
+    dd = w.K
+    kern = {"carve_fwd": (fwd_ms, fwd_bytes(dd, L) * th), "carve_bwd": (bwd_ms, bwd_bytes(dd, L) * th)}
+    dom = max(kern, key=lambda k: kern[k][0])
+    dms, dbytes = kern[dom]
+    achieved = dbytes / (dms * 1e-3) / 1e9
+    flops = (fwd_flops(dd, L, w.R) + bwd_flops(dd, L, w.R)) * th * ws
+    tensor_frac = flops / (ms * 1e-3) / (peaks["bf16"] * 1e12 * ws)
+    traffic = load_traffic(dom)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, host, dv_, step, stream, ws, w, bwd_out)
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and ws == 1:
+        v, cores, sample = cpu_oracle_sample(w, d, dO)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "heads": w.H, "d": w.K,
+                   "chunk": L, "rank": w.R, "mc_mode": mode, "parallelism": f"dp{ws}",
+                   "l2": "no flush: step working set ~3 GB >> 126 MB L2"},
+        "tensor_frac": tensor_frac,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm"], "traffic": traffic, "peak_source": peaks["source"]},
+        "kernels_ms": {"carve_fwd": fwd_ms, "carve_bwd": bwd_ms},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p))
+    return j.get(kernel)
+
+
+def measure_e2e(args, host, dv_, step, stream, ws, w, grads):
+    """Same step through the public API with host buffers: pinned H2D copies of the step's
+    inputs, the kernels, and D2H copies of every gradient, all inside the timed region."""
+    import torch
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    grads_host = {k: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for k, t in grads.items()}
+    d2h = sum(t.numel() * t.element_size() for t in grads.values())
+
+    def e2e_step():
+        for k in host:
+            dv_[k].copy_(host[k], non_blocking=True)
+        step(dv_)
+        for k, t in grads.items():
+            grads_host[k].copy_(t, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(1, min(args.steps, 5))
+    barrier_sync(ws)
+    start.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    end.record(stream)
+    barrier_sync(ws)
+    ms = max_over_ranks(start.elapsed_time(end), ws) / steps
+    return {"value": w.B * w.T * ws / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="carve", choices=["carve", "reference"])
+    ap.add_argument("--workload", default="train", choices=["train"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = I.TRAIN_1P3B
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_train(args, w)
+
+
+if __name__ == "__main__":
+    main()

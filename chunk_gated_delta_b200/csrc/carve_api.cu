@@ -1,0 +1,144 @@
+// Host side of the C ABI declared in include/carve.h: argument validation, buffer sizing and
+// kernel dispatch.  Nothing here allocates, frees or synchronises.
+#include <cuda_runtime.h>
+
+#include "../../include/carve.h"
+#include "carve_device.cuh"
+
+namespace carve {
+cudaError_t launch_fwd_simt(int K, int V, bool bf16, const FwdArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
+cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
+                        const float *g_logit, const float *bx, const float *w_logit, const float *A,
+                        const float *Bm, float *S, float *mstate, int *pos, void *o, int B, int H,
+                        int R, int L, int mc_mode, cudaStream_t st);
+}  // namespace carve
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void *p) { return p == nullptr || aligned16(p); }
+
+// shape checks shared by every entry point; `seq` adds the sequence-length rules
+carve_status check_dims(const carve_dims *d, bool seq) {
+    if (!d) return CARVE_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H < 1 || d->dk < 1 || d->dv < 1 || d->rank < 1 || d->chunk < 1)
+        return CARVE_ERR_INVALID_ARG;
+    if (d->io != CARVE_IO_FP32 && d->io != CARVE_IO_BF16) return CARVE_ERR_INVALID_ARG;
+    if (d->mc_mode != CARVE_MC_BOUNDARY_STATE && d->mc_mode != CARVE_MC_PREV_MEAN_O) return CARVE_ERR_INVALID_ARG;
+    if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return CARVE_ERR_UNSUPPORTED;
+    if (d->rank > 64) return CARVE_ERR_UNSUPPORTED;
+    if ((long long)d->B * d->H > (1LL << 30)) return CARVE_ERR_UNSUPPORTED;
+    if (seq) {
+        if (d->T < 1) return CARVE_ERR_INVALID_ARG;
+        if (d->chunk != 16 && d->chunk != 32 && d->chunk != 64 && d->chunk != 128) return CARVE_ERR_UNSUPPORTED;
+        if (d->T % carve::kSub != 0) return CARVE_ERR_UNSUPPORTED;
+        if ((long long)d->B * d->T * d->H * (d->dk > d->dv ? d->dk : d->dv) > (1LL << 40)) return CARVE_ERR_UNSUPPORTED;
+    }
+    return CARVE_OK;
+}
+
+size_t n_chunks(const carve_dims *d) { return (size_t)((d->T + d->chunk - 1) / d->chunk); }
+
+}  // namespace
+
+extern "C" {
+
+const char *carve_status_string(carve_status s) {
+    switch (s) {
+        case CARVE_OK: return "CARVE_OK";
+        case CARVE_ERR_INVALID_ARG: return "CARVE_ERR_INVALID_ARG";
+        case CARVE_ERR_UNSUPPORTED: return "CARVE_ERR_UNSUPPORTED";
+        case CARVE_ERR_CUDA: return "CARVE_ERR_CUDA";
+        case CARVE_ERR_TIMEOUT: return "CARVE_ERR_TIMEOUT";
+    }
+    return "CARVE_ERR_UNKNOWN";
+}
+
+size_t carve_saved_bytes(const carve_dims *d) {
+    if (check_dims(d, true) != CARVE_OK) return 0;
+    const size_t units = (size_t)d->B * d->H;
+    const size_t states = units * (size_t)(d->T / carve::kSub) * d->dv * d->dk;
+    const size_t aux = units * n_chunks(d) * (size_t)(d->dv + d->rank + d->dk);
+    return sizeof(float) * (states + aux);
+}
+
+size_t carve_bwd_workspace_bytes(const carve_dims *d) {
+    if (check_dims(d, true) != CARVE_OK) return 0;
+    return sizeof(float) * (size_t)d->B * d->H * ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv);
+}
+
+carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
+                       const float *g_logit, const float *bx, const float *w_logit,
+                       const float *A, const float *Bm, const float *S0,
+                       const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
+                       void *saved, void *stream) {
+    carve_status st = check_dims(d, true);
+    if (st != CARVE_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
+        !ok_ptr(A) || !ok_ptr(Bm) || !ok_ptr(o) || !ok_opt(S0) || !ok_opt(m_prev_in) || !ok_opt(S_final) ||
+        !ok_opt(m_prev_out) || !ok_opt(saved))
+        return CARVE_ERR_INVALID_ARG;
+    carve::FwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
+    a.S0 = S0; a.m_prev_in = m_prev_in; a.o = o; a.S_final = S_final; a.m_prev_out = m_prev_out;
+    if (saved) {
+        const size_t units = (size_t)d->B * d->H;
+        a.saved_states = static_cast<float *>(saved);
+        a.saved_aux = a.saved_states + units * (size_t)(d->T / carve::kSub) * d->dv * d->dk;
+    }
+    a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
+    cudaError_t e = carve::launch_fwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const void *v,
+                       const float *g_logit, const float *bx, const float *w_logit,
+                       const float *A, const float *Bm, const float *S0,
+                       const float *m_prev_in, const void *saved, const void *dO,
+                       const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
+                       void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
+                       float *dB, float *dS0, float *dm_prev_in, void *workspace,
+                       void *stream) {
+    carve_status st = check_dims(d, true);
+    if (st != CARVE_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
+        !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(S0) || !ok_opt(m_prev_in) || !ok_ptr(saved) || !ok_ptr(dO) ||
+        !ok_opt(dS_final) || !ok_opt(dm_prev_out) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
+        !ok_ptr(dg_logit) || !ok_ptr(dbx) || !ok_ptr(dw_logit) || !ok_ptr(dA) || !ok_ptr(dB) || !ok_opt(dS0) ||
+        !ok_opt(dm_prev_in) || !ok_ptr(workspace))
+        return CARVE_ERR_INVALID_ARG;
+    (void)S0;
+    (void)m_prev_in;  // their effect is captured by the saved states and content signals
+    carve::BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
+    const size_t units = (size_t)d->B * d->H;
+    a.saved_states = static_cast<const float *>(saved);
+    a.saved_aux = a.saved_states + units * (size_t)(d->T / carve::kSub) * d->dv * d->dk;
+    a.dO = dO; a.dS_final = dS_final; a.dm_prev_out = dm_prev_out;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg_logit = dg_logit; a.dbx = dbx; a.dw_logit = dw_logit;
+    a.dS0 = dS0; a.dm_prev_in = dm_prev_in; a.ws = static_cast<float *>(workspace);
+    a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
+    cudaError_t e = carve::launch_bwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_step(const carve_dims *d, const void *q, const void *k, const void *v,
+                        const float *g_logit, const float *bx, const float *w_logit,
+                        const float *A, const float *Bm, float *S, float *mstate, int32_t *pos,
+                        void *o, void *stream) {
+    carve_status st = check_dims(d, false);
+    if (st != CARVE_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
+        !ok_ptr(A) || !ok_ptr(Bm) || !ok_ptr(S) || !ok_ptr(o))
+        return CARVE_ERR_INVALID_ARG;
+    if (d->mc_mode == CARVE_MC_PREV_MEAN_O && (!ok_ptr(mstate) || !ok_ptr(pos))) return CARVE_ERR_INVALID_ARG;
+    cudaError_t e = carve::launch_step(d->dk, d->dv, d->io == CARVE_IO_BF16, q, k, v, g_logit, bx, w_logit, A, Bm, S,
+                                       mstate, pos, o, d->B, d->H, d->rank, d->chunk, d->mc_mode,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+}  // extern "C"

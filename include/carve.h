@@ -1,0 +1,143 @@
+/*
+ * carve.h -- C ABI of the B200 (sm_100a) CARVE recurrence library (libcarve.so).
+ *
+ * CARVE ("Content-Aware Recurrent with Value Efficiency for Chunk-Parallel Linear
+ * Attention") keeps, per batch element b and head h, a state S in R^{dv x dk} and updates it
+ * token by token with a key-axis gated delta rule (CARVE blog, liuzhao09.github.io,
+ * section 2.1; gist.science technical summary, section 2):
+ *
+ *   for each chunk c of `chunk` tokens:
+ *     m_c   = S_[c-1] . mean_{t in c} q_t            (mc_mode 0, chunk-boundary state readout,
+ *                                                     paperdance abstract)
+ *           | mean_{t in c-1} o_t                     (mc_mode 1, previous-chunk mean output,
+ *                                                     CARVE blog section 2.2)
+ *     Delta = A (Bm m_c)                              (U_b = A.Bm, zero-initialisable low rank)
+ *     for t in c:
+ *       a_t = exp(-softplus(g_logit_t)) * sigmoid(bx_t + Delta)      (key axis, length dk)
+ *       w_t = sigmoid(w_logit_t)                                      (one scalar per head)
+ *       S_t = S_{t-1} Diag(a_t) + w_t (v_t - S_{t-1} Diag(a_t) k_t) k_t^T
+ *       o_t = S_t q_t
+ *
+ * The library evaluates this chunk-parallel in WY form on the GPU (one triangular solve per
+ * chunk shared by all value channels; CARVE blog section 2.3).  Every entry point is
+ * stream-ordered on the caller's stream, allocates nothing, frees nothing and never
+ * synchronises the device.  All pointers are DEVICE pointers unless stated otherwise; the
+ * caller owns every buffer.  Arguments are validated on the host before any launch; a
+ * rejected call launches nothing and returns a non-zero status.  No entry point keeps
+ * mutable global state, so concurrent calls on different streams with disjoint buffers are
+ * safe.
+ *
+ * Tensor layouts (contiguous, row-major; "io" = CARVE_IO_FP32 -> float, CARVE_IO_BF16 ->
+ * bfloat16 stored as 16-bit words):
+ *   q, k           [B, T, H, dk]  io        v, o           [B, T, H, dv]  io
+ *   g_logit, bx    [B, T, H, dk]  float     w_logit        [B, T, H]      float
+ *   A              [H, dk, rank]  float     Bm             [H, rank, dv]  float
+ *   S0, S_final    [B, H, dv, dk] float     m vectors      [B, H, dv]     float
+ * Gradients have the layout and dtype of the tensor they belong to.  Every device pointer
+ * must be 16-byte aligned.
+ *
+ * Supported shapes: dk, dv in {64, 128}; 1 <= rank <= 64; chunk in {16, 32, 64, 128};
+ * T a multiple of 16 (a shorter last chunk is allowed: its mean runs over its own tokens).
+ */
+#ifndef CARVE_H
+#define CARVE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CARVE_OK = 0,
+    CARVE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad dimension or enum value    */
+    CARVE_ERR_UNSUPPORTED = 2,  /* well-formed but outside the supported shape set above    */
+    CARVE_ERR_CUDA = 3,         /* a CUDA launch or attribute call failed                   */
+    CARVE_ERR_TIMEOUT = 4       /* a bounded device-side wait expired (reported, not hung)  */
+} carve_status;
+
+typedef enum { CARVE_IO_FP32 = 0, CARVE_IO_BF16 = 1 } carve_io;
+
+typedef enum {
+    CARVE_MC_BOUNDARY_STATE = 0, /* m_c = S_[c-1] mean(q_c)           */
+    CARVE_MC_PREV_MEAN_O = 1     /* m_c = mean of chunk c-1's outputs */
+} carve_mc_mode;
+
+/* Problem description shared by every entry point.  io and mc_mode take the enum values
+ * above.  For carve_step, T is ignored and chunk is the block length of mc_mode 1. */
+typedef struct {
+    int B, H, T, dk, dv, rank, chunk;
+    int io;
+    int mc_mode;
+} carve_dims;
+
+/* Human-readable name of a status code (static storage). */
+const char *carve_status_string(carve_status s);
+
+/* Size in bytes of the `saved` buffer that carve_fwd fills for carve_bwd (chunk-boundary
+ * states and per-chunk content signals).  0 if the dims are invalid. */
+size_t carve_saved_bytes(const carve_dims *d);
+
+/* Size in bytes of the scratch buffer carve_bwd needs.  0 if the dims are invalid. */
+size_t carve_bwd_workspace_bytes(const carve_dims *d);
+
+/*
+ * carve_fwd -- the forward recurrence over T tokens (the chunked WY evaluation of the
+ * definition above; CARVE blog sections 2.1-2.3, paperdance abstract).
+ *   S0          nullable: initial state (treated as 0 when NULL)
+ *   m_prev_in   nullable: mc_mode 1 content signal for the first chunk (0 when NULL)
+ *   o           out: outputs
+ *   S_final     nullable out: state after the last token
+ *   m_prev_out  nullable out: mean output of the last chunk (the m_prev_in of a chained call)
+ *   saved       nullable out: carve_saved_bytes(d) bytes, required if carve_bwd follows
+ *   stream      a cudaStream_t (NULL = legacy default stream)
+ */
+carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
+                       const float *g_logit, const float *bx, const float *w_logit,
+                       const float *A, const float *Bm, const float *S0,
+                       const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
+                       void *saved, void *stream);
+
+/*
+ * carve_bwd -- reverse sweep over the chunks: gradients of
+ *   sum(dO*o) + sum(dS_final*S_final) + sum(dm_prev_out*m_prev_out)
+ * with respect to every input of carve_fwd.  The forward inputs and the `saved` buffer of
+ * the matching carve_fwd call must be passed unchanged.  dA and dB are overwritten (summed
+ * over the batch), not accumulated.
+ *   dS_final, dm_prev_out   nullable (0 when NULL)
+ *   dS0, dm_prev_in         nullable outputs
+ *   workspace               carve_bwd_workspace_bytes(d) bytes of scratch
+ */
+carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const void *v,
+                       const float *g_logit, const float *bx, const float *w_logit,
+                       const float *A, const float *Bm, const float *S0,
+                       const float *m_prev_in, const void *saved, const void *dO,
+                       const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
+                       void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
+                       float *dB, float *dS0, float *dm_prev_in, void *workspace,
+                       void *stream);
+
+/*
+ * carve_step -- one decode token for every (b,h) (the recurrence above with T = 1;
+ * inference costs O(dv dk) per token, CARVE blog Table 1).
+ *   mc_mode 0: content signal read from the state before this token, m = S q (the chunk
+ *              mean over future tokens does not exist while decoding; this is the L = 1
+ *              readout).
+ *   mc_mode 1: content signal = mean output of the previous complete block of d->chunk
+ *              tokens.  mstate [B,H,2,dv] float holds (sum of o in the current block, mean
+ *              of the previous block) and pos [B,H] int32 the tokens consumed so far; both
+ *              are updated in place.  Unused (may be NULL) in mc_mode 0.
+ * Inputs: q, k [B,H,dk] io; v [B,H,dv] io; g_logit, bx [B,H,dk] float; w_logit [B,H]
+ * float.  S [B,H,dv,dk] float is read and written in place; o [B,H,dv] io.
+ */
+carve_status carve_step(const carve_dims *d, const void *q, const void *k, const void *v,
+                        const float *g_logit, const float *bx, const float *w_logit,
+                        const float *A, const float *Bm, float *S, float *mstate, int32_t *pos,
+                        void *o, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CARVE_H */

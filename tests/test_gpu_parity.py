@@ -1,0 +1,243 @@
+"""GPU (libcarve.so through its C ABI) against the fp64 oracle, element by element.
+
+Tolerance: relative L2 over each whole tensor, 1e-5 with fp32 I/O and 2e-2 with bf16
+q/k/v/o (fp32 gates, state and accumulation).  The oracle reads the bf16-rounded inputs
+exactly.  Full-size workloads are compared on sampled (batch, head) units, which are
+independent except for dA/dB (sampled heads keep every batch element so those sums are
+exact).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import chunk_gated_delta_b200 as carve
+import oracle
+from chunk_gated_delta_b200 import inputs as I
+from tests.helpers import TOL, host, rel_l2, sub_units, to_dev
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ("dq", "dk", "dv", "dg_logit", "dbx", "dw_logit", "dA", "dB")
+
+
+def gpu_fwd(dev, dd, L, mode, S0=None, mp=None):
+    return carve.carve_fwd(dd["q"], dd["k"], dd["v"], dd["g_logit"], dd["bx"], dd["w_logit"], dd["A"], dd["B"],
+                           chunk=L, mc_mode=mode, S0=S0, m_prev_in=mp)
+
+
+def gpu_bwd(dd, saved, L, mode, dS_final=None, dm_prev_out=None):
+    return carve.carve_bwd(dd["q"], dd["k"], dd["v"], dd["g_logit"], dd["bx"], dd["w_logit"], dd["A"], dd["B"],
+                           saved, dd["dO"], chunk=L, mc_mode=mode, dS_final=dS_final, dm_prev_out=dm_prev_out)
+
+
+def check(name, got, ref, tol):
+    e = rel_l2(got, ref)
+    assert e <= tol, f"{name}: rel-L2 {e:.3e} > {tol:.1e}"
+    return e
+
+
+def run_case(cuda_device, w, d, dO, L, mode, S0=None, mp=None, dSf=None, dmo=None, units=None, bwd=True):
+    """GPU fwd(+bwd) on the whole workload; oracle on `units` = (bs, hs) (all by default)."""
+    import torch
+    dd = to_dev(d if dO is None else dict(d, dO=dO), w.io, cuda_device)
+    tS0 = None if S0 is None else torch.from_numpy(S0).to(cuda_device)
+    tmp = None if mp is None else torch.from_numpy(mp).to(cuda_device)
+    out = gpu_fwd(cuda_device, dd, L, mode, tS0, tmp)
+    g = None
+    if bwd:
+        tdS = None if dSf is None else torch.from_numpy(dSf).to(cuda_device)
+        tdm = None if dmo is None else torch.from_numpy(dmo).to(cuda_device)
+        g = gpu_bwd(dd, out["saved"], L, mode, tdS, tdm)
+    torch.cuda.synchronize()
+    bs, hs = units if units is not None else (slice(None), slice(None))
+    od = sub_units(d, bs, hs)
+    sl = lambda x: None if x is None else x[bs][:, hs]   # noqa: E731
+    r = oracle.fwd(od, L=L, mc_mode=mode, S0=sl(S0), m_prev=sl(mp))
+    tol = TOL[w.io]
+    errs = {}
+    errs["o"] = check("o", host(out["o"])[bs][:, :, hs], r["o"], tol)
+    errs["S_final"] = check("S_final", host(out["S_final"])[bs][:, hs], r["S_final"], tol)
+    errs["m_prev_out"] = check("m_prev_out", host(out["m_prev_out"])[bs][:, hs], r["m_prev_out"], tol)
+    if bwd:
+        rg = oracle.bwd(od, L, dO[bs][:, :, hs], mc_mode=mode, S0=sl(S0), m_prev=sl(mp), dS_final=sl(dSf),
+                        dm_prev_out=sl(dmo))
+        for key in GRADS:
+            gk = host(g[key])
+            gk = gk[hs] if key in ("dA", "dB") else gk[bs][:, :, hs]
+            errs[key] = check(key, gk, rg[key], tol)
+        errs["dS0"] = check("dS0", host(g["dS0"])[bs][:, hs], rg["dS0"], tol)
+        if mode == 1:
+            errs["dm_prev_in"] = check("dm_prev_in", host(g["dm_prev_in"])[bs][:, hs], rg["dm_prev_in"], tol)
+    return errs
+
+
+def small(w, **kw):
+    w = dataclasses.replace(w, **kw)
+    d = I.make_inputs(w)
+    dO = I.make_grad_out(w)
+    return w, d, dO
+
+
+# ---------------------------------------------------------------------------------------
+# tiny fp32 workload (B1 H2 T256 d64 L64, rank 16): forward and backward at 1e-5
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", [0, 1])
+def test_tiny_fp32(cuda_device, mode):
+    w, d, dO = small(I.TINY_FP32)
+    errs = run_case(cuda_device, w, d, dO, w.L, mode)
+    print(w.name, mode, {k: f"{v:.2e}" for k, v in errs.items()})
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_tiny_fp32_carried_state_and_signal(cuda_device, mode):
+    """Non-zero S0, m_prev_in, dS_final and dm_prev_out, a ragged last chunk (T = 80, L = 32)."""
+    w, d, dO = small(I.TINY_FP32, T=80, L=32, seed=77)
+    d["A"] *= 10.0
+    d["B"] *= 10.0
+    S0 = I.make_state(w, 0.1)
+    mp = I.normal(1, 2, (w.B, w.H, w.V)).astype(np.float32)
+    dSf = I.normal(1, 3, (w.B, w.H, w.V, w.K)).astype(np.float32)
+    dmo = I.normal(1, 4, (w.B, w.H, w.V)).astype(np.float32)
+    run_case(cuda_device, w, d, dO, 32, mode, S0=S0, mp=mp, dSf=dSf, dmo=dmo)
+
+
+@pytest.mark.parametrize("K,V", [(64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("io", ["fp32", "bf16"])
+def test_shapes_and_dtypes(cuda_device, K, V, io):
+    w, d, dO = small(I.TINY_FP32, B=2, H=3, T=96, K=K, V=V, R=8, L=32, io=io, seed=K + V)
+    d["A"] *= 10.0
+    d["B"] *= 10.0
+    for mode in (0, 1):
+        run_case(cuda_device, w, d, dO, 32, mode)
+
+
+@pytest.mark.parametrize("L", [16, 32, 64, 128])
+def test_chunk_lengths_bf16(cuda_device, L):
+    w, d, dO = small(I.FWD_1P3B, B=1, H=4, T=384, L=L, seed=5 + L)
+    d["A"] *= 10.0
+    d["B"] *= 10.0
+    for mode in (0, 1):
+        run_case(cuda_device, w, d, dO, L, mode)
+
+
+def test_zero_projection_is_chunk_length_invariant_bitwise(cuda_device):
+    """U_b = 0 (A = 0): the erase gate is sigmoid(bx + 0) = sigmoid(bx) exactly, so the GPU
+    result cannot depend on the gate grouping L at all -- bitwise -- and matches the oracle's
+    key-axis baseline (content path removed)."""
+    import torch
+    w, d, dO = small(I.FWD_1P3B, B=2, H=2, T=256, seed=9)
+    d["A"][:] = 0.0
+    dd = to_dev(d, w.io, cuda_device)
+    outs = [gpu_fwd(cuda_device, dd, L, 0) for L in (16, 32, 64, 128)]
+    outs += [gpu_fwd(cuda_device, dd, 64, 1)]
+    torch.cuda.synchronize()
+    for x in outs[1:]:
+        assert torch.equal(x["o"], outs[0]["o"]) and torch.equal(x["S_final"], outs[0]["S_final"])
+    base = oracle.fwd(d, L=64, content_off=True)
+    check("o", host(outs[0]["o"]), base["o"], TOL["bf16"])
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_chaining_is_bitwise(cuda_device, mode):
+    """fwd(T) == fwd(first half) then fwd(second half) carrying S and m (checkpoint/resume)."""
+    import torch
+    w, d, dO = small(I.FWD_1P3B, B=2, H=3, T=512, seed=31)
+    d["A"] *= 10.0
+    d["B"] *= 10.0
+    dd = to_dev(d, w.io, cuda_device)
+    full = gpu_fwd(cuda_device, dd, 64, mode)
+    half = {k: (v[:, :256].contiguous() if v.dim() >= 3 and k not in ("A", "B") else v) for k, v in dd.items()}
+    rest = {k: (v[:, 256:].contiguous() if v.dim() >= 3 and k not in ("A", "B") else v) for k, v in dd.items()}
+    a = gpu_fwd(cuda_device, half, 64, mode)
+    b = gpu_fwd(cuda_device, rest, 64, mode, S0=a["S_final"], mp=a["m_prev_out"])
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([a["o"], b["o"]], dim=1), full["o"])
+    assert torch.equal(b["S_final"], full["S_final"])
+    assert torch.equal(b["m_prev_out"], full["m_prev_out"])
+
+
+# ---------------------------------------------------------------------------------------
+# full-size workloads
+# ---------------------------------------------------------------------------------------
+def test_fwd_1p3b_layer(cuda_device):
+    """B4 H16 T2048 d128 L64 rank 32, bf16 forward; 8 sampled units."""
+    w = I.FWD_1P3B
+    d = I.make_inputs(w)
+    errs = run_case(cuda_device, w, d, None, w.L, 0, units=([0, 3], [0, 5, 10, 15]), bwd=False)
+    print(w.name, {k: f"{v:.2e}" for k, v in errs.items()})
+
+
+def test_train_1p3b_layer(cuda_device):
+    """B8 H16 T4096 d128 L64 rank 32, bf16 forward + backward; heads 0 and 9 (every batch)."""
+    w = I.TRAIN_1P3B
+    d = I.make_inputs(w)
+    dO = I.make_grad_out(w)
+    errs = run_case(cuda_device, w, d, dO, w.L, 0, units=(list(range(w.B)), [0, 9]))
+    print(w.name, {k: f"{v:.2e}" for k, v in errs.items()})
+
+
+@pytest.fixture(scope="module")
+def long_inputs():
+    w = I.long_context(64, 0)
+    return I.make_inputs(w), I.make_grad_out(w)
+
+
+@pytest.mark.parametrize("L", [32, 64, 128])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_long_context(cuda_device, long_inputs, L, mode):
+    """B1 H16 T65536 d128, bf16 forward + backward at L in {32, 64, 128}, both readouts;
+    one sampled head (the oracle is sequential per unit)."""
+    w = I.long_context(L, mode)
+    d, dO = long_inputs
+    errs = run_case(cuda_device, w, d, dO, L, mode, units=([0], [3]))
+    print(w.name, {k: f"{v:.2e}" for k, v in errs.items()})
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_decode_1000_steps(cuda_device, mode):
+    """B256 H16 d128: 1000 consecutive decode steps, fp32 state ~ N(0, 0.05^2) in place,
+    bf16 q/k/v, per-token gates (a pool of 64 seeded token sets cycled).  Six sampled units
+    are replayed by the oracle step by step; every step's output and the final state are
+    compared."""
+    import torch
+    w = I.DECODE
+    L = 64
+    pool = I.make_decode_pool(w, pool=64)
+    S_np = I.make_state(w, 0.05)
+    dev = cuda_device
+    tp = to_dev({k: pool[k] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}, "bf16", dev)
+    A = torch.from_numpy(pool["A"]).to(dev)
+    Bm = torch.from_numpy(pool["B"]).to(dev)
+    S = torch.from_numpy(S_np).to(dev)
+    mstate = torch.zeros((w.B, w.H, 2, w.V), dtype=torch.float32, device=dev)
+    pos = torch.zeros((w.B, w.H), dtype=torch.int32, device=dev)
+    units = [(0, 0), (17, 3), (100, 8), (128, 15), (200, 1), (255, 12)]
+    bi = [u[0] for u in units]
+    hi = [u[1] for u in units]
+    outs = []
+    for j in range(w.steps):
+        p = j % 64
+        o = carve.carve_step(tp["q"][p], tp["k"][p], tp["v"][p], tp["g_logit"][p], tp["bx"][p], tp["w_logit"][p], A,
+                             Bm, S, mc_mode=mode, chunk=L, mstate=mstate, pos=pos)
+        outs.append(o[bi, hi].float())
+    torch.cuda.synchronize()
+    go = torch.stack(outs).cpu().numpy()
+    # oracle: the same units, token by token
+    Sr = S_np[bi, hi][:, None].astype(np.float64).copy()          # [6,1,V,K]
+    A_r = pool["A"][hi][:, None]                                    # per-unit head factors
+    ms = np.zeros((len(units), 1, 2, w.V))
+    ps = np.zeros((len(units), 1), dtype=np.int32)
+    ref = np.zeros_like(go)
+    for n, (b, h) in enumerate(units):
+        Sn = Sr[n:n + 1]
+        msn, psn = ms[n:n + 1], ps[n:n + 1]
+        for j in range(w.steps):
+            p = j % 64
+            tok = {k: pool[k][p][b:b + 1, h:h + 1] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}
+            tok = {k: np.asarray(v, dtype=np.float64) for k, v in tok.items()}
+            ref[j, n] = oracle.step(tok, A_r[n], pool["B"][h][None], Sn, L=L, mc_mode=mode, mstate=msn, pos=psn)[0, 0]
+    check("o (all steps)", go, ref, TOL["bf16"])
+    check("S after 1000 steps", host(S)[bi, hi], Sr[:, 0], TOL["bf16"])
+    if mode == 1:
+        assert torch.all(pos == w.steps)
