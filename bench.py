@@ -336,14 +336,17 @@ def measure_e2e(args, host, dv_, step, stream, ws, w, grads):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="carve", choices=["carve", "reference"])
     ap.add_argument("--workload", default="train", choices=["train"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
     args = ap.parse_args()
     w = I.TRAIN_1P3B
+    if args.batch:
+        w = dataclasses.replace(w, B=args.batch, name=w.name.replace("_B8_", f"_B{args.batch}_"))
     if args.impl == "reference":
         run_reference(args, w)
     else:
