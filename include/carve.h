@@ -23,7 +23,8 @@
  * stream-ordered on the caller's stream, allocates nothing, frees nothing and never
  * synchronises the device.  All pointers are DEVICE pointers unless stated otherwise; the
  * caller owns every buffer.  Arguments are validated on the host before any launch; a
- * rejected call launches nothing and returns a non-zero status.  No entry point keeps
+ * rejected call launches nothing and returns a non-zero status.  Apart from
+ * carve_bwd_noalloc (which shares one scratch array, see below), no entry point keeps
  * mutable global state, so concurrent calls on different streams with disjoint buffers are
  * safe.
  *
@@ -117,6 +118,32 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
                        void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
                        float *dB, float *dS0, float *dm_prev_in, void *workspace,
                        void *stream);
+
+/*
+ * carve_bwd_noalloc -- carve_bwd without a workspace argument, for callers that cannot
+ * allocate device memory when they run the backward (for example a plugin inside a host
+ * framework that owns all device memory and passes in only input and output buffers, or a
+ * latency-critical loop that must avoid cudaMalloc's implicit synchronisation).  The pages
+ * have no counterpart to this entry point; it only changes where the scratch lives.
+ *
+ * Arguments, layouts, results and errors are those of carve_bwd.  The scratch is a 4 MiB
+ * array inside the library, present on every GPU that loads it until the process exits, so
+ * the call allocates nothing.  Limit: carve_bwd_workspace_bytes(d) <= 4 MiB, that is
+ * B*H*(dk*rank + rank*dv) <= 1,048,576; larger problems return CARVE_ERR_UNSUPPORTED
+ * without launching anything.
+ * The first call on each device looks up the array's device address (with that device
+ * current) and caches it; make that first call before any stream capture begins.
+ * Every call shares the one array: calls that overlap on the GPU (different streams, or
+ * threads racing on one device) corrupt each other's dA/dB.  Serialise them.
+ */
+carve_status carve_bwd_noalloc(const carve_dims *d, const void *q, const void *k, const void *v,
+                               const float *g_logit, const float *bx, const float *w_logit,
+                               const float *A, const float *Bm, const float *S0,
+                               const float *m_prev_in, const void *saved, const void *dO,
+                               const float *dS_final, const float *dm_prev_out, void *dq,
+                               void *dk, void *dv, float *dg_logit, float *dbx,
+                               float *dw_logit, float *dA, float *dB, float *dS0,
+                               float *dm_prev_in, void *stream);
 
 /*
  * carve_step -- one decode token for every (b,h) (the recurrence above with T = 1;
