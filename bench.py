@@ -145,7 +145,7 @@ def max_over_ranks(x: float, ws: int) -> float:
     return float(t.item())
 
 
-def cpu_oracle_sample(w, d, dO, target_s=12.0, max_T=None):
+def cpu_oracle_sample(w, d, dO, target_s=12.0, max_T=None, fwd_only=False):
     """Time the fp64 oracle (fwd + bwd) on batch element 0 (all heads) over a prefix of the
     sequence, doubling the prefix until the run takes at least target_s / 2 seconds.
     Returns (tokens/s of the whole layer, cores used, sample description)."""
@@ -156,12 +156,14 @@ def cpu_oracle_sample(w, d, dO, target_s=12.0, max_T=None):
         sub = {k: (v[:1, :T] if v.ndim >= 3 and k not in ("A", "B") else v) for k, v in d.items()}
         t0 = time.perf_counter()
         oracle.fwd(sub, L=w.L, mc_mode=w.mc_mode)
-        oracle.bwd(sub, w.L, dO[:1, :T], mc_mode=w.mc_mode)
+        if not fwd_only:
+            oracle.bwd(sub, w.L, dO[:1, :T], mc_mode=w.mc_mode)
         dt = time.perf_counter() - t0
         if dt >= target_s / 2 or T >= max_T:
             break
         T = min(max_T, T * 2)
-    return T / dt, oracle.threads(), f"oracle fwd+bwd, batch 0 (all {w.H} heads), first {T} of {w.T} tokens"
+    what = "fwd" if fwd_only else "fwd+bwd"
+    return T / dt, oracle.threads(), f"oracle {what}, batch 0 (all {w.H} heads), first {T} of {w.T} tokens"
 
 
 # ---------------------------------------------------------------------------------------
@@ -195,7 +197,7 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def run_train(args, w):
+def run_train(args, w, fwd_only=False):
     import torch
     import chunk_gated_delta_b200 as carve
     ws, rank, local = dist_setup()
@@ -216,9 +218,11 @@ def run_train(args, w):
     torch.cuda.synchronize()
     L, mode = w.L, w.mc_mode
     fwd_out = carve.carve_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
-                              dv_["B"], chunk=L, mc_mode=mode)
-    bwd_out = carve.carve_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
-                              dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode)
+                              dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only)
+    bwd_out = None
+    if not fwd_only:
+        bwd_out = carve.carve_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
+                                  dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode)
     workspace = torch.empty(carve.bwd_workspace_bytes(carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode)),
                             dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -227,9 +231,13 @@ def run_train(args, w):
         if ev is not None:
             ev[0].record(stream)
         carve.carve_fwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"], chunk=L,
-                        mc_mode=mode, out=fwd_out)
+                        mc_mode=mode, out=fwd_out, save_for_bwd=not fwd_only)
         if ev is not None:
             ev[1].record(stream)
+        if fwd_only:
+            if ev is not None:
+                ev[2].record(stream)
+            return
         carve.carve_bwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"],
                         fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace)
         if ev is not None:
@@ -258,23 +266,26 @@ def run_train(args, w):
 
     th = w.B * w.T * w.H          # token-heads of one rank's launch
     dd = w.K
-    kern = {"carve_fwd": (fwd_ms, fwd_bytes(dd, L) * th), "carve_bwd": (bwd_ms, bwd_bytes(dd, L) * th)}
+    if fwd_only:
+        kern = {"carve_fwd": (fwd_ms, 2052 * th)}
+    else:
+        kern = {"carve_fwd": (fwd_ms, fwd_bytes(dd, L) * th), "carve_bwd": (bwd_ms, bwd_bytes(dd, L) * th)}
     dom = max(kern, key=lambda k: kern[k][0])
     dms, dbytes = kern[dom]
     achieved = dbytes / (dms * 1e-3) / 1e9
-    flops = (fwd_flops(dd, L, w.R) + bwd_flops(dd, L, w.R)) * th * ws
+    flops = (fwd_flops(dd, L, w.R) + (0 if fwd_only else bwd_flops(dd, L, w.R))) * th * ws
     tensor_frac = flops / (ms * 1e-3) / (peaks["bf16"] * 1e12 * ws)
     traffic = load_traffic(dom)
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(args, host, dv_, step, stream, ws, w, bwd_out)
+        e2e = measure_e2e(args, host, dv_, step, stream, ws, w, {"o": fwd_out["o"]} if fwd_only else bwd_out)
     cpu = None
     if not args.no_cpu_baseline and rank == 0 and ws == 1:
-        v, cores, sample = cpu_oracle_sample(w, d, dO)
+        v, cores, sample = cpu_oracle_sample(w, d, dO, fwd_only=fwd_only)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "metric": "fwd tokens/s per layer (B200, 16 heads, d=128)" if fwd_only else METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "heads": w.H, "d": w.K,
@@ -284,7 +295,7 @@ def run_train(args, w):
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm"], "traffic": traffic, "peak_source": peaks["source"]},
         "kernels_ms": {"carve_fwd": fwd_ms, "carve_bwd": bwd_ms},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (1 if fwd_only else 3) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0:
@@ -339,7 +350,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="carve", choices=["carve", "reference"])
-    ap.add_argument("--workload", default="train", choices=["train"])
+    ap.add_argument("--workload", default="train", choices=["train", "fwd"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
@@ -347,10 +358,12 @@ def main():
     w = I.TRAIN_1P3B
     if args.batch:
         w = dataclasses.replace(w, B=args.batch, name=w.name.replace("_B8_", f"_B{args.batch}_"))
+    if args.workload == "fwd":
+        w = I.FWD_1P3B
     if args.impl == "reference":
         run_reference(args, w)
     else:
-        run_train(args, w)
+        run_train(args, w, fwd_only=args.workload == "fwd")
 
 
 if __name__ == "__main__":

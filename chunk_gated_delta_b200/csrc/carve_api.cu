@@ -7,6 +7,8 @@
 
 namespace carve {
 cudaError_t launch_fwd_simt(int K, int V, bool bf16, const FwdArgs &a, cudaStream_t st);
+cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st);
+int tc_compute_chunk(int L);
 cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit, const float *A,
@@ -40,6 +42,14 @@ carve_status check_dims(const carve_dims *d, bool seq) {
 }
 
 size_t n_chunks(const carve_dims *d) { return (size_t)((d->T + d->chunk - 1) / d->chunk); }
+
+// The tensor-core kernels cover bf16 I/O with dk = dv = 128, rank <= 32 and gate chunks of 32,
+// 64 or 128 tokens when T is a multiple of the compute chunk; everything else runs the SIMT
+// kernels.
+bool use_tc_fwd(const carve_dims *d) {
+    const int C = carve::tc_compute_chunk(d->chunk);
+    return d->io == CARVE_IO_BF16 && d->dk == 128 && d->dv == 128 && d->rank <= 32 && C > 0 && d->T % C == 0;
+}
 
 }  // namespace
 
@@ -89,7 +99,11 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
         a.saved_aux = a.saved_states + units * (size_t)(d->T / carve::kSub) * d->dv * d->dk;
     }
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
-    cudaError_t e = carve::launch_fwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (use_tc_fwd(d) && saved == nullptr)
+        e = carve::launch_fwd_tc(a, static_cast<cudaStream_t>(stream));
+    else
+        e = carve::launch_fwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 

@@ -25,6 +25,42 @@ __device__ __forceinline__ float log_retention(float g_logit, float beta) {
     return -softplus_f(g_logit) - softplus_f(-beta);
 }
 
+// Content signal of a chunk: z = Bh m (R outputs, dot products over V) then
+// Delta = Ah z (K outputs over R).  Bh is [R][V], Ah is [K][R] (row-major, global or shared);
+// every thread of the CTA must call this.  Eight threads share each z output and
+// kThreads / K share each Delta output, so the loads of one output are issued together.
+template <int K, int V>
+__device__ __forceinline__ void content_signal(const float *Bh, const float *Ah, const float *m, float *z,
+                                               float *delta, int R) {
+    const int tid = threadIdx.x;
+    for (int j0 = 0; j0 < R; j0 += kThreads / 8) {
+        const int j = j0 + tid / 8, part = tid % 8;
+        float acc = 0.f;
+        if (j < R) {
+            const float *row = Bh + (size_t)j * V;
+#pragma unroll
+            for (int r = part; r < V; r += 8) acc += row[r] * m[r];
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (j < R && part == 0) z[j] = acc;
+    }
+    __syncthreads();
+    constexpr int TPO = kThreads / K;
+    {
+        const int kk = tid / TPO, part = tid % TPO;
+        const float *row = Ah + (size_t)kk * R;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = part; j < R; j += TPO) acc += row[j] * z[j];
+#pragma unroll
+        for (int off = TPO / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (part == 0) delta[kk] = acc;
+    }
+    __syncthreads();
+}
+
 struct FwdArgs {
     const void *q, *k, *v;
     const float *g_logit, *bx, *w_logit, *A, *Bm, *S0, *m_prev_in;

@@ -94,17 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
             mvec[tid] = mprev[tid];
         }
         __syncthreads();
-        if (tid < R) {
-            float z = 0.f;
-            for (int r = 0; r < V; ++r) z += a.Bm[((size_t)h * R + tid) * V + r] * mvec[r];
-            zvec[tid] = z;
-        }
-        __syncthreads();
-        if (tid < K) {
-            float d = 0.f;
-            for (int j = 0; j < R; ++j) d += a.A[((size_t)h * K + tid) * R + j] * zvec[j];
-            delta[tid] = d;
-        }
+        content_signal<K, V>(a.Bm + (size_t)h * R * V, a.A + (size_t)h * K * R, mvec, zvec, delta, R);
         if (tid < V) osum[tid] = 0.f;
         __syncthreads();
         if (a.saved_aux) {
@@ -525,16 +515,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
             __syncthreads();
         }
         // ---- chunk start: Delta = A z, z = Bm m
-        if (tid < R) {
+        for (int j0 = 0; j0 < R; j0 += kThreads / 8) {   // dz = A^T dDelta, 8 threads per output
+            const int j = j0 + tid / 8, part = tid % 8;
             float s = 0.f;
-            for (int i = 0; i < K; ++i) s += a.A[((size_t)h * K + i) * R + tid] * ddelta[i];
-            dzv[tid] = s;
+            if (j < R)
+#pragma unroll
+                for (int i = part; i < K; i += 8) s += a.A[((size_t)h * K + i) * R + j] * ddelta[i];
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            if (j < R && part == 0) dzv[j] = s;
         }
         __syncthreads();
         for (int idx = tid; idx < K * R; idx += kThreads) wsu[idx] += ddelta[idx / R] * zvec[idx % R];
         for (int idx = tid; idx < R * V; idx += kThreads) wsu[K * R + idx] += dzv[idx / V] * mvec[idx % V];
         if (tid < V) {
             float s = 0.f;
+#pragma unroll 8
             for (int j = 0; j < R; ++j) s += a.Bm[((size_t)h * R + j) * V + tid] * dzv[j];
             dmv[tid] = s;
         }

@@ -1,0 +1,499 @@
+// CARVE forward, tensor-core kernel for bf16 q/k/v/o with dk = dv = 128.
+//
+// One CTA (8 warps) per (batch, head) unit sweeps the sequence in compute chunks of
+// C = 16*NB tokens (C = min(chunk, 64); a 128-token gate chunk is two compute chunks sharing
+// one content signal).  Warp w owns state rows v in [16w, 16w+16): its 16x128 slice of the
+// fp32 state lives in registers as mma accumulator fragments for the whole sweep, so the
+// state never round-trips through memory except when it is saved for the backward.
+//
+// Per compute chunk (CARVE blog section 2.3: one WY solve shared by all value channels):
+//   gates      a_t = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)})), floored at e^-10, and its
+//              reciprocal (free), per key channel
+//   operands   mid-block referenced q*e^{Lam_t - Lam_m}, k*e^{Lam_t - Lam_m}, k*e^{Lam_m - Lam_s}
+//              (m = middle of the token's 16-block) built from running products of a and 1/a,
+//              so every factor lies in [e^-80, e^80]; chunk-level factors (block products) carry
+//              the rest and are all <= 1
+//   Gram       Akk, Aqk: block (i,j) = rows_i . diag(e^{Lam_m(i) - Lam_m(j)}) . cols_j^T
+//   G          S0 [Kt; Qt]^T   (Kt = k e^{Lam}, Qt = q e^{Lam})            per warp, mma
+//   solve      X = Diag(w)(V - Kt S0^T);  U_i = (X_i - sum_j U_j M_ij^T) T_ii^T,  T_ii = (I + D A_ii)^-1
+//   output     O^T = S0 Qt^T + U^T Aqk^T                                  per warp, mma
+//   state      S = S Diag(gamma) + U^T Kbar,  Kbar = k e^{Lam_C - Lam}         per warp, mma
+// Raw q/k/v rows are prefetched into shared memory by the bulk-copy (TMA) engine while the
+// previous chunk computes.  The floor a >= e^-10 bounds the deviation from the exact
+// recurrence by e^-10 per step in channels that are being erased anyway.
+#include "carve_device.cuh"
+#include "carve_mma.cuh"
+
+namespace carve {
+
+constexpr int kLdOp = 136;                            // bf16 row stride of 128-wide operand tiles
+constexpr float kAMin = 4.5399929762484854e-05f;      // e^-10
+constexpr float kInvAMin = 22026.465794806718f;       // e^10
+constexpr int kTcMaxRank = 32;                        // low-rank factors staged in shared memory
+
+__device__ int g_tc_timeout;  // set when a bounded wait gives up (never expected)
+
+template <int NB>
+struct __align__(16) TcFwdSmem {
+    static constexpr int C = 16 * NB, LDA = C + 8, NPAIR = NB * (NB - 1) / 2 > 0 ? NB * (NB - 1) / 2 : 1;
+    __nv_bfloat16 rq[C * 128], rk[C * 128], rv[C * 128];
+    __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp], qt[C * kLdOp], kt[C * kLdOp];
+    __nv_bfloat16 aqk[C * LDA], mkk[C * LDA];
+    __nv_bfloat16 tii[NB * 16 * 24];
+    float akk_d[NB * 16 * 17];
+    float p7[NB * 128], r15[NB * 128], dblk[NB * 128], em[NB * 128], fm[NB * 128], cij[NPAIR * 128];
+    float gam[128], wv[C], qbar[128], mvec[128], osum[128], mprev[128], zvec[64], delta[128];
+    float Ah[128 * kTcMaxRank], Bh[kTcMaxRank * 128];   // the head's low-rank factors
+    uint64_t bar;
+    // the output tile is staged in qt once the S-GEMM has consumed it
+    __device__ __nv_bfloat16 *ost() { return qt; }
+};
+
+__device__ __forceinline__ int pair_index(int i, int j) { return i * (i - 1) / 2 + j; }
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <int NB>
+__global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a) {
+    using SM = TcFwdSmem<NB>;
+    constexpr int C = SM::C, LDA = SM::LDA;
+    constexpr int NP = (128 * NB + 255) / 256;  // (channel, block) pairs per thread in the gate phase
+    extern __shared__ __align__(128) unsigned char smraw[];
+    SM &sm = *reinterpret_cast<SM *>(smraw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, c4 = lane & 3;
+    const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
+    const int b = u / H, h = u % H;
+    const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
+    const __nv_bfloat16 *kk = static_cast<const __nv_bfloat16 *>(a.k);
+    const __nv_bfloat16 *vv = static_cast<const __nv_bfloat16 *>(a.v);
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
+    const size_t tstride = (size_t)H * 128;
+    const size_t base_bh = (size_t)b * T * tstride + (size_t)h * 128;   // token 0 of this unit
+    const int v0 = 16 * warp + g, v1 = v0 + 8;
+
+    float s[16][4];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int col = 8 * j + 2 * c4;
+        if (a.S0) {
+            const float *S0 = a.S0 + (size_t)u * 128 * 128;
+            s[j][0] = S0[v0 * 128 + col];
+            s[j][1] = S0[v0 * 128 + col + 1];
+            s[j][2] = S0[v1 * 128 + col];
+            s[j][3] = S0[v1 * 128 + col + 1];
+        } else {
+            s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+        }
+    }
+    if (tid == 0) {
+        mbar_init(&sm.bar, 1);
+        fence_mbar_init();
+    }
+    if (tid < 128) {
+        sm.mprev[tid] = a.m_prev_in ? a.m_prev_in[(size_t)u * 128 + tid] : 0.f;
+        sm.osum[tid] = 0.f;
+    }
+    for (int idx = tid; idx < 128 * R; idx += 256) {
+        sm.Ah[idx] = a.A[(size_t)h * 128 * R + idx];
+        sm.Bh[idx] = a.Bm[(size_t)h * R * 128 + idx];
+    }
+    __syncthreads();
+
+    // raw tile rows of chunk cc: which = 0 (q and k, with the barrier's byte count) or 1 (v)
+    auto issue = [&](int cc, int which) {
+        if (warp != 0) return;
+        if (which == 0 && lane == 0) mbar_expect_tx(&sm.bar, 3u * C * 256u);
+        __syncwarp();
+        for (int r = lane; r < C; r += 32) {
+            const size_t off = base_bh + (size_t)(cc * C + r) * tstride;
+            if (which == 0) {
+                bulk_g2s(sm.rq + r * 128, q + off, 256, &sm.bar);
+                bulk_g2s(sm.rk + r * 128, kk + off, 256, &sm.bar);
+            } else {
+                bulk_g2s(sm.rv + r * 128, vv + off, 256, &sm.bar);
+            }
+        }
+    };
+    issue(0, 0);
+    issue(0, 1);
+    uint32_t phase = 0;
+
+    for (int cc = 0; cc < NCC; ++cc) {
+        const int t0 = cc * C, gc = cc / CPG;
+        const bool first = (cc % CPG) == 0, last = (cc % CPG) == CPG - 1 || cc == NCC - 1;
+        const int n = min(L, T - gc * L);
+        // gate inputs of this chunk, into registers (their latency overlaps the readout)
+        float glr[NP][16], bxr[NP][16];
+#pragma unroll
+        for (int x = 0; x < NP; ++x) {
+            const int p = tid + 256 * x, kch = p & 127, i = p >> 7;
+            if (p < 128 * NB) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const size_t gi = ((size_t)b * T + t0 + 16 * i + t) * tstride + (size_t)h * 128 + kch;
+                    glr[x][t] = a.g_logit[gi];
+                    bxr[x][t] = a.bx[gi];
+                }
+            }
+        }
+        if (!mbar_wait(&sm.bar, phase)) atomicOr(&g_tc_timeout, 1);
+        phase ^= 1u;
+        if (a.saved_states) {
+            float *st = a.saved_states + ((size_t)u * NCC + cc) * 128 * 128;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int col = 8 * j + 2 * c4;
+                *reinterpret_cast<float2 *>(st + v0 * 128 + col) = make_float2(s[j][0], s[j][1]);
+                *reinterpret_cast<float2 *>(st + v1 * 128 + col) = make_float2(s[j][2], s[j][3]);
+            }
+        }
+        // ---- content signal at a gate-chunk start
+        if (first) {
+            if (a.mc_mode == 0) {
+                if (tid < 128) {
+                    float acc = 0.f;
+                    if (CPG == 1) {
+                        for (int t = 0; t < C; ++t) acc += bf(sm.rq[t * 128 + tid]);
+                    } else {
+#pragma unroll 8
+                        for (int t = 0; t < n; ++t) acc += bf(q[base_bh + (size_t)(gc * L + t) * tstride + tid]);
+                    }
+                    sm.qbar[tid] = acc / (float)n;
+                }
+                __syncthreads();
+                float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int col = 8 * j + 2 * c4;
+                    const float q0 = sm.qbar[col], q1 = sm.qbar[col + 1];
+                    p0 += s[j][0] * q0 + s[j][1] * q1;
+                    p1 += s[j][2] * q0 + s[j][3] * q1;
+                }
+                p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+                p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+                if (c4 == 0) {
+                    sm.mvec[v0] = p0;
+                    sm.mvec[v1] = p1;
+                }
+            } else if (tid < 128) {
+                sm.mvec[tid] = sm.mprev[tid];
+            }
+            __syncthreads();
+            content_signal<128, 128>(sm.Bh, sm.Ah, sm.mvec, sm.zvec, sm.delta, R);
+            if (tid < 128) sm.osum[tid] = 0.f;
+            if (a.saved_aux) {
+                float *aux = a.saved_aux + ((size_t)u * NG + gc) * (256 + R);
+                if (tid < 128) {
+                    aux[tid] = sm.mvec[tid];
+                    aux[128 + R + tid] = sm.delta[tid];
+                }
+                if (tid < R) aux[128 + tid] = sm.zvec[tid];
+            }
+        }
+        // ---- gates and mid-block referenced operands, one (channel, 16-block) pair at a time
+#pragma unroll
+        for (int x = 0; x < NP; ++x) {
+            const int p = tid + 256 * x, kch = p & 127, i = p >> 7;
+            if (p < 128 * NB) {
+                const float dl = sm.delta[kch];
+                float av[16], ia[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const float D = (1.f + __expf(glr[x][t])) * (1.f + __expf(-(bxr[x][t] + dl)));
+                    const float r = __fdividef(1.f, D);
+                    const bool floor = !(r >= kAMin);
+                    av[t] = floor ? kAMin : r;
+                    ia[t] = floor ? kInvAMin : D;
+                }
+                float rf[16], cf[16];
+                rf[7] = cf[7] = 1.f;
+#pragma unroll
+                for (int t = 8; t < 16; ++t) {
+                    rf[t] = rf[t - 1] * av[t];
+                    cf[t] = cf[t - 1] * ia[t];
+                }
+#pragma unroll
+                for (int t = 6; t >= 0; --t) {
+                    cf[t] = cf[t + 1] * av[t + 1];
+                    rf[t] = rf[t + 1] * ia[t + 1];
+                }
+                float p7 = 1.f;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) p7 *= av[t];
+                sm.p7[i * 128 + kch] = p7;
+                sm.r15[i * 128 + kch] = rf[15];
+                sm.dblk[i * 128 + kch] = p7 * rf[15];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int row = 16 * i + t;
+                    const float qv = bf(sm.rq[row * 128 + kch]), kv = bf(sm.rk[row * 128 + kch]);
+                    sm.qm[row * kLdOp + kch] = __float2bfloat16_rn(qv * rf[t]);
+                    sm.krm[row * kLdOp + kch] = __float2bfloat16_rn(kv * rf[t]);
+                    sm.kcm[row * kLdOp + kch] = __float2bfloat16_rn(kv * cf[t]);
+                }
+            }
+        }
+        if (tid < C) sm.wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + t0 + tid) * H + h]);
+        __syncthreads();
+        // ---- chunk-level factors per channel
+        if (tid < 128) {
+            float E = 1.f;
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                sm.em[i * 128 + tid] = E * sm.p7[i * 128 + tid];
+                E *= sm.dblk[i * 128 + tid];
+            }
+            sm.gam[tid] = E;
+            float F = 1.f;
+#pragma unroll
+            for (int i = NB - 1; i >= 0; --i) {
+                sm.fm[i * 128 + tid] = sm.r15[i * 128 + tid] * F;
+                F *= sm.dblk[i * 128 + tid];
+            }
+#pragma unroll
+            for (int i = 1; i < NB; ++i) {
+                float prod = 1.f;
+#pragma unroll
+                for (int j = i - 1; j >= 0; --j) {
+                    prod *= sm.r15[j * 128 + tid] * sm.p7[(j + 1) * 128 + tid];   // e^{Lam_m(j+1) - Lam_m(j)}
+                    sm.cij[pair_index(i, j) * 128 + tid] = prod;
+                }
+            }
+        }
+        __syncthreads();
+        for (int idx = tid; idx < C * 128; idx += 256) {
+            const int t = idx >> 7, kch = idx & 127;
+            const float f = sm.em[(t >> 4) * 128 + kch];
+            sm.qt[t * kLdOp + kch] = __float2bfloat16_rn(bf(sm.qm[t * kLdOp + kch]) * f);
+            sm.kt[t * kLdOp + kch] = __float2bfloat16_rn(bf(sm.krm[t * kLdOp + kch]) * f);
+        }
+        __syncthreads();
+        // ---- Gram blocks (warp = type x row block); T_ii on the Akk warps
+        {
+            const int type = warp >> 2, i = warp & 3;
+            if (i < NB) {
+                const __nv_bfloat16 *rowop = type ? sm.qm : sm.krm;
+                for (int j = 0; j <= i; ++j) {
+                    float acc[2][4] = {};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        uint32_t af[4], bfr[4];
+                        load_a(af, rowop, kLdOp, 16 * i, 16 * ks, lane);
+                        load_b_nk(bfr, sm.kcm, kLdOp, 16 * j, 16 * ks, lane);
+                        if (j < i) {
+                            const float *f = sm.cij + pair_index(i, j) * 128 + 16 * ks + 2 * c4;
+                            bfr[0] = scale_bf16x2(bfr[0], f[0], f[1]);
+                            bfr[1] = scale_bf16x2(bfr[1], f[8], f[9]);
+                            bfr[2] = scale_bf16x2(bfr[2], f[0], f[1]);
+                            bfr[3] = scale_bf16x2(bfr[3], f[8], f[9]);
+                        }
+                        mma_bf16(acc[0], af, bfr[0], bfr[1]);
+                        mma_bf16(acc[1], af, bfr[2], bfr[3]);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int tr = 16 * i + g + ((e >> 1) << 3);
+                            const int sc = 16 * j + 8 * nt + 2 * c4 + (e & 1);
+                            const float val = acc[nt][e];
+                            if (type == 0) {
+                                const bool ok = sc < tr;
+                                sm.mkk[tr * LDA + sc] = __float2bfloat16_rn(ok ? sm.wv[tr] * val : 0.f);
+                                if (j == i) sm.akk_d[(16 * i + tr - 16 * i) * 17 + (sc - 16 * j)] = ok ? val : 0.f;
+                            } else {
+                                sm.aqk[tr * LDA + sc] = __float2bfloat16_rn(sc <= tr ? val : 0.f);
+                            }
+                        }
+                }
+                if (type == 0) {
+                    __syncwarp();
+                    if (lane < 16) {   // column `lane` of T_ii = (I + Diag(w) A_ii)^-1
+                        float col[16];
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) {
+                            float x = (t == lane) ? 1.f : 0.f;
+                            const float w = sm.wv[16 * i + t];
+#pragma unroll
+                            for (int s2 = 0; s2 < t; ++s2) x -= w * sm.akk_d[(16 * i + t) * 17 + s2] * col[s2];
+                            col[t] = x;
+                        }
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) sm.tii[(i * 16 + t) * 24 + lane] = __float2bfloat16_rn(col[t]);
+                    }
+                }
+            }
+        }
+        // ---- G = S0 [Kt; Qt]^T  (rows v of this warp)
+        float ga[4 * NB][4];
+#pragma unroll
+        for (int j = 0; j < 4 * NB; ++j) ga[j][0] = ga[j][1] = ga[j][2] = ga[j][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t af[4];
+            af[0] = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
+            af[1] = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
+            af[2] = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+            af[3] = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+            for (int np = 0; np < 2 * NB; ++np) {
+                uint32_t bfr[4];
+                load_b_nk(bfr, np < NB ? sm.kt : sm.qt, kLdOp, 16 * (np % NB), 16 * ks, lane);
+                mma_bf16(ga[2 * np], af, bfr[0], bfr[1]);
+                mma_bf16(ga[2 * np + 1], af, bfr[2], bfr[3]);
+            }
+        }
+        __syncthreads();
+        if (cc + 1 < NCC) issue(cc + 1, 0);
+        // ---- X = Diag(w)(V - Kt S0^T), as X^T (rows v, cols t)
+#pragma unroll
+        for (int j = 0; j < 2 * NB; ++j) {
+            const int t = 8 * j + 2 * c4;
+            const float w0 = sm.wv[t], w1 = sm.wv[t + 1];
+            ga[j][0] = w0 * (bf(sm.rv[t * 128 + v0]) - ga[j][0]);
+            ga[j][1] = w1 * (bf(sm.rv[(t + 1) * 128 + v0]) - ga[j][1]);
+            ga[j][2] = w0 * (bf(sm.rv[t * 128 + v1]) - ga[j][2]);
+            ga[j][3] = w1 * (bf(sm.rv[(t + 1) * 128 + v1]) - ga[j][3]);
+        }
+        // ---- blocked solve:  U_i^T = (X_i^T - sum_{j<i} U_j^T M_ij^T) T_ii^T
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+#pragma unroll
+            for (int j = 0; j < i; ++j) {
+                uint32_t ua[4], bfr[4];
+                ua[0] = pack_bf16(-ga[2 * j][0], -ga[2 * j][1]);
+                ua[1] = pack_bf16(-ga[2 * j][2], -ga[2 * j][3]);
+                ua[2] = pack_bf16(-ga[2 * j + 1][0], -ga[2 * j + 1][1]);
+                ua[3] = pack_bf16(-ga[2 * j + 1][2], -ga[2 * j + 1][3]);
+                load_b_nk(bfr, sm.mkk, LDA, 16 * i, 16 * j, lane);
+                mma_bf16(ga[2 * i], ua, bfr[0], bfr[1]);
+                mma_bf16(ga[2 * i + 1], ua, bfr[2], bfr[3]);
+            }
+            uint32_t ya[4], bfr[4];
+            ya[0] = pack_bf16(ga[2 * i][0], ga[2 * i][1]);
+            ya[1] = pack_bf16(ga[2 * i][2], ga[2 * i][3]);
+            ya[2] = pack_bf16(ga[2 * i + 1][0], ga[2 * i + 1][1]);
+            ya[3] = pack_bf16(ga[2 * i + 1][2], ga[2 * i + 1][3]);
+            load_b_nk(bfr, sm.tii + i * 16 * 24, 24, 0, 0, lane);
+            float un[2][4] = {};
+            mma_bf16(un[0], ya, bfr[0], bfr[1]);
+            mma_bf16(un[1], ya, bfr[2], bfr[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ga[2 * i][e] = un[0][e];
+                ga[2 * i + 1][e] = un[1][e];
+            }
+        }
+        // ---- O^T = S0 Qt^T + U^T Aqk^T
+#pragma unroll
+        for (int i = 0; i < NB; ++i)
+#pragma unroll
+            for (int j = 0; j <= i; ++j) {
+                uint32_t ua[4], bfr[4];
+                ua[0] = pack_bf16(ga[2 * j][0], ga[2 * j][1]);
+                ua[1] = pack_bf16(ga[2 * j][2], ga[2 * j][3]);
+                ua[2] = pack_bf16(ga[2 * j + 1][0], ga[2 * j + 1][1]);
+                ua[3] = pack_bf16(ga[2 * j + 1][2], ga[2 * j + 1][3]);
+                load_b_nk(bfr, sm.aqk, LDA, 16 * i, 16 * j, lane);
+                mma_bf16(ga[2 * NB + 2 * i], ua, bfr[0], bfr[1]);
+                mma_bf16(ga[2 * NB + 2 * i + 1], ua, bfr[2], bfr[3]);
+            }
+        {
+            float os0 = 0.f, os1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 2 * NB; ++j) {
+                const int t = 8 * j + 2 * c4;
+                const float *y = ga[2 * NB + j];
+                sm.ost()[t * kLdOp + v0] = __float2bfloat16_rn(y[0]);
+                sm.ost()[(t + 1) * kLdOp + v0] = __float2bfloat16_rn(y[1]);
+                sm.ost()[t * kLdOp + v1] = __float2bfloat16_rn(y[2]);
+                sm.ost()[(t + 1) * kLdOp + v1] = __float2bfloat16_rn(y[3]);
+                os0 += y[0] + y[1];
+                os1 += y[2] + y[3];
+            }
+            os0 += __shfl_xor_sync(0xffffffffu, os0, 1);
+            os0 += __shfl_xor_sync(0xffffffffu, os0, 2);
+            os1 += __shfl_xor_sync(0xffffffffu, os1, 1);
+            os1 += __shfl_xor_sync(0xffffffffu, os1, 2);
+            if (c4 == 0) {
+                sm.osum[v0] += os0;
+                sm.osum[v1] += os1;
+            }
+        }
+        // ---- S = S Diag(gamma) + U^T Kbar
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int col = 8 * j + 2 * c4;
+            const float g0 = sm.gam[col], g1 = sm.gam[col + 1];
+            s[j][0] *= g0;
+            s[j][1] *= g1;
+            s[j][2] *= g0;
+            s[j][3] *= g1;
+        }
+#pragma unroll
+        for (int js = 0; js < NB; ++js) {
+            uint32_t ua[4];
+            ua[0] = pack_bf16(ga[2 * js][0], ga[2 * js][1]);
+            ua[1] = pack_bf16(ga[2 * js][2], ga[2 * js][3]);
+            ua[2] = pack_bf16(ga[2 * js + 1][0], ga[2 * js + 1][1]);
+            ua[3] = pack_bf16(ga[2 * js + 1][2], ga[2 * js + 1][3]);
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bfr[4];
+                load_b_kn(bfr, sm.kcm, kLdOp, 16 * np, 16 * js, lane);
+                const float f0 = sm.fm[js * 128 + 16 * np + g], f1 = sm.fm[js * 128 + 16 * np + 8 + g];
+                bfr[0] = scale_bf16x2(bfr[0], f0, f0);
+                bfr[1] = scale_bf16x2(bfr[1], f0, f0);
+                bfr[2] = scale_bf16x2(bfr[2], f1, f1);
+                bfr[3] = scale_bf16x2(bfr[3], f1, f1);
+                mma_bf16(s[2 * np], ua, bfr[0], bfr[1]);
+                mma_bf16(s[2 * np + 1], ua, bfr[2], bfr[3]);
+            }
+        }
+        __syncthreads();
+        if (cc + 1 < NCC) issue(cc + 1, 1);
+        for (int idx = tid; idx < C * 16; idx += 256) {
+            const int t = idx >> 4, part = idx & 15;
+            *reinterpret_cast<uint4 *>(o + base_bh + (size_t)(t0 + t) * tstride + part * 8) =
+                *reinterpret_cast<const uint4 *>(sm.ost() + t * kLdOp + part * 8);
+        }
+        if (last) {
+            if (tid < 128) sm.mprev[tid] = sm.osum[tid] / (float)n;
+        }
+        __syncthreads();
+    }
+    if (a.S_final) {
+        float *Sf = a.S_final + (size_t)u * 128 * 128;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int col = 8 * j + 2 * c4;
+            *reinterpret_cast<float2 *>(Sf + v0 * 128 + col) = make_float2(s[j][0], s[j][1]);
+            *reinterpret_cast<float2 *>(Sf + v1 * 128 + col) = make_float2(s[j][2], s[j][3]);
+        }
+    }
+    if (a.m_prev_out && tid < 128) a.m_prev_out[(size_t)u * 128 + tid] = sm.mprev[tid];
+}
+
+template <int NB>
+cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
+    auto kern = tc_fwd_kernel<NB>;
+    const int bytes = (int)sizeof(TcFwdSmem<NB>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<a.B * a.H, 256, bytes, st>>>(a);
+    return cudaGetLastError();
+}
+
+// Compute chunk of the tensor-core path for a gate chunk L (0 = not supported).
+int tc_compute_chunk(int L) { return L == 32 ? 32 : (L == 64 || L == 128) ? 64 : 0; }
+
+cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st) {
+    return tc_compute_chunk(a.L) == 32 ? launch_tc_fwd_t<2>(a, st) : launch_tc_fwd_t<4>(a, st);
+}
+
+size_t tc_fwd_smem(int L) { return tc_compute_chunk(L) == 32 ? sizeof(TcFwdSmem<2>) : sizeof(TcFwdSmem<4>); }
+
+}  // namespace carve

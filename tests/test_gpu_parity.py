@@ -21,9 +21,9 @@ pytestmark = pytest.mark.gpu
 GRADS = ("dq", "dk", "dv", "dg_logit", "dbx", "dw_logit", "dA", "dB")
 
 
-def gpu_fwd(dev, dd, L, mode, S0=None, mp=None):
+def gpu_fwd(dev, dd, L, mode, S0=None, mp=None, save=True):
     return carve.carve_fwd(dd["q"], dd["k"], dd["v"], dd["g_logit"], dd["bx"], dd["w_logit"], dd["A"], dd["B"],
-                           chunk=L, mc_mode=mode, S0=S0, m_prev_in=mp)
+                           chunk=L, mc_mode=mode, S0=S0, m_prev_in=mp, save_for_bwd=save)
 
 
 def gpu_bwd(dd, saved, L, mode, dS_final=None, dm_prev_out=None):
@@ -43,7 +43,7 @@ def run_case(cuda_device, w, d, dO, L, mode, S0=None, mp=None, dSf=None, dmo=Non
     dd = to_dev(d if dO is None else dict(d, dO=dO), w.io, cuda_device)
     tS0 = None if S0 is None else torch.from_numpy(S0).to(cuda_device)
     tmp = None if mp is None else torch.from_numpy(mp).to(cuda_device)
-    out = gpu_fwd(cuda_device, dd, L, mode, tS0, tmp)
+    out = gpu_fwd(cuda_device, dd, L, mode, tS0, tmp, save=bwd)
     g = None
     if bwd:
         tdS = None if dSf is None else torch.from_numpy(dSf).to(cuda_device)
@@ -121,21 +121,26 @@ def test_chunk_lengths_bf16(cuda_device, L):
         run_case(cuda_device, w, d, dO, L, mode)
 
 
-def test_zero_projection_is_chunk_length_invariant_bitwise(cuda_device):
-    """U_b = 0 (A = 0): the erase gate is sigmoid(bx + 0) = sigmoid(bx) exactly, so the GPU
-    result cannot depend on the gate grouping L at all -- bitwise -- and matches the oracle's
-    key-axis baseline (content path removed)."""
+def test_zero_projection_is_chunk_length_invariant(cuda_device):
+    """U_b = 0 (A = 0): the erase gate is sigmoid(bx + 0) = sigmoid(bx) exactly, so the gate
+    grouping L cannot matter.  Kernels that split the sequence into the same compute chunks
+    (L = 64 and 128 on the tensor-core path, both readouts) agree bitwise; every L agrees with
+    the oracle's key-axis baseline (content path removed) within tolerance."""
     import torch
     w, d, dO = small(I.FWD_1P3B, B=2, H=2, T=256, seed=9)
     d["A"][:] = 0.0
     dd = to_dev(d, w.io, cuda_device)
-    outs = [gpu_fwd(cuda_device, dd, L, 0) for L in (16, 32, 64, 128)]
-    outs += [gpu_fwd(cuda_device, dd, 64, 1)]
+    same = [gpu_fwd(cuda_device, dd, 64, 0, save=False), gpu_fwd(cuda_device, dd, 128, 0, save=False),
+            gpu_fwd(cuda_device, dd, 64, 1, save=False), gpu_fwd(cuda_device, dd, 128, 1, save=False)]
     torch.cuda.synchronize()
-    for x in outs[1:]:
-        assert torch.equal(x["o"], outs[0]["o"]) and torch.equal(x["S_final"], outs[0]["S_final"])
+    for x in same[1:]:
+        assert torch.equal(x["o"], same[0]["o"]) and torch.equal(x["S_final"], same[0]["S_final"])
     base = oracle.fwd(d, L=64, content_off=True)
-    check("o", host(outs[0]["o"]), base["o"], TOL["bf16"])
+    for L in (16, 32, 64, 128):
+        for save in (False, True):
+            x = gpu_fwd(cuda_device, dd, L, 0, save=save)
+            check(f"o L={L} save={save}", host(x["o"]), base["o"], TOL["bf16"])
+            check(f"S L={L} save={save}", host(x["S_final"]), base["S_final"], TOL["bf16"])
 
 
 @pytest.mark.parametrize("mode", [0, 1])
@@ -146,11 +151,11 @@ def test_chaining_is_bitwise(cuda_device, mode):
     d["A"] *= 10.0
     d["B"] *= 10.0
     dd = to_dev(d, w.io, cuda_device)
-    full = gpu_fwd(cuda_device, dd, 64, mode)
+    full = gpu_fwd(cuda_device, dd, 64, mode, save=False)
     half = {k: (v[:, :256].contiguous() if v.dim() >= 3 and k not in ("A", "B") else v) for k, v in dd.items()}
     rest = {k: (v[:, 256:].contiguous() if v.dim() >= 3 and k not in ("A", "B") else v) for k, v in dd.items()}
-    a = gpu_fwd(cuda_device, half, 64, mode)
-    b = gpu_fwd(cuda_device, rest, 64, mode, S0=a["S_final"], mp=a["m_prev_out"])
+    a = gpu_fwd(cuda_device, half, 64, mode, save=False)
+    b = gpu_fwd(cuda_device, rest, 64, mode, S0=a["S_final"], mp=a["m_prev_out"], save=False)
     torch.cuda.synchronize()
     assert torch.equal(torch.cat([a["o"], b["o"]], dim=1), full["o"])
     assert torch.equal(b["S_final"], full["S_final"])
