@@ -7,7 +7,8 @@
 
 namespace carve {
 cudaError_t launch_fwd_simt(int K, int V, bool bf16, const FwdArgs &a, cudaStream_t st);
-cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st);
+cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st);
+cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 int tc_compute_chunk(int L);
 cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
@@ -44,12 +45,22 @@ carve_status check_dims(const carve_dims *d, bool seq) {
 size_t n_chunks(const carve_dims *d) { return (size_t)((d->T + d->chunk - 1) / d->chunk); }
 
 // The tensor-core kernels cover bf16 I/O with dk = dv = 128, rank <= 32 and gate chunks of 32,
-// 64 or 128 tokens when T is a multiple of the compute chunk; everything else runs the SIMT
-// kernels.
-bool use_tc_fwd(const carve_dims *d) {
-    const int C = carve::tc_compute_chunk(d->chunk);
-    return d->io == CARVE_IO_BF16 && d->dk == 128 && d->dv == 128 && d->rank <= 32 && C > 0 && d->T % C == 0;
+// 64 or 128 tokens; everything else runs the SIMT kernels.  The forward alone uses compute
+// chunks of min(chunk, 64) tokens (32 when T is not a multiple of that); a forward that saves
+// for the backward, and the backward, use 32-token compute chunks (T a multiple of 32).
+bool tc_shape(const carve_dims *d) {
+    return d->io == CARVE_IO_BF16 && d->dk == 128 && d->dv == 128 && d->rank <= 32 &&
+           carve::tc_compute_chunk(d->chunk) > 0;
 }
+
+int tc_fwd_chunk(const carve_dims *d) {
+    if (!tc_shape(d)) return 0;
+    const int C = carve::tc_compute_chunk(d->chunk);
+    if (d->T % C == 0) return C;
+    return d->T % 32 == 0 ? 32 : 0;
+}
+
+bool use_tc_bwd(const carve_dims *d) { return tc_shape(d) && d->T % 32 == 0; }
 
 }  // namespace
 
@@ -69,7 +80,8 @@ const char *carve_status_string(carve_status s) {
 size_t carve_saved_bytes(const carve_dims *d) {
     if (check_dims(d, true) != CARVE_OK) return 0;
     const size_t units = (size_t)d->B * d->H;
-    const size_t states = units * (size_t)(d->T / carve::kSub) * d->dv * d->dk;
+    const size_t n16 = (size_t)(d->T / carve::kSub), n32 = use_tc_bwd(d) ? (size_t)(d->T / 32 + 1) : 0;
+    const size_t states = units * (n16 > n32 ? n16 : n32) * d->dv * d->dk;
     const size_t aux = units * n_chunks(d) * (size_t)(d->dv + d->rank + d->dk);
     return sizeof(float) * (states + aux);
 }
@@ -93,17 +105,22 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
     carve::FwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
     a.S0 = S0; a.m_prev_in = m_prev_in; a.o = o; a.S_final = S_final; a.m_prev_out = m_prev_out;
+    const size_t units = (size_t)d->B * d->H;
+    const bool tc_saved = use_tc_bwd(d);
     if (saved) {
-        const size_t units = (size_t)d->B * d->H;
         a.saved_states = static_cast<float *>(saved);
-        a.saved_aux = a.saved_states + units * (size_t)(d->T / carve::kSub) * d->dv * d->dk;
+        const size_t nstates = tc_saved ? (size_t)(d->T / 32 + 1) : (size_t)(d->T / carve::kSub);
+        a.saved_aux = a.saved_states + units * nstates * d->dv * d->dk;
     }
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
     cudaError_t e;
-    if (use_tc_fwd(d) && saved == nullptr)
-        e = carve::launch_fwd_tc(a, static_cast<cudaStream_t>(stream));
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (saved != nullptr && tc_saved)
+        e = carve::launch_fwd_tc(a, 32, cs);
+    else if (saved == nullptr && tc_fwd_chunk(d) > 0)
+        e = carve::launch_fwd_tc(a, tc_fwd_chunk(d), cs);
     else
-        e = carve::launch_fwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, static_cast<cudaStream_t>(stream));
+        e = carve::launch_fwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, cs);
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 
@@ -128,14 +145,17 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
     carve::BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
     const size_t units = (size_t)d->B * d->H;
+    const bool tc = use_tc_bwd(d);
     a.saved_states = static_cast<const float *>(saved);
-    a.saved_aux = a.saved_states + units * (size_t)(d->T / carve::kSub) * d->dv * d->dk;
+    const size_t nstates = tc ? (size_t)(d->T / 32 + 1) : (size_t)(d->T / carve::kSub);
+    a.saved_aux = a.saved_states + units * nstates * d->dv * d->dk;
     a.dO = dO; a.dS_final = dS_final; a.dm_prev_out = dm_prev_out;
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg_logit = dg_logit; a.dbx = dbx; a.dw_logit = dw_logit;
     a.dS0 = dS0; a.dm_prev_in = dm_prev_in; a.ws = static_cast<float *>(workspace);
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
-    cudaError_t e = carve::launch_bwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
-                                          static_cast<cudaStream_t>(stream));
+    cudaError_t e = tc ? carve::launch_bwd_tc(a, dA, dB, static_cast<cudaStream_t>(stream))
+                       : carve::launch_bwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
+                                                static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 

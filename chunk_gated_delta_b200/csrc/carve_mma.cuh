@@ -9,6 +9,7 @@
 // Two adjacent C tiles (cols n0..n0+15) therefore repack into one A fragment without any
 // data movement between lanes.
 #pragma once
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -109,5 +110,24 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+
+// Tiled TMA load of a 3-D box (coordinates innermost first) into shared memory, completing
+// on `bar` as transaction bytes.  c0 * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];\n" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Host: tensor map over a [rows, H, inner] token-major tensor (inner = channels, contiguous),
+// box = [box_rows tokens, 1 head, inner channels]; elem_bytes 2 (bf16) or 4 (fp32).
+cudaError_t make_token_tile_map(CUtensorMap *map, const void *base, int elem_bytes, int inner, int H,
+                                long long rows, int box_rows);
 
 }  // namespace carve

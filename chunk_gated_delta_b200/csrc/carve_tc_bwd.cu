@@ -1,0 +1,820 @@
+// CARVE backward, tensor-core kernel for bf16 q/k/v/o with dk = dv = 128.
+//
+// One CTA (8 warps) per (batch, head) unit sweeps the compute chunks of 32 tokens in reverse.
+// Warp w owns rows v in [16w, 16w+16) of the carried state gradient dS, kept in registers as
+// mma accumulator fragments.  Per chunk, from the saved chunk-start state S0 and the saved
+// content signal Delta:
+//   recompute  gates (as the forward), Gram blocks Akk/Aqk, T_ii, R = V - Kt S0^T,
+//              U (blocked WY solve) and E = R - Akk U (the prediction errors v - S Diag(a) k)
+//   per warp   dU^T = dO^T Aqk + dS1 Kbar^T;  dY^T = dU^T M^-1 (blocked back substitution);
+//              dR = Diag(w) dY;  dw_t = sum_v dY E;  dS0 = dS1 Diag(gamma) + dO^T Qt - dR^T Kt
+//   cross-warp dAqk = dO U^T, dAkk = -dR U^T (reductions over v), then, per (token block,
+//              channel quarter), with every decay factor folded into a B operand:
+//                Gq  = dO (S0 Em) + dAqk (Kcm C)          -> dq   = r Gq
+//                Gkr = -dR (S0 Em) + dAkk (Kcm C)         -> dk   = r Gkr + Gkc / r
+//                Gkc = dAqk^T (Qm C) + dAkk^T (Krm C)
+//                Gkb = U (dS1 Fm)                          (the Kbar part of Gkc)
+//                dLam = Qm Gq + Krm Gkr - Kcm (Gkc + Gkb)
+//                       (+ sum_s Kbar_s dKbar_s + gamma colsum(S0 * dS1) at the chunk's last token)
+//   gates      dl = reverse cumsum of dLam; d g_logit = -sigma(g_logit) dl; dbx = sigma(-beta) dl
+// (Qm, Krm, Kcm: mid-block referenced operands; Em, Fm, C: the block-level decay factors of the
+// forward.)  The content path (dz = A^T dDelta, dm = B^T dz) closes each gate chunk.
+// Terms that cancel pairwise in the reverse cumulative sum of dLam (a Gram entry's row and
+// column token; Kbar_s against the chunk's last token) are formed from the same rounded values
+// on both sides, so the cancellation stays exact to fp32 rounding.
+#include "carve_tc_common.cuh"
+
+namespace carve {
+
+constexpr int kBC = 32;     // compute chunk of the backward
+constexpr int kBNB = 2;     // 16-token blocks per compute chunk
+constexpr int kLdT = 40;    // bf16 row stride of 32-wide tiles
+
+struct BwdMaps {
+    CUtensorMap q, k, v, dO;
+};
+
+struct __align__(16) TcBwdSmem {
+    __nv_bfloat16 rq[kBC * 128], rk[kBC * 128], rv[kBC * 128], rdo[kBC * 128];  // TMA tiles
+    __nv_bfloat16 dop[kBC * kLdOp];
+    __nv_bfloat16 qm[kBC * kLdOp], krm[kBC * kLdOp], kcm[kBC * kLdOp];
+    __nv_bfloat16 s0b[128 * kLdOp], ds1b[128 * kLdOp];
+    __nv_bfloat16 ub[kBC * kLdOp], drb[kBC * kLdOp];
+    __nv_bfloat16 aqk[kBC * kLdT], akk[kBC * kLdT], mkk[kBC * kLdT], daqk[kBC * kLdT], dakk[kBC * kLdT];
+    __nv_bfloat16 tii[kBNB * 16 * 24];
+    float akk_d[kBC * 17];
+    float rfac[kBC * 129], dlam[kBC * 129];
+    float p7[kBNB * 128], r15[kBNB * 128], dblk[kBNB * 128], em[kBNB * 128], fm[kBNB * 128], cij[128];
+    float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], btot[kBNB * 128], pdd[kBNB * 128];
+    float bpart[kBNB * 128];
+    float delta[128], ddelta[128], mvec[128], zvec[64], dzv[64], dmv[128], dox[128], vecK[128], qbar[128];
+    uint64_t bar;
+};
+
+__device__ int g_tc_bwd_timeout;
+
+__global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_constant__ BwdMaps maps) {
+    constexpr int C = kBC, NB = kBNB;
+    extern __shared__ __align__(128) unsigned char smraw[];
+    TcBwdSmem &sm = *reinterpret_cast<TcBwdSmem *>(smraw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, c4 = lane & 3;
+    const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
+    const int b = u / H, h = u % H;
+    const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
+    __nv_bfloat16 *dq = static_cast<__nv_bfloat16 *>(a.dq), *dk = static_cast<__nv_bfloat16 *>(a.dk);
+    __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv);
+    const size_t tstride = (size_t)H * 128;
+    const size_t base_bh = (size_t)b * T * tstride + (size_t)h * 128;
+    const int v0 = 16 * warp + g, v1 = v0 + 8;
+    const float *states = a.saved_states + (size_t)u * (NCC + 1) * 128 * 128;
+    float *wsu = a.ws + (size_t)u * (256 * R);
+    const int kch = tid & 127, ib = tid >> 7;   // (channel, 16-block) owned in the gate phases
+
+    float ds[16][4];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int col = 8 * j + 2 * c4;
+        if (a.dS_final) {
+            const float *D = a.dS_final + (size_t)u * 128 * 128;
+            ds[j][0] = D[v0 * 128 + col];
+            ds[j][1] = D[v0 * 128 + col + 1];
+            ds[j][2] = D[v1 * 128 + col];
+            ds[j][3] = D[v1 * 128 + col + 1];
+        } else {
+            ds[j][0] = ds[j][1] = ds[j][2] = ds[j][3] = 0.f;
+        }
+    }
+
+    // column sums over this warp's rows of (dS .* S), into sm.xp[warp]
+    auto colsum_partial = [&](const float *S) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int col = 8 * j + 2 * c4;
+            const float2 s0 = *reinterpret_cast<const float2 *>(S + v0 * 128 + col);
+            const float2 s1 = *reinterpret_cast<const float2 *>(S + v1 * 128 + col);
+            float p0 = ds[j][0] * s0.x + ds[j][2] * s1.x;
+            float p1 = ds[j][1] * s0.y + ds[j][3] * s1.y;
+#pragma unroll
+            for (int off = 4; off <= 16; off <<= 1) {
+                p0 += __shfl_xor_sync(0xffffffffu, p0, off);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, off);
+            }
+            if (g == 0) {
+                sm.xp[warp * 128 + col] = p0;
+                sm.xp[warp * 128 + col + 1] = p1;
+            }
+        }
+    };
+
+    if (tid == 0) {
+        mbar_init(&sm.bar, 1);
+        fence_mbar_init();
+    }
+    if (tid < 128) {
+        const int nl = T - (NG - 1) * L;
+        sm.dox[tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * 128 + tid] / (float)nl : 0.f;
+    }
+    for (int idx = tid; idx < 256 * R; idx += 256) wsu[idx] = 0.f;
+    auto issue = [&](int cc) {
+        if (tid != 0) return;
+        const int row = b * T + cc * C;
+        mbar_expect_tx(&sm.bar, 4u * C * 256u);
+        tma_load_3d(sm.rq, &maps.q, 0, h, row, &sm.bar);
+        tma_load_3d(sm.rk, &maps.k, 0, h, row, &sm.bar);
+        tma_load_3d(sm.rv, &maps.v, 0, h, row, &sm.bar);
+        tma_load_3d(sm.rdo, &maps.dO, 0, h, row, &sm.bar);
+    };
+    issue(NCC - 1);
+    uint32_t phase = 0;
+    __syncthreads();
+
+    for (int cc = NCC - 1; cc >= 0; --cc) {
+        const int t0 = cc * C, gc = cc / CPG;
+        const bool gate_end = (cc % CPG) == CPG - 1 || cc == NCC - 1;
+        const bool gate_start = (cc % CPG) == 0;
+        const int n = min(L, T - gc * L);
+        float glr[16], bxr[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const size_t gi = base_bh + (size_t)(t0 + 16 * ib + t) * tstride + kch;
+            glr[t] = a.g_logit[gi];
+            bxr[t] = a.bx[gi];
+        }
+        if (gate_end) {
+            const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (256 + R);
+            if (tid < 128) {
+                sm.mvec[tid] = aux[tid];
+                sm.delta[tid] = aux[128 + R + tid];
+                sm.ddelta[tid] = 0.f;
+            }
+            if (tid < R) sm.zvec[tid] = aux[128 + tid];
+        }
+        {   // this chunk's start state and the carried gradient, as bf16 tiles
+            const float *S0 = states + (size_t)cc * 128 * 128;
+            const int r = tid >> 1, half = tid & 1;
+            const float4 *src = reinterpret_cast<const float4 *>(S0 + r * 128 + half * 64);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const float4 f0 = src[2 * x], f1 = src[2 * x + 1];
+                uint4 o4;
+                o4.x = pack_bf16(f0.x, f0.y);
+                o4.y = pack_bf16(f0.z, f0.w);
+                o4.z = pack_bf16(f1.x, f1.y);
+                o4.w = pack_bf16(f1.z, f1.w);
+                *reinterpret_cast<uint4 *>(sm.s0b + r * kLdOp + half * 64 + 8 * x) = o4;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int col = 8 * j + 2 * c4;
+                *reinterpret_cast<uint32_t *>(sm.ds1b + v0 * kLdOp + col) = pack_bf16(ds[j][0], ds[j][1]);
+                *reinterpret_cast<uint32_t *>(sm.ds1b + v1 * kLdOp + col) = pack_bf16(ds[j][2], ds[j][3]);
+            }
+        }
+        colsum_partial(states + (size_t)cc * 128 * 128);   // for gamma * dgamma
+        if (!mbar_wait(&sm.bar, phase)) atomicOr(&g_tc_bwd_timeout, 1);
+        phase ^= 1u;
+        __syncthreads();
+        if (tid < 128) {
+            float x = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x += sm.xp[w * 128 + tid];
+            sm.s0ds[tid] = x;
+        }
+        // dO plus the content-signal gradient carried from the next gate chunk, padded
+        for (int idx = tid; idx < C * 16; idx += 256) {
+            const int t = idx >> 4, part = idx & 15;
+            const uint4 x = *reinterpret_cast<const uint4 *>(sm.rdo + t * 128 + part * 8);
+            const __nv_bfloat16 *xv = reinterpret_cast<const __nv_bfloat16 *>(&x);
+            const float *dx = sm.dox + part * 8;
+            uint4 y;
+            y.x = pack_bf16(bf(xv[0]) + dx[0], bf(xv[1]) + dx[1]);
+            y.y = pack_bf16(bf(xv[2]) + dx[2], bf(xv[3]) + dx[3]);
+            y.z = pack_bf16(bf(xv[4]) + dx[4], bf(xv[5]) + dx[5]);
+            y.w = pack_bf16(bf(xv[6]) + dx[6], bf(xv[7]) + dx[7]);
+            *reinterpret_cast<uint4 *>(sm.dop + t * kLdOp + part * 8) = y;
+        }
+        // ---- recompute: gates and mid-block referenced operands (as the forward)
+        {
+            const float dl = sm.delta[kch];
+            float av[16], ia[16], rf[16], cf[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) retention(glr[t], bxr[t] + dl, av[t], ia[t]);
+            mid_reference(av, ia, rf, cf);
+            float p7 = 1.f;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) p7 *= av[t];
+            sm.p7[ib * 128 + kch] = p7;
+            sm.r15[ib * 128 + kch] = rf[15];
+            sm.dblk[ib * 128 + kch] = p7 * rf[15];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const int row = 16 * ib + t;
+                const float qv = bf(sm.rq[row * 128 + kch]), kv = bf(sm.rk[row * 128 + kch]);
+                sm.qm[row * kLdOp + kch] = __float2bfloat16_rn(qv * rf[t]);
+                sm.krm[row * kLdOp + kch] = __float2bfloat16_rn(kv * rf[t]);
+                sm.kcm[row * kLdOp + kch] = __float2bfloat16_rn(kv * cf[t]);
+                sm.rfac[row * 129 + kch] = rf[t];
+            }
+        }
+        if (tid < C) sm.wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + t0 + tid) * H + h]);
+        __syncthreads();
+        if (tid < 128) {
+            float E = 1.f;
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                sm.em[i * 128 + tid] = E * sm.p7[i * 128 + tid];
+                E *= sm.dblk[i * 128 + tid];
+            }
+            sm.gam[tid] = E;
+            float F = 1.f;
+#pragma unroll
+            for (int i = NB - 1; i >= 0; --i) {
+                sm.fm[i * 128 + tid] = sm.r15[i * 128 + tid] * F;
+                F *= sm.dblk[i * 128 + tid];
+            }
+            sm.cij[tid] = sm.r15[tid] * sm.p7[128 + tid];   // e^{Lam_m(1) - Lam_m(0)}
+        }
+        __syncthreads();
+        // ---- Gram blocks (warps 0-3: type x row block), T_ii on the Akk warps
+        if (warp < 4) {
+            const int type = warp >> 1, i = warp & 1;
+            const __nv_bfloat16 *rowop = type ? sm.qm : sm.krm;
+            for (int j = 0; j <= i; ++j) {
+                float acc[2][4] = {};
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    uint32_t af[4], bfr[4];
+                    load_a(af, rowop, kLdOp, 16 * i, 16 * ks, lane);
+                    load_b_nk(bfr, sm.kcm, kLdOp, 16 * j, 16 * ks, lane);
+                    if (j < i) {
+                        const float *f = sm.cij + 16 * ks + 2 * c4;
+                        bfr[0] = scale_bf16x2(bfr[0], f[0], f[1]);
+                        bfr[1] = scale_bf16x2(bfr[1], f[8], f[9]);
+                        bfr[2] = scale_bf16x2(bfr[2], f[0], f[1]);
+                        bfr[3] = scale_bf16x2(bfr[3], f[8], f[9]);
+                    }
+                    mma_bf16(acc[0], af, bfr[0], bfr[1]);
+                    mma_bf16(acc[1], af, bfr[2], bfr[3]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int tr = 16 * i + g + ((e >> 1) << 3);
+                        const int sc = 16 * j + 8 * nt + 2 * c4 + (e & 1);
+                        const float val = acc[nt][e];
+                        if (type == 0) {
+                            const bool ok = sc < tr;
+                            sm.akk[tr * kLdT + sc] = __float2bfloat16_rn(ok ? val : 0.f);
+                            sm.mkk[tr * kLdT + sc] = __float2bfloat16_rn(ok ? sm.wv[tr] * val : 0.f);
+                            if (j == i) sm.akk_d[tr * 17 + (sc - 16 * j)] = ok ? val : 0.f;
+                        } else {
+                            sm.aqk[tr * kLdT + sc] = __float2bfloat16_rn(sc <= tr ? val : 0.f);
+                        }
+                    }
+            }
+            if (type == 0) {
+                __syncwarp();
+                if (lane < 16) {
+                    float col[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        float x = (t == lane) ? 1.f : 0.f;
+                        const float w = sm.wv[16 * i + t];
+#pragma unroll
+                        for (int s2 = 0; s2 < t; ++s2) x -= w * sm.akk_d[(16 * i + t) * 17 + s2] * col[s2];
+                        col[t] = x;
+                    }
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) sm.tii[(i * 16 + t) * 24 + lane] = __float2bfloat16_rn(col[t]);
+                }
+            }
+        }
+        // ---- R = V - S0 Kt^T  (rows v of this warp, cols t)
+        float rr[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) rr[j][0] = rr[j][1] = rr[j][2] = rr[j][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t af[4];
+            load_a(af, sm.s0b, kLdOp, 16 * warp, 16 * ks, lane);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bfr[4];
+                load_b_nk(bfr, sm.krm, kLdOp, 16 * np, 16 * ks, lane);
+                const float *f = sm.em + np * 128 + 16 * ks + 2 * c4;
+                bfr[0] = scale_bf16x2(bfr[0], f[0], f[1]);
+                bfr[1] = scale_bf16x2(bfr[1], f[8], f[9]);
+                bfr[2] = scale_bf16x2(bfr[2], f[0], f[1]);
+                bfr[3] = scale_bf16x2(bfr[3], f[8], f[9]);
+                mma_bf16(rr[2 * np], af, bfr[0], bfr[1]);
+                mma_bf16(rr[2 * np + 1], af, bfr[2], bfr[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = 8 * j + 2 * c4;
+            rr[j][0] = bf(sm.rv[t * 128 + v0]) - rr[j][0];
+            rr[j][1] = bf(sm.rv[(t + 1) * 128 + v0]) - rr[j][1];
+            rr[j][2] = bf(sm.rv[t * 128 + v1]) - rr[j][2];
+            rr[j][3] = bf(sm.rv[(t + 1) * 128 + v1]) - rr[j][3];
+        }
+        __syncthreads();
+        // ---- U (blocked WY solve), E = R - Akk U, U -> shared tile
+        float ga[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = 8 * j + 2 * c4;
+            const float w0 = sm.wv[t], w1 = sm.wv[t + 1];
+            ga[j][0] = w0 * rr[j][0];
+            ga[j][1] = w1 * rr[j][1];
+            ga[j][2] = w0 * rr[j][2];
+            ga[j][3] = w1 * rr[j][3];
+        }
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+#pragma unroll
+            for (int j = 0; j < i; ++j) {
+                uint32_t ua[4], bfr[4];
+                ua[0] = pack_bf16(ga[2 * j][0], ga[2 * j][1]);
+                ua[1] = pack_bf16(ga[2 * j][2], ga[2 * j][3]);
+                ua[2] = pack_bf16(ga[2 * j + 1][0], ga[2 * j + 1][1]);
+                ua[3] = pack_bf16(ga[2 * j + 1][2], ga[2 * j + 1][3]);
+                negate_frag(ua);
+                load_b_nk(bfr, sm.mkk, kLdT, 16 * i, 16 * j, lane);
+                mma_bf16(ga[2 * i], ua, bfr[0], bfr[1]);
+                mma_bf16(ga[2 * i + 1], ua, bfr[2], bfr[3]);
+            }
+            uint32_t ya[4], bfr[4];
+            ya[0] = pack_bf16(ga[2 * i][0], ga[2 * i][1]);
+            ya[1] = pack_bf16(ga[2 * i][2], ga[2 * i][3]);
+            ya[2] = pack_bf16(ga[2 * i + 1][0], ga[2 * i + 1][1]);
+            ya[3] = pack_bf16(ga[2 * i + 1][2], ga[2 * i + 1][3]);
+            load_b_nk(bfr, sm.tii + i * 16 * 24, 24, 0, 0, lane);
+            float un[2][4] = {};
+            mma_bf16(un[0], ya, bfr[0], bfr[1]);
+            mma_bf16(un[1], ya, bfr[2], bfr[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ga[2 * i][e] = un[0][e];
+                ga[2 * i + 1][e] = un[1][e];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < NB; ++i)
+#pragma unroll
+            for (int j = 0; j <= i; ++j) {
+                uint32_t ua[4], bfr[4];
+                ua[0] = pack_bf16(ga[2 * j][0], ga[2 * j][1]);
+                ua[1] = pack_bf16(ga[2 * j][2], ga[2 * j][3]);
+                ua[2] = pack_bf16(ga[2 * j + 1][0], ga[2 * j + 1][1]);
+                ua[3] = pack_bf16(ga[2 * j + 1][2], ga[2 * j + 1][3]);
+                negate_frag(ua);
+                load_b_nk(bfr, sm.akk, kLdT, 16 * i, 16 * j, lane);
+                mma_bf16(rr[2 * i], ua, bfr[0], bfr[1]);
+                mma_bf16(rr[2 * i + 1], ua, bfr[2], bfr[3]);
+            }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = 8 * j + 2 * c4;
+            sm.ub[t * kLdOp + v0] = __float2bfloat16_rn(ga[j][0]);
+            sm.ub[(t + 1) * kLdOp + v0] = __float2bfloat16_rn(ga[j][1]);
+            sm.ub[t * kLdOp + v1] = __float2bfloat16_rn(ga[j][2]);
+            sm.ub[(t + 1) * kLdOp + v1] = __float2bfloat16_rn(ga[j][3]);
+        }
+        // ---- dU^T = dO^T Aqk + dS1 Kbar^T
+        float du[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) du[j][0] = du[j][1] = du[j][2] = du[j][3] = 0.f;
+#pragma unroll
+        for (int js = 0; js < NB; ++js)
+#pragma unroll
+            for (int kt = js; kt < NB; ++kt) {
+                uint32_t af[4], bfr[4];
+                load_a_t(af, sm.dop, kLdOp, 16 * warp, 16 * kt, lane);
+                load_b_kn(bfr, sm.aqk, kLdT, 16 * js, 16 * kt, lane);
+                mma_bf16(du[2 * js], af, bfr[0], bfr[1]);
+                mma_bf16(du[2 * js + 1], af, bfr[2], bfr[3]);
+            }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t af[4];
+            af[0] = pack_bf16(ds[2 * ks][0], ds[2 * ks][1]);
+            af[1] = pack_bf16(ds[2 * ks][2], ds[2 * ks][3]);
+            af[2] = pack_bf16(ds[2 * ks + 1][0], ds[2 * ks + 1][1]);
+            af[3] = pack_bf16(ds[2 * ks + 1][2], ds[2 * ks + 1][3]);
+#pragma unroll
+            for (int js = 0; js < NB; ++js) {
+                uint32_t bfr[4];
+                load_b_nk(bfr, sm.kcm, kLdOp, 16 * js, 16 * ks, lane);
+                const float *f = sm.fm + js * 128 + 16 * ks + 2 * c4;
+                bfr[0] = scale_bf16x2(bfr[0], f[0], f[1]);
+                bfr[1] = scale_bf16x2(bfr[1], f[8], f[9]);
+                bfr[2] = scale_bf16x2(bfr[2], f[0], f[1]);
+                bfr[3] = scale_bf16x2(bfr[3], f[8], f[9]);
+                mma_bf16(du[2 * js], af, bfr[0], bfr[1]);
+                mma_bf16(du[2 * js + 1], af, bfr[2], bfr[3]);
+            }
+        }
+        // ---- dY^T = dU^T M^-1:  dY_j = (dU_j - sum_{i>j} dY_i M_ij) T_jj
+#pragma unroll
+        for (int j = NB - 1; j >= 0; --j) {
+#pragma unroll
+            for (int i = j + 1; i < NB; ++i) {
+                uint32_t ya[4], bfr[4];
+                ya[0] = pack_bf16(du[2 * i][0], du[2 * i][1]);
+                ya[1] = pack_bf16(du[2 * i][2], du[2 * i][3]);
+                ya[2] = pack_bf16(du[2 * i + 1][0], du[2 * i + 1][1]);
+                ya[3] = pack_bf16(du[2 * i + 1][2], du[2 * i + 1][3]);
+                negate_frag(ya);
+                load_b_kn(bfr, sm.mkk, kLdT, 16 * j, 16 * i, lane);
+                mma_bf16(du[2 * j], ya, bfr[0], bfr[1]);
+                mma_bf16(du[2 * j + 1], ya, bfr[2], bfr[3]);
+            }
+            uint32_t za[4], bfr[4];
+            za[0] = pack_bf16(du[2 * j][0], du[2 * j][1]);
+            za[1] = pack_bf16(du[2 * j][2], du[2 * j][3]);
+            za[2] = pack_bf16(du[2 * j + 1][0], du[2 * j + 1][1]);
+            za[3] = pack_bf16(du[2 * j + 1][2], du[2 * j + 1][3]);
+            load_b_kn(bfr, sm.tii + j * 16 * 24, 24, 0, 0, lane);
+            float un[2][4] = {};
+            mma_bf16(un[0], za, bfr[0], bfr[1]);
+            mma_bf16(un[1], za, bfr[2], bfr[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                du[2 * j][e] = un[0][e];
+                du[2 * j + 1][e] = un[1][e];
+            }
+        }
+        // ---- dR = Diag(w) dY (-> shared tile, dv), dw partials
+        float dr[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = 8 * j + 2 * c4;
+            const float w0 = sm.wv[t], w1 = sm.wv[t + 1];
+            dr[j][0] = w0 * du[j][0];
+            dr[j][1] = w1 * du[j][1];
+            dr[j][2] = w0 * du[j][2];
+            dr[j][3] = w1 * du[j][3];
+            sm.drb[t * kLdOp + v0] = __float2bfloat16_rn(dr[j][0]);
+            sm.drb[(t + 1) * kLdOp + v0] = __float2bfloat16_rn(dr[j][1]);
+            sm.drb[t * kLdOp + v1] = __float2bfloat16_rn(dr[j][2]);
+            sm.drb[(t + 1) * kLdOp + v1] = __float2bfloat16_rn(dr[j][3]);
+            float p0 = du[j][0] * rr[j][0] + du[j][2] * rr[j][2];
+            float p1 = du[j][1] * rr[j][1] + du[j][3] * rr[j][3];
+#pragma unroll
+            for (int off = 4; off <= 16; off <<= 1) {
+                p0 += __shfl_xor_sync(0xffffffffu, p0, off);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, off);
+            }
+            if (g == 0) {
+                sm.dwp[warp * C + t] = p0;
+                sm.dwp[warp * C + t + 1] = p1;
+            }
+        }
+        // ---- dS0 = dS1 Diag(gamma) + dO^T Qt - dR^T Kt
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int col = 8 * j + 2 * c4;
+            const float g0 = sm.gam[col], g1 = sm.gam[col + 1];
+            ds[j][0] *= g0;
+            ds[j][1] *= g1;
+            ds[j][2] *= g0;
+            ds[j][3] *= g1;
+        }
+#pragma unroll
+        for (int kt = 0; kt < NB; ++kt) {
+            uint32_t ao[4], ar[4];
+            load_a_t(ao, sm.dop, kLdOp, 16 * warp, 16 * kt, lane);
+            ar[0] = pack_bf16(dr[2 * kt][0], dr[2 * kt][1]);
+            ar[1] = pack_bf16(dr[2 * kt][2], dr[2 * kt][3]);
+            ar[2] = pack_bf16(dr[2 * kt + 1][0], dr[2 * kt + 1][1]);
+            ar[3] = pack_bf16(dr[2 * kt + 1][2], dr[2 * kt + 1][3]);
+            negate_frag(ar);
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bq[4], bk[4];
+                load_b_kn(bq, sm.qm, kLdOp, 16 * np, 16 * kt, lane);
+                load_b_kn(bk, sm.krm, kLdOp, 16 * np, 16 * kt, lane);
+                const float f0 = sm.em[kt * 128 + 16 * np + g], f1 = sm.em[kt * 128 + 16 * np + 8 + g];
+                bq[0] = scale_bf16x2(bq[0], f0, f0);
+                bq[1] = scale_bf16x2(bq[1], f0, f0);
+                bq[2] = scale_bf16x2(bq[2], f1, f1);
+                bq[3] = scale_bf16x2(bq[3], f1, f1);
+                bk[0] = scale_bf16x2(bk[0], f0, f0);
+                bk[1] = scale_bf16x2(bk[1], f0, f0);
+                bk[2] = scale_bf16x2(bk[2], f1, f1);
+                bk[3] = scale_bf16x2(bk[3], f1, f1);
+                mma_bf16(ds[2 * np], ao, bq[0], bq[1]);
+                mma_bf16(ds[2 * np + 1], ao, bq[2], bq[3]);
+                mma_bf16(ds[2 * np], ar, bk[0], bk[1]);
+                mma_bf16(ds[2 * np + 1], ar, bk[2], bk[3]);
+            }
+        }
+        __syncthreads();
+        // ---- dAqk = dO U^T (s <= t), dAkk = -dR U^T (s < t): reductions over v, six 16x16 tiles
+        if (warp < 6) {
+            const int type = warp / 3, blk = warp % 3;
+            const int i = blk == 0 ? 0 : 1, j = blk == 2 ? 1 : 0;
+            float acc[2][4] = {};
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t af[4], bfr[4];
+                load_a(af, type ? sm.drb : sm.dop, kLdOp, 16 * i, 16 * ks, lane);
+                load_b_nk(bfr, sm.ub, kLdOp, 16 * j, 16 * ks, lane);
+                mma_bf16(acc[0], af, bfr[0], bfr[1]);
+                mma_bf16(acc[1], af, bfr[2], bfr[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tr = 16 * i + g + ((e >> 1) << 3);
+                    const int sc = 16 * j + 8 * nt + 2 * c4 + (e & 1);
+                    if (type == 0) sm.daqk[tr * kLdT + sc] = __float2bfloat16_rn(sc <= tr ? acc[nt][e] : 0.f);
+                    else sm.dakk[tr * kLdT + sc] = __float2bfloat16_rn(sc < tr ? -acc[nt][e] : 0.f);
+                }
+        }
+        __syncthreads();
+        // ---- per (token block, channel quarter): Gq, Gkr, Gkc, Gkb -> dq, dk, dLam
+        // Paired terms that cancel in the reverse cumulative sum of dLam are built from the same
+        // rounded operands on both sides: the off-diagonal decay factor C is applied to fp32
+        // products, never to one side's bf16 operand.
+        {
+            const int ib2 = warp >> 2, ch0 = 32 * (warp & 3);
+            float gq[4][4], gkr[4][4], gkc[4][4], gkb[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) gq[j][e] = gkr[j][e] = gkc[j][e] = gkb[j][e] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t ao[4], ar[4], au[4];
+                load_a(ao, sm.dop, kLdOp, 16 * ib2, 16 * ks, lane);
+                load_a(ar, sm.drb, kLdOp, 16 * ib2, 16 * ks, lane);
+                negate_frag(ar);
+                load_a(au, sm.ub, kLdOp, 16 * ib2, 16 * ks, lane);
+#pragma unroll
+                for (int np2 = 0; np2 < 2; ++np2) {
+                    const int n0 = ch0 + 16 * np2;
+                    uint32_t bs[4], bd[4];
+                    load_b_kn(bs, sm.s0b, kLdOp, n0, 16 * ks, lane);
+                    load_b_kn(bd, sm.ds1b, kLdOp, n0, 16 * ks, lane);
+                    const float e0 = sm.em[ib2 * 128 + n0 + g], e1 = sm.em[ib2 * 128 + n0 + 8 + g];
+                    const float f0 = sm.fm[ib2 * 128 + n0 + g], f1 = sm.fm[ib2 * 128 + n0 + 8 + g];
+                    bs[0] = scale_bf16x2(bs[0], e0, e0);
+                    bs[1] = scale_bf16x2(bs[1], e0, e0);
+                    bs[2] = scale_bf16x2(bs[2], e1, e1);
+                    bs[3] = scale_bf16x2(bs[3], e1, e1);
+                    bd[0] = scale_bf16x2(bd[0], f0, f0);
+                    bd[1] = scale_bf16x2(bd[1], f0, f0);
+                    bd[2] = scale_bf16x2(bd[2], f1, f1);
+                    bd[3] = scale_bf16x2(bd[3], f1, f1);
+                    mma_bf16(gq[2 * np2], ao, bs[0], bs[1]);
+                    mma_bf16(gq[2 * np2 + 1], ao, bs[2], bs[3]);
+                    mma_bf16(gkr[2 * np2], ar, bs[0], bs[1]);
+                    mma_bf16(gkr[2 * np2 + 1], ar, bs[2], bs[3]);
+                    mma_bf16(gkb[2 * np2], au, bd[0], bd[1]);
+                    mma_bf16(gkb[2 * np2 + 1], au, bd[2], bd[3]);
+                }
+            }
+            // Gram blocks: rows t of this block against columns s of block j (row side) and
+            // columns s of this block against rows t of block i2 (column side)
+#pragma unroll
+            for (int j2 = 0; j2 < NB; ++j2) {
+                const bool row_side = j2 <= ib2;   // pair (ib2, j2)
+                const bool col_side = j2 >= ib2;   // pair (j2, ib2)
+                const bool offdiag = j2 != ib2;
+                float tq[4][4], tk[4][4], tc[4][4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) tq[j][e] = tk[j][e] = tc[j][e] = 0.f;
+                if (row_side) {
+                    uint32_t aq[4], ak[4];
+                    load_a(aq, sm.daqk, kLdT, 16 * ib2, 16 * j2, lane);
+                    load_a(ak, sm.dakk, kLdT, 16 * ib2, 16 * j2, lane);
+#pragma unroll
+                    for (int np2 = 0; np2 < 2; ++np2) {
+                        uint32_t bc[4];
+                        load_b_kn(bc, sm.kcm, kLdOp, ch0 + 16 * np2, 16 * j2, lane);
+                        mma_bf16(tq[2 * np2], aq, bc[0], bc[1]);
+                        mma_bf16(tq[2 * np2 + 1], aq, bc[2], bc[3]);
+                        mma_bf16(tk[2 * np2], ak, bc[0], bc[1]);
+                        mma_bf16(tk[2 * np2 + 1], ak, bc[2], bc[3]);
+                    }
+                }
+                if (col_side) {
+                    uint32_t aq[4], ak[4];
+                    load_a_t(aq, sm.daqk, kLdT, 16 * ib2, 16 * j2, lane);
+                    load_a_t(ak, sm.dakk, kLdT, 16 * ib2, 16 * j2, lane);
+#pragma unroll
+                    for (int np2 = 0; np2 < 2; ++np2) {
+                        uint32_t bq[4], bk[4];
+                        load_b_kn(bq, sm.qm, kLdOp, ch0 + 16 * np2, 16 * j2, lane);
+                        load_b_kn(bk, sm.krm, kLdOp, ch0 + 16 * np2, 16 * j2, lane);
+                        mma_bf16(tc[2 * np2], aq, bq[0], bq[1]);
+                        mma_bf16(tc[2 * np2 + 1], aq, bq[2], bq[3]);
+                        mma_bf16(tc[2 * np2], ak, bk[0], bk[1]);
+                        mma_bf16(tc[2 * np2 + 1], ak, bk[2], bk[3]);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float c = offdiag ? sm.cij[ch0 + 8 * nt + 2 * c4 + (e & 1)] : 1.f;
+                        gq[nt][e] += c * tq[nt][e];
+                        gkr[nt][e] += c * tk[nt][e];
+                        gkc[nt][e] += c * tc[nt][e];
+                    }
+            }
+            float bsum[4][2];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) bsum[nt][0] = bsum[nt][1] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int t = 16 * ib2 + g + 8 * hh;
+                    const int ch = ch0 + 8 * nt + 2 * c4;
+                    float dqv[2], dkv[2];
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int e = 2 * hh + e2, c = ch + e2;
+                        const float r = sm.rfac[t * 129 + c];
+                        const float ri = __fdividef(1.f, r);
+                        const float Gq = gq[nt][e], Gkr = gkr[nt][e], Gkc = gkc[nt][e] + gkb[nt][e];
+                        const float qmv = bf(sm.qm[t * kLdOp + c]), krv = bf(sm.krm[t * kLdOp + c]);
+                        const float kcv = bf(sm.kcm[t * kLdOp + c]);
+                        dqv[e2] = r * Gq;
+                        dkv[e2] = r * Gkr + ri * Gkc;
+                        sm.dlam[t * 129 + c] = qmv * Gq + krv * Gkr - kcv * Gkc;
+                        bsum[nt][e2] += kcv * gkb[nt][e];     // Kbar_t dKbar_t
+                    }
+                    const size_t gi = base_bh + (size_t)(t0 + t) * tstride + ch;
+                    *reinterpret_cast<uint32_t *>(dq + gi) = pack_bf16(dqv[0], dqv[1]);
+                    *reinterpret_cast<uint32_t *>(dk + gi) = pack_bf16(dkv[0], dkv[1]);
+                }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    float x = bsum[nt][e2];
+#pragma unroll
+                    for (int off = 4; off <= 16; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+                    if (g == 0) sm.bpart[ib2 * 128 + ch0 + 8 * nt + 2 * c4 + e2] = x;
+                }
+        }
+        __syncthreads();
+        // ---- reverse cumulative sum of dLam within the chunk, gate gradients
+        {
+            float tot = 0.f;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) tot += sm.dlam[(16 * ib + t) * 129 + kch];
+            float xl = sm.gam[kch] * sm.s0ds[kch];
+#pragma unroll
+            for (int i2 = 0; i2 < NB; ++i2) xl += sm.bpart[i2 * 128 + kch];
+            if (ib == NB - 1) tot += xl;
+            sm.btot[ib * 128 + kch] = tot;
+        }
+        if (tid < C) {
+            float dw = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) dw += sm.dwp[w * C + tid];
+            const float w = sm.wv[tid];
+            a.dw_logit[((size_t)b * T + t0 + tid) * H + h] = dw * w * (1.f - w);
+        }
+        for (int idx = tid; idx < C * 16; idx += 256) {   // dv = dR
+            const int t = idx >> 4, part = idx & 15;
+            *reinterpret_cast<uint4 *>(dv + base_bh + (size_t)(t0 + t) * tstride + part * 8) =
+                *reinterpret_cast<const uint4 *>(sm.drb + t * kLdOp + part * 8);
+        }
+        __syncthreads();
+        {
+            float run = 0.f;
+#pragma unroll
+            for (int i2 = 0; i2 < NB; ++i2)
+                if (i2 > ib) run += sm.btot[i2 * 128 + kch];
+            const float dl = sm.delta[kch];
+            float xl = sm.gam[kch] * sm.s0ds[kch];
+#pragma unroll
+            for (int i2 = 0; i2 < NB; ++i2) xl += sm.bpart[i2 * 128 + kch];
+            float pdd = 0.f;
+#pragma unroll
+            for (int t = 15; t >= 0; --t) {
+                run += sm.dlam[(16 * ib + t) * 129 + kch];
+                if (ib == NB - 1 && t == 15) run += xl;
+                const float e1 = __expf(glr[t]), e2 = __expf(-(bxr[t] + dl));
+                const float D = (1.f + e1) * (1.f + e2);
+                const bool floor = !(__fdividef(1.f, D) >= kAMin);
+                const float dglv = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run;
+                const float dbv = floor ? 0.f : __fdividef(e2, 1.f + e2) * run;
+                const size_t gi = base_bh + (size_t)(t0 + 16 * ib + t) * tstride + kch;
+                a.dg_logit[gi] = dglv;
+                a.dbx[gi] = dbv;
+                pdd += dbv;
+            }
+            sm.pdd[ib * 128 + kch] = pdd;
+        }
+        __syncthreads();
+        if (tid < 128) sm.ddelta[tid] += sm.pdd[tid] + sm.pdd[128 + tid];
+        __syncthreads();
+        // ---- content path at the gate chunk's first token
+        if (gate_start) {
+            for (int j0 = 0; j0 < R; j0 += 32) {   // dz = A^T dDelta, 8 threads per output
+                const int j = j0 + tid / 8, part = tid % 8;
+                float s = 0.f;
+                if (j < R)
+#pragma unroll
+                    for (int i = part; i < 128; i += 8) s += a.A[((size_t)h * 128 + i) * R + j] * sm.ddelta[i];
+                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                if (j < R && part == 0) sm.dzv[j] = s;
+            }
+            __syncthreads();
+            for (int idx = tid; idx < 128 * R; idx += 256) wsu[idx] += sm.ddelta[idx / R] * sm.zvec[idx % R];
+            for (int idx = tid; idx < R * 128; idx += 256) wsu[128 * R + idx] += sm.dzv[idx / 128] * sm.mvec[idx % 128];
+            if (tid < 128) {
+                float s = 0.f;
+#pragma unroll 8
+                for (int j = 0; j < R; ++j) s += a.Bm[((size_t)h * R + j) * 128 + tid] * sm.dzv[j];
+                sm.dmv[tid] = s;
+            }
+            __syncthreads();
+            if (a.mc_mode == 0) {
+                // m = S0 qbar:  dS0 += dm qbar^T,  dq_t += S0^T dm / n  for every t of the gate chunk
+                if (tid < 128) {
+                    float acc = 0.f;
+#pragma unroll 8
+                    for (int t = 0; t < n; ++t) acc += bf(q[base_bh + (size_t)(gc * L + t) * tstride + tid]);
+                    sm.qbar[tid] = acc / (float)n;
+                    const float *S0 = states + (size_t)cc * 128 * 128;
+                    float s = 0.f;
+#pragma unroll 8
+                    for (int r = 0; r < 128; ++r) s += S0[r * 128 + tid] * sm.dmv[r];
+                    sm.vecK[tid] = s / (float)n;
+                    sm.dox[tid] = 0.f;
+                }
+                __syncthreads();
+                const float m0 = sm.dmv[v0], m1 = sm.dmv[v1];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int col = 8 * j + 2 * c4;
+                    const float q0 = sm.qbar[col], q1 = sm.qbar[col + 1];
+                    ds[j][0] += m0 * q0;
+                    ds[j][1] += m0 * q1;
+                    ds[j][2] += m1 * q0;
+                    ds[j][3] += m1 * q1;
+                }
+                for (int idx = tid; idx < n * 64; idx += 256) {
+                    const int t = idx >> 6, c2 = (idx & 63) * 2;
+                    __nv_bfloat16 *p = dq + base_bh + (size_t)(gc * L + t) * tstride + c2;
+                    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(p);
+                    *reinterpret_cast<uint32_t *>(p) = pack_bf16(bf(x.x) + sm.vecK[c2], bf(x.y) + sm.vecK[c2 + 1]);
+                }
+            } else if (tid < 128) {
+                sm.dox[tid] = gc > 0 ? sm.dmv[tid] / (float)L : 0.f;
+                if (gc == 0 && a.dm_prev_in) a.dm_prev_in[(size_t)u * 128 + tid] = sm.dmv[tid];
+            }
+        }
+        if (cc > 0) issue(cc - 1);
+        __syncthreads();
+    }
+    if (a.dS0) {
+        float *D = a.dS0 + (size_t)u * 128 * 128;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int col = 8 * j + 2 * c4;
+            *reinterpret_cast<float2 *>(D + v0 * 128 + col) = make_float2(ds[j][0], ds[j][1]);
+            *reinterpret_cast<float2 *>(D + v1 * 128 + col) = make_float2(ds[j][2], ds[j][3]);
+        }
+    }
+    if (a.mc_mode == 0 && a.dm_prev_in && tid < 128) a.dm_prev_in[(size_t)u * 128 + tid] = 0.f;
+}
+
+__global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, int B, int H, int KR, int RV);
+
+cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st) {
+    const int bytes = (int)sizeof(TcBwdSmem);
+    cudaError_t e = cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    const long long rows = (long long)a.B * a.T;
+    BwdMaps maps;
+    if ((e = make_token_tile_map(&maps.q, a.q, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&maps.k, a.k, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&maps.v, a.v, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&maps.dO, a.dO, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
+    tc_bwd_kernel<<<a.B * a.H, 256, bytes, st>>>(a, maps);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int KR = 128 * a.R, RV = a.R * 128;
+    dim3 grid((KR + RV + 255) / 256, a.H);
+    reduce_dAdB_kernel<<<grid, 256, 0, st>>>(a.ws, dA, dB, a.B, a.H, KR, RV);
+    return cudaGetLastError();
+}
+
+size_t tc_bwd_smem() { return sizeof(TcBwdSmem); }
+
+}  // namespace carve

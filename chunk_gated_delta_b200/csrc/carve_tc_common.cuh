@@ -1,0 +1,48 @@
+// Constants and small helpers shared by the tensor-core forward and backward kernels.
+#pragma once
+#include "carve_device.cuh"
+#include "carve_mma.cuh"
+
+namespace carve {
+
+constexpr int kLdOp = 136;                            // bf16 row stride of 128-wide tiles
+constexpr float kAMin = 4.5399929762484854e-05f;      // e^-10: floor of the per-step retention
+constexpr float kInvAMin = 22026.465794806718f;       // e^10
+
+__device__ __forceinline__ int pair_index(int i, int j) { return i * (i - 1) / 2 + j; }
+__device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Per-step retention of one (token, channel) in product form: a = sigma(-g_logit) sigma(beta)
+// = 1 / ((1 + e^{g_logit})(1 + e^{-beta})), floored at e^-10; also returns 1/a.
+__device__ __forceinline__ void retention(float g_logit, float beta, float &a, float &inv_a) {
+    const float D = (1.f + __expf(g_logit)) * (1.f + __expf(-beta));
+    const float r = __fdividef(1.f, D);
+    const bool floor = !(r >= kAMin);
+    a = floor ? kAMin : r;
+    inv_a = floor ? kInvAMin : D;
+}
+
+// Mid-block references of one 16-token block from its retentions av (and reciprocals ia):
+// rf[t] = e^{Lam_t - Lam_7}, cf[t] = 1 / rf[t], both as running products from token 7.
+__device__ __forceinline__ void mid_reference(const float (&av)[16], const float (&ia)[16], float (&rf)[16],
+                                              float (&cf)[16]) {
+    rf[7] = cf[7] = 1.f;
+#pragma unroll
+    for (int t = 8; t < 16; ++t) {
+        rf[t] = rf[t - 1] * av[t];
+        cf[t] = cf[t - 1] * ia[t];
+    }
+#pragma unroll
+    for (int t = 6; t >= 0; --t) {
+        cf[t] = cf[t + 1] * av[t + 1];
+        rf[t] = rf[t + 1] * ia[t + 1];
+    }
+}
+
+// A fragment of the negated operand (sign flip of both bf16 halves)
+__device__ __forceinline__ void negate_frag(uint32_t (&a)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) a[e] ^= 0x80008000u;
+}
+
+}  // namespace carve

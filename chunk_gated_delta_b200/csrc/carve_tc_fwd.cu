@@ -21,14 +21,10 @@
 // Raw q/k/v rows are prefetched into shared memory by the bulk-copy (TMA) engine while the
 // previous chunk computes.  The floor a >= e^-10 bounds the deviation from the exact
 // recurrence by e^-10 per step in channels that are being erased anyway.
-#include "carve_device.cuh"
-#include "carve_mma.cuh"
+#include "carve_tc_common.cuh"
 
 namespace carve {
 
-constexpr int kLdOp = 136;                            // bf16 row stride of 128-wide operand tiles
-constexpr float kAMin = 4.5399929762484854e-05f;      // e^-10
-constexpr float kInvAMin = 22026.465794806718f;       // e^10
 constexpr int kTcMaxRank = 32;                        // low-rank factors staged in shared memory
 
 __device__ int g_tc_timeout;  // set when a bounded wait gives up (never expected)
@@ -49,12 +45,12 @@ struct __align__(16) TcFwdSmem {
     __device__ __nv_bfloat16 *ost() { return qt; }
 };
 
-__device__ __forceinline__ int pair_index(int i, int j) { return i * (i - 1) / 2 + j; }
-
-__device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
+struct TileMaps {
+    CUtensorMap q, k, v;
+};
 
 template <int NB>
-__global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_constant__ TileMaps maps) {
     using SM = TcFwdSmem<NB>;
     constexpr int C = SM::C, LDA = SM::LDA;
     constexpr int NP = (128 * NB + 255) / 256;  // (channel, block) pairs per thread in the gate phase
@@ -100,21 +96,24 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a) {
     }
     __syncthreads();
 
-    // raw tile rows of chunk cc: which = 0 (q and k, with the barrier's byte count) or 1 (v)
+    // raw q/k/v tiles of chunk cc by TMA (one tensor copy per tile): which = 0 -> q and k
+    // (arming the barrier with the byte count of all three), 1 -> v
     auto issue = [&](int cc, int which) {
-        if (warp != 0) return;
-        if (which == 0 && lane == 0) mbar_expect_tx(&sm.bar, 3u * C * 256u);
-        __syncwarp();
-        for (int r = lane; r < C; r += 32) {
-            const size_t off = base_bh + (size_t)(cc * C + r) * tstride;
-            if (which == 0) {
-                bulk_g2s(sm.rq + r * 128, q + off, 256, &sm.bar);
-                bulk_g2s(sm.rk + r * 128, kk + off, 256, &sm.bar);
-            } else {
-                bulk_g2s(sm.rv + r * 128, vv + off, 256, &sm.bar);
-            }
+        if (tid != 0) return;
+        const int row = b * T + cc * C;
+        if (which == 0) {
+            mbar_expect_tx(&sm.bar, 3u * C * 256u);
+            tma_load_3d(sm.rq, &maps.q, 0, h, row, &sm.bar);
+            tma_load_3d(sm.rk, &maps.k, 0, h, row, &sm.bar);
+        } else {
+            tma_load_3d(sm.rv, &maps.v, 0, h, row, &sm.bar);
         }
     };
+    if (tid == 0) {
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+    }
     issue(0, 0);
     issue(0, 1);
     uint32_t phase = 0;
@@ -140,7 +139,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a) {
         if (!mbar_wait(&sm.bar, phase)) atomicOr(&g_tc_timeout, 1);
         phase ^= 1u;
         if (a.saved_states) {
-            float *st = a.saved_states + ((size_t)u * NCC + cc) * 128 * 128;
+            float *st = a.saved_states + ((size_t)u * (NCC + 1) + cc) * 128 * 128;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int col = 8 * j + 2 * c4;
@@ -199,27 +198,10 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a) {
             const int p = tid + 256 * x, kch = p & 127, i = p >> 7;
             if (p < 128 * NB) {
                 const float dl = sm.delta[kch];
-                float av[16], ia[16];
+                float av[16], ia[16], rf[16], cf[16];
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float D = (1.f + __expf(glr[x][t])) * (1.f + __expf(-(bxr[x][t] + dl)));
-                    const float r = __fdividef(1.f, D);
-                    const bool floor = !(r >= kAMin);
-                    av[t] = floor ? kAMin : r;
-                    ia[t] = floor ? kInvAMin : D;
-                }
-                float rf[16], cf[16];
-                rf[7] = cf[7] = 1.f;
-#pragma unroll
-                for (int t = 8; t < 16; ++t) {
-                    rf[t] = rf[t - 1] * av[t];
-                    cf[t] = cf[t - 1] * ia[t];
-                }
-#pragma unroll
-                for (int t = 6; t >= 0; --t) {
-                    cf[t] = cf[t + 1] * av[t + 1];
-                    rf[t] = rf[t + 1] * ia[t + 1];
-                }
+                for (int t = 0; t < 16; ++t) retention(glr[x][t], bxr[x][t] + dl, av[t], ia[t]);
+                mid_reference(av, ia, rf, cf);
                 float p7 = 1.f;
 #pragma unroll
                 for (int t = 0; t < 8; ++t) p7 *= av[t];
@@ -465,6 +447,15 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a) {
         }
         __syncthreads();
     }
+    if (a.saved_states) {   // the state after the last token closes the list of boundary states
+        float *st = a.saved_states + ((size_t)u * (NCC + 1) + NCC) * 128 * 128;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int col = 8 * j + 2 * c4;
+            *reinterpret_cast<float2 *>(st + v0 * 128 + col) = make_float2(s[j][0], s[j][1]);
+            *reinterpret_cast<float2 *>(st + v1 * 128 + col) = make_float2(s[j][2], s[j][3]);
+        }
+    }
     if (a.S_final) {
         float *Sf = a.S_final + (size_t)u * 128 * 128;
 #pragma unroll
@@ -483,15 +474,24 @@ cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
     const int bytes = (int)sizeof(TcFwdSmem<NB>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    kern<<<a.B * a.H, 256, bytes, st>>>(a);
+    const int C = 16 * NB;
+    const long long rows = (long long)a.B * a.T;
+    TileMaps maps;
+    if ((e = make_token_tile_map(&maps.q, a.q, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&maps.k, a.k, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
+    if ((e = make_token_tile_map(&maps.v, a.v, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
+    kern<<<a.B * a.H, 256, bytes, st>>>(a, maps);
     return cudaGetLastError();
 }
 
-// Compute chunk of the tensor-core path for a gate chunk L (0 = not supported).
+// Compute chunk of the tensor-core forward for a gate chunk L (0 = not supported).
 int tc_compute_chunk(int L) { return L == 32 ? 32 : (L == 64 || L == 128) ? 64 : 0; }
 
-cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st) {
-    return tc_compute_chunk(a.L) == 32 ? launch_tc_fwd_t<2>(a, st) : launch_tc_fwd_t<4>(a, st);
+// C = 32 or 64 tokens per compute chunk.  With a.saved_states set, the state at every
+// compute-chunk boundary (T/C + 1 states per unit, the last one after the final token) and the
+// per-gate-chunk content signals are written for the backward.
+cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st) {
+    return C == 32 ? launch_tc_fwd_t<2>(a, st) : launch_tc_fwd_t<4>(a, st);
 }
 
 size_t tc_fwd_smem(int L) { return tc_compute_chunk(L) == 32 ? sizeof(TcFwdSmem<2>) : sizeof(TcFwdSmem<4>); }
