@@ -62,6 +62,15 @@ int tc_fwd_chunk(const carve_dims *d) {
 
 bool use_tc_bwd(const carve_dims *d) { return tc_shape(d) && d->T % 32 == 0; }
 
+// Bytes of the boundary states at the head of the `saved` buffer: fp32 states every 16 tokens
+// for the SIMT kernels; bf16 states every 32 tokens, rows padded to 136, for the tensor-core
+// kernels.  The per-chunk content signals (fp32) follow.
+size_t saved_states_bytes(const carve_dims *d) {
+    const size_t units = (size_t)d->B * d->H;
+    if (use_tc_bwd(d)) return units * (size_t)(d->T / 32) * 128 * 136 * 2;
+    return units * (size_t)(d->T / carve::kSub) * d->dv * d->dk * sizeof(float);
+}
+
 }  // namespace
 
 extern "C" {
@@ -80,15 +89,16 @@ const char *carve_status_string(carve_status s) {
 size_t carve_saved_bytes(const carve_dims *d) {
     if (check_dims(d, true) != CARVE_OK) return 0;
     const size_t units = (size_t)d->B * d->H;
-    const size_t n16 = (size_t)(d->T / carve::kSub), n32 = use_tc_bwd(d) ? (size_t)(d->T / 32 + 1) : 0;
-    const size_t states = units * (n16 > n32 ? n16 : n32) * d->dv * d->dk;
-    const size_t aux = units * n_chunks(d) * (size_t)(d->dv + d->rank + d->dk);
-    return sizeof(float) * (states + aux);
+    const size_t rec = use_tc_bwd(d) ? (size_t)(384 + d->rank) : (size_t)(d->dv + d->rank + d->dk);
+    return saved_states_bytes(d) + sizeof(float) * units * n_chunks(d) * rec;
 }
 
 size_t carve_bwd_workspace_bytes(const carve_dims *d) {
     if (check_dims(d, true) != CARVE_OK) return 0;
-    return sizeof(float) * (size_t)d->B * d->H * ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv);
+    const size_t units = (size_t)d->B * d->H;
+    if (use_tc_bwd(d))   // per gate chunk: dDelta and dz (160 floats) and the readout vector of dq
+        return sizeof(float) * units * n_chunks(d) * (160 + (size_t)d->dk);
+    return sizeof(float) * units * ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv);
 }
 
 carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
@@ -105,12 +115,10 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
     carve::FwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
     a.S0 = S0; a.m_prev_in = m_prev_in; a.o = o; a.S_final = S_final; a.m_prev_out = m_prev_out;
-    const size_t units = (size_t)d->B * d->H;
     const bool tc_saved = use_tc_bwd(d);
     if (saved) {
         a.saved_states = static_cast<float *>(saved);
-        const size_t nstates = tc_saved ? (size_t)(d->T / 32 + 1) : (size_t)(d->T / carve::kSub);
-        a.saved_aux = a.saved_states + units * nstates * d->dv * d->dk;
+        a.saved_aux = reinterpret_cast<float *>(static_cast<char *>(saved) + saved_states_bytes(d));
     }
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
     cudaError_t e;
@@ -144,11 +152,9 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
     (void)m_prev_in;  // their effect is captured by the saved states and content signals
     carve::BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
-    const size_t units = (size_t)d->B * d->H;
     const bool tc = use_tc_bwd(d);
     a.saved_states = static_cast<const float *>(saved);
-    const size_t nstates = tc ? (size_t)(d->T / 32 + 1) : (size_t)(d->T / carve::kSub);
-    a.saved_aux = a.saved_states + units * nstates * d->dv * d->dk;
+    a.saved_aux = reinterpret_cast<const float *>(static_cast<const char *>(saved) + saved_states_bytes(d));
     a.dO = dO; a.dS_final = dS_final; a.dm_prev_out = dm_prev_out;
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg_logit = dg_logit; a.dbx = dbx; a.dw_logit = dw_logit;
     a.dS0 = dS0; a.dm_prev_in = dm_prev_in; a.ws = static_cast<float *>(workspace);

@@ -25,10 +25,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// bf16x2 operand times a pair of factors (rounded to bf16), one packed multiply
 __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float f_lo, float f_hi) {
-    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&v);
-    float2 y = __bfloat1622float2(x);
-    return pack_bf16(y.x * f_lo, y.y * f_hi);
+    const uint32_t f = pack_bf16(f_lo, f_hi);
+    const __nv_bfloat162 r =
+        __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&v), *reinterpret_cast<const __nv_bfloat162 *>(&f));
+    return *reinterpret_cast<const uint32_t *>(&r);
 }
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {

@@ -18,7 +18,9 @@
 //                       (+ sum_s Kbar_s dKbar_s + gamma colsum(S0 * dS1) at the chunk's last token)
 //   gates      dl = reverse cumsum of dLam; d g_logit = -sigma(g_logit) dl; dbx = sigma(-beta) dl
 // (Qm, Krm, Kcm: mid-block referenced operands; Em, Fm, C: the block-level decay factors of the
-// forward.)  The content path (dz = A^T dDelta, dm = B^T dz) closes each gate chunk.
+// forward.)  The content path (dz = A^T dDelta, dm = B^T dz) closes each gate chunk; with the
+// boundary-state readout its term in dq (S0^T dm / n for every token of the gate chunk) is
+// stored per gate chunk and added by a parallel pass after the sweep.
 // Terms that cancel pairwise in the reverse cumulative sum of dLam (a Gram entry's row and
 // column token; Kbar_s against the chunk's last token) are formed from the same rounded values
 // on both sides, so the cancellation stays exact to fp32 rounding.
@@ -48,7 +50,7 @@ struct __align__(16) TcBwdSmem {
     float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], btot[kBNB * 128], pdd[kBNB * 128];
     float bpart[kBNB * 128];
     float delta[128], ddelta[128], mvec[128], zvec[64], dzv[64], dmv[128], dox[128], vecK[128], qbar[128];
-    uint64_t bar;
+    uint64_t bar, bar_s0;
 };
 
 __device__ int g_tc_bwd_timeout;
@@ -67,8 +69,12 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     const size_t tstride = (size_t)H * 128;
     const size_t base_bh = (size_t)b * T * tstride + (size_t)h * 128;
     const int v0 = 16 * warp + g, v1 = v0 + 8;
-    const float *states = a.saved_states + (size_t)u * (NCC + 1) * 128 * 128;
-    float *wsu = a.ws + (size_t)u * (256 * R);
+    // bf16 chunk-start states written by the forward, rows padded to kLdOp
+    const __nv_bfloat16 *states = reinterpret_cast<const __nv_bfloat16 *>(a.saved_states) + (size_t)u * NCC * 128 * kLdOp;
+    // workspace: per gate chunk dDelta (128) and dz (32) for the dA / dB reduction, then the
+    // readout vectors of dq (128 per gate chunk)
+    float *wsg = a.ws + (size_t)u * NG * 160;
+    float *wsv = a.ws + (size_t)a.B * a.H * NG * 160 + (size_t)u * NG * 128;
     const int kch = tid & 127, ib = tid >> 7;   // (channel, 16-block) owned in the gate phases
 
     float ds[16][4];
@@ -86,36 +92,52 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         }
     }
 
-    // column sums over this warp's rows of (dS .* S), into sm.xp[warp]
-    auto colsum_partial = [&](const float *S) {
+    // column sums over this warp's rows of (dS .* S0), S0 from the bf16 tile, into sm.xp[warp];
+    // the reduction over the 8 row lanes halves the live values at each exchange
+    auto colsum_partial = [&]() {
+        float v[16][2];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int col = 8 * j + 2 * c4;
-            const float2 s0 = *reinterpret_cast<const float2 *>(S + v0 * 128 + col);
-            const float2 s1 = *reinterpret_cast<const float2 *>(S + v1 * 128 + col);
-            float p0 = ds[j][0] * s0.x + ds[j][2] * s1.x;
-            float p1 = ds[j][1] * s0.y + ds[j][3] * s1.y;
+            const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + v0 * kLdOp + col);
+            const __nv_bfloat162 s1 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + v1 * kLdOp + col);
+            v[j][0] = ds[j][0] * bf(s0.x) + ds[j][2] * bf(s1.x);
+            v[j][1] = ds[j][1] * bf(s0.y) + ds[j][3] * bf(s1.y);
+        }
+        const bool up1 = g & 4, up2 = g & 2, up3 = g & 1;
+        float w1[8][2], w2[4][2], w3[2][2];
 #pragma unroll
-            for (int off = 4; off <= 16; off <<= 1) {
-                p0 += __shfl_xor_sync(0xffffffffu, p0, off);
-                p1 += __shfl_xor_sync(0xffffffffu, p1, off);
-            }
-            if (g == 0) {
-                sm.xp[warp * 128 + col] = p0;
-                sm.xp[warp * 128 + col + 1] = p1;
-            }
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                w1[j][e] = (up1 ? v[j + 8][e] : v[j][e]) + __shfl_xor_sync(0xffffffffu, up1 ? v[j][e] : v[j + 8][e], 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                w2[j][e] = (up2 ? w1[j + 4][e] : w1[j][e]) + __shfl_xor_sync(0xffffffffu, up2 ? w1[j][e] : w1[j + 4][e], 8);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                w3[j][e] = (up3 ? w2[j + 2][e] : w2[j][e]) + __shfl_xor_sync(0xffffffffu, up3 ? w2[j][e] : w2[j + 2][e], 4);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int jj = j + (up3 ? 2 : 0) + (up2 ? 4 : 0) + (up1 ? 8 : 0);
+            sm.xp[warp * 128 + 8 * jj + 2 * c4] = w3[j][0];
+            sm.xp[warp * 128 + 8 * jj + 2 * c4 + 1] = w3[j][1];
         }
     };
 
     if (tid == 0) {
         mbar_init(&sm.bar, 1);
+        mbar_init(&sm.bar_s0, 1);
         fence_mbar_init();
     }
     if (tid < 128) {
         const int nl = T - (NG - 1) * L;
         sm.dox[tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * 128 + tid] / (float)nl : 0.f;
     }
-    for (int idx = tid; idx < 256 * R; idx += 256) wsu[idx] = 0.f;
     auto issue = [&](int cc) {
         if (tid != 0) return;
         const int row = b * T + cc * C;
@@ -125,45 +147,43 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         tma_load_3d(sm.rv, &maps.v, 0, h, row, &sm.bar);
         tma_load_3d(sm.rdo, &maps.dO, 0, h, row, &sm.bar);
     };
+    auto issue_s0 = [&](int cc) {
+        if (tid != 0) return;
+        mbar_expect_tx(&sm.bar_s0, 128u * kLdOp * 2u);
+        bulk_g2s(sm.s0b, states + (size_t)cc * 128 * kLdOp, 128u * kLdOp * 2u, &sm.bar_s0);
+    };
     issue(NCC - 1);
+    issue_s0(NCC - 1);
     uint32_t phase = 0;
     __syncthreads();
+    // gate logits of the chunk about to be processed, loaded one chunk ahead
+    float glr[16], bxr[16];
+    auto load_gates = [&](int cc) {
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const size_t gi = base_bh + (size_t)(cc * C + 16 * ib + t) * tstride + kch;
+            glr[t] = a.g_logit[gi];
+            bxr[t] = a.bx[gi];
+        }
+    };
+    load_gates(NCC - 1);
 
     for (int cc = NCC - 1; cc >= 0; --cc) {
         const int t0 = cc * C, gc = cc / CPG;
         const bool gate_end = (cc % CPG) == CPG - 1 || cc == NCC - 1;
         const bool gate_start = (cc % CPG) == 0;
         const int n = min(L, T - gc * L);
-        float glr[16], bxr[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const size_t gi = base_bh + (size_t)(t0 + 16 * ib + t) * tstride + kch;
-            glr[t] = a.g_logit[gi];
-            bxr[t] = a.bx[gi];
-        }
         if (gate_end) {
-            const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (256 + R);
+            const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (384 + R);
             if (tid < 128) {
                 sm.mvec[tid] = aux[tid];
                 sm.delta[tid] = aux[128 + R + tid];
+                sm.qbar[tid] = aux[256 + R + tid];
                 sm.ddelta[tid] = 0.f;
             }
             if (tid < R) sm.zvec[tid] = aux[128 + tid];
         }
-        {   // this chunk's start state and the carried gradient, as bf16 tiles
-            const float *S0 = states + (size_t)cc * 128 * 128;
-            const int r = tid >> 1, half = tid & 1;
-            const float4 *src = reinterpret_cast<const float4 *>(S0 + r * 128 + half * 64);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const float4 f0 = src[2 * x], f1 = src[2 * x + 1];
-                uint4 o4;
-                o4.x = pack_bf16(f0.x, f0.y);
-                o4.y = pack_bf16(f0.z, f0.w);
-                o4.z = pack_bf16(f1.x, f1.y);
-                o4.w = pack_bf16(f1.z, f1.w);
-                *reinterpret_cast<uint4 *>(sm.s0b + r * kLdOp + half * 64 + 8 * x) = o4;
-            }
+        {   // the carried gradient as a bf16 tile
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int col = 8 * j + 2 * c4;
@@ -171,16 +191,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 *reinterpret_cast<uint32_t *>(sm.ds1b + v1 * kLdOp + col) = pack_bf16(ds[j][2], ds[j][3]);
             }
         }
-        colsum_partial(states + (size_t)cc * 128 * 128);   // for gamma * dgamma
         if (!mbar_wait(&sm.bar, phase)) atomicOr(&g_tc_bwd_timeout, 1);
-        phase ^= 1u;
         __syncthreads();
-        if (tid < 128) {
-            float x = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) x += sm.xp[w * 128 + tid];
-            sm.s0ds[tid] = x;
-        }
         // dO plus the content-signal gradient carried from the next gate chunk, padded
         for (int idx = tid; idx < C * 16; idx += 256) {
             const int t = idx >> 4, part = idx & 15;
@@ -235,7 +247,16 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             }
             sm.cij[tid] = sm.r15[tid] * sm.p7[128 + tid];   // e^{Lam_m(1) - Lam_m(0)}
         }
+        if (!mbar_wait(&sm.bar_s0, phase)) atomicOr(&g_tc_bwd_timeout, 2);
+        phase ^= 1u;
+        colsum_partial();   // for gamma * dgamma
         __syncthreads();
+        if (tid < 128) {
+            float x = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x += sm.xp[w * 128 + tid];
+            sm.s0ds[tid] = x;
+        }
         // ---- Gram blocks (warps 0-3: type x row block), T_ii on the Akk warps
         if (warp < 4) {
             const int type = warp >> 1, i = warp & 1;
@@ -321,6 +342,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             rr[j][3] = bf(sm.rv[(t + 1) * 128 + v1]) - rr[j][3];
         }
         __syncthreads();
+        if (cc > 0) issue(cc - 1);   // q, k, v and dO of this chunk are no longer read
         // ---- U (blocked WY solve), E = R - Akk U, U -> shared tile
         float ga[4][4];
 #pragma unroll
@@ -711,15 +733,21 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 const bool floor = !(__fdividef(1.f, D) >= kAMin);
                 const float dglv = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run;
                 const float dbv = floor ? 0.f : __fdividef(e2, 1.f + e2) * run;
-                const size_t gi = base_bh + (size_t)(t0 + 16 * ib + t) * tstride + kch;
-                a.dg_logit[gi] = dglv;
-                a.dbx[gi] = dbv;
+                sm.dlam[(16 * ib + t) * 129 + kch] = dglv;   // staged: this thread's own column
+                sm.rfac[(16 * ib + t) * 129 + kch] = dbv;
                 pdd += dbv;
             }
             sm.pdd[ib * 128 + kch] = pdd;
         }
         __syncthreads();
         if (tid < 128) sm.ddelta[tid] += sm.pdd[tid] + sm.pdd[128 + tid];
+        for (int idx = tid; idx < C * 32; idx += 256) {   // d g_logit, dbx: four channels per store
+            const int t = idx >> 5, c = (idx & 31) * 4;
+            const float *gsrc = sm.dlam + t * 129 + c, *bsrc = sm.rfac + t * 129 + c;
+            const size_t gi = base_bh + (size_t)(t0 + t) * tstride + c;
+            *reinterpret_cast<float4 *>(a.dg_logit + gi) = make_float4(gsrc[0], gsrc[1], gsrc[2], gsrc[3]);
+            *reinterpret_cast<float4 *>(a.dbx + gi) = make_float4(bsrc[0], bsrc[1], bsrc[2], bsrc[3]);
+        }
         __syncthreads();
         // ---- content path at the gate chunk's first token
         if (gate_start) {
@@ -735,30 +763,35 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 if (j < R && part == 0) sm.dzv[j] = s;
             }
             __syncthreads();
-            for (int idx = tid; idx < 128 * R; idx += 256) wsu[idx] += sm.ddelta[idx / R] * sm.zvec[idx % R];
-            for (int idx = tid; idx < R * 128; idx += 256) wsu[128 * R + idx] += sm.dzv[idx / 128] * sm.mvec[idx % 128];
-            if (tid < 128) {
-                float s = 0.f;
+            if (tid < 128) wsg[(size_t)gc * 160 + tid] = sm.ddelta[tid];
+            if (tid < R) wsg[(size_t)gc * 160 + 128 + tid] = sm.dzv[tid];
+            {   // dm = B^T dz, two threads per output
+                const int vv = tid >> 1, half = tid & 1;
+                float sacc = 0.f;
 #pragma unroll 8
-                for (int j = 0; j < R; ++j) s += a.Bm[((size_t)h * R + j) * 128 + tid] * sm.dzv[j];
-                sm.dmv[tid] = s;
+                for (int j = half; j < R; j += 2) sacc += a.Bm[((size_t)h * R + j) * 128 + vv] * sm.dzv[j];
+                sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+                if (half == 0) sm.dmv[vv] = sacc;
             }
             __syncthreads();
             if (a.mc_mode == 0) {
-                // m = S0 qbar:  dS0 += dm qbar^T,  dq_t += S0^T dm / n  for every t of the gate chunk
-                if (tid < 128) {
-                    float acc = 0.f;
-#pragma unroll 8
-                    for (int t = 0; t < n; ++t) acc += bf(q[base_bh + (size_t)(gc * L + t) * tstride + tid]);
-                    sm.qbar[tid] = acc / (float)n;
-                    const float *S0 = states + (size_t)cc * 128 * 128;
-                    float s = 0.f;
-#pragma unroll 8
-                    for (int r = 0; r < 128; ++r) s += S0[r * 128 + tid] * sm.dmv[r];
-                    sm.vecK[tid] = s / (float)n;
-                    sm.dox[tid] = 0.f;
+                // m = S0 qbar:  dS0 += dm qbar^T here;  dq_t += S0^T dm / n for every t of the gate
+                // chunk is added by the readout pass after this kernel (vector stored per gate chunk)
+                {
+                    const int ch = tid & 127, half = tid >> 7;
+                    float sa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int r = 0; r < 64; r += 4)
+#pragma unroll
+                        for (int x = 0; x < 4; ++x)
+                            sa[x] += bf(sm.s0b[(64 * half + r + x) * kLdOp + ch]) * sm.dmv[64 * half + r + x];
+                    sm.pdd[half * 128 + ch] = (sa[0] + sa[1]) + (sa[2] + sa[3]);
                 }
                 __syncthreads();
+                if (tid < 128) {
+                    wsv[(size_t)gc * 128 + tid] = (sm.pdd[tid] + sm.pdd[128 + tid]) / (float)n;
+                    sm.dox[tid] = 0.f;
+                }
                 const float m0 = sm.dmv[v0], m1 = sm.dmv[v1];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -769,19 +802,16 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     ds[j][2] += m1 * q0;
                     ds[j][3] += m1 * q1;
                 }
-                for (int idx = tid; idx < n * 64; idx += 256) {
-                    const int t = idx >> 6, c2 = (idx & 63) * 2;
-                    __nv_bfloat16 *p = dq + base_bh + (size_t)(gc * L + t) * tstride + c2;
-                    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(p);
-                    *reinterpret_cast<uint32_t *>(p) = pack_bf16(bf(x.x) + sm.vecK[c2], bf(x.y) + sm.vecK[c2 + 1]);
-                }
             } else if (tid < 128) {
                 sm.dox[tid] = gc > 0 ? sm.dmv[tid] / (float)L : 0.f;
                 if (gc == 0 && a.dm_prev_in) a.dm_prev_in[(size_t)u * 128 + tid] = sm.dmv[tid];
             }
         }
-        if (cc > 0) issue(cc - 1);
         __syncthreads();
+        if (cc > 0) {
+            issue_s0(cc - 1);
+            load_gates(cc - 1);
+        }
     }
     if (a.dS0) {
         float *D = a.dS0 + (size_t)u * 128 * 128;
@@ -795,7 +825,49 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     if (a.mc_mode == 0 && a.dm_prev_in && tid < 128) a.dm_prev_in[(size_t)u * 128 + tid] = 0.f;
 }
 
-__global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, int B, int H, int KR, int RV);
+
+// dA[h] = sum_{b, gate chunk} dDelta z^T,  dB[h] = sum dz m^T  (z, m from the saved records),
+// summed in a fixed order
+__global__ void reduce_dAdB_tc_kernel(const float *wsg, const float *aux, float *dA, float *dB, int B, int H, int NG,
+                                      int R) {
+    const int h = blockIdx.y, x = blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= 256 * R) return;
+    const bool isA = x < 128 * R;
+    const int y = isA ? x : x - 128 * R;
+    const int r0 = isA ? y / R : y / 128, r1 = isA ? y % R : y % 128;
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b) {
+        const size_t u = (size_t)b * H + h;
+        for (int gc = 0; gc < NG; ++gc) {
+            const float *g = wsg + (u * NG + gc) * 160, *rec = aux + (u * NG + gc) * (384 + R);
+            acc += isA ? g[r0] * rec[128 + r1] : g[128 + r0] * rec[r1];
+        }
+    }
+    if (isA) dA[(size_t)h * 128 * R + y] = acc;
+    else dB[(size_t)h * R * 128 + y] = acc;
+}
+
+// dq_t += vec[unit][gate chunk of t] (the content-readout term of the default readout), 8
+// channels per thread
+__global__ void dq_readout_kernel(__nv_bfloat16 *dq, const float *vec, int H, int T, int L, size_t rows) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows * 16) return;
+    const size_t row = i >> 4;                  // (b, t, h)
+    const int part = (int)(i & 15), h = (int)(row % H);
+    const size_t bt = row / H;
+    const int t = (int)(bt % T), b = (int)(bt / T);
+    const int NG = (T + L - 1) / L;
+    const float *vk = vec + (((size_t)b * H + h) * NG + t / L) * 128 + part * 8;
+    uint4 *p = reinterpret_cast<uint4 *>(dq + row * 128 + part * 8);
+    uint4 x = *p;
+    __nv_bfloat162 *xv = reinterpret_cast<__nv_bfloat162 *>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(xv[e]);
+        xv[e] = __floats2bfloat162_rn(f.x + vk[2 * e], f.y + vk[2 * e + 1]);
+    }
+    *p = x;
+}
 
 cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st) {
     const int bytes = (int)sizeof(TcBwdSmem);
@@ -809,9 +881,16 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
     if ((e = make_token_tile_map(&maps.dO, a.dO, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
     tc_bwd_kernel<<<a.B * a.H, 256, bytes, st>>>(a, maps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int KR = 128 * a.R, RV = a.R * 128;
-    dim3 grid((KR + RV + 255) / 256, a.H);
-    reduce_dAdB_kernel<<<grid, 256, 0, st>>>(a.ws, dA, dB, a.B, a.H, KR, RV);
+    if (a.mc_mode == 0) {
+        const size_t rows = (size_t)a.B * a.T * a.H;
+        const float *vec = a.ws + (size_t)a.B * a.H * ((a.T + a.L - 1) / a.L) * 160;
+        dq_readout_kernel<<<(unsigned)((rows * 16 + 255) / 256), 256, 0, st>>>(static_cast<__nv_bfloat16 *>(a.dq), vec,
+                                                                              a.H, a.T, a.L, rows);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const int NG = (a.T + a.L - 1) / a.L;
+    dim3 grid((256 * a.R + 255) / 256, a.H);
+    reduce_dAdB_tc_kernel<<<grid, 256, 0, st>>>(a.ws, a.saved_aux, dA, dB, a.B, a.H, NG, a.R);
     return cudaGetLastError();
 }
 

@@ -32,7 +32,14 @@ __device__ int g_tc_timeout;  // set when a bounded wait gives up (never expecte
 template <int NB>
 struct __align__(16) TcFwdSmem {
     static constexpr int C = 16 * NB, LDA = C + 8, NPAIR = NB * (NB - 1) / 2 > 0 ? NB * (NB - 1) / 2 : 1;
-    __nv_bfloat16 rq[C * 128], rk[C * 128], rv[C * 128];
+    // 32-token chunks: every input tile of the next chunk (q, k, v and the fp32 gate logits)
+    // is brought in by TMA into a second stage while this chunk computes.  64-token chunks do
+    // not fit twice: one stage, gate logits through registers.
+    static constexpr int ST = NB == 2 ? 2 : 1;
+    static constexpr bool GT = NB == 2;
+    static constexpr int GSZ = GT ? C * 128 : 4;
+    __nv_bfloat16 rq[ST][C * 128], rk[ST][C * 128], rv[ST][C * 128];
+    float rgl[ST][GSZ], rbx[ST][GSZ];
     __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp], qt[C * kLdOp], kt[C * kLdOp];
     __nv_bfloat16 aqk[C * LDA], mkk[C * LDA];
     __nv_bfloat16 tii[NB * 16 * 24];
@@ -40,13 +47,13 @@ struct __align__(16) TcFwdSmem {
     float p7[NB * 128], r15[NB * 128], dblk[NB * 128], em[NB * 128], fm[NB * 128], cij[NPAIR * 128];
     float gam[128], wv[C], qbar[128], mvec[128], osum[128], mprev[128], zvec[64], delta[128];
     float Ah[128 * kTcMaxRank], Bh[kTcMaxRank * 128];   // the head's low-rank factors
-    uint64_t bar;
+    uint64_t bar[ST];
     // the output tile is staged in qt once the S-GEMM has consumed it
     __device__ __nv_bfloat16 *ost() { return qt; }
 };
 
 struct TileMaps {
-    CUtensorMap q, k, v;
+    CUtensorMap q, k, v, gl, bx;
 };
 
 template <int NB>
@@ -83,7 +90,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         }
     }
     if (tid == 0) {
-        mbar_init(&sm.bar, 1);
+        for (int i = 0; i < SM::ST; ++i) mbar_init(&sm.bar[i], 1);
         fence_mbar_init();
     }
     if (tid < 128) {
@@ -96,64 +103,83 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     }
     __syncthreads();
 
-    // raw q/k/v tiles of chunk cc by TMA (one tensor copy per tile): which = 0 -> q and k
-    // (arming the barrier with the byte count of all three), 1 -> v
+    // Input tiles of chunk cc by TMA (one tensor copy per tile) into stage cc % ST.  With two
+    // stages everything is issued at once, one chunk ahead; with one stage q/k (which = 0,
+    // arming the barrier) go out mid-chunk and v (which = 1) at the end of the previous chunk.
     auto issue = [&](int cc, int which) {
         if (tid != 0) return;
-        const int row = b * T + cc * C;
+        const int row = b * T + cc * C, st = cc % SM::ST;
+        uint64_t *bar = &sm.bar[st];
         if (which == 0) {
-            mbar_expect_tx(&sm.bar, 3u * C * 256u);
-            tma_load_3d(sm.rq, &maps.q, 0, h, row, &sm.bar);
-            tma_load_3d(sm.rk, &maps.k, 0, h, row, &sm.bar);
-        } else {
-            tma_load_3d(sm.rv, &maps.v, 0, h, row, &sm.bar);
+            mbar_expect_tx(bar, 3u * C * 256u + (SM::GT ? 2u * C * 512u : 0u));
+            tma_load_3d(sm.rq[st], &maps.q, 0, h, row, bar);
+            tma_load_3d(sm.rk[st], &maps.k, 0, h, row, bar);
+            if (SM::GT) {
+                tma_load_3d(sm.rgl[st], &maps.gl, 0, h, row, bar);
+                tma_load_3d(sm.rbx[st], &maps.bx, 0, h, row, bar);
+            }
         }
+        if (which == 1 || SM::ST == 2) tma_load_3d(sm.rv[st], &maps.v, 0, h, row, bar);
     };
     if (tid == 0) {
         tma_prefetch_desc(&maps.q);
         tma_prefetch_desc(&maps.k);
         tma_prefetch_desc(&maps.v);
+        if (SM::GT) {
+            tma_prefetch_desc(&maps.gl);
+            tma_prefetch_desc(&maps.bx);
+        }
     }
     issue(0, 0);
-    issue(0, 1);
-    uint32_t phase = 0;
+    if (SM::ST == 1) issue(0, 1);
+    uint32_t phase_bits = 0u;   // bit st: parity to wait for on stage st
+    float wnext = tid < C ? a.w_logit[((size_t)b * T + tid) * H + h] : 0.f;
 
     for (int cc = 0; cc < NCC; ++cc) {
         const int t0 = cc * C, gc = cc / CPG;
         const bool first = (cc % CPG) == 0, last = (cc % CPG) == CPG - 1 || cc == NCC - 1;
         const int n = min(L, T - gc * L);
-        // gate inputs of this chunk, into registers (their latency overlaps the readout)
+        const int st = cc % SM::ST;
+        // gate inputs of this chunk, into registers (one-stage layout only; their latency
+        // overlaps the readout)
         float glr[NP][16], bxr[NP][16];
+        if (!SM::GT) {
 #pragma unroll
-        for (int x = 0; x < NP; ++x) {
-            const int p = tid + 256 * x, kch = p & 127, i = p >> 7;
-            if (p < 128 * NB) {
+            for (int x = 0; x < NP; ++x) {
+                const int p = tid + 256 * x, kch = p & 127, i = p >> 7;
+                if (p < 128 * NB) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const size_t gi = ((size_t)b * T + t0 + 16 * i + t) * tstride + (size_t)h * 128 + kch;
-                    glr[x][t] = a.g_logit[gi];
-                    bxr[x][t] = a.bx[gi];
+                    for (int t = 0; t < 16; ++t) {
+                        const size_t gi = ((size_t)b * T + t0 + 16 * i + t) * tstride + (size_t)h * 128 + kch;
+                        glr[x][t] = a.g_logit[gi];
+                        bxr[x][t] = a.bx[gi];
+                    }
                 }
             }
         }
-        if (!mbar_wait(&sm.bar, phase)) atomicOr(&g_tc_timeout, 1);
-        phase ^= 1u;
-        if (a.saved_states) {
-            float *st = a.saved_states + ((size_t)u * (NCC + 1) + cc) * 128 * 128;
+        if (!mbar_wait(&sm.bar[st], (phase_bits >> st) & 1u)) atomicOr(&g_tc_timeout, 1);
+        phase_bits ^= 1u << st;
+        if (SM::ST == 2 && cc + 1 < NCC) issue(cc + 1, 0);   // the other stage is free since last chunk
+        const float wcur = wnext;
+        if (tid < C && cc + 1 < NCC) wnext = a.w_logit[((size_t)b * T + t0 + C + tid) * H + h];
+        if (a.saved_states) {   // bf16 copy of the chunk-start state, rows padded to 136
+            __nv_bfloat16 *stb = reinterpret_cast<__nv_bfloat16 *>(a.saved_states) + ((size_t)u * NCC + cc) * 128 * kLdOp;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int col = 8 * j + 2 * c4;
-                *reinterpret_cast<float2 *>(st + v0 * 128 + col) = make_float2(s[j][0], s[j][1]);
-                *reinterpret_cast<float2 *>(st + v1 * 128 + col) = make_float2(s[j][2], s[j][3]);
+                *reinterpret_cast<uint32_t *>(stb + v0 * kLdOp + col) = pack_bf16(s[j][0], s[j][1]);
+                *reinterpret_cast<uint32_t *>(stb + v1 * kLdOp + col) = pack_bf16(s[j][2], s[j][3]);
             }
         }
         // ---- content signal at a gate-chunk start
         if (first) {
             if (a.mc_mode == 0) {
-                if (tid < 128) {
+                if (tid < 128 && a.saved_aux) {   // written by the chunk-mean prologue
+                    sm.qbar[tid] = a.saved_aux[((size_t)u * NG + gc) * (384 + R) + 256 + R + tid];
+                } else if (tid < 128) {
                     float acc = 0.f;
                     if (CPG == 1) {
-                        for (int t = 0; t < C; ++t) acc += bf(sm.rq[t * 128 + tid]);
+                        for (int t = 0; t < C; ++t) acc += bf(sm.rq[st][t * 128 + tid]);
                     } else {
 #pragma unroll 8
                         for (int t = 0; t < n; ++t) acc += bf(q[base_bh + (size_t)(gc * L + t) * tstride + tid]);
@@ -184,7 +210,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             content_signal<128, 128>(sm.Bh, sm.Ah, sm.mvec, sm.zvec, sm.delta, R);
             if (tid < 128) sm.osum[tid] = 0.f;
             if (a.saved_aux) {
-                float *aux = a.saved_aux + ((size_t)u * NG + gc) * (256 + R);
+                float *aux = a.saved_aux + ((size_t)u * NG + gc) * (384 + R);
                 if (tid < 128) {
                     aux[tid] = sm.mvec[tid];
                     aux[128 + R + tid] = sm.delta[tid];
@@ -200,7 +226,15 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 const float dl = sm.delta[kch];
                 float av[16], ia[16], rf[16], cf[16];
 #pragma unroll
-                for (int t = 0; t < 16; ++t) retention(glr[x][t], bxr[x][t] + dl, av[t], ia[t]);
+                if (SM::GT) {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        retention(sm.rgl[st][(16 * i + t) * 128 + kch], sm.rbx[st][(16 * i + t) * 128 + kch] + dl, av[t],
+                                  ia[t]);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) retention(glr[x][t], bxr[x][t] + dl, av[t], ia[t]);
+                }
                 mid_reference(av, ia, rf, cf);
                 float p7 = 1.f;
 #pragma unroll
@@ -211,14 +245,14 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int row = 16 * i + t;
-                    const float qv = bf(sm.rq[row * 128 + kch]), kv = bf(sm.rk[row * 128 + kch]);
+                    const float qv = bf(sm.rq[st][row * 128 + kch]), kv = bf(sm.rk[st][row * 128 + kch]);
                     sm.qm[row * kLdOp + kch] = __float2bfloat16_rn(qv * rf[t]);
                     sm.krm[row * kLdOp + kch] = __float2bfloat16_rn(kv * rf[t]);
                     sm.kcm[row * kLdOp + kch] = __float2bfloat16_rn(kv * cf[t]);
                 }
             }
         }
-        if (tid < C) sm.wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + t0 + tid) * H + h]);
+        if (tid < C) sm.wv[tid] = sigmoid_f(wcur);
         __syncthreads();
         // ---- chunk-level factors per channel
         if (tid < 128) {
@@ -329,16 +363,16 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             }
         }
         __syncthreads();
-        if (cc + 1 < NCC) issue(cc + 1, 0);
+        if (SM::ST == 1 && cc + 1 < NCC) issue(cc + 1, 0);
         // ---- X = Diag(w)(V - Kt S0^T), as X^T (rows v, cols t)
 #pragma unroll
         for (int j = 0; j < 2 * NB; ++j) {
             const int t = 8 * j + 2 * c4;
             const float w0 = sm.wv[t], w1 = sm.wv[t + 1];
-            ga[j][0] = w0 * (bf(sm.rv[t * 128 + v0]) - ga[j][0]);
-            ga[j][1] = w1 * (bf(sm.rv[(t + 1) * 128 + v0]) - ga[j][1]);
-            ga[j][2] = w0 * (bf(sm.rv[t * 128 + v1]) - ga[j][2]);
-            ga[j][3] = w1 * (bf(sm.rv[(t + 1) * 128 + v1]) - ga[j][3]);
+            ga[j][0] = w0 * (bf(sm.rv[st][t * 128 + v0]) - ga[j][0]);
+            ga[j][1] = w1 * (bf(sm.rv[st][(t + 1) * 128 + v0]) - ga[j][1]);
+            ga[j][2] = w0 * (bf(sm.rv[st][t * 128 + v1]) - ga[j][2]);
+            ga[j][3] = w1 * (bf(sm.rv[st][(t + 1) * 128 + v1]) - ga[j][3]);
         }
         // ---- blocked solve:  U_i^T = (X_i^T - sum_{j<i} U_j^T M_ij^T) T_ii^T
 #pragma unroll
@@ -436,7 +470,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             }
         }
         __syncthreads();
-        if (cc + 1 < NCC) issue(cc + 1, 1);
+        if (SM::ST == 1 && cc + 1 < NCC) issue(cc + 1, 1);
         for (int idx = tid; idx < C * 16; idx += 256) {
             const int t = idx >> 4, part = idx & 15;
             *reinterpret_cast<uint4 *>(o + base_bh + (size_t)(t0 + t) * tstride + part * 8) =
@@ -446,15 +480,6 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             if (tid < 128) sm.mprev[tid] = sm.osum[tid] / (float)n;
         }
         __syncthreads();
-    }
-    if (a.saved_states) {   // the state after the last token closes the list of boundary states
-        float *st = a.saved_states + ((size_t)u * (NCC + 1) + NCC) * 128 * 128;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int col = 8 * j + 2 * c4;
-            *reinterpret_cast<float2 *>(st + v0 * 128 + col) = make_float2(s[j][0], s[j][1]);
-            *reinterpret_cast<float2 *>(st + v1 * 128 + col) = make_float2(s[j][2], s[j][3]);
-        }
     }
     if (a.S_final) {
         float *Sf = a.S_final + (size_t)u * 128 * 128;
@@ -466,6 +491,22 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         }
     }
     if (a.m_prev_out && tid < 128) a.m_prev_out[(size_t)u * 128 + tid] = sm.mprev[tid];
+}
+
+// Per (unit, gate chunk): mean of q over the gate chunk's tokens, into the saved aux record
+// (offset 256 + R of each 384 + R floats).  One CTA per record, one thread per channel.
+__global__ void __launch_bounds__(128) qbar_kernel(const __nv_bfloat16 *q, float *aux, int H, int T, int L, int R) {
+    const int rec = blockIdx.x, NG = (T + L - 1) / L;
+    const int u = rec / NG, gc = rec % NG, b = u / H, h = u % H, tid = threadIdx.x;
+    const int n = min(L, T - gc * L);
+    const __nv_bfloat16 *src = q + ((size_t)b * T + (size_t)gc * L) * H * 128 + (size_t)h * 128 + tid;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int t = 0;
+    for (; t + 4 <= n; t += 4)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[x] += bf(src[(size_t)(t + x) * H * 128]);
+    for (; t < n; ++t) acc[0] += bf(src[(size_t)t * H * 128]);
+    aux[(size_t)rec * (384 + R) + 256 + R + tid] = (acc[0] + acc[1] + acc[2] + acc[3]) / (float)n;
 }
 
 template <int NB>
@@ -480,6 +521,16 @@ cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
     if ((e = make_token_tile_map(&maps.q, a.q, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
     if ((e = make_token_tile_map(&maps.k, a.k, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
     if ((e = make_token_tile_map(&maps.v, a.v, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
+    if (TcFwdSmem<NB>::GT) {
+        if ((e = make_token_tile_map(&maps.gl, a.g_logit, 4, 128, a.H, rows, C)) != cudaSuccess) return e;
+        if ((e = make_token_tile_map(&maps.bx, a.bx, 4, 128, a.H, rows, C)) != cudaSuccess) return e;
+    }
+    if (a.saved_aux && a.mc_mode == 0) {
+        const int NG = (a.T + a.L - 1) / a.L;
+        qbar_kernel<<<a.B * a.H * NG, 128, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.q), a.saved_aux, a.H, a.T,
+                                                    a.L, a.R);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     kern<<<a.B * a.H, 256, bytes, st>>>(a, maps);
     return cudaGetLastError();
 }
@@ -487,9 +538,10 @@ cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
 // Compute chunk of the tensor-core forward for a gate chunk L (0 = not supported).
 int tc_compute_chunk(int L) { return L == 32 ? 32 : (L == 64 || L == 128) ? 64 : 0; }
 
-// C = 32 or 64 tokens per compute chunk.  With a.saved_states set, the state at every
-// compute-chunk boundary (T/C + 1 states per unit, the last one after the final token) and the
-// per-gate-chunk content signals are written for the backward.
+// C = 32 or 64 tokens per compute chunk.  With a.saved_states set (32-token chunks), a bf16
+// copy of the state at every compute-chunk start ([T/32][128][136] per unit, rows padded) and
+// per gate chunk the record (m, z, Delta, mean q) of 384 + R floats are written for the
+// backward.
 cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st) {
     return C == 32 ? launch_tc_fwd_t<2>(a, st) : launch_tc_fwd_t<4>(a, st);
 }
