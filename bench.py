@@ -19,7 +19,6 @@ import dataclasses
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -57,6 +56,15 @@ def bwd_flops(d, L, r):
     return 14 * L * d + 14 * d * d + L * L
 
 
+def launches_per_step(w, fwd_only):
+    """Kernels one step launches on the tensor-core path (bf16, d = 128): the forward (plus the
+    chunk-mean prologue when it saves for the backward in mode 0); the backward, the dq
+    readout pass (mode 0) and the dA/dB reduction."""
+    if fwd_only:
+        return 1
+    return (2 if w.mc_mode == 0 else 1) + (3 if w.mc_mode == 0 else 2)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -68,48 +76,75 @@ def load_peaks():
 
 # ---------------------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """SM clock, power and throttle reasons of this process's GPU, polled through NVML every
+    `period` seconds on a host thread during the timed region (read-only queries); the
+    samples are also written to gpurun_out/clocks_rank<i>.csv."""
+    NAMES = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+             ("sw_power_cap", 0x4))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    def __init__(self, index: int, period: float = 0.005):
+        self.index, self.period = index, period
+        self.rows, self.err = [], None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
 
-    def __enter__(self):
+    def _handle(self, nv):
+        import torch
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                                         stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+            p = torch.cuda.get_device_properties(self.index)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:   # noqa: BLE001 - older torch without PCI fields: CUDA order
+            return nv.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _run(self):
+        nv = self.nv
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                self.rows.append((time.time(), nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                  nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0, int(reasons_fn(self.h))))
+            except Exception as e:   # noqa: BLE001
+                self.err = str(e)
+                return
+            self.stop.wait(self.period)
+
+    def __enter__(self):
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv, self.h = nv, self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception as e:   # noqa: BLE001
+            self.nv, self.err = None, f"nvml: {e}"
+            return self
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.f.close()
+        if self.nv is None:
+            return
+        self.stop.set()
+        self.thread.join(timeout=5)
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            with open(self.path, "w") as f:
+                f.write("time,sm_mhz,sm_max_mhz,power_w,reasons_mask\n")
+                for t, mhz, pw, rs in self.rows:
+                    f.write(f"{t:.3f},{mhz},{self.max_mhz},{pw:.1f},{rs:#x}\n")
+        except OSError:
+            pass
+        self.nv.nvmlShutdown()
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.count(",") >= 8]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows]
-        mx = max(float(r[2]) for r in rows)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(float(r[3]) for r in rows)}
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled: " + str(self.err)]}
+        reasons = sorted({n for _, _, _, rs in self.rows for n, bit in self.NAMES if rs & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.rows), "power_w_max": max(r[2] for r in self.rows)}
 
 
 # ---------------------------------------------------------------------------------------
@@ -287,7 +322,7 @@ def run_train(args, w, fwd_only=False):
     line = {
         "metric": "fwd tokens/s per layer (B200, 16 heads, d=128)" if fwd_only else METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "heads": w.H, "d": w.K,
                    "chunk": L, "rank": w.R, "mc_mode": mode, "parallelism": f"dp{ws}",
                    "l2": "no flush: step working set ~3 GB >> 126 MB L2"},
@@ -295,7 +330,7 @@ def run_train(args, w, fwd_only=False):
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm"], "traffic": traffic, "peak_source": peaks["source"]},
         "kernels_ms": {"carve_fwd": fwd_ms, "carve_bwd": bwd_ms},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (1 if fwd_only else 3) * args.steps,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, fwd_only) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0:

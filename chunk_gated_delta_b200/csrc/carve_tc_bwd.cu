@@ -63,7 +63,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
     const int b = u / H, h = u % H;
     const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
     __nv_bfloat16 *dq = static_cast<__nv_bfloat16 *>(a.dq), *dk = static_cast<__nv_bfloat16 *>(a.dk);
     __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv);
     const size_t tstride = (size_t)H * 128;

@@ -68,8 +68,6 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     const int b = u / H, h = u % H;
     const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
-    const __nv_bfloat16 *kk = static_cast<const __nv_bfloat16 *>(a.k);
-    const __nv_bfloat16 *vv = static_cast<const __nv_bfloat16 *>(a.v);
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
     const size_t tstride = (size_t)H * 128;
     const size_t base_bh = (size_t)b * T * tstride + (size_t)h * 128;   // token 0 of this unit
@@ -225,7 +223,6 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             if (p < 128 * NB) {
                 const float dl = sm.delta[kch];
                 float av[16], ia[16], rf[16], cf[16];
-#pragma unroll
                 if (SM::GT) {
 #pragma unroll
                     for (int t = 0; t < 16; ++t)

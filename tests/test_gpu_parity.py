@@ -121,6 +121,22 @@ def test_chunk_lengths_bf16(cuda_device, L):
         run_case(cuda_device, w, d, dO, L, mode)
 
 
+@pytest.mark.parametrize("T,L", [(352, 64), (352, 128), (320, 128), (448, 64)])
+def test_saved_state_paths_bf16(cuda_device, T, L):
+    """Gate chunks of 64 and 128 tokens over the 32-token chunks that the training path saves
+    and reverses, with T a multiple of 64 or only of 32 (gate chunks of 128 may end ragged).
+    Carried S0, m_prev_in, dS_final and dm_prev_out."""
+    w, d, dO = small(I.FWD_1P3B, B=1, H=3, T=T, L=L, seed=T + L)
+    d["A"] *= 10.0
+    d["B"] *= 10.0
+    S0 = I.make_state(w, 0.05)
+    mp = I.normal(2, 2, (w.B, w.H, w.V)).astype(np.float32)
+    dSf = I.normal(2, 3, (w.B, w.H, w.V, w.K)).astype(np.float32)
+    dmo = I.normal(2, 4, (w.B, w.H, w.V)).astype(np.float32)
+    for mode in (0, 1):
+        run_case(cuda_device, w, d, dO, L, mode, S0=S0, mp=mp, dSf=dSf, dmo=dmo)
+
+
 def test_zero_projection_is_chunk_length_invariant(cuda_device):
     """U_b = 0 (A = 0): the erase gate is sigmoid(bx + 0) = sigmoid(bx) exactly, so the gate
     grouping L cannot matter.  Kernels that split the sequence into the same compute chunks
