@@ -5,7 +5,7 @@ bf16 q/k/v/o, fp32 gates) -- one step = carve_fwd (saving what the backward need
 against a seeded upstream gradient.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl carve|reference]
-                  [--workload train|fwd|long|decode] [--no-e2e] [--no-cpu-baseline]
+                  [--workload train|fwd|decode] [--no-e2e] [--no-cpu-baseline]
 
 Timing: CUDA events on the launch stream, W untimed warm-up steps, then K timed steps
 bracketed by a barrier and a device synchronize, max over ranks.  The working set of a step
@@ -149,35 +149,20 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------------------
 def dist_setup():
-    import torch
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return ws, rank, local
+    from chunk_gated_delta_b200 import dist as cdist
+    return cdist.setup("nccl")
 
 
 def barrier_sync(ws):
     import torch
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
+    from chunk_gated_delta_b200 import dist as cdist
+    cdist.barrier(torch.device("cuda", torch.cuda.current_device()))
 
 
 def max_over_ranks(x: float, ws: int) -> float:
-    if ws == 1:
-        return x
     import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from chunk_gated_delta_b200 import dist as cdist
+    return cdist.max_over_ranks(x, torch.device("cuda", torch.cuda.current_device()))
 
 
 def cpu_oracle_sample(w, d, dO, target_s=12.0, max_T=None, fwd_only=False):
@@ -203,32 +188,53 @@ def cpu_oracle_sample(w, d, dO, target_s=12.0, max_T=None, fwd_only=False):
 
 # ---------------------------------------------------------------------------------------
 def run_reference(args, w):
-    """The reference arm: the fp64 oracle on the host cores, bounded sample per step."""
+    """The reference arm: the fp64 oracle on the host cores, one bounded sample per step (batch
+    element 0, every head: 256 tokens for the sequence workloads, batch 0-15 for decode),
+    reported in this workload's metric and unit."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if ws > 1 and rank != 0:
         return
     import oracle
-    Tp = 256
-    d = I.make_inputs(w, T=Tp)
-    dO = I.make_grad_out(w, T=Tp)
-    sub = {k: (v[:1] if v.ndim >= 3 and k not in ("A", "B") else v) for k, v in d.items()}
-    for _ in range(args.warmup):
-        oracle.fwd(sub, L=w.L)
-        oracle.bwd(sub, w.L, dO[:1])
+    decode = args.workload == "decode"
+    fwd_only = args.workload == "fwd"
+    if decode:
+        Bs, P = 16, 64
+        pool = I.make_decode_pool(w, pool=P)
+        S64 = I.make_state(w, 0.05)[:Bs].astype(np.float64)
+        keys = ("q", "k", "v", "g_logit", "bx", "w_logit")
+
+        def one(j):
+            oracle.step({k: pool[k][j % P][:Bs] for k in keys}, pool["A"], pool["B"], S64, L=1, mc_mode=w.mc_mode)
+    else:
+        Tp = 256
+        d = I.make_inputs(w, T=Tp)
+        dO = I.make_grad_out(w, T=Tp)
+        sub = {k: (v[:1] if v.ndim >= 3 and k not in ("A", "B") else v) for k, v in d.items()}
+
+        def one(j):
+            oracle.fwd(sub, L=w.L, mc_mode=w.mc_mode)
+            if not fwd_only:
+                oracle.bwd(sub, w.L, dO[:1], mc_mode=w.mc_mode)
+    for j in range(args.warmup):
+        one(j)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.fwd(sub, L=w.L)
-        oracle.bwd(sub, w.L, dO[:1])
+    for j in range(args.steps):
+        one(j)
     dt = (time.perf_counter() - t0) / args.steps
-    v = Tp / dt
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+    if decode:
+        v, unit, metric = Bs / w.B / dt, "steps/s", "decode steps/s (B200, B=256, 16 heads, d=128)"
+        sample = f"oracle decode step on batch 0-{Bs - 1} of {w.B} (all {w.H} heads), scaled to {w.B}"
+    else:
+        v, unit = Tp / dt, "tokens/s"
+        metric = "fwd tokens/s per layer (B200, 16 heads, d=128)" if fwd_only else METRIC
+        sample = f"oracle {'fwd' if fwd_only else 'fwd+bwd'} on batch 0 (all {w.H} heads), {Tp} tokens per step"
+    line = {"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "sample": f"batch 0, all {w.H} heads, first {Tp} tokens per step"},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-                             "sample": f"oracle fwd+bwd on batch 0 (all {w.H} heads), {Tp} tokens per step"},
-            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "config": {"workload": w.name, "sample": sample},
+            "cpu_baseline": {"value": v, "unit": unit, "cores": oracle.threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -255,9 +261,12 @@ def run_train(args, w, fwd_only=False):
     fwd_out = carve.carve_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
                               dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only)
     bwd_out = None
-    if not fwd_only:
+    if not fwd_only:   # dA and dB as views of one flat buffer: the step's only collective
+        from chunk_gated_delta_b200 import dist as cdist
+        dAB, dA_, dB_ = cdist.grad_buffer(w.H, w.K, w.V, w.R, dev)
         bwd_out = carve.carve_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
-                                  dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode)
+                                  dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode,
+                                  out={"dA": dA_, "dB": dB_})
     workspace = torch.empty(carve.bwd_workspace_bytes(carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode)),
                             dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -278,9 +287,7 @@ def run_train(args, w, fwd_only=False):
         if ev is not None:
             ev[2].record(stream)
         if ws > 1:
-            import torch.distributed as dist
-            dist.all_reduce(bwd_out["dA"])
-            dist.all_reduce(bwd_out["dB"])
+            cdist.allreduce_(dAB)
 
     for _ in range(args.warmup):
         step(dv_)
@@ -340,6 +347,112 @@ def run_train(args, w, fwd_only=False):
         dist.destroy_process_group()
 
 
+# Decode: per (b,h) and step, the fp32 state read and written (8 d^2 = 131,072 B at d = 128),
+# q, k, v (768 B), g_logit and bx (1,024 B), w_logit (4 B) and o (256 B).
+def step_bytes(d):
+    return 8 * d * d + 3 * 2 * d + 2 * 4 * d + 4 + 2 * d
+
+
+def run_decode(args, w):
+    """One bench step = one carve_step (one token for every (b,h)) of the decode workload,
+    reading token set j % 64 of a seeded pool held on the device; the state stays resident."""
+    import torch
+    import chunk_gated_delta_b200 as carve
+    ws, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    seed = w.seed + 7919 * rank
+    P = 64
+    pool = I.make_decode_pool(w, pool=P, seed=seed)
+    S_host = I.make_state(w, 0.05, seed=seed)
+    host = {}
+    for k, v in pool.items():
+        t = torch.from_numpy(v)
+        host[k] = (t.to(torch.bfloat16) if k in ("q", "k", "v") else t).pin_memory()
+    dp = {k: v.to(dev) for k, v in host.items()}
+    S = torch.from_numpy(S_host).to(dev)
+    o = torch.empty((w.B, w.H, w.V), dtype=torch.bfloat16, device=dev)
+    keys = ("q", "k", "v", "g_logit", "bx", "w_logit")
+    stream = torch.cuda.current_stream()
+
+    def step(x):
+        carve.carve_step(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], dp["A"], dp["B"], S,
+                         mc_mode=w.mc_mode, chunk=1, o=o)
+
+    for j in range(args.warmup):
+        step({k: dp[k][j % P] for k in keys})
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier_sync(ws)
+        start.record(stream)
+        for j in range(args.steps):
+            step({k: dp[k][j % P] for k in keys})
+        end.record(stream)
+        barrier_sync(ws)
+    ms = max_over_ranks(start.elapsed_time(end), ws) / args.steps
+    value = ws / (ms * 1e-3)            # steps/s of the whole job (each rank: its own batch shard)
+    units = w.B * w.H
+    achieved = step_bytes(w.K) * units / (ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:   # the step's token set from pinned host memory, o back to the host
+        stage = {k: torch.empty_like(dp[k][0]) for k in keys}
+        o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h2d = sum(host[k][0].numel() * host[k][0].element_size() for k in keys)
+        d2h = o.numel() * o.element_size()
+
+        def e2e_step(j):
+            for k in keys:
+                stage[k].copy_(host[k][j % P], non_blocking=True)
+            step(stage)
+            o_host.copy_(o, non_blocking=True)
+
+        for j in range(2):
+            e2e_step(j)
+        n = max(1, args.steps)
+        barrier_sync(ws)
+        start.record(stream)
+        for j in range(n):
+            e2e_step(j)
+        end.record(stream)
+        barrier_sync(ws)
+        ems = max_over_ranks(start.elapsed_time(end), ws) / n
+        e2e = {"value": ws / (ems * 1e-3), "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": n}
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and ws == 1:
+        import oracle
+        Bs = 16
+        S64 = S_host[:Bs].astype(np.float64)
+        A64, B64 = pool["A"], pool["B"]
+        t0, n = time.perf_counter(), 0
+        while time.perf_counter() - t0 < 6.0:
+            tok = {k: pool[k][n % P][:Bs] for k in keys}
+            oracle.step(tok, A64, B64, S64, L=1, mc_mode=w.mc_mode)
+            n += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": n / dt * Bs / w.B, "unit": "steps/s", "cores": oracle.threads(), "kind": "oracle",
+               "sample": f"oracle decode, {n} steps on batch 0-{Bs - 1} of {w.B} (all {w.H} heads), scaled to {w.B}"}
+    line = {
+        "metric": "decode steps/s (B200, B=256, 16 heads, d=128)", "value": value, "unit": "steps/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B * ws, "heads": w.H, "d": w.K, "rank": w.R,
+                   "mc_mode": w.mc_mode, "parallelism": f"dp{ws}", "tokens_per_s": value * w.B,
+                   "l2": "no flush: 256 MB state and 470 MB token pool >> 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": "carve_step", "achieved": achieved, "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm"], "traffic": load_traffic("carve_step"),
+                     "peak_source": peaks["source"]},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def load_traffic(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if it is current."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -385,18 +498,21 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="carve", choices=["carve", "reference"])
-    ap.add_argument("--workload", default="train", choices=["train", "fwd"])
+    ap.add_argument("--workload", default="train", choices=["train", "fwd", "decode"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
+    ap.add_argument("--seq-len", type=int, default=None, help="override T (smaller cases for profiling)")
     args = ap.parse_args()
-    w = I.TRAIN_1P3B
+    w = {"fwd": I.FWD_1P3B, "decode": I.DECODE}.get(args.workload, I.TRAIN_1P3B)
     if args.batch:
-        w = dataclasses.replace(w, B=args.batch, name=w.name.replace("_B8_", f"_B{args.batch}_"))
-    if args.workload == "fwd":
-        w = I.FWD_1P3B
+        w = dataclasses.replace(w, B=args.batch, name=w.name.replace(f"_B{w.B}_", f"_B{args.batch}_"))
+    if args.seq_len:
+        w = dataclasses.replace(w, T=args.seq_len, name=w.name.replace(f"_T{w.T}_", f"_T{args.seq_len}_"))
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.workload == "decode":
+        run_decode(args, w)
     else:
         run_train(args, w, fwd_only=args.workload == "fwd")
 

@@ -31,6 +31,9 @@ namespace carve {
 constexpr int kBC = 32;     // compute chunk of the backward
 constexpr int kBNB = 2;     // 16-token blocks per compute chunk
 constexpr int kLdT = 40;    // bf16 row stride of 32-wide tiles
+constexpr int kTcMaxRankBwd = 32;   // rank limit of the tensor-core path
+constexpr int kLdF = 136;   // fp32 row stride of the per-(token, channel) tables: the fragment
+                            // lane pattern (row g, column pair c4) reads float2 without conflicts
 
 struct BwdMaps {
     CUtensorMap q, k, v, dO;
@@ -45,7 +48,7 @@ struct __align__(16) TcBwdSmem {
     __nv_bfloat16 aqk[kBC * kLdT], akk[kBC * kLdT], mkk[kBC * kLdT], daqk[kBC * kLdT], dakk[kBC * kLdT];
     __nv_bfloat16 tii[kBNB * 16 * 24];
     float akk_d[kBC * 17];
-    float rfac[kBC * 129], dlam[kBC * 129];
+    float rfac[kBC * kLdF], dlam[kBC * kLdF];
     float p7[kBNB * 128], r15[kBNB * 128], dblk[kBNB * 128], em[kBNB * 128], fm[kBNB * 128], cij[128];
     float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], btot[kBNB * 128], pdd[kBNB * 128];
     float bpart[kBNB * 128];
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 sm.qm[row * kLdOp + kch] = __float2bfloat16_rn(qv * rf[t]);
                 sm.krm[row * kLdOp + kch] = __float2bfloat16_rn(kv * rf[t]);
                 sm.kcm[row * kLdOp + kch] = __float2bfloat16_rn(kv * cf[t]);
-                sm.rfac[row * 129 + kch] = rf[t];
+                sm.rfac[row * kLdF + kch] = rf[t];
             }
         }
         if (tid < C) sm.wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + t0 + tid) * H + h]);
@@ -660,20 +663,25 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 for (int hh = 0; hh < 2; ++hh) {
                     const int t = 16 * ib2 + g + 8 * hh;
                     const int ch = ch0 + 8 * nt + 2 * c4;
-                    float dqv[2], dkv[2];
+                    float dqv[2], dkv[2], dlv[2];
+                    const float2 r2 = *reinterpret_cast<const float2 *>(sm.rfac + t * kLdF + ch);
+                    const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.qm + t * kLdOp + ch);
+                    const __nv_bfloat162 kr2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.krm + t * kLdOp + ch);
+                    const __nv_bfloat162 kc2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.kcm + t * kLdOp + ch);
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
-                        const int e = 2 * hh + e2, c = ch + e2;
-                        const float r = sm.rfac[t * 129 + c];
+                        const int e = 2 * hh + e2;
+                        const float r = e2 ? r2.y : r2.x;
                         const float ri = __fdividef(1.f, r);
                         const float Gq = gq[nt][e], Gkr = gkr[nt][e], Gkc = gkc[nt][e] + gkb[nt][e];
-                        const float qmv = bf(sm.qm[t * kLdOp + c]), krv = bf(sm.krm[t * kLdOp + c]);
-                        const float kcv = bf(sm.kcm[t * kLdOp + c]);
+                        const float qmv = bf(e2 ? q2.y : q2.x), krv = bf(e2 ? kr2.y : kr2.x);
+                        const float kcv = bf(e2 ? kc2.y : kc2.x);
                         dqv[e2] = r * Gq;
                         dkv[e2] = r * Gkr + ri * Gkc;
-                        sm.dlam[t * 129 + c] = qmv * Gq + krv * Gkr - kcv * Gkc;
+                        dlv[e2] = qmv * Gq + krv * Gkr - kcv * Gkc;
                         bsum[nt][e2] += kcv * gkb[nt][e];     // Kbar_t dKbar_t
                     }
+                    *reinterpret_cast<float2 *>(sm.dlam + t * kLdF + ch) = make_float2(dlv[0], dlv[1]);
                     const size_t gi = base_bh + (size_t)(t0 + t) * tstride + ch;
                     *reinterpret_cast<uint32_t *>(dq + gi) = pack_bf16(dqv[0], dqv[1]);
                     *reinterpret_cast<uint32_t *>(dk + gi) = pack_bf16(dkv[0], dkv[1]);
@@ -693,7 +701,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         {
             float tot = 0.f;
 #pragma unroll
-            for (int t = 0; t < 16; ++t) tot += sm.dlam[(16 * ib + t) * 129 + kch];
+            for (int t = 0; t < 16; ++t) tot += sm.dlam[(16 * ib + t) * kLdF + kch];
             float xl = sm.gam[kch] * sm.s0ds[kch];
 #pragma unroll
             for (int i2 = 0; i2 < NB; ++i2) xl += sm.bpart[i2 * 128 + kch];
@@ -725,15 +733,15 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             float pdd = 0.f;
 #pragma unroll
             for (int t = 15; t >= 0; --t) {
-                run += sm.dlam[(16 * ib + t) * 129 + kch];
+                run += sm.dlam[(16 * ib + t) * kLdF + kch];
                 if (ib == NB - 1 && t == 15) run += xl;
                 const float e1 = __expf(glr[t]), e2 = __expf(-(bxr[t] + dl));
                 const float D = (1.f + e1) * (1.f + e2);
                 const bool floor = !(__fdividef(1.f, D) >= kAMin);
                 const float dglv = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run;
                 const float dbv = floor ? 0.f : __fdividef(e2, 1.f + e2) * run;
-                sm.dlam[(16 * ib + t) * 129 + kch] = dglv;   // staged: this thread's own column
-                sm.rfac[(16 * ib + t) * 129 + kch] = dbv;
+                sm.dlam[(16 * ib + t) * kLdF + kch] = dglv;   // staged: this thread's own column
+                sm.rfac[(16 * ib + t) * kLdF + kch] = dbv;
                 pdd += dbv;
             }
             sm.pdd[ib * 128 + kch] = pdd;
@@ -742,7 +750,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         if (tid < 128) sm.ddelta[tid] += sm.pdd[tid] + sm.pdd[128 + tid];
         for (int idx = tid; idx < C * 32; idx += 256) {   // d g_logit, dbx: four channels per store
             const int t = idx >> 5, c = (idx & 31) * 4;
-            const float *gsrc = sm.dlam + t * 129 + c, *bsrc = sm.rfac + t * 129 + c;
+            const float *gsrc = sm.dlam + t * kLdF + c, *bsrc = sm.rfac + t * kLdF + c;
             const size_t gi = base_bh + (size_t)(t0 + t) * tstride + c;
             *reinterpret_cast<float4 *>(a.dg_logit + gi) = make_float4(gsrc[0], gsrc[1], gsrc[2], gsrc[3]);
             *reinterpret_cast<float4 *>(a.dbx + gi) = make_float4(bsrc[0], bsrc[1], bsrc[2], bsrc[3]);
@@ -826,24 +834,60 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 
 
 // dA[h] = sum_{b, gate chunk} dDelta z^T,  dB[h] = sum dz m^T  (z, m from the saved records),
-// summed in a fixed order
-__global__ void reduce_dAdB_tc_kernel(const float *wsg, const float *aux, float *dA, float *dB, int B, int H, int NG,
-                                      int R) {
-    const int h = blockIdx.y, x = blockIdx.x * blockDim.x + threadIdx.x;
-    if (x >= 256 * R) return;
-    const bool isA = x < 128 * R;
-    const int y = isA ? x : x - 128 * R;
-    const int r0 = isA ? y / R : y / 128, r1 = isA ? y % R : y % 128;
-    float acc = 0.f;
-    for (int b = 0; b < B; ++b) {
-        const size_t u = (size_t)b * H + h;
-        for (int gc = 0; gc < NG; ++gc) {
-            const float *g = wsg + (u * NG + gc) * 160, *rec = aux + (u * NG + gc) * (384 + R);
-            acc += isA ? g[r0] * rec[128 + r1] : g[128 + r0] * rec[r1];
+// summed in a fixed order.  Grid (H, slices of kRedOut outputs); the records of the head are
+// staged kRedRec at a time in shared memory with every load of a stage issued together.
+constexpr int kRedRec = 32, kRedOut = 1024;
+__global__ void __launch_bounds__(256) reduce_dAdB_tc_kernel(const float *wsg, const float *aux, float *dA, float *dB,
+                                                             int B, int H, int NG, int R) {
+    __shared__ __align__(16) float gd[kRedRec][128], rm[kRedRec][128], gz[kRedRec][kTcMaxRankBwd],
+        rz[kRedRec][kTcMaxRankBwd];
+    const int h = blockIdx.x, tid = threadIdx.x, NR = B * NG;
+    int oidx[4];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) oidx[x] = blockIdx.y * kRedOut + x * 256 + tid;
+    for (int i0 = 0; i0 < NR; i0 += kRedRec) {
+        const int nr = min(kRedRec, NR - i0);
+        for (int idx = tid; idx < nr * 64; idx += 256) {   // dDelta and m, four floats per load
+            const int i = idx >> 6, part = idx & 63, rec = i0 + i;
+            const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
+            if (part < 32) {
+                *reinterpret_cast<float4 *>(&gd[i][4 * part]) =
+                    *reinterpret_cast<const float4 *>(wsg + (u * NG + gc) * 160 + 4 * part);
+            } else {
+                const float *r = aux + (u * NG + gc) * (384 + R) + 4 * (part - 32);
+                rm[i][4 * (part - 32)] = r[0];
+                rm[i][4 * (part - 32) + 1] = r[1];
+                rm[i][4 * (part - 32) + 2] = r[2];
+                rm[i][4 * (part - 32) + 3] = r[3];
+            }
         }
+        for (int idx = tid; idx < nr * R; idx += 256) {   // dz and z
+            const int i = idx / R, j = idx % R, rec = i0 + i;
+            const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
+            gz[i][j] = wsg[(u * NG + gc) * 160 + 128 + j];
+            rz[i][j] = aux[(u * NG + gc) * (384 + R) + 128 + j];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int o = oidx[x];
+            if (o < 128 * R) {
+                const int k = o / R, j = o % R;
+                for (int i = 0; i < nr; ++i) acc[x] += gd[i][k] * rz[i][j];
+            } else if (o < 256 * R) {
+                const int j = (o - 128 * R) / 128, v = (o - 128 * R) % 128;
+                for (int i = 0; i < nr; ++i) acc[x] += gz[i][j] * rm[i][v];
+            }
+        }
+        __syncthreads();
     }
-    if (isA) dA[(size_t)h * 128 * R + y] = acc;
-    else dB[(size_t)h * R * 128 + y] = acc;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        const int o = oidx[x];
+        if (o < 128 * R) dA[(size_t)h * 128 * R + o] = acc[x];
+        else if (o < 256 * R) dB[(size_t)h * R * 128 + (o - 128 * R)] = acc[x];
+    }
 }
 
 // dq_t += vec[unit][gate chunk of t] (the content-readout term of the default readout), 8
@@ -888,7 +932,7 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int NG = (a.T + a.L - 1) / a.L;
-    dim3 grid((256 * a.R + 255) / 256, a.H);
+    dim3 grid(a.H, (256 * a.R + kRedOut - 1) / kRedOut);
     reduce_dAdB_tc_kernel<<<grid, 256, 0, st>>>(a.ws, a.saved_aux, dA, dB, a.B, a.H, NG, a.R);
     return cudaGetLastError();
 }

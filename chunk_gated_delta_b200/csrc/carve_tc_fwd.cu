@@ -490,20 +490,42 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     if (a.m_prev_out && tid < 128) a.m_prev_out[(size_t)u * 128 + tid] = sm.mprev[tid];
 }
 
-// Per (unit, gate chunk): mean of q over the gate chunk's tokens, into the saved aux record
-// (offset 256 + R of each 384 + R floats).  One CTA per record, one thread per channel.
-__global__ void __launch_bounds__(128) qbar_kernel(const __nv_bfloat16 *q, float *aux, int H, int T, int L, int R) {
-    const int rec = blockIdx.x, NG = (T + L - 1) / L;
-    const int u = rec / NG, gc = rec % NG, b = u / H, h = u % H, tid = threadIdx.x;
+// Per (batch, gate chunk): mean of q over the gate chunk's tokens for every head, into the saved
+// aux records (offset 256 + R of each 384 + R floats).  A token's H*128 channels are one
+// contiguous row; each thread owns 8 consecutive channels (one 16-byte load per token).
+__global__ void __launch_bounds__(256) qbar_kernel(const __nv_bfloat16 *q, float *aux, int H, int T, int L, int R) {
+    const int NG = (T + L - 1) / L, b = blockIdx.x / NG, gc = blockIdx.x % NG;
     const int n = min(L, T - gc * L);
-    const __nv_bfloat16 *src = q + ((size_t)b * T + (size_t)gc * L) * H * 128 + (size_t)h * 128 + tid;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int t = 0;
-    for (; t + 4 <= n; t += 4)
+    const size_t row = (size_t)H * 128;
+    const __nv_bfloat16 *src = q + ((size_t)b * T + (size_t)gc * L) * row;
+    for (int c8 = threadIdx.x; c8 < H * 16; c8 += blockDim.x) {
+        float acc[2][8] = {};
+        int t = 0;
+        for (; t + 2 <= n; t += 2)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) acc[x] += bf(src[(size_t)(t + x) * H * 128]);
-    for (; t < n; ++t) acc[0] += bf(src[(size_t)t * H * 128]);
-    aux[(size_t)rec * (384 + R) + 256 + R + tid] = (acc[0] + acc[1] + acc[2] + acc[3]) / (float)n;
+            for (int x = 0; x < 2; ++x) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)(t + x) * row + c8 * 8);
+                const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc[x][2 * e] += bf(p[e].x);
+                    acc[x][2 * e + 1] += bf(p[e].y);
+                }
+            }
+        for (; t < n; ++t) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)t * row + c8 * 8);
+            const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[0][2 * e] += bf(p[e].x);
+                acc[0][2 * e + 1] += bf(p[e].y);
+            }
+        }
+        const int h = c8 / 16, ch = (c8 % 16) * 8;
+        float *dst = aux + (((size_t)b * H + h) * NG + gc) * (384 + R) + 256 + R + ch;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst[e] = (acc[0][e] + acc[1][e]) / (float)n;
+    }
 }
 
 template <int NB>
@@ -524,8 +546,8 @@ cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
     }
     if (a.saved_aux && a.mc_mode == 0) {
         const int NG = (a.T + a.L - 1) / a.L;
-        qbar_kernel<<<a.B * a.H * NG, 128, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.q), a.saved_aux, a.H, a.T,
-                                                    a.L, a.R);
+        qbar_kernel<<<a.B * NG, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.q), a.saved_aux, a.H, a.T, a.L,
+                                              a.R);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     kern<<<a.B * a.H, 256, bytes, st>>>(a, maps);
