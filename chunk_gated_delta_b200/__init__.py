@@ -57,7 +57,9 @@ def load():
     lib.carve_fwd.argtypes = [D] + [P] * 15
     lib.carve_bwd.argtypes = [D] + [P] * 25
     lib.carve_step.argtypes = [D] + [P] * 13
-    for f in (lib.carve_fwd, lib.carve_bwd, lib.carve_step):
+    lib.carve_check.argtypes = [P]
+    lib.carve_selftest_timeout.argtypes = [ctypes.c_uint32, P]
+    for f in (lib.carve_fwd, lib.carve_bwd, lib.carve_step, lib.carve_check, lib.carve_selftest_timeout):
         f.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -110,6 +112,12 @@ def bwd_workspace_bytes(d: Dims) -> int:
 def _check(fn, rc):
     if rc != 0:
         raise CarveError(fn, rc)
+
+
+def carve_check(stream=None) -> int:
+    """Wait for `stream` and return the library's status: 0 (CARVE_OK), or the code of a CUDA
+    error or of a bounded device-side wait that gave up since the last check."""
+    return int(load().carve_check(_stream(stream)))
 
 
 def carve_fwd(q, k, v, g_logit, bx, w_logit, A, B, chunk: int, mc_mode: int = 0, S0=None, m_prev_in=None,

@@ -10,6 +10,10 @@ cudaError_t launch_fwd_simt(int K, int V, bool bf16, const FwdArgs &a, cudaStrea
 cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st);
 cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 int tc_compute_chunk(int L);
+int tc_fwd_take_timeout();
+int tc_bwd_take_timeout();
+int step_take_timeout();
+cudaError_t launch_selftest_timeout(uint32_t iterations, cudaStream_t st);
 cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit, const float *A,
@@ -179,6 +183,19 @@ carve_status carve_step(const carve_dims *d, const void *q, const void *k, const
                                        mstate, pos, o, d->B, d->H, d->rank, d->chunk, d->mc_mode,
                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_check(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CARVE_ERR_CUDA;
+    const int t = carve::tc_fwd_take_timeout() | carve::tc_bwd_take_timeout() | carve::step_take_timeout();
+    return t ? CARVE_ERR_TIMEOUT : CARVE_OK;
+}
+
+carve_status carve_selftest_timeout(uint32_t iterations, void *stream) {
+    if (iterations < 1 || iterations > 1000000) return CARVE_ERR_INVALID_ARG;
+    return carve::launch_selftest_timeout(iterations, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CARVE_OK
+               : CARVE_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,16 +1,23 @@
-// CARVE single-token decode step: one CTA per (batch, head), state read once and written
-// once (CARVE blog, Table 1: inference costs O(dv dk) per token).
+// CARVE single-token decode step (CARVE blog, Table 1: inference costs O(dv dk) per token).
 //
-// With P = S Diag(a) the token's update and output expand to three matrix-vector products
-// over the same state rows, so the state is loaded into registers once:
+// With P = S Diag(a) the token's update and output expand to matrix-vector products over the
+// same state rows, so each (batch, head) state is read once and written once:
 //   m  = S q                     (mc_mode 0: content signal from the state before the token)
 //   a  = exp(-softplus(g_logit)) * sigmoid(bx + A (Bm m)),  w = sigmoid(w_logit)
 //   p  = S (a*k),  e = v - p
 //   o  = S (a*q) + w e (k.q)     (= S' q)
 //   S' = S Diag(a) + w e k^T
-// Each row of S is held by TPR threads as float4 groups interleaved so that a warp's loads
-// and stores cover contiguous 16-byte segments.
+//
+// The step moves 8 dv dk bytes of state per (b,h) and little else, so the kernel is built
+// around the copy engine: one persistent CTA per SM walks its share of the (b,h) units with
+// three shared-memory stages.  A unit's whole state arrives by one bulk copy issued two units
+// ahead and leaves by one bulk store from the same stage, so loads, stores and the arithmetic
+// of three units overlap.  The unit's token vectors and its head's slices of the low-rank
+// factors are prefetched into registers one unit ahead.  Each state row is read by TPR
+// threads as float4 groups in a row-rotated order (conflict-free shared-memory banks) and
+// kept in registers between the content-signal pass and the update pass.
 #include "carve_device.cuh"
+#include "carve_mma.cuh"
 
 namespace carve {
 
@@ -23,114 +30,288 @@ struct StepArgs {
     int B, H, R, L, mc_mode;
 };
 
-template <int K, int V, typename IO>
-__global__ void __launch_bounds__(kThreads) step_kernel(StepArgs a) {
-    constexpr int TPR = kThreads / V;        // threads per state row
-    constexpr int G4 = K / 4 / TPR;          // float4 groups per thread
-    __shared__ float qv[K], kv[K], av[K], mv[V], zv[64], red[kThreads / 32];
-    __shared__ float s_w, s_kq;
-    const int tid = threadIdx.x, u = blockIdx.x, h = u % a.H;
-    const int row = tid / TPR, seg = tid % TPR;
-    const IO *q = static_cast<const IO *>(a.q) + (size_t)u * K;
-    const IO *k = static_cast<const IO *>(a.k) + (size_t)u * K;
-    const IO *vv = static_cast<const IO *>(a.v) + (size_t)u * V;
-    float4 *Srow = reinterpret_cast<float4 *>(a.S + ((size_t)u * V + row) * K);
+constexpr int kStepThreads = 256;
+constexpr int kStepStages = 3;
+constexpr int kStepMaxRank = 64;
 
-    float4 s[G4];
-#pragma unroll
-    for (int j = 0; j < G4; ++j) s[j] = Srow[seg + TPR * j];
-    if (tid < K) {
-        qv[tid] = ld_io(q + tid);
-        kv[tid] = ld_io(k + tid);
+__device__ int g_step_timeout;  // set when a bounded wait gives up (never expected)
+
+template <int K, int V>
+struct __align__(16) StepSmem {
+    float S[kStepStages][V * K];
+    float qv[K], kv[K], glv[K], bxv[K], av[K], akv[K], aqv[K];
+    float vv[V], mv[V], msum[V], zv[kStepMaxRank];
+    float w, kq;
+    uint64_t bar[kStepStages];
+};
+
+template <int K, int V, typename IO>
+__global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n_units) {
+    constexpr int TPR = kStepThreads / V;     // threads per state row
+    constexpr int G4 = K / 4 / TPR;           // float4 groups per thread
+    constexpr int TPK = kStepThreads / K;     // threads per Delta output
+    constexpr int VP = V / 8;                 // entries of a z dot product per thread (8 per output)
+    constexpr int AP = kStepMaxRank / TPK;    // entries of a Delta dot product per thread
+    constexpr uint32_t kBytes = V * K * 4;
+    extern __shared__ __align__(128) unsigned char smraw[];
+    StepSmem<K, V> &sm = *reinterpret_cast<StepSmem<K, V> *>(smraw);
+    const int tid = threadIdx.x, row = tid / TPR, seg = tid % TPR, H = a.H, R = a.R;
+    const int first = blockIdx.x, stride = gridDim.x;
+    const int nmine = first < n_units ? (n_units - 1 - first) / stride + 1 : 0;
+
+    if (tid == 0) {
+        for (int st = 0; st < kStepStages; ++st) mbar_init(&sm.bar[st], 1);
+        fence_mbar_init();
     }
     __syncthreads();
-    // content signal
-    if (a.mc_mode == 0) {
-        float part = 0.f;
-#pragma unroll
-        for (int j = 0; j < G4; ++j) {
-            const int c = 4 * (seg + TPR * j);
-            part += s[j].x * qv[c] + s[j].y * qv[c + 1] + s[j].z * qv[c + 2] + s[j].w * qv[c + 3];
+    auto issue = [&](int i) {   // the state of this CTA's i-th unit into stage i % 3
+        if (tid == 0 && i < nmine) {
+            const int u = first + i * stride, st = i % kStepStages;
+            mbar_expect_tx(&sm.bar[st], kBytes);
+            bulk_g2s(sm.S[st], a.S + (size_t)u * V * K, kBytes, &sm.bar[st]);
         }
-#pragma unroll
-        for (int off = TPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        if (seg == 0) mv[row] = part;
-    } else if (tid < V) {
-        float *msum = a.mstate + (size_t)u * 2 * V, *mprev = msum + V;
-        const int p = a.pos[u];
-        float m = mprev[tid];
-        if (p > 0 && p % a.L == 0) {
-            m = msum[tid] / (float)a.L;
-            mprev[tid] = m;
-            msum[tid] = 0.f;
+    };
+    issue(0);
+    issue(1);
+
+    // token vectors of a unit (channel tid / row tid) and the mean-output carry (mc_mode 1)
+    float pq = 0.f, pk = 0.f, pgl = 0.f, pbx = 0.f, pv = 0.f, pwl = 0.f, pms = 0.f, pmp = 0.f;
+    int ppos = 0;
+    auto prefetch_tokens = [&](int i) {
+        if (i >= nmine) return;
+        const int u = first + i * stride;
+        if (tid < K) {
+            pq = ld_io(static_cast<const IO *>(a.q) + (size_t)u * K + tid);
+            pk = ld_io(static_cast<const IO *>(a.k) + (size_t)u * K + tid);
+            pgl = a.g_logit[(size_t)u * K + tid];
+            pbx = a.bx[(size_t)u * K + tid];
         }
-        mv[tid] = m;
-    }
-    // k.q (warp 0)
-    if (tid < 32) {
-        float x = 0.f;
-        for (int i = tid; i < K; i += 32) x += kv[i] * qv[i];
+        if (tid < V) {
+            pv = ld_io(static_cast<const IO *>(a.v) + (size_t)u * V + tid);
+            if (a.mc_mode == 1) {
+                pms = a.mstate[(size_t)u * 2 * V + tid];
+                pmp = a.mstate[(size_t)u * 2 * V + V + tid];
+                ppos = a.pos[u];
+            }
+        }
+        if (tid == 0) pwl = a.w_logit[u];
+    };
+    // the head's slices of Bm (for z, 8 threads per output) and A (for Delta, TPK per output)
+    float pB[2][VP], pA[AP];
+    auto prefetch_factors = [&](int i) {
+        if (i >= nmine) return;
+        const int h = (first + i * stride) % H;
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        for (int zp = 0; zp < 2; ++zp) {
+            const int j = 32 * zp + tid / 8, part = tid % 8;
+#pragma unroll
+            for (int x = 0; x < VP; ++x) pB[zp][x] = j < R ? a.Bm[((size_t)h * R + j) * V + part + 8 * x] : 0.f;
+        }
+        const int kk = tid / TPK, part = tid % TPK;
+#pragma unroll
+        for (int x = 0; x < AP; ++x) {
+            const int r = part + TPK * x;
+            pA[x] = r < R ? a.A[((size_t)h * K + kk) * R + r] : 0.f;
+        }
+    };
+    prefetch_tokens(0);
+    prefetch_factors(0);
+
+    bool failed = false;
+    int i = 0;
+    for (; i < nmine; ++i) {
+        const int u = first + i * stride, st = i % kStepStages;
+        float *Sst = sm.S[st];
+        // ---- token vectors into shared memory, next unit's into registers
+        if (tid < K) {
+            sm.qv[tid] = pq;
+            sm.kv[tid] = pk;
+            sm.glv[tid] = pgl;
+            sm.bxv[tid] = pbx;
+        }
+        if (tid < V) {
+            sm.vv[tid] = pv;
+            if (a.mc_mode == 1) {   // running block mean of o: close the block every L tokens
+                float m = pmp, msum = pms;
+                if (ppos > 0 && ppos % a.L == 0) {
+                    m = msum / (float)a.L;
+                    a.mstate[(size_t)u * 2 * V + V + tid] = m;
+                    msum = 0.f;
+                }
+                sm.mv[tid] = m;
+                sm.msum[tid] = msum;
+            }
+        }
         if (tid == 0) {
-            s_kq = x;
-            s_w = sigmoid_f(a.w_logit[u]);
+            sm.w = sigmoid_f(pwl);
+            if (a.mc_mode == 1) a.pos[u] = ppos + 1;
+        }
+        prefetch_tokens(i + 1);
+        __syncthreads();
+        // ---- state rows into registers; content signal m = S q (mc_mode 0); k.q
+        const bool ok = mbar_wait(&sm.bar[st], (uint32_t)(i / kStepStages) & 1u);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        float4 s[G4];
+        {
+            float part = 0.f;
+#pragma unroll
+            for (int j = 0; j < G4; ++j) {
+                const int f = seg + TPR * ((j + row) % G4);
+                s[j] = reinterpret_cast<const float4 *>(Sst)[row * (K / 4) + f];
+                const float4 qq = reinterpret_cast<const float4 *>(sm.qv)[f];
+                part += s[j].x * qq.x + s[j].y * qq.y + s[j].z * qq.z + s[j].w * qq.w;
+            }
+            if (a.mc_mode == 0) {
+#pragma unroll
+                for (int off = TPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+                if (seg == 0) sm.mv[row] = part;
+            }
+        }
+        if (tid >= kStepThreads - 32) {   // last warp: k.q
+            float x = 0.f;
+            for (int c = tid - (kStepThreads - 32); c < K; c += 32) x += sm.kv[c] * sm.qv[c];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+            if (tid == kStepThreads - 32) sm.kq = x;
+        }
+        __syncthreads();
+        // ---- z = Bm m
+#pragma unroll
+        for (int zp = 0; zp < 2; ++zp) {
+            if (32 * zp < R) {
+                const int j = 32 * zp + tid / 8, part = tid % 8;
+                float acc = 0.f;
+#pragma unroll
+                for (int x = 0; x < VP; ++x) acc += pB[zp][x] * sm.mv[part + 8 * x];
+                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                if (part == 0 && j < R) sm.zv[j] = acc;
+            }
+        }
+        __syncthreads();
+        // ---- Delta = A z, gates
+        {
+            const int kk = tid / TPK, part = tid % TPK;
+            float acc = 0.f;
+#pragma unroll
+            for (int x = 0; x < AP; ++x)
+                if (part + TPK * x < R) acc += pA[x] * sm.zv[part + TPK * x];
+#pragma unroll
+            for (int off = TPK / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (part == 0) {
+                const float av = expf(log_retention(sm.glv[kk], sm.bxv[kk] + acc));
+                sm.av[kk] = av;
+                sm.akv[kk] = av * sm.kv[kk];
+                sm.aqv[kk] = av * sm.qv[kk];
+            }
+        }
+        prefetch_factors(i + 1);
+        if (tid == 0) {   // the stage of unit i - 1 takes unit i + 2 once its store has read it
+            bulk_wait_read<0>();
+            issue(i + 2);
+        }
+        __syncthreads();
+        // ---- p = S (a*k), S (a*q); update; output
+        {
+            float p = 0.f, s2 = 0.f;
+#pragma unroll
+            for (int j = 0; j < G4; ++j) {
+                const int f = seg + TPR * ((j + row) % G4);
+                const float4 ak = reinterpret_cast<const float4 *>(sm.akv)[f];
+                const float4 aq = reinterpret_cast<const float4 *>(sm.aqv)[f];
+                p += s[j].x * ak.x + s[j].y * ak.y + s[j].z * ak.z + s[j].w * ak.w;
+                s2 += s[j].x * aq.x + s[j].y * aq.y + s[j].z * aq.z + s[j].w * aq.w;
+            }
+#pragma unroll
+            for (int off = TPR / 2; off >= 1; off >>= 1) {
+                p += __shfl_xor_sync(0xffffffffu, p, off);
+                s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+            }
+            const float we = sm.w * (sm.vv[row] - p);
+#pragma unroll
+            for (int j = 0; j < G4; ++j) {
+                const int f = seg + TPR * ((j + row) % G4);
+                const float4 av = reinterpret_cast<const float4 *>(sm.av)[f];
+                const float4 kv = reinterpret_cast<const float4 *>(sm.kv)[f];
+                float4 x = s[j];
+                x.x = x.x * av.x + we * kv.x;
+                x.y = x.y * av.y + we * kv.y;
+                x.z = x.z * av.z + we * kv.z;
+                x.w = x.w * av.w + we * kv.w;
+                reinterpret_cast<float4 *>(Sst)[row * (K / 4) + f] = x;
+            }
+            if (seg == 0) {
+                const float ov = s2 + we * sm.kq;
+                st_io(static_cast<IO *>(a.o) + (size_t)u * V + row, ov);
+                if (a.mc_mode == 1) a.mstate[(size_t)u * 2 * V + row] = sm.msum[row] + ov;
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_s2g(a.S + (size_t)u * V * K, Sst, kBytes);
+            bulk_commit();
         }
     }
-    __syncthreads();
-    if (tid < a.R) {
-        float z = 0.f;
-        const float *Bh = a.Bm + ((size_t)h * a.R + tid) * V;
-        for (int r = 0; r < V; ++r) z += Bh[r] * mv[r];
-        zv[tid] = z;
+    if (failed) {   // drain the loads still in flight into this CTA's stages, bounded
+        if (tid == 0) {
+            atomicOr(&g_step_timeout, 1);
+            for (int j = i; j < min(i + 2, nmine); ++j) mbar_wait(&sm.bar[j % kStepStages], (uint32_t)(j / kStepStages) & 1u);
+        }
     }
-    __syncthreads();
-    if (tid < K) {
-        float d = 0.f;
-        const float *Ah = a.A + ((size_t)h * K + tid) * a.R;
-        for (int j = 0; j < a.R; ++j) d += Ah[j] * zv[j];
-        const size_t g = (size_t)u * K + tid;
-        av[tid] = expf(log_retention(a.g_logit[g], a.bx[g] + d));
+    if (tid == 0) bulk_wait<0>();
+}
+
+// A single thread waits, bounded, on a barrier that nothing arrives on (the expiry path of
+// every bounded wait in this library, exercised on purpose).
+__global__ void selftest_timeout_kernel(uint32_t iterations) {
+    __shared__ uint64_t bar;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0u, iterations)) atomicOr(&g_step_timeout, 2);
+}
+
+cudaError_t launch_selftest_timeout(uint32_t iterations, cudaStream_t st) {
+    selftest_timeout_kernel<<<1, 1, 0, st>>>(iterations);
+    return cudaGetLastError();
+}
+
+// Device status word of this file: returns and clears it.
+int step_take_timeout() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_step_timeout, sizeof(int)) != cudaSuccess) return 0;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_step_timeout, &z, sizeof(int));
     }
-    __syncthreads();
-    float p = 0.f, s2 = 0.f;
-#pragma unroll
-    for (int j = 0; j < G4; ++j) {
-        const int c = 4 * (seg + TPR * j);
-        const float a0 = av[c], a1 = av[c + 1], a2 = av[c + 2], a3 = av[c + 3];
-        p += s[j].x * a0 * kv[c] + s[j].y * a1 * kv[c + 1] + s[j].z * a2 * kv[c + 2] + s[j].w * a3 * kv[c + 3];
-        s2 += s[j].x * a0 * qv[c] + s[j].y * a1 * qv[c + 1] + s[j].z * a2 * qv[c + 2] + s[j].w * a3 * qv[c + 3];
+    return v;
+}
+
+static int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
     }
-#pragma unroll
-    for (int off = TPR / 2; off >= 1; off >>= 1) {
-        p += __shfl_xor_sync(0xffffffffu, p, off);
-        s2 += __shfl_xor_sync(0xffffffffu, s2, off);
-    }
-    const float w = s_w;
-    const float e = ld_io(vv + row) - p;
-    const float we = w * e;
-#pragma unroll
-    for (int j = 0; j < G4; ++j) {
-        const int c = 4 * (seg + TPR * j);
-        float4 x = s[j];
-        x.x = x.x * av[c] + we * kv[c];
-        x.y = x.y * av[c + 1] + we * kv[c + 1];
-        x.z = x.z * av[c + 2] + we * kv[c + 2];
-        x.w = x.w * av[c + 3] + we * kv[c + 3];
-        Srow[seg + TPR * j] = x;
-    }
-    if (seg == 0) {
-        const float ov = s2 + we * s_kq;
-        st_io(static_cast<IO *>(a.o) + (size_t)u * V + row, ov);
-        if (a.mc_mode == 1) a.mstate[(size_t)u * 2 * V + row] += ov;
-    }
-    if (a.mc_mode == 1 && tid == 0) a.pos[u] += 1;
-    (void)red;
+    return cached[dev];
 }
 
 template <int K, int V, typename IO>
 cudaError_t launch_step_t(const StepArgs &a, cudaStream_t st) {
-    step_kernel<K, V, IO><<<a.B * a.H, kThreads, 0, st>>>(a);
+    auto kern = step_kernel<K, V, IO>;
+    const int bytes = (int)sizeof(StepSmem<K, V>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    const int units = a.B * a.H;
+    const int grid = units < sm_count() ? units : sm_count();
+    kern<<<grid, kStepThreads, bytes, st>>>(a, units);
     return cudaGetLastError();
 }
 

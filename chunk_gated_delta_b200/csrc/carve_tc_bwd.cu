@@ -939,4 +939,15 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
 
 size_t tc_bwd_smem() { return sizeof(TcBwdSmem); }
 
+// Device status word of this file: returns and clears it.
+int tc_bwd_take_timeout() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_bwd_timeout, sizeof(int)) != cudaSuccess) return 0;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_tc_bwd_timeout, &z, sizeof(int));
+    }
+    return v;
+}
+
 }  // namespace carve

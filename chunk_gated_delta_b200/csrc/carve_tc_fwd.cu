@@ -567,4 +567,15 @@ cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st) {
 
 size_t tc_fwd_smem(int L) { return tc_compute_chunk(L) == 32 ? sizeof(TcFwdSmem<2>) : sizeof(TcFwdSmem<4>); }
 
+// Device status word of this file: returns and clears it.
+int tc_fwd_take_timeout() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_timeout, sizeof(int)) != cudaSuccess) return 0;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_tc_timeout, &z, sizeof(int));
+    }
+    return v;
+}
+
 }  // namespace carve

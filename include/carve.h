@@ -164,6 +164,26 @@ carve_status carve_step(const carve_dims *d, const void *q, const void *k, const
                         const float *A, const float *Bm, float *S, float *mstate, int32_t *pos,
                         void *o, void *stream);
 
+/*
+ * carve_check -- blocks the host until the work queued on `stream` has finished, then
+ * reports what the device saw: CARVE_ERR_CUDA if the stream reports an error,
+ * CARVE_ERR_TIMEOUT if a bounded device-side wait of a carve kernel (a shared-memory
+ * barrier waiting for a bulk copy) gave up since the previous carve_check, else CARVE_OK.
+ * The device status words are cleared by the call.  A kernel whose wait gives up records
+ * it, stops its sweep, waits (again bounded) for its own copies in flight and returns, so
+ * the CUDA context stays usable; the outputs of that call are undefined.  The pages have
+ * no counterpart to this entry point.
+ */
+carve_status carve_check(void *stream);
+
+/*
+ * carve_selftest_timeout -- test hook for the path above: launches one thread that waits
+ * on a shared-memory barrier nothing arrives on, bounded by `iterations` polls (1 to
+ * 1,000,000), so the wait always gives up and records it; the next carve_check returns
+ * CARVE_ERR_TIMEOUT.  Nothing else is touched.  No counterpart in the pages.
+ */
+carve_status carve_selftest_timeout(uint32_t iterations, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,8 +26,9 @@ def declared_functions():
 
 
 def test_header_declares_the_boundary():
-    assert declared_functions() == ["carve_bwd", "carve_bwd_noalloc", "carve_bwd_workspace_bytes", "carve_fwd",
-                                    "carve_saved_bytes", "carve_status_string", "carve_step"]
+    assert declared_functions() == ["carve_bwd", "carve_bwd_noalloc", "carve_bwd_workspace_bytes", "carve_check",
+                                    "carve_fwd", "carve_saved_bytes", "carve_selftest_timeout",
+                                    "carve_status_string", "carve_step"]
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -101,3 +102,9 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.carve_step(ctypes.byref(ds), *([P] * 9), None, None, P, None) == 1   # needs mstate and pos
     assert lib.carve_step(ctypes.byref(d), *([P] * 8), None, None, None, P, None) == 1  # S missing
     assert lib.carve_fwd(None, *fwd_ok) == 1
+
+
+def test_selftest_timeout_bounds_checked_on_host(lib):
+    """Out-of-range poll counts are rejected before any launch."""
+    assert lib.carve_selftest_timeout(0, None) == 1
+    assert lib.carve_selftest_timeout(1_000_001, None) == 1

@@ -262,3 +262,39 @@ def test_decode_1000_steps(cuda_device, mode):
     check("S after 1000 steps", host(S)[bi, hi], Sr[:, 0], TOL["bf16"])
     if mode == 1:
         assert torch.all(pos == w.steps)
+
+
+@pytest.mark.parametrize("K,V", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("io", ["fp32", "bf16"])
+def test_decode_shapes_all_units(cuda_device, K, V, io):
+    """336 (b,h) units (more than one per SM, so every CTA cycles its state stages), rank 48
+    (two passes of the z product), 40 steps in each mode (mc_mode 1 with 4-token blocks);
+    every unit's outputs and final state against the oracle."""
+    import torch
+    w = dataclasses.replace(I.DECODE, B=3, H=112, K=K, V=V, R=48, io=io, seed=900 + K + V)
+    steps, L = 40, 4
+    pool = I.make_decode_pool(w, pool=steps)
+    for mode in (0, 1):
+        S_np = I.make_state(w, 0.05)
+        tp = to_dev({k: pool[k] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}, io, cuda_device)
+        A = torch.from_numpy(pool["A"]).to(cuda_device)
+        Bm = torch.from_numpy(pool["B"]).to(cuda_device)
+        S = torch.from_numpy(S_np).to(cuda_device)
+        mstate = torch.zeros((w.B, w.H, 2, V), dtype=torch.float32, device=cuda_device)
+        pos = torch.zeros((w.B, w.H), dtype=torch.int32, device=cuda_device)
+        outs = []
+        for j in range(steps):
+            o = carve.carve_step(tp["q"][j], tp["k"][j], tp["v"][j], tp["g_logit"][j], tp["bx"][j], tp["w_logit"][j],
+                                 A, Bm, S, mc_mode=mode, chunk=L, mstate=mstate, pos=pos)
+            outs.append(host(o))
+        assert carve.carve_check() == 0
+        Sr = S_np.astype(np.float64).copy()
+        ms = np.zeros((w.B, w.H, 2, V))
+        ps = np.zeros((w.B, w.H), dtype=np.int32)
+        ref = [oracle.step({k: pool[k][j] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}, pool["A"], pool["B"],
+                           Sr, L=L, mc_mode=mode, mstate=ms, pos=ps) for j in range(steps)]
+        check(f"o mode {mode}", np.stack(outs), np.stack(ref), TOL[io])
+        check(f"S mode {mode}", host(S), Sr, TOL[io])
+        if mode == 1:
+            check("mstate", host(mstate), ms, TOL[io])
+            assert torch.all(pos == steps)
