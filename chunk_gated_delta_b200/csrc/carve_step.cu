@@ -8,14 +8,15 @@
 //   o  = S (a*q) + w e (k.q)     (= S' q)
 //   S' = S Diag(a) + w e k^T
 //
-// The step moves 8 dv dk bytes of state per (b,h) and little else, so the kernel is built
-// around the copy engine: one persistent CTA per SM walks its share of the (b,h) units with
-// three shared-memory stages.  A unit's whole state arrives by one bulk copy issued two units
-// ahead and leaves by one bulk store from the same stage, so loads, stores and the arithmetic
-// of three units overlap.  The unit's token vectors and its head's slices of the low-rank
-// factors are prefetched into registers one unit ahead.  Each state row is read by TPR
-// threads as float4 groups in a row-rotated order (conflict-free shared-memory banks) and
-// kept in registers between the content-signal pass and the update pass.
+// The step moves 8 dv dk bytes of state per (b,h) and little else.  One persistent CTA per
+// SM walks its share of the (b,h) units with NGRP independent groups of 256 threads (each
+// with its own named barrier and its own shared-memory stage), so the dependent chain of one
+// unit (content signal -> z -> Delta -> gates -> update) overlaps the other group's.  A
+// unit's state arrives in the group's stage by one bulk copy; the first pass moves it into
+// registers, after which the stage is refilled with the group's next unit while this one
+// finishes.  The updated state is stored from registers: each row is held by TPR threads as
+// float4 groups in a row-rotated order, which keeps the shared-memory reads conflict-free
+// and every 32-byte sector of the global stores whole.
 #include "carve_device.cuh"
 #include "carve_mma.cuh"
 
@@ -30,110 +31,80 @@ struct StepArgs {
     int B, H, R, L, mc_mode;
 };
 
-constexpr int kStepThreads = 256;
-constexpr int kStepStages = 3;
+constexpr int kGroupThreads = 256;   // threads per unit group
 constexpr int kStepMaxRank = 64;
 
 __device__ int g_step_timeout;  // set when a bounded wait gives up (never expected)
 
 template <int K, int V>
-struct __align__(16) StepSmem {
-    float S[kStepStages][V * K];
+struct __align__(16) StepGroupSmem {
+    float S[V * K];
     float qv[K], kv[K], glv[K], bxv[K], av[K], akv[K], aqv[K];
     float vv[V], mv[V], msum[V], zv[kStepMaxRank];
     float w, kq;
-    uint64_t bar[kStepStages];
+    uint64_t bar;
 };
 
-template <int K, int V, typename IO>
-__global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n_units) {
-    constexpr int TPR = kStepThreads / V;     // threads per state row
-    constexpr int G4 = K / 4 / TPR;           // float4 groups per thread
-    constexpr int TPK = kStepThreads / K;     // threads per Delta output
-    constexpr int VP = V / 8;                 // entries of a z dot product per thread (8 per output)
-    constexpr int AP = kStepMaxRank / TPK;    // entries of a Delta dot product per thread
+// Barrier over the 256 threads of group `id` (named barrier 1 + id).
+__device__ __forceinline__ void group_sync(int id) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(1 + id), "r"(kGroupThreads) : "memory");
+}
+// The same barrier, returning whether any thread of the group passed `v` true.
+__device__ __forceinline__ bool group_sync_or(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(1 + id), "r"(kGroupThreads)
+        : "memory");
+    return r != 0;
+}
+
+// RMAX: rank bound of the factor slices held in registers (32, or 64 with one group).
+template <int K, int V, typename IO, int RMAX, int NGRP>
+__global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a, int n_units) {
+    constexpr int TPR = kGroupThreads / V;     // threads per state row
+    constexpr int G4 = K / 4 / TPR;            // float4 groups per thread
+    constexpr int TPK = kGroupThreads / K;     // threads per Delta output
+    constexpr int VP = V / 8;                  // entries of a z dot product per thread (8 per output)
+    constexpr int ZP = RMAX / 32;              // passes of 32 z outputs
+    constexpr int AP = RMAX / TPK;             // entries of a Delta dot product per thread
     constexpr uint32_t kBytes = V * K * 4;
     extern __shared__ __align__(128) unsigned char smraw[];
-    StepSmem<K, V> &sm = *reinterpret_cast<StepSmem<K, V> *>(smraw);
-    const int tid = threadIdx.x, row = tid / TPR, seg = tid % TPR, H = a.H, R = a.R;
+    const int grp = threadIdx.x / kGroupThreads, tid = threadIdx.x % kGroupThreads;
+    StepGroupSmem<K, V> &sm = reinterpret_cast<StepGroupSmem<K, V> *>(smraw)[grp];
+    const int row = tid / TPR, seg = tid % TPR, H = a.H, R = a.R;
+    // this group's units: first + (NGRP i + grp) stride, i = 0, 1, ...
     const int first = blockIdx.x, stride = gridDim.x;
-    const int nmine = first < n_units ? (n_units - 1 - first) / stride + 1 : 0;
+    const int mine = first < n_units ? (n_units - 1 - first) / stride + 1 : 0;
+    const int nmine = mine > grp ? (mine - 1 - grp) / NGRP + 1 : 0;
+    auto unit_of = [&](int i) { return first + (NGRP * i + grp) * stride; };
 
     if (tid == 0) {
-        for (int st = 0; st < kStepStages; ++st) mbar_init(&sm.bar[st], 1);
+        mbar_init(&sm.bar, 1);
         fence_mbar_init();
+        if (nmine > 0) {
+            mbar_expect_tx(&sm.bar, kBytes);
+            bulk_g2s(sm.S, a.S + (size_t)unit_of(0) * V * K, kBytes, &sm.bar);
+        }
     }
-    __syncthreads();
-    auto issue = [&](int i) {   // the state of this CTA's i-th unit into stage i % 3
-        if (tid == 0 && i < nmine) {
-            const int u = first + i * stride, st = i % kStepStages;
-            mbar_expect_tx(&sm.bar[st], kBytes);
-            bulk_g2s(sm.S[st], a.S + (size_t)u * V * K, kBytes, &sm.bar[st]);
-        }
-    };
-    issue(0);
-    issue(1);
+    group_sync(grp);
 
-    // token vectors of a unit (channel tid / row tid) and the mean-output carry (mc_mode 1)
-    float pq = 0.f, pk = 0.f, pgl = 0.f, pbx = 0.f, pv = 0.f, pwl = 0.f, pms = 0.f, pmp = 0.f;
-    int ppos = 0;
-    auto prefetch_tokens = [&](int i) {
-        if (i >= nmine) return;
-        const int u = first + i * stride;
+    for (int i = 0; i < nmine; ++i) {
+        const int u = unit_of(i), h = u % H;
+        // ---- token vectors into shared memory, the head's factor slices into registers
         if (tid < K) {
-            pq = ld_io(static_cast<const IO *>(a.q) + (size_t)u * K + tid);
-            pk = ld_io(static_cast<const IO *>(a.k) + (size_t)u * K + tid);
-            pgl = a.g_logit[(size_t)u * K + tid];
-            pbx = a.bx[(size_t)u * K + tid];
+            sm.qv[tid] = ld_io(static_cast<const IO *>(a.q) + (size_t)u * K + tid);
+            sm.kv[tid] = ld_io(static_cast<const IO *>(a.k) + (size_t)u * K + tid);
+            sm.glv[tid] = a.g_logit[(size_t)u * K + tid];
+            sm.bxv[tid] = a.bx[(size_t)u * K + tid];
         }
         if (tid < V) {
-            pv = ld_io(static_cast<const IO *>(a.v) + (size_t)u * V + tid);
-            if (a.mc_mode == 1) {
-                pms = a.mstate[(size_t)u * 2 * V + tid];
-                pmp = a.mstate[(size_t)u * 2 * V + V + tid];
-                ppos = a.pos[u];
-            }
-        }
-        if (tid == 0) pwl = a.w_logit[u];
-    };
-    // the head's slices of Bm (for z, 8 threads per output) and A (for Delta, TPK per output)
-    float pB[2][VP], pA[AP];
-    auto prefetch_factors = [&](int i) {
-        if (i >= nmine) return;
-        const int h = (first + i * stride) % H;
-#pragma unroll
-        for (int zp = 0; zp < 2; ++zp) {
-            const int j = 32 * zp + tid / 8, part = tid % 8;
-#pragma unroll
-            for (int x = 0; x < VP; ++x) pB[zp][x] = j < R ? a.Bm[((size_t)h * R + j) * V + part + 8 * x] : 0.f;
-        }
-        const int kk = tid / TPK, part = tid % TPK;
-#pragma unroll
-        for (int x = 0; x < AP; ++x) {
-            const int r = part + TPK * x;
-            pA[x] = r < R ? a.A[((size_t)h * K + kk) * R + r] : 0.f;
-        }
-    };
-    prefetch_tokens(0);
-    prefetch_factors(0);
-
-    bool failed = false;
-    int i = 0;
-    for (; i < nmine; ++i) {
-        const int u = first + i * stride, st = i % kStepStages;
-        float *Sst = sm.S[st];
-        // ---- token vectors into shared memory, next unit's into registers
-        if (tid < K) {
-            sm.qv[tid] = pq;
-            sm.kv[tid] = pk;
-            sm.glv[tid] = pgl;
-            sm.bxv[tid] = pbx;
-        }
-        if (tid < V) {
-            sm.vv[tid] = pv;
+            sm.vv[tid] = ld_io(static_cast<const IO *>(a.v) + (size_t)u * V + tid);
             if (a.mc_mode == 1) {   // running block mean of o: close the block every L tokens
-                float m = pmp, msum = pms;
-                if (ppos > 0 && ppos % a.L == 0) {
+                const int p = a.pos[u];
+                float m = a.mstate[(size_t)u * 2 * V + V + tid], msum = a.mstate[(size_t)u * 2 * V + tid];
+                if (p > 0 && p % a.L == 0) {
                     m = msum / (float)a.L;
                     a.mstate[(size_t)u * 2 * V + V + tid] = m;
                     msum = 0.f;
@@ -142,16 +113,29 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
                 sm.msum[tid] = msum;
             }
         }
-        if (tid == 0) {
-            sm.w = sigmoid_f(pwl);
-            if (a.mc_mode == 1) a.pos[u] = ppos + 1;
+        if (tid == 0) sm.w = sigmoid_f(a.w_logit[u]);
+        float pB[ZP][VP], pA[AP];
+#pragma unroll
+        for (int zp = 0; zp < ZP; ++zp) {
+            const int j = 32 * zp + tid / 8, part = tid % 8;
+#pragma unroll
+            for (int x = 0; x < VP; ++x) pB[zp][x] = j < R ? a.Bm[((size_t)h * R + j) * V + part + 8 * x] : 0.f;
         }
-        prefetch_tokens(i + 1);
-        __syncthreads();
+        {
+            const int kk = tid / TPK, part = tid % TPK;
+#pragma unroll
+            for (int x = 0; x < AP; ++x) {
+                const int r = part + TPK * x;
+                pA[x] = r < R ? a.A[((size_t)h * K + kk) * R + r] : 0.f;
+            }
+        }
         // ---- state rows into registers; content signal m = S q (mc_mode 0); k.q
-        const bool ok = mbar_wait(&sm.bar[st], (uint32_t)(i / kStepStages) & 1u);
-        if (__syncthreads_or(!ok)) {
-            failed = true;
+        const bool ok = mbar_wait(&sm.bar, (uint32_t)i & 1u);
+        if (group_sync_or(grp, !ok)) {   // record; drain the copy still in flight (bounded); leave
+            if (tid == 0) {
+                atomicOr(&g_step_timeout, 1);
+                mbar_wait(&sm.bar, (uint32_t)i & 1u);
+            }
             break;
         }
         float4 s[G4];
@@ -160,7 +144,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
 #pragma unroll
             for (int j = 0; j < G4; ++j) {
                 const int f = seg + TPR * ((j + row) % G4);
-                s[j] = reinterpret_cast<const float4 *>(Sst)[row * (K / 4) + f];
+                s[j] = reinterpret_cast<const float4 *>(sm.S)[row * (K / 4) + f];
                 const float4 qq = reinterpret_cast<const float4 *>(sm.qv)[f];
                 part += s[j].x * qq.x + s[j].y * qq.y + s[j].z * qq.z + s[j].w * qq.w;
             }
@@ -170,17 +154,21 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
                 if (seg == 0) sm.mv[row] = part;
             }
         }
-        if (tid >= kStepThreads - 32) {   // last warp: k.q
+        if (tid >= kGroupThreads - 32) {   // last warp: k.q
             float x = 0.f;
-            for (int c = tid - (kStepThreads - 32); c < K; c += 32) x += sm.kv[c] * sm.qv[c];
+            for (int c = tid - (kGroupThreads - 32); c < K; c += 32) x += sm.kv[c] * sm.qv[c];
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-            if (tid == kStepThreads - 32) sm.kq = x;
+            if (tid == kGroupThreads - 32) sm.kq = x;
         }
-        __syncthreads();
+        group_sync(grp);
+        if (tid == 0 && i + 1 < nmine) {   // the stage is free: the group's next unit
+            mbar_expect_tx(&sm.bar, kBytes);
+            bulk_g2s(sm.S, a.S + (size_t)unit_of(i + 1) * V * K, kBytes, &sm.bar);
+        }
         // ---- z = Bm m
 #pragma unroll
-        for (int zp = 0; zp < 2; ++zp) {
+        for (int zp = 0; zp < ZP; ++zp) {
             if (32 * zp < R) {
                 const int j = 32 * zp + tid / 8, part = tid % 8;
                 float acc = 0.f;
@@ -192,7 +180,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
                 if (part == 0 && j < R) sm.zv[j] = acc;
             }
         }
-        __syncthreads();
+        group_sync(grp);
         // ---- Delta = A z, gates
         {
             const int kk = tid / TPK, part = tid % TPK;
@@ -209,13 +197,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
                 sm.aqv[kk] = av * sm.qv[kk];
             }
         }
-        prefetch_factors(i + 1);
-        if (tid == 0) {   // the stage of unit i - 1 takes unit i + 2 once its store has read it
-            bulk_wait_read<0>();
-            issue(i + 2);
-        }
-        __syncthreads();
-        // ---- p = S (a*k), S (a*q); update; output
+        group_sync(grp);
+        // ---- p = S (a*k), S (a*q); update (stored from registers); output
         {
             float p = 0.f, s2 = 0.f;
 #pragma unroll
@@ -232,6 +215,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
                 s2 += __shfl_xor_sync(0xffffffffu, s2, off);
             }
             const float we = sm.w * (sm.vv[row] - p);
+            float4 *Sg = reinterpret_cast<float4 *>(a.S + (size_t)u * V * K) + row * (K / 4);
 #pragma unroll
             for (int j = 0; j < G4; ++j) {
                 const int f = seg + TPR * ((j + row) % G4);
@@ -242,7 +226,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
                 x.y = x.y * av.y + we * kv.y;
                 x.z = x.z * av.z + we * kv.z;
                 x.w = x.w * av.w + we * kv.w;
-                reinterpret_cast<float4 *>(Sst)[row * (K / 4) + f] = x;
+                Sg[f] = x;
             }
             if (seg == 0) {
                 const float ov = s2 + we * sm.kq;
@@ -250,20 +234,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a, int n
                 if (a.mc_mode == 1) a.mstate[(size_t)u * 2 * V + row] = sm.msum[row] + ov;
             }
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_s2g(a.S + (size_t)u * V * K, Sst, kBytes);
-            bulk_commit();
-        }
+        if (tid == 0 && a.mc_mode == 1) a.pos[u] += 1;
+        group_sync(grp);   // the vectors of this unit are read; the next unit may overwrite them
     }
-    if (failed) {   // drain the loads still in flight into this CTA's stages, bounded
-        if (tid == 0) {
-            atomicOr(&g_step_timeout, 1);
-            for (int j = i; j < min(i + 2, nmine); ++j) mbar_wait(&sm.bar[j % kStepStages], (uint32_t)(j / kStepStages) & 1u);
-        }
-    }
-    if (tid == 0) bulk_wait<0>();
 }
 
 // A single thread waits, bounded, on a barrier that nothing arrives on (the expiry path of
@@ -303,24 +276,29 @@ static int sm_count() {
     return cached[dev];
 }
 
-template <int K, int V, typename IO>
+template <int K, int V, typename IO, int RMAX, int NGRP>
 cudaError_t launch_step_t(const StepArgs &a, cudaStream_t st) {
-    auto kern = step_kernel<K, V, IO>;
-    const int bytes = (int)sizeof(StepSmem<K, V>);
+    auto kern = step_kernel<K, V, IO, RMAX, NGRP>;
+    const int bytes = (int)sizeof(StepGroupSmem<K, V>) * NGRP;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     const int units = a.B * a.H;
     const int grid = units < sm_count() ? units : sm_count();
-    kern<<<grid, kStepThreads, bytes, st>>>(a, units);
+    kern<<<grid, kGroupThreads * NGRP, bytes, st>>>(a, units);
     return cudaGetLastError();
+}
+
+template <int K, int V, typename IO>
+cudaError_t launch_step_r(const StepArgs &a, cudaStream_t st) {
+    return a.R <= 32 ? launch_step_t<K, V, IO, 32, 2>(a, st) : launch_step_t<K, V, IO, 64, 1>(a, st);
 }
 
 template <typename IO>
 cudaError_t dispatch_step(int K, int V, const StepArgs &a, cudaStream_t st) {
-    if (K == 64 && V == 64) return launch_step_t<64, 64, IO>(a, st);
-    if (K == 64 && V == 128) return launch_step_t<64, 128, IO>(a, st);
-    if (K == 128 && V == 64) return launch_step_t<128, 64, IO>(a, st);
-    return launch_step_t<128, 128, IO>(a, st);
+    if (K == 64 && V == 64) return launch_step_r<64, 64, IO>(a, st);
+    if (K == 64 && V == 128) return launch_step_r<64, 128, IO>(a, st);
+    if (K == 128 && V == 64) return launch_step_r<128, 64, IO>(a, st);
+    return launch_step_r<128, 128, IO>(a, st);
 }
 
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
