@@ -61,6 +61,9 @@ __device__ __forceinline__ void content_signal(const float *Bh, const float *Ah,
     __syncthreads();
 }
 
+// Host: raise `kern`'s dynamic shared-memory limit to `bytes` on the current device, once.
+cudaError_t set_smem_once(const void *kern, int bytes);
+
 struct FwdArgs {
     const void *q, *k, *v;
     const float *g_logit, *bx, *w_logit, *A, *Bm, *S0, *m_prev_in;

@@ -587,7 +587,7 @@ __global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, int B,
 template <int K, int V, typename IO>
 cudaError_t launch_fwd_simt_t(const FwdArgs &a, cudaStream_t st) {
     auto kern = fwd_simt_kernel<K, V, IO>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FwdSmem<K, V>::bytes);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)FwdSmem<K, V>::bytes);
     if (e != cudaSuccess) return e;
     kern<<<a.B * a.H, kThreads, FwdSmem<K, V>::bytes, st>>>(a);
     return cudaGetLastError();
@@ -596,7 +596,7 @@ cudaError_t launch_fwd_simt_t(const FwdArgs &a, cudaStream_t st) {
 template <int K, int V, typename IO>
 cudaError_t launch_bwd_simt_t(const BwdArgs &a, float *dA, float *dB, cudaStream_t st) {
     auto kern = bwd_simt_kernel<K, V, IO>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwdSmem<K, V>::bytes);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)BwdSmem<K, V>::bytes);
     if (e != cudaSuccess) return e;
     kern<<<a.B * a.H, kThreads, BwdSmem<K, V>::bytes, st>>>(a);
     e = cudaGetLastError();

@@ -14,9 +14,13 @@
 // unit (content signal -> z -> Delta -> gates -> update) overlaps the other group's.  A
 // unit's state arrives in the group's stage by one bulk copy; the first pass moves it into
 // registers, after which the stage is refilled with the group's next unit while this one
-// finishes.  The updated state is stored from registers: each row is held by TPR threads as
-// float4 groups in a row-rotated order, which keeps the shared-memory reads conflict-free
-// and every 32-byte sector of the global stores whole.
+// finishes.  The updated state is stored from registers.  Thread layout: the 8 lanes of a
+// lane octet share a row group and split the columns (lane seg holds float4 columns
+// seg, seg + 8, ...), and a thread holds the rows rg, rg + 32, ... of its row group rg.  A
+// warp's reads of a state row are then 128 contiguous bytes per octet, its reads of the
+// q / k / a vectors are broadcasts (every octet reads the same 128 bytes), and each global
+// store instruction writes whole 128-byte lines.  Row sums over an octet use a transposing
+// reduction that halves the values exchanged at each of its three steps.
 #include "carve_device.cuh"
 #include "carve_mma.cuh"
 
@@ -39,7 +43,7 @@ __device__ int g_step_timeout;  // set when a bounded wait gives up (never expec
 template <int K, int V>
 struct __align__(16) StepGroupSmem {
     float S[V * K];
-    float qv[K], kv[K], glv[K], bxv[K], av[K], akv[K], aqv[K];
+    float qv[K], kv[K], glv[K], bxv[K], av[K];
     float vv[V], mv[V], msum[V], zv[kStepMaxRank];
     float w, kq;
     uint64_t bar;
@@ -60,11 +64,37 @@ __device__ __forceinline__ bool group_sync_or(int id, bool v) {
     return r != 0;
 }
 
+// Sums x[0..N) over the 8 lanes of an aligned lane octet (lanes differing in bits 0-2 of the
+// lane index; `seg` = those bits) and returns the total of x[seg >> (3 - log2 N)].
+template <int N>
+__device__ __forceinline__ float octet_reduce(const float (&x)[N], int seg) {
+    static_assert(N == 2 || N == 4 || N == 8, "octet_reduce: N in {2, 4, 8}");
+    float y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = j < N ? x[j] : 0.f;
+    int n = N;
+#pragma unroll
+    for (int bit = 4; bit >= 1; bit >>= 1) {
+        if (n > 1) {
+            const int h = n / 2;
+            const bool up = (seg & bit) != 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (j < h) y[j] = (up ? y[j + h] : y[j]) + __shfl_xor_sync(0xffffffffu, up ? y[j] : y[j + h], bit);
+            n = h;
+        } else {
+            y[0] += __shfl_xor_sync(0xffffffffu, y[0], bit);
+        }
+    }
+    return y[0];
+}
+
 // RMAX: rank bound of the factor slices held in registers (32, or 64 with one group).
 template <int K, int V, typename IO, int RMAX, int NGRP>
 __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a, int n_units) {
-    constexpr int TPR = kGroupThreads / V;     // threads per state row
-    constexpr int G4 = K / 4 / TPR;            // float4 groups per thread
+    constexpr int RPT = V / 32;                // state rows per thread: rg + 32 i
+    constexpr int CPT = K / 32;                // float4 columns per row per thread: seg + 8 jj
+    constexpr int LRPT = RPT == 4 ? 2 : 1;     // log2 RPT
     constexpr int TPK = kGroupThreads / K;     // threads per Delta output
     constexpr int VP = V / 8;                  // entries of a z dot product per thread (8 per output)
     constexpr int ZP = RMAX / 32;              // passes of 32 z outputs
@@ -73,7 +103,7 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
     extern __shared__ __align__(128) unsigned char smraw[];
     const int grp = threadIdx.x / kGroupThreads, tid = threadIdx.x % kGroupThreads;
     StepGroupSmem<K, V> &sm = reinterpret_cast<StepGroupSmem<K, V> *>(smraw)[grp];
-    const int row = tid / TPR, seg = tid % TPR, H = a.H, R = a.R;
+    const int seg = tid % 8, rg = tid / 8, lane = tid % 32, H = a.H, R = a.R;
     // this group's units: first + (NGRP i + grp) stride, i = 0, 1, ...
     const int first = blockIdx.x, stride = gridDim.x;
     const int mine = first < n_units ? (n_units - 1 - first) / stride + 1 : 0;
@@ -138,20 +168,24 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
             }
             break;
         }
-        float4 s[G4];
+        float4 s[RPT][CPT];
         {
-            float part = 0.f;
+            const float4 *S4 = reinterpret_cast<const float4 *>(sm.S);
+            float part[RPT];
 #pragma unroll
-            for (int j = 0; j < G4; ++j) {
-                const int f = seg + TPR * ((j + row) % G4);
-                s[j] = reinterpret_cast<const float4 *>(sm.S)[row * (K / 4) + f];
-                const float4 qq = reinterpret_cast<const float4 *>(sm.qv)[f];
-                part += s[j].x * qq.x + s[j].y * qq.y + s[j].z * qq.z + s[j].w * qq.w;
+            for (int i2 = 0; i2 < RPT; ++i2) part[i2] = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < CPT; ++jj) {
+                const float4 qq = reinterpret_cast<const float4 *>(sm.qv)[seg + 8 * jj];
+#pragma unroll
+                for (int i2 = 0; i2 < RPT; ++i2) {
+                    s[i2][jj] = S4[(rg + 32 * i2) * (K / 4) + seg + 8 * jj];
+                    part[i2] += s[i2][jj].x * qq.x + s[i2][jj].y * qq.y + s[i2][jj].z * qq.z + s[i2][jj].w * qq.w;
+                }
             }
             if (a.mc_mode == 0) {
-#pragma unroll
-                for (int off = TPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-                if (seg == 0) sm.mv[row] = part;
+                const float m = octet_reduce<RPT>(part, seg);   // row rg + 32 (seg >> (3 - LRPT))
+                if ((seg & ((8 >> LRPT) - 1)) == 0) sm.mv[rg + 32 * (seg >> (3 - LRPT))] = m;
             }
         }
         if (tid >= kGroupThreads - 32) {   // last warp: k.q
@@ -191,47 +225,64 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
 #pragma unroll
             for (int off = TPK / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             if (part == 0) {
-                const float av = expf(log_retention(sm.glv[kk], sm.bxv[kk] + acc));
+                // a = sigma(-g_logit) sigma(bx + Delta) = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)}))
+                const float e1 = __expf(sm.glv[kk]), e2 = __expf(-(sm.bxv[kk] + acc));
+                const float av = __fdividef(1.f, (1.f + e1) * (1.f + e2));
                 sm.av[kk] = av;
-                sm.akv[kk] = av * sm.kv[kk];
-                sm.aqv[kk] = av * sm.qv[kk];
             }
         }
         group_sync(grp);
-        // ---- p = S (a*k), S (a*q); update (stored from registers); output
+        // ---- p = (S a).k, s2 = (S a).q per row; update (stored from registers); output
         {
-            float p = 0.f, s2 = 0.f;
+            float ps[2 * RPT];   // p of rows 0..RPT-1, then s2
 #pragma unroll
-            for (int j = 0; j < G4; ++j) {
-                const int f = seg + TPR * ((j + row) % G4);
-                const float4 ak = reinterpret_cast<const float4 *>(sm.akv)[f];
-                const float4 aq = reinterpret_cast<const float4 *>(sm.aqv)[f];
-                p += s[j].x * ak.x + s[j].y * ak.y + s[j].z * ak.z + s[j].w * ak.w;
-                s2 += s[j].x * aq.x + s[j].y * aq.y + s[j].z * aq.z + s[j].w * aq.w;
-            }
+            for (int x = 0; x < 2 * RPT; ++x) ps[x] = 0.f;
 #pragma unroll
-            for (int off = TPR / 2; off >= 1; off >>= 1) {
-                p += __shfl_xor_sync(0xffffffffu, p, off);
-                s2 += __shfl_xor_sync(0xffffffffu, s2, off);
-            }
-            const float we = sm.w * (sm.vv[row] - p);
-            float4 *Sg = reinterpret_cast<float4 *>(a.S + (size_t)u * V * K) + row * (K / 4);
+            for (int jj = 0; jj < CPT; ++jj) {
+                const float4 av = reinterpret_cast<const float4 *>(sm.av)[seg + 8 * jj];
+                const float4 kv = reinterpret_cast<const float4 *>(sm.kv)[seg + 8 * jj];
+                const float4 qv = reinterpret_cast<const float4 *>(sm.qv)[seg + 8 * jj];
 #pragma unroll
-            for (int j = 0; j < G4; ++j) {
-                const int f = seg + TPR * ((j + row) % G4);
-                const float4 av = reinterpret_cast<const float4 *>(sm.av)[f];
-                const float4 kv = reinterpret_cast<const float4 *>(sm.kv)[f];
-                float4 x = s[j];
-                x.x = x.x * av.x + we * kv.x;
-                x.y = x.y * av.y + we * kv.y;
-                x.z = x.z * av.z + we * kv.z;
-                x.w = x.w * av.w + we * kv.w;
-                Sg[f] = x;
+                for (int i2 = 0; i2 < RPT; ++i2) {
+                    float4 &x = s[i2][jj];
+                    x.x *= av.x;
+                    x.y *= av.y;
+                    x.z *= av.z;
+                    x.w *= av.w;
+                    ps[i2] += x.x * kv.x + x.y * kv.y + x.z * kv.z + x.w * kv.w;
+                    ps[RPT + i2] += x.x * qv.x + x.y * qv.y + x.z * qv.z + x.w * qv.w;
+                }
             }
-            if (seg == 0) {
-                const float ov = s2 + we * sm.kq;
-                st_io(static_cast<IO *>(a.o) + (size_t)u * V + row, ov);
-                if (a.mc_mode == 1) a.mstate[(size_t)u * 2 * V + row] = sm.msum[row] + ov;
+            // lane seg now holds ps[idx] summed over the octet, idx = seg >> (2 - LRPT)
+            const float tot = octet_reduce<2 * RPT>(ps, seg);
+            const int idx = seg >> (2 - LRPT), ri = idx % RPT;
+            const int row_i = rg + 32 * ri;
+            const float we_mine = idx < RPT ? sm.w * (sm.vv[row_i] - tot) : 0.f;
+            float we[RPT];
+#pragma unroll
+            for (int i2 = 0; i2 < RPT; ++i2) we[i2] = __shfl_sync(0xffffffffu, we_mine, (lane & ~7) | (i2 << (2 - LRPT)));
+            float4 *Sg = reinterpret_cast<float4 *>(a.S + (size_t)u * V * K);
+#pragma unroll
+            for (int jj = 0; jj < CPT; ++jj) {   // S' = S Diag(a) + w e k^T
+                const float4 kv = reinterpret_cast<const float4 *>(sm.kv)[seg + 8 * jj];
+#pragma unroll
+                for (int i2 = 0; i2 < RPT; ++i2) {
+                    float4 x = s[i2][jj];
+                    x.x += we[i2] * kv.x;
+                    x.y += we[i2] * kv.y;
+                    x.z += we[i2] * kv.z;
+                    x.w += we[i2] * kv.w;
+                    Sg[(rg + 32 * i2) * (K / 4) + seg + 8 * jj] = x;
+                }
+            }
+            if (idx >= RPT && (seg & ((4 >> LRPT) - 1)) == 0) {   // one lane per row: the output
+                float wr = we[0];
+#pragma unroll
+                for (int i2 = 1; i2 < RPT; ++i2)
+                    if (ri == i2) wr = we[i2];
+                const float ov = tot + wr * sm.kq;
+                st_io(static_cast<IO *>(a.o) + (size_t)u * V + row_i, ov);
+                if (a.mc_mode == 1) a.mstate[(size_t)u * 2 * V + row_i] = sm.msum[row_i] + ov;
             }
         }
         if (tid == 0 && a.mc_mode == 1) a.pos[u] += 1;
@@ -280,7 +331,7 @@ template <int K, int V, typename IO, int RMAX, int NGRP>
 cudaError_t launch_step_t(const StepArgs &a, cudaStream_t st) {
     auto kern = step_kernel<K, V, IO, RMAX, NGRP>;
     const int bytes = (int)sizeof(StepGroupSmem<K, V>) * NGRP;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), bytes);
     if (e != cudaSuccess) return e;
     const int units = a.B * a.H;
     const int grid = units < sm_count() ? units : sm_count();

@@ -914,7 +914,7 @@ __global__ void dq_readout_kernel(__nv_bfloat16 *dq, const float *vec, int H, in
 
 cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st) {
     const int bytes = (int)sizeof(TcBwdSmem);
-    cudaError_t e = cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(tc_bwd_kernel), bytes);
     if (e != cudaSuccess) return e;
     const long long rows = (long long)a.B * a.T;
     BwdMaps maps;

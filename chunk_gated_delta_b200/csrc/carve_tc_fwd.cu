@@ -532,7 +532,7 @@ template <int NB>
 cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
     auto kern = tc_fwd_kernel<NB>;
     const int bytes = (int)sizeof(TcFwdSmem<NB>);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), bytes);
     if (e != cudaSuccess) return e;
     const int C = 16 * NB;
     const long long rows = (long long)a.B * a.T;

@@ -1,5 +1,9 @@
-// Host-side construction of TMA tensor maps for the token-major [B*T, H, channels] tensors.
+// Host-side helpers: TMA tensor maps for the token-major [B*T, H, channels] tensors, and the
+// once-per-device dynamic shared-memory opt-in of the kernels.
 #include <cudaTypedefs.h>
+
+#include <mutex>
+#include <vector>
 
 #include "carve_mma.cuh"
 
@@ -29,6 +33,27 @@ cudaError_t make_token_tile_map(CUtensorMap *map, const void *base, int elem_byt
     CUresult r = enc(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The opt-in above 48 KB of dynamic shared memory is a per-device attribute of the kernel that
+// persists, so it is set on the first launch on each device only (launches stay one driver
+// call; safe to call from several threads).
+cudaError_t set_smem_once(const void *kern, int bytes) {
+    struct Entry {
+        const void *kern;
+        int dev, bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry &x : done)
+        if (x.kern == kern && x.dev == dev && x.bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.push_back(Entry{kern, dev, bytes});
+    return e;
 }
 
 }  // namespace carve
