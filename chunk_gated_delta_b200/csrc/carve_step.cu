@@ -40,14 +40,31 @@ constexpr int kStepMaxRank = 64;
 
 __device__ int g_step_timeout;  // set when a bounded wait gives up (never expected)
 
-template <int K, int V>
+// A unit's token vectors as stored in global memory (q, k, v in the I/O type).
+template <int K, int V, typename IO>
+struct __align__(16) StepTokens {
+    IO q[K], k[K], v[V];
+    float gl[K], bx[K], wl[4];
+};
+
+template <int K, int V, typename IO>
 struct __align__(16) StepGroupSmem {
     float S[V * K];
+    StepTokens<K, V, IO> tok[2];   // this unit's and the next unit's, filled by cp.async
     float qv[K], kv[K], glv[K], bxv[K], av[K];
     float vv[V], mv[V], msum[V], zv[kStepMaxRank];
     float w, kq;
     uint64_t bar;
 };
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 // Barrier over the 256 threads of group `id` (named barrier 1 + id).
 __device__ __forceinline__ void group_sync(int id) {
@@ -102,13 +119,36 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
     constexpr uint32_t kBytes = V * K * 4;
     extern __shared__ __align__(128) unsigned char smraw[];
     const int grp = threadIdx.x / kGroupThreads, tid = threadIdx.x % kGroupThreads;
-    StepGroupSmem<K, V> &sm = reinterpret_cast<StepGroupSmem<K, V> *>(smraw)[grp];
+    StepGroupSmem<K, V, IO> &sm = reinterpret_cast<StepGroupSmem<K, V, IO> *>(smraw)[grp];
     const int seg = tid % 8, rg = tid / 8, lane = tid % 32, H = a.H, R = a.R;
     // this group's units: first + (NGRP i + grp) stride, i = 0, 1, ...
     const int first = blockIdx.x, stride = gridDim.x;
     const int mine = first < n_units ? (n_units - 1 - first) / stride + 1 : 0;
     const int nmine = mine > grp ? (mine - 1 - grp) / NGRP + 1 : 0;
     auto unit_of = [&](int i) { return first + (NGRP * i + grp) * stride; };
+
+    // token vectors of the group's i-th unit into tok[i & 1], 16 bytes per copy
+    auto fetch_tokens = [&](int i) {
+        if (i >= nmine) return;
+        const int u = unit_of(i);
+        StepTokens<K, V, IO> &t = sm.tok[i & 1];
+        constexpr int CQ = K * (int)sizeof(IO) / 16, CV = V * (int)sizeof(IO) / 16, CG = K * 4 / 16;
+        for (int c = tid; c < 2 * CQ + CV + 2 * CG; c += kGroupThreads) {
+            if (c < CQ) cp_async16(reinterpret_cast<char *>(t.q) + 16 * c,
+                                   static_cast<const char *>(a.q) + (size_t)u * K * sizeof(IO) + 16 * c);
+            else if (c < 2 * CQ) cp_async16(reinterpret_cast<char *>(t.k) + 16 * (c - CQ),
+                                            static_cast<const char *>(a.k) + (size_t)u * K * sizeof(IO) + 16 * (c - CQ));
+            else if (c < 2 * CQ + CV)
+                cp_async16(reinterpret_cast<char *>(t.v) + 16 * (c - 2 * CQ),
+                           static_cast<const char *>(a.v) + (size_t)u * V * sizeof(IO) + 16 * (c - 2 * CQ));
+            else if (c < 2 * CQ + CV + CG)
+                cp_async16(t.gl + 4 * (c - 2 * CQ - CV), a.g_logit + (size_t)u * K + 4 * (c - 2 * CQ - CV));
+            else
+                cp_async16(t.bx + 4 * (c - 2 * CQ - CV - CG), a.bx + (size_t)u * K + 4 * (c - 2 * CQ - CV - CG));
+        }
+        if (tid == kGroupThreads - 1) cp_async4(t.wl, a.w_logit + u);
+        cp_async_commit();
+    };
 
     if (tid == 0) {
         mbar_init(&sm.bar, 1);
@@ -118,19 +158,28 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
             bulk_g2s(sm.S, a.S + (size_t)unit_of(0) * V * K, kBytes, &sm.bar);
         }
     }
+    fetch_tokens(0);
     group_sync(grp);
 
     for (int i = 0; i < nmine; ++i) {
         const int u = unit_of(i), h = u % H;
-        // ---- token vectors into shared memory, the head's factor slices into registers
-        if (tid < K) {
-            sm.qv[tid] = ld_io(static_cast<const IO *>(a.q) + (size_t)u * K + tid);
-            sm.kv[tid] = ld_io(static_cast<const IO *>(a.k) + (size_t)u * K + tid);
-            sm.glv[tid] = a.g_logit[(size_t)u * K + tid];
-            sm.bxv[tid] = a.bx[(size_t)u * K + tid];
+        // ---- token vectors (prefetched) into fp32 working copies, the next unit's requested;
+        //      the head's factor slices into registers
+        cp_async_wait_all();
+        group_sync(grp);
+        {
+            const StepTokens<K, V, IO> &t = sm.tok[i & 1];
+            if (tid < K) {
+                sm.qv[tid] = ld_io(t.q + tid);
+                sm.kv[tid] = ld_io(t.k + tid);
+                sm.glv[tid] = t.gl[tid];
+                sm.bxv[tid] = t.bx[tid];
+            }
+            if (tid < V) sm.vv[tid] = ld_io(t.v + tid);
+            if (tid == 0) sm.w = sigmoid_f(t.wl[0]);
         }
+        fetch_tokens(i + 1);   // tok[(i + 1) & 1] was last read before the barrier above
         if (tid < V) {
-            sm.vv[tid] = ld_io(static_cast<const IO *>(a.v) + (size_t)u * V + tid);
             if (a.mc_mode == 1) {   // running block mean of o: close the block every L tokens
                 const int p = a.pos[u];
                 float m = a.mstate[(size_t)u * 2 * V + V + tid], msum = a.mstate[(size_t)u * 2 * V + tid];
@@ -143,7 +192,6 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
                 sm.msum[tid] = msum;
             }
         }
-        if (tid == 0) sm.w = sigmoid_f(a.w_logit[u]);
         float pB[ZP][VP], pA[AP];
 #pragma unroll
         for (int zp = 0; zp < ZP; ++zp) {
@@ -330,7 +378,7 @@ static int sm_count() {
 template <int K, int V, typename IO, int RMAX, int NGRP>
 cudaError_t launch_step_t(const StepArgs &a, cudaStream_t st) {
     auto kern = step_kernel<K, V, IO, RMAX, NGRP>;
-    const int bytes = (int)sizeof(StepGroupSmem<K, V>) * NGRP;
+    const int bytes = (int)sizeof(StepGroupSmem<K, V, IO>) * NGRP;
     cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), bytes);
     if (e != cudaSuccess) return e;
     const int units = a.B * a.H;
