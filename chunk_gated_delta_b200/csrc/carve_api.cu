@@ -10,6 +10,7 @@ cudaError_t launch_fwd_simt(int K, int V, bool bf16, const FwdArgs &a, cudaStrea
 cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st);
 cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 int tc_compute_chunk(int L);
+int tc_reduce_slices(int B, int NG);
 int tc_fwd_take_timeout();
 int tc_bwd_take_timeout();
 int step_take_timeout();
@@ -100,8 +101,10 @@ size_t carve_saved_bytes(const carve_dims *d) {
 size_t carve_bwd_workspace_bytes(const carve_dims *d) {
     if (check_dims(d, true) != CARVE_OK) return 0;
     const size_t units = (size_t)d->B * d->H;
-    if (use_tc_bwd(d))   // per gate chunk: dDelta and dz (160 floats) and the readout vector of dq
-        return sizeof(float) * units * n_chunks(d) * (160 + (size_t)d->dk);
+    if (use_tc_bwd(d))   // per gate chunk: dDelta and dz (160 floats) and the readout vector of dq;
+                         // then the per-slice partial sums of dA and dB
+        return sizeof(float) * (units * n_chunks(d) * (160 + (size_t)d->dk) +
+                                (size_t)carve::tc_reduce_slices(d->B, (int)n_chunks(d)) * d->H * 256 * d->rank);
     return sizeof(float) * units * ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv);
 }
 

@@ -49,8 +49,8 @@ struct __align__(16) TcBwdSmem {
     __nv_bfloat16 tii[kBNB * 16 * 24];
     float akk_d[kBC * 17];
     float rfac[kBC * kLdF], dlam[kBC * kLdF];
-    float p7[kBNB * 128], r15[kBNB * 128], dblk[kBNB * 128], em[kBNB * 128], fm[kBNB * 128], cij[128];
-    float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], btot[kBNB * 128], pdd[kBNB * 128];
+    float p7[kBNB * 128], r15[kBNB * 128], em[kBNB * 128], fm[kBNB * 128], cij[128];
+    float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], htot[2 * kBNB * 128], pdd[2 * kBNB * 128];
     float bpart[kBNB * 128];
     float delta[128], ddelta[128], mvec[128], zvec[64], dzv[64], dmv[128], dox[128], vecK[128], qbar[128];
     uint64_t bar, bar_s0;
@@ -77,7 +77,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     // readout vectors of dq (128 per gate chunk)
     float *wsg = a.ws + (size_t)u * NG * 160;
     float *wsv = a.ws + (size_t)a.B * a.H * NG * 160 + (size_t)u * NG * 128;
-    const int kch = tid & 127, ib = tid >> 7;   // (channel, 16-block) owned in the gate phases
+    // gate phases: channel pair c0 = 2 cp, 2 cp + 1 over tokens 8 hf + [0, 8) of 16-token block ib
+    const int cp = tid & 63, hf = (tid >> 6) & 1, ib = tid >> 7, c0 = 2 * cp;
 
     float ds[16][4];
 #pragma unroll
@@ -159,13 +160,13 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     uint32_t phase = 0;
     __syncthreads();
     // gate logits of the chunk about to be processed, loaded one chunk ahead
-    float glr[16], bxr[16];
+    float2 glr[8], bxr[8];
     auto load_gates = [&](int cc) {
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const size_t gi = base_bh + (size_t)(cc * C + 16 * ib + t) * tstride + kch;
-            glr[t] = a.g_logit[gi];
-            bxr[t] = a.bx[gi];
+        for (int t = 0; t < 8; ++t) {
+            const size_t gi = base_bh + (size_t)(cc * C + 16 * ib + 8 * hf + t) * tstride + c0;
+            glr[t] = *reinterpret_cast<const float2 *>(a.g_logit + gi);
+            bxr[t] = *reinterpret_cast<const float2 *>(a.bx + gi);
         }
     };
     load_gates(NCC - 1);
@@ -208,44 +209,76 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             y.w = pack_bf16(bf(xv[6]) + dx[6], bf(xv[7]) + dx[7]);
             *reinterpret_cast<uint4 *>(sm.dop + t * kLdOp + part * 8) = y;
         }
-        // ---- recompute: gates and mid-block referenced operands (as the forward)
+        // ---- recompute: gates and mid-block referenced operands (as the forward: running
+        //      products outward from the block's token 7, two channels per thread)
         {
-            const float dl = sm.delta[kch];
-            float av[16], ia[16], rf[16], cf[16];
+            const float dl0 = sm.delta[c0], dl1 = sm.delta[c0 + 1];
+            float av[2][8], ia[2][8], rf[2][8], cf[2][8];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) retention(glr[t], bxr[t] + dl, av[t], ia[t]);
-            mid_reference(av, ia, rf, cf);
-            float p7 = 1.f;
+            for (int t = 0; t < 8; ++t) {
+                retention(glr[t].x, bxr[t].x + dl0, av[0][t], ia[0][t]);
+                retention(glr[t].y, bxr[t].y + dl1, av[1][t], ia[1][t]);
+            }
+            if (hf == 0) {
 #pragma unroll
-            for (int t = 0; t < 8; ++t) p7 *= av[t];
-            sm.p7[ib * 128 + kch] = p7;
-            sm.r15[ib * 128 + kch] = rf[15];
-            sm.dblk[ib * 128 + kch] = p7 * rf[15];
+                for (int e = 0; e < 2; ++e) {
+                    rf[e][7] = cf[e][7] = 1.f;
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const int row = 16 * ib + t;
-                const float qv = bf(sm.rq[row * 128 + kch]), kv = bf(sm.rk[row * 128 + kch]);
-                sm.qm[row * kLdOp + kch] = __float2bfloat16_rn(qv * rf[t]);
-                sm.krm[row * kLdOp + kch] = __float2bfloat16_rn(kv * rf[t]);
-                sm.kcm[row * kLdOp + kch] = __float2bfloat16_rn(kv * cf[t]);
-                sm.rfac[row * kLdF + kch] = rf[t];
+                    for (int t = 6; t >= 0; --t) {
+                        cf[e][t] = cf[e][t + 1] * av[e][t + 1];
+                        rf[e][t] = rf[e][t + 1] * ia[e][t + 1];
+                    }
+                }
+                float p0 = 1.f, p1 = 1.f;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    p0 *= av[0][t];
+                    p1 *= av[1][t];
+                }
+                *reinterpret_cast<float2 *>(&sm.p7[ib * 128 + c0]) = make_float2(p0, p1);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    rf[e][0] = av[e][0];
+                    cf[e][0] = ia[e][0];
+#pragma unroll
+                    for (int t = 1; t < 8; ++t) {
+                        rf[e][t] = rf[e][t - 1] * av[e][t];
+                        cf[e][t] = cf[e][t - 1] * ia[e][t];
+                    }
+                }
+                *reinterpret_cast<float2 *>(&sm.r15[ib * 128 + c0]) = make_float2(rf[0][7], rf[1][7]);
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int row = 16 * ib + 8 * hf + t;
+                const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(&sm.rq[row * 128 + c0]);
+                const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(&sm.rk[row * 128 + c0]);
+                const float k0 = bf(k2.x), k1 = bf(k2.y);
+                *reinterpret_cast<uint32_t *>(&sm.qm[row * kLdOp + c0]) = pack_bf16(bf(q2.x) * rf[0][t], bf(q2.y) * rf[1][t]);
+                *reinterpret_cast<uint32_t *>(&sm.krm[row * kLdOp + c0]) = pack_bf16(k0 * rf[0][t], k1 * rf[1][t]);
+                *reinterpret_cast<uint32_t *>(&sm.kcm[row * kLdOp + c0]) = pack_bf16(k0 * cf[0][t], k1 * cf[1][t]);
+                *reinterpret_cast<float2 *>(&sm.rfac[row * kLdF + c0]) = make_float2(rf[0][t], rf[1][t]);
             }
         }
         if (tid < C) sm.wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + t0 + tid) * H + h]);
         __syncthreads();
         if (tid < 128) {
+            float dblk[NB];   // decay over each 16-token block
+#pragma unroll
+            for (int i = 0; i < NB; ++i) dblk[i] = sm.p7[i * 128 + tid] * sm.r15[i * 128 + tid];
             float E = 1.f;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
                 sm.em[i * 128 + tid] = E * sm.p7[i * 128 + tid];
-                E *= sm.dblk[i * 128 + tid];
+                E *= dblk[i];
             }
             sm.gam[tid] = E;
             float F = 1.f;
 #pragma unroll
             for (int i = NB - 1; i >= 0; --i) {
                 sm.fm[i * 128 + tid] = sm.r15[i * 128 + tid] * F;
-                F *= sm.dblk[i * 128 + tid];
+                F *= dblk[i];
             }
             sm.cij[tid] = sm.r15[tid] * sm.p7[128 + tid];   // e^{Lam_m(1) - Lam_m(0)}
         }
@@ -697,16 +730,29 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 }
         }
         __syncthreads();
-        // ---- reverse cumulative sum of dLam within the chunk, gate gradients
+        // ---- reverse cumulative sum of dLam within the chunk, gate gradients.  Half-block
+        //      totals first (the chunk's last-token term xl joins the last half), then each
+        //      thread scans its 8 tokens from the total of everything after them.
+        auto last_token_term = [&](int c) {
+            float xl = sm.gam[c] * sm.s0ds[c];
+#pragma unroll
+            for (int i2 = 0; i2 < NB; ++i2) xl += sm.bpart[i2 * 128 + c];
+            return xl;
+        };
+        const int hb = 2 * ib + hf;   // half-block index, 0 .. 2 NB - 1
         {
-            float tot = 0.f;
+            float t0s = 0.f, t1s = 0.f;
 #pragma unroll
-            for (int t = 0; t < 16; ++t) tot += sm.dlam[(16 * ib + t) * kLdF + kch];
-            float xl = sm.gam[kch] * sm.s0ds[kch];
-#pragma unroll
-            for (int i2 = 0; i2 < NB; ++i2) xl += sm.bpart[i2 * 128 + kch];
-            if (ib == NB - 1) tot += xl;
-            sm.btot[ib * 128 + kch] = tot;
+            for (int t = 0; t < 8; ++t) {
+                const float2 d2 = *reinterpret_cast<const float2 *>(&sm.dlam[(16 * ib + 8 * hf + t) * kLdF + c0]);
+                t0s += d2.x;
+                t1s += d2.y;
+            }
+            if (hb == 2 * NB - 1) {
+                t0s += last_token_term(c0);
+                t1s += last_token_term(c0 + 1);
+            }
+            *reinterpret_cast<float2 *>(&sm.htot[hb * 128 + c0]) = make_float2(t0s, t1s);
         }
         if (tid < C) {
             float dw = 0.f;
@@ -722,32 +768,47 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         }
         __syncthreads();
         {
-            float run = 0.f;
+            float run[2] = {0.f, 0.f};
 #pragma unroll
-            for (int i2 = 0; i2 < NB; ++i2)
-                if (i2 > ib) run += sm.btot[i2 * 128 + kch];
-            const float dl = sm.delta[kch];
-            float xl = sm.gam[kch] * sm.s0ds[kch];
+            for (int h2 = 0; h2 < 2 * NB; ++h2)
+                if (h2 > hb) {
+                    const float2 x = *reinterpret_cast<const float2 *>(&sm.htot[h2 * 128 + c0]);
+                    run[0] += x.x;
+                    run[1] += x.y;
+                }
+            const float dl[2] = {sm.delta[c0], sm.delta[c0 + 1]};
+            const float xl[2] = {hb == 2 * NB - 1 ? last_token_term(c0) : 0.f,
+                                 hb == 2 * NB - 1 ? last_token_term(c0 + 1) : 0.f};
+            float pdd[2] = {0.f, 0.f};
 #pragma unroll
-            for (int i2 = 0; i2 < NB; ++i2) xl += sm.bpart[i2 * 128 + kch];
-            float pdd = 0.f;
+            for (int t = 7; t >= 0; --t) {
+                const int row = 16 * ib + 8 * hf + t;
+                const float2 d2 = *reinterpret_cast<const float2 *>(&sm.dlam[row * kLdF + c0]);
+                float dg[2], db[2];
 #pragma unroll
-            for (int t = 15; t >= 0; --t) {
-                run += sm.dlam[(16 * ib + t) * kLdF + kch];
-                if (ib == NB - 1 && t == 15) run += xl;
-                const float e1 = __expf(glr[t]), e2 = __expf(-(bxr[t] + dl));
-                const float D = (1.f + e1) * (1.f + e2);
-                const bool floor = !(__fdividef(1.f, D) >= kAMin);
-                const float dglv = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run;
-                const float dbv = floor ? 0.f : __fdividef(e2, 1.f + e2) * run;
-                sm.dlam[(16 * ib + t) * kLdF + kch] = dglv;   // staged: this thread's own column
-                sm.rfac[(16 * ib + t) * kLdF + kch] = dbv;
-                pdd += dbv;
+                for (int e = 0; e < 2; ++e) {
+                    run[e] += e ? d2.y : d2.x;
+                    if (t == 7) run[e] += xl[e];
+                    const float e1 = __expf(e ? glr[t].y : glr[t].x), e2 = __expf(-((e ? bxr[t].y : bxr[t].x) + dl[e]));
+                    const float D = (1.f + e1) * (1.f + e2);
+                    const bool floor = !(__fdividef(1.f, D) >= kAMin);
+                    dg[e] = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run[e];
+                    db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
+                    pdd[e] += db[e];
+                }
+                // staged in this thread's own positions for the vectorised stores below
+                *reinterpret_cast<float2 *>(&sm.dlam[row * kLdF + c0]) = make_float2(dg[0], dg[1]);
+                *reinterpret_cast<float2 *>(&sm.rfac[row * kLdF + c0]) = make_float2(db[0], db[1]);
             }
-            sm.pdd[ib * 128 + kch] = pdd;
+            *reinterpret_cast<float2 *>(&sm.pdd[hb * 128 + c0]) = make_float2(pdd[0], pdd[1]);
         }
         __syncthreads();
-        if (tid < 128) sm.ddelta[tid] += sm.pdd[tid] + sm.pdd[128 + tid];
+        if (tid < 128) {
+            float x = 0.f;
+#pragma unroll
+            for (int h2 = 0; h2 < 2 * NB; ++h2) x += sm.pdd[h2 * 128 + tid];
+            sm.ddelta[tid] += x;
+        }
         for (int idx = tid; idx < C * 32; idx += 256) {   // d g_logit, dbx: four channels per store
             const int t = idx >> 5, c = (idx & 31) * 4;
             const float *gsrc = sm.dlam + t * kLdF + c, *bsrc = sm.rfac + t * kLdF + c;
@@ -834,32 +895,32 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 
 
 // dA[h] = sum_{b, gate chunk} dDelta z^T,  dB[h] = sum dz m^T  (z, m from the saved records),
-// summed in a fixed order.  Grid (H, slices of kRedOut outputs); the records of the head are
-// staged kRedRec at a time in shared memory with every load of a stage issued together.
-constexpr int kRedRec = 32, kRedOut = 1024;
-__global__ void __launch_bounds__(256) reduce_dAdB_tc_kernel(const float *wsg, const float *aux, float *dA, float *dB,
-                                                             int B, int H, int NG, int R) {
+// summed in a fixed order in two passes.  Pass 1, grid (H, slices of kRedSlice records): the
+// slice's records are staged kRedRec at a time in shared memory and each thread accumulates R
+// of the head's 256 R outputs; the partial sums go to the workspace.  Pass 2 adds the slices
+// in order.
+constexpr int kRedRec = 32, kRedSlice = 64;
+__global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *wsg, const float *aux, float *part,
+                                                                  int B, int H, int NG, int R) {
     __shared__ __align__(16) float gd[kRedRec][128], rm[kRedRec][128], gz[kRedRec][kTcMaxRankBwd],
         rz[kRedRec][kTcMaxRankBwd];
-    const int h = blockIdx.x, tid = threadIdx.x, NR = B * NG;
-    int oidx[4];
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x, NR = B * NG;
+    const int r0 = sl * kRedSlice, r1 = min(NR, r0 + kRedSlice);
+    float acc[kTcMaxRankBwd];
 #pragma unroll
-    for (int x = 0; x < 4; ++x) oidx[x] = blockIdx.y * kRedOut + x * 256 + tid;
-    for (int i0 = 0; i0 < NR; i0 += kRedRec) {
-        const int nr = min(kRedRec, NR - i0);
+    for (int x = 0; x < kTcMaxRankBwd; ++x) acc[x] = 0.f;
+    for (int i0 = r0; i0 < r1; i0 += kRedRec) {
+        const int nr = min(kRedRec, r1 - i0);
         for (int idx = tid; idx < nr * 64; idx += 256) {   // dDelta and m, four floats per load
-            const int i = idx >> 6, part = idx & 63, rec = i0 + i;
+            const int i = idx >> 6, part4 = idx & 63, rec = i0 + i;
             const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
-            if (part < 32) {
-                *reinterpret_cast<float4 *>(&gd[i][4 * part]) =
-                    *reinterpret_cast<const float4 *>(wsg + (u * NG + gc) * 160 + 4 * part);
+            if (part4 < 32) {
+                *reinterpret_cast<float4 *>(&gd[i][4 * part4]) =
+                    *reinterpret_cast<const float4 *>(wsg + (u * NG + gc) * 160 + 4 * part4);
             } else {
-                const float *r = aux + (u * NG + gc) * (384 + R) + 4 * (part - 32);
-                rm[i][4 * (part - 32)] = r[0];
-                rm[i][4 * (part - 32) + 1] = r[1];
-                rm[i][4 * (part - 32) + 2] = r[2];
-                rm[i][4 * (part - 32) + 3] = r[3];
+                const float *r = aux + (u * NG + gc) * (384 + R) + 4 * (part4 - 32);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) rm[i][4 * (part4 - 32) + e] = r[e];
             }
         }
         for (int idx = tid; idx < nr * R; idx += 256) {   // dz and z
@@ -870,25 +931,39 @@ __global__ void __launch_bounds__(256) reduce_dAdB_tc_kernel(const float *wsg, c
         }
         __syncthreads();
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int o = oidx[x];
-            if (o < 128 * R) {
-                const int k = o / R, j = o % R;
-                for (int i = 0; i < nr; ++i) acc[x] += gd[i][k] * rz[i][j];
-            } else if (o < 256 * R) {
-                const int j = (o - 128 * R) / 128, v = (o - 128 * R) % 128;
-                for (int i = 0; i < nr; ++i) acc[x] += gz[i][j] * rm[i][v];
+        for (int x = 0; x < kTcMaxRankBwd; ++x) {
+            if (x < R) {
+                const int o = tid + 256 * x;   // outputs 0 .. 256 R - 1
+                if (o < 128 * R) {
+                    const int k = o / R, j = o % R;
+                    for (int i = 0; i < nr; ++i) acc[x] += gd[i][k] * rz[i][j];
+                } else {
+                    const int j = (o - 128 * R) / 128, v = (o - 128 * R) % 128;
+                    for (int i = 0; i < nr; ++i) acc[x] += gz[i][j] * rm[i][v];
+                }
             }
         }
         __syncthreads();
     }
+    float *dst = part + ((size_t)sl * H + h) * 256 * R;
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        const int o = oidx[x];
-        if (o < 128 * R) dA[(size_t)h * 128 * R + o] = acc[x];
-        else if (o < 256 * R) dB[(size_t)h * R * 128 + (o - 128 * R)] = acc[x];
-    }
+    for (int x = 0; x < kTcMaxRankBwd; ++x)
+        if (x < R) dst[tid + 256 * x] = acc[x];
 }
+
+__global__ void __launch_bounds__(256) reduce_dAdB_final_kernel(const float *part, float *dA, float *dB, int H,
+                                                                int R, int S) {
+    const int idx = blockIdx.x * 256 + threadIdx.x;
+    if (idx >= H * 256 * R) return;
+    const int h = idx / (256 * R), o = idx % (256 * R);
+    float acc = 0.f;
+    for (int sl = 0; sl < S; ++sl) acc += part[((size_t)sl * H + h) * 256 * R + o];
+    if (o < 128 * R) dA[(size_t)h * 128 * R + o] = acc;
+    else dB[(size_t)h * R * 128 + (o - 128 * R)] = acc;
+}
+
+// Record slices of the dA / dB reduction (B * NG records per head, kRedSlice per slice).
+int tc_reduce_slices(int B, int NG) { return (B * NG + kRedSlice - 1) / kRedSlice; }
 
 // dq_t += vec[unit][gate chunk of t] (the content-readout term of the default readout), 8
 // channels per thread
@@ -931,9 +1006,11 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
                                                                               a.H, a.T, a.L, rows);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const int NG = (a.T + a.L - 1) / a.L;
-    dim3 grid(a.H, (256 * a.R + kRedOut - 1) / kRedOut);
-    reduce_dAdB_tc_kernel<<<grid, 256, 0, st>>>(a.ws, a.saved_aux, dA, dB, a.B, a.H, NG, a.R);
+    const int NG = (a.T + a.L - 1) / a.L, S = tc_reduce_slices(a.B, NG);
+    float *part = a.ws + (size_t)a.B * a.H * NG * (160 + 128);
+    reduce_dAdB_partial_kernel<<<dim3(a.H, S), 256, 0, st>>>(a.ws, a.saved_aux, part, a.B, a.H, NG, a.R);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    reduce_dAdB_final_kernel<<<(a.H * 256 * a.R + 255) / 256, 256, 0, st>>>(part, dA, dB, a.H, a.R, S);
     return cudaGetLastError();
 }
 

@@ -44,7 +44,7 @@ struct __align__(16) TcFwdSmem {
     __nv_bfloat16 aqk[C * LDA], mkk[C * LDA];
     __nv_bfloat16 tii[NB * 16 * 24];
     float akk_d[NB * 16 * 17];
-    float p7[NB * 128], r15[NB * 128], dblk[NB * 128], em[NB * 128], fm[NB * 128], cij[NPAIR * 128];
+    float p7[NB * 128], r15[NB * 128], em[NB * 128], fm[NB * 128], cij[NPAIR * 128];
     float gam[128], wv[C], qbar[128], mvec[128], osum[128], mprev[128], zvec[64], delta[128];
     float Ah[128 * kTcMaxRank], Bh[kTcMaxRank * 128];   // the head's low-rank factors
     uint64_t bar[ST];
@@ -140,17 +140,20 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         const int st = cc % SM::ST;
         // gate inputs of this chunk, into registers (one-stage layout only; their latency
         // overlaps the readout)
-        float glr[NP][16], bxr[NP][16];
+        // (gate work item p: channel pair cp = p & 63, half hf = (p >> 6) & 1 of 16-token block
+        //  i = p >> 7: tokens 16 i + 8 hf + [0, 8) of channels 2 cp, 2 cp + 1)
+        float2 glr[NP][8], bxr[NP][8];
         if (!SM::GT) {
 #pragma unroll
             for (int x = 0; x < NP; ++x) {
-                const int p = tid + 256 * x, kch = p & 127, i = p >> 7;
+                const int p = tid + 256 * x, cp = p & 63, hf = (p >> 6) & 1, i = p >> 7;
                 if (p < 128 * NB) {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        const size_t gi = ((size_t)b * T + t0 + 16 * i + t) * tstride + (size_t)h * 128 + kch;
-                        glr[x][t] = a.g_logit[gi];
-                        bxr[x][t] = a.bx[gi];
+                    for (int t = 0; t < 8; ++t) {
+                        const size_t gi =
+                            ((size_t)b * T + t0 + 16 * i + 8 * hf + t) * tstride + (size_t)h * 128 + 2 * cp;
+                        glr[x][t] = *reinterpret_cast<const float2 *>(a.g_logit + gi);
+                        bxr[x][t] = *reinterpret_cast<const float2 *>(a.bx + gi);
                     }
                 }
             }
@@ -216,36 +219,69 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 if (tid < R) aux[128 + tid] = sm.zvec[tid];
             }
         }
-        // ---- gates and mid-block referenced operands, one (channel, 16-block) pair at a time
+        // ---- gates and mid-block referenced operands: per work item, two channels over half a
+        //      16-token block, factors referenced to the block's token 7 (running products
+        //      outward from it: backward over tokens 0-7, forward over tokens 8-15)
 #pragma unroll
         for (int x = 0; x < NP; ++x) {
-            const int p = tid + 256 * x, kch = p & 127, i = p >> 7;
+            const int p = tid + 256 * x, cp = p & 63, hf = (p >> 6) & 1, i = p >> 7, c0 = 2 * cp;
             if (p < 128 * NB) {
-                const float dl = sm.delta[kch];
-                float av[16], ia[16], rf[16], cf[16];
-                if (SM::GT) {
+                const float dl0 = sm.delta[c0], dl1 = sm.delta[c0 + 1];
+                float av[2][8], ia[2][8];
 #pragma unroll
-                    for (int t = 0; t < 16; ++t)
-                        retention(sm.rgl[st][(16 * i + t) * 128 + kch], sm.rbx[st][(16 * i + t) * 128 + kch] + dl, av[t],
-                                  ia[t]);
+                for (int t = 0; t < 8; ++t) {
+                    float2 gv, bv;
+                    if (SM::GT) {
+                        const int row = 16 * i + 8 * hf + t;
+                        gv = *reinterpret_cast<const float2 *>(&sm.rgl[st][row * 128 + c0]);
+                        bv = *reinterpret_cast<const float2 *>(&sm.rbx[st][row * 128 + c0]);
+                    } else {
+                        gv = glr[x][t];
+                        bv = bxr[x][t];
+                    }
+                    retention(gv.x, bv.x + dl0, av[0][t], ia[0][t]);
+                    retention(gv.y, bv.y + dl1, av[1][t], ia[1][t]);
+                }
+                float rf[2][8], cf[2][8];
+                if (hf == 0) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        rf[e][7] = cf[e][7] = 1.f;
+#pragma unroll
+                        for (int t = 6; t >= 0; --t) {
+                            cf[e][t] = cf[e][t + 1] * av[e][t + 1];
+                            rf[e][t] = rf[e][t + 1] * ia[e][t + 1];
+                        }
+                    }
+                    float p0 = 1.f, p1 = 1.f;
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        p0 *= av[0][t];
+                        p1 *= av[1][t];
+                    }
+                    *reinterpret_cast<float2 *>(&sm.p7[i * 128 + c0]) = make_float2(p0, p1);
                 } else {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) retention(glr[x][t], bxr[x][t] + dl, av[t], ia[t]);
+                    for (int e = 0; e < 2; ++e) {
+                        rf[e][0] = av[e][0];
+                        cf[e][0] = ia[e][0];
+#pragma unroll
+                        for (int t = 1; t < 8; ++t) {
+                            rf[e][t] = rf[e][t - 1] * av[e][t];
+                            cf[e][t] = cf[e][t - 1] * ia[e][t];
+                        }
+                    }
+                    *reinterpret_cast<float2 *>(&sm.r15[i * 128 + c0]) = make_float2(rf[0][7], rf[1][7]);
                 }
-                mid_reference(av, ia, rf, cf);
-                float p7 = 1.f;
 #pragma unroll
-                for (int t = 0; t < 8; ++t) p7 *= av[t];
-                sm.p7[i * 128 + kch] = p7;
-                sm.r15[i * 128 + kch] = rf[15];
-                sm.dblk[i * 128 + kch] = p7 * rf[15];
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int row = 16 * i + t;
-                    const float qv = bf(sm.rq[st][row * 128 + kch]), kv = bf(sm.rk[st][row * 128 + kch]);
-                    sm.qm[row * kLdOp + kch] = __float2bfloat16_rn(qv * rf[t]);
-                    sm.krm[row * kLdOp + kch] = __float2bfloat16_rn(kv * rf[t]);
-                    sm.kcm[row * kLdOp + kch] = __float2bfloat16_rn(kv * cf[t]);
+                for (int t = 0; t < 8; ++t) {
+                    const int row = 16 * i + 8 * hf + t;
+                    const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(&sm.rq[st][row * 128 + c0]);
+                    const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(&sm.rk[st][row * 128 + c0]);
+                    const float k0 = bf(k2.x), k1 = bf(k2.y);
+                    *reinterpret_cast<uint32_t *>(&sm.qm[row * kLdOp + c0]) = pack_bf16(bf(q2.x) * rf[0][t], bf(q2.y) * rf[1][t]);
+                    *reinterpret_cast<uint32_t *>(&sm.krm[row * kLdOp + c0]) = pack_bf16(k0 * rf[0][t], k1 * rf[1][t]);
+                    *reinterpret_cast<uint32_t *>(&sm.kcm[row * kLdOp + c0]) = pack_bf16(k0 * cf[0][t], k1 * cf[1][t]);
                 }
             }
         }
@@ -253,18 +289,21 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         __syncthreads();
         // ---- chunk-level factors per channel
         if (tid < 128) {
+            float dblk[NB];   // decay over each 16-token block
+#pragma unroll
+            for (int i = 0; i < NB; ++i) dblk[i] = sm.p7[i * 128 + tid] * sm.r15[i * 128 + tid];
             float E = 1.f;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
                 sm.em[i * 128 + tid] = E * sm.p7[i * 128 + tid];
-                E *= sm.dblk[i * 128 + tid];
+                E *= dblk[i];
             }
             sm.gam[tid] = E;
             float F = 1.f;
 #pragma unroll
             for (int i = NB - 1; i >= 0; --i) {
                 sm.fm[i * 128 + tid] = sm.r15[i * 128 + tid] * F;
-                F *= sm.dblk[i * 128 + tid];
+                F *= dblk[i];
             }
 #pragma unroll
             for (int i = 1; i < NB; ++i) {

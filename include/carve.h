@@ -129,8 +129,9 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
  * Arguments, layouts, results and errors are those of carve_bwd.  The scratch is a 4 MiB
  * array inside the library, present on every GPU that loads it until the process exits, so
  * the call allocates nothing.  Limit: carve_bwd_workspace_bytes(d) <= 4 MiB, that is
- * B*H*(dk*rank + rank*dv) floats, or B*H*ceil(T/chunk)*288 floats when the tensor-core
- * kernels run (bf16, dk = dv = 128, rank <= 32); larger problems return
+ * B*H*(dk*rank + rank*dv) floats, or, when the tensor-core kernels run (bf16,
+ * dk = dv = 128, rank <= 32), B*H*NG*288 + ceil(B*NG/64)*H*256*rank floats with
+ * NG = ceil(T/chunk); larger problems return
  * CARVE_ERR_UNSUPPORTED without launching anything.
  * The first call on each device looks up the array's device address (with that device
  * current) and caches it; make that first call before any stream capture begins.
