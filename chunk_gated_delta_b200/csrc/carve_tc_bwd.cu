@@ -170,6 +170,23 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         }
     };
     load_gates(NCC - 1);
+    // the saved record of the next gate chunk and the write logits of the next compute chunk,
+    // loaded one iteration ahead
+    float pm = 0.f, pd = 0.f, pq = 0.f, pz = 0.f, pw = 0.f;
+    auto load_aux = [&](int gc) {
+        const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (384 + R);
+        if (tid < 128) {
+            pm = aux[tid];
+            pd = aux[128 + R + tid];
+            pq = aux[256 + R + tid];
+        }
+        if (tid < R) pz = aux[128 + tid];
+    };
+    auto load_w = [&](int cc) {
+        if (tid < C) pw = a.w_logit[((size_t)b * T + (size_t)cc * C + tid) * H + h];
+    };
+    load_aux((NCC - 1) / CPG);
+    load_w(NCC - 1);
 
     for (int cc = NCC - 1; cc >= 0; --cc) {
         const int t0 = cc * C, gc = cc / CPG;
@@ -177,14 +194,13 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         const bool gate_start = (cc % CPG) == 0;
         const int n = min(L, T - gc * L);
         if (gate_end) {
-            const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (384 + R);
             if (tid < 128) {
-                sm.mvec[tid] = aux[tid];
-                sm.delta[tid] = aux[128 + R + tid];
-                sm.qbar[tid] = aux[256 + R + tid];
+                sm.mvec[tid] = pm;
+                sm.delta[tid] = pd;
+                sm.qbar[tid] = pq;
                 sm.ddelta[tid] = 0.f;
             }
-            if (tid < R) sm.zvec[tid] = aux[128 + tid];
+            if (tid < R) sm.zvec[tid] = pz;
         }
         {   // the carried gradient as a bf16 tile
 #pragma unroll
@@ -261,7 +277,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 *reinterpret_cast<float2 *>(&sm.rfac[row * kLdF + c0]) = make_float2(rf[0][t], rf[1][t]);
             }
         }
-        if (tid < C) sm.wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + t0 + tid) * H + h]);
+        if (tid < C) sm.wv[tid] = sigmoid_f(pw);
         __syncthreads();
         if (tid < 128) {
             float dblk[NB];   // decay over each 16-token block
@@ -879,6 +895,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         if (cc > 0) {
             issue_s0(cc - 1);
             load_gates(cc - 1);
+            load_w(cc - 1);
+            if (gate_start) load_aux((cc - 1) / CPG);   // chunk cc - 1 ends the previous gate chunk
         }
     }
     if (a.dS0) {

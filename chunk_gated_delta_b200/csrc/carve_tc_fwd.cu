@@ -132,6 +132,13 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     if (SM::ST == 1) issue(0, 1);
     uint32_t phase_bits = 0u;   // bit st: parity to wait for on stage st
     float wnext = tid < C ? a.w_logit[((size_t)b * T + tid) * H + h] : 0.f;
+    // mean q of the next gate chunk from the saved record (mode 0 with saving), one chunk ahead
+    auto load_qbar = [&](int gc) {
+        return (a.saved_aux && a.mc_mode == 0 && tid < 128 && gc < NG)
+                   ? a.saved_aux[((size_t)u * NG + gc) * (384 + R) + 256 + R + tid]
+                   : 0.f;
+    };
+    float pqb = load_qbar(0);
 
     for (int cc = 0; cc < NCC; ++cc) {
         const int t0 = cc * C, gc = cc / CPG;
@@ -175,8 +182,9 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         // ---- content signal at a gate-chunk start
         if (first) {
             if (a.mc_mode == 0) {
-                if (tid < 128 && a.saved_aux) {   // written by the chunk-mean prologue
-                    sm.qbar[tid] = a.saved_aux[((size_t)u * NG + gc) * (384 + R) + 256 + R + tid];
+                if (tid < 128 && a.saved_aux) {   // written by the chunk-mean prologue, prefetched
+                    sm.qbar[tid] = pqb;
+                    pqb = load_qbar(gc + 1);
                 } else if (tid < 128) {
                     float acc = 0.f;
                     if (CPG == 1) {
