@@ -350,14 +350,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 __syncwarp();
                 if (lane < 16) {
                     float col[16];
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        float x = (t == lane) ? 1.f : 0.f;
-                        const float w = sm.wv[16 * i + t];
-#pragma unroll
-                        for (int s2 = 0; s2 < t; ++s2) x -= w * sm.akk_d[(16 * i + t) * 17 + s2] * col[s2];
-                        col[t] = x;
-                    }
+                    unit_lower_inverse_column(sm.akk_d + 16 * i * 17, 17, sm.wv + 16 * i, lane, col);
 #pragma unroll
                     for (int t = 0; t < 16; ++t) sm.tii[(i * 16 + t) * 24 + lane] = __float2bfloat16_rn(col[t]);
                 }
@@ -924,9 +917,10 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
         rz[kRedRec][kTcMaxRankBwd];
     const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x, NR = B * NG;
     const int r0 = sl * kRedSlice, r1 = min(NR, r0 + kRedSlice);
-    float acc[kTcMaxRankBwd];
-#pragma unroll
-    for (int x = 0; x < kTcMaxRankBwd; ++x) acc[x] = 0.f;
+    // each thread: a 4x4 tile of dA (rows k = 4 ka + a, columns j = 4 ja + b) and of dB
+    // (rows j = 4 jb + a, columns v = 4 vb + b); the operands of a record are float4 reads
+    const int ka = tid >> 3, ja = tid & 7, jb = tid >> 5, vb = tid & 31;
+    float accA[4][4] = {}, accB[4][4] = {};
     for (int i0 = r0; i0 < r1; i0 += kRedRec) {
         const int nr = min(kRedRec, r1 - i0);
         for (int idx = tid; idx < nr * 64; idx += 256) {   // dDelta and m, four floats per load
@@ -941,32 +935,41 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
                 for (int e = 0; e < 4; ++e) rm[i][4 * (part4 - 32) + e] = r[e];
             }
         }
-        for (int idx = tid; idx < nr * R; idx += 256) {   // dz and z
-            const int i = idx / R, j = idx % R, rec = i0 + i;
+        for (int idx = tid; idx < nr * kTcMaxRankBwd; idx += 256) {   // dz and z (zero beyond R)
+            const int i = idx / kTcMaxRankBwd, j = idx % kTcMaxRankBwd, rec = i0 + i;
             const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
-            gz[i][j] = wsg[(u * NG + gc) * 160 + 128 + j];
-            rz[i][j] = aux[(u * NG + gc) * (384 + R) + 128 + j];
+            gz[i][j] = j < R ? wsg[(u * NG + gc) * 160 + 128 + j] : 0.f;
+            rz[i][j] = j < R ? aux[(u * NG + gc) * (384 + R) + 128 + j] : 0.f;
         }
         __syncthreads();
+        for (int i = 0; i < nr; ++i) {
+            const float4 g4 = *reinterpret_cast<const float4 *>(&gd[i][4 * ka]);
+            const float4 z4 = *reinterpret_cast<const float4 *>(&rz[i][4 * ja]);
+            const float4 y4 = *reinterpret_cast<const float4 *>(&gz[i][4 * jb]);
+            const float4 m4 = *reinterpret_cast<const float4 *>(&rm[i][4 * vb]);
+            const float ga[4] = {g4.x, g4.y, g4.z, g4.w}, za[4] = {z4.x, z4.y, z4.z, z4.w};
+            const float ya[4] = {y4.x, y4.y, y4.z, y4.w}, ma[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-        for (int x = 0; x < kTcMaxRankBwd; ++x) {
-            if (x < R) {
-                const int o = tid + 256 * x;   // outputs 0 .. 256 R - 1
-                if (o < 128 * R) {
-                    const int k = o / R, j = o % R;
-                    for (int i = 0; i < nr; ++i) acc[x] += gd[i][k] * rz[i][j];
-                } else {
-                    const int j = (o - 128 * R) / 128, v = (o - 128 * R) % 128;
-                    for (int i = 0; i < nr; ++i) acc[x] += gz[i][j] * rm[i][v];
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    accA[x][y] += ga[x] * za[y];
+                    accB[x][y] += ya[x] * ma[y];
                 }
-            }
         }
         __syncthreads();
     }
+    // partial sums in output order: dA (k, j) at k R + j, then dB (j, v) at 128 R + 128 j + v
     float *dst = part + ((size_t)sl * H + h) * 256 * R;
 #pragma unroll
-    for (int x = 0; x < kTcMaxRankBwd; ++x)
-        if (x < R) dst[tid + 256 * x] = acc[x];
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+            const int k = 4 * ka + x, j = 4 * ja + y;
+            if (j < R) dst[k * R + j] = accA[x][y];
+            const int j2 = 4 * jb + x, v = 4 * vb + y;
+            if (j2 < R) dst[128 * R + 128 * j2 + v] = accB[x][y];
+        }
 }
 
 __global__ void __launch_bounds__(256) reduce_dAdB_final_kernel(const float *part, float *dA, float *dB, int H,

@@ -39,6 +39,23 @@ __device__ __forceinline__ void mid_reference(const float (&av)[16], const float
     }
 }
 
+// Column c of T = (I + Diag(w) A)^-1 for a strictly lower-triangular 16x16 block A (row t at
+// A + t * lda) and weights w[0..16): x_t = [t == c] - w_t sum_{s<t} A_ts x_s, evaluated
+// right-looking (each x_s, once final, is added into every later row's sum at once), so the
+// dependent chain is 16 steps deep instead of one step per term.
+__device__ __forceinline__ void unit_lower_inverse_column(const float *A, int lda, const float *w, int c,
+                                                          float (&x)[16]) {
+    float acc[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        x[s] = (s == c ? 1.f : 0.f) - w[s] * acc[s];
+#pragma unroll
+        for (int t = s + 1; t < 16; ++t) acc[t] += A[t * lda + s] * x[s];
+    }
+}
+
 // A fragment of the negated operand (sign flip of both bf16 halves)
 __device__ __forceinline__ void negate_frag(uint32_t (&a)[4]) {
 #pragma unroll

@@ -373,14 +373,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                     __syncwarp();
                     if (lane < 16) {   // column `lane` of T_ii = (I + Diag(w) A_ii)^-1
                         float col[16];
-#pragma unroll
-                        for (int t = 0; t < 16; ++t) {
-                            float x = (t == lane) ? 1.f : 0.f;
-                            const float w = sm.wv[16 * i + t];
-#pragma unroll
-                            for (int s2 = 0; s2 < t; ++s2) x -= w * sm.akk_d[(16 * i + t) * 17 + s2] * col[s2];
-                            col[t] = x;
-                        }
+                        unit_lower_inverse_column(sm.akk_d + 16 * i * 17, 17, sm.wv + 16 * i, lane, col);
 #pragma unroll
                         for (int t = 0; t < 16; ++t) sm.tii[(i * 16 + t) * 24 + lane] = __float2bfloat16_rn(col[t]);
                     }
