@@ -44,7 +44,7 @@ struct __align__(16) TcFwdSmem {
     __nv_bfloat16 aqk[C * LDA], mkk[C * LDA];
     __nv_bfloat16 tii[NB * 16 * 24];
     float akk_d[NB * 16 * 17];
-    float p7[NB * 128], r15[NB * 128], em[NB * 128], fm[NB * 128], cij[NPAIR * 128];
+    float p7[NB * 128], r15[NB * 128], fm[NB * 128], cij[NPAIR * 128];
     float gam[128], wv[C], qbar[128], mvec[128], osum[128], mprev[128], zvec[64], delta[128];
     float Ah[128 * kTcMaxRank], Bh[kTcMaxRank * 128];   // the head's low-rank factors
     uint64_t bar[ST];
@@ -295,17 +295,31 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         }
         if (tid < C) sm.wv[tid] = sigmoid_f(wcur);
         __syncthreads();
-        // ---- chunk-level factors per channel
+        // ---- decayed operands Qt = Qm Em, Kt = Krm Em: one (channel, 16-token block) item per
+        //      thread, each forming its own prefix of block decays; chunk-level factors per
+        //      channel alongside
+#pragma unroll
+        for (int x = 0; x < NP; ++x) {
+            const int p = tid + 256 * x, ch = p & 127, i = p >> 7;
+            if (p < 128 * NB) {
+                float E = 1.f;
+                for (int j = 0; j < i; ++j) E *= sm.p7[j * 128 + ch] * sm.r15[j * 128 + ch];
+                const float em = E * sm.p7[i * 128 + ch];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int row = 16 * i + t;
+                    sm.qt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
+                    sm.kt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+                }
+            }
+        }
         if (tid < 128) {
             float dblk[NB];   // decay over each 16-token block
 #pragma unroll
             for (int i = 0; i < NB; ++i) dblk[i] = sm.p7[i * 128 + tid] * sm.r15[i * 128 + tid];
             float E = 1.f;
 #pragma unroll
-            for (int i = 0; i < NB; ++i) {
-                sm.em[i * 128 + tid] = E * sm.p7[i * 128 + tid];
-                E *= dblk[i];
-            }
+            for (int i = 0; i < NB; ++i) E *= dblk[i];
             sm.gam[tid] = E;
             float F = 1.f;
 #pragma unroll
@@ -322,13 +336,6 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                     sm.cij[pair_index(i, j) * 128 + tid] = prod;
                 }
             }
-        }
-        __syncthreads();
-        for (int idx = tid; idx < C * 128; idx += 256) {
-            const int t = idx >> 7, kch = idx & 127;
-            const float f = sm.em[(t >> 4) * 128 + kch];
-            sm.qt[t * kLdOp + kch] = __float2bfloat16_rn(bf(sm.qm[t * kLdOp + kch]) * f);
-            sm.kt[t * kLdOp + kch] = __float2bfloat16_rn(bf(sm.krm[t * kLdOp + kch]) * f);
         }
         __syncthreads();
         // ---- Gram blocks (warp = type x row block); T_ii on the Akk warps
