@@ -79,6 +79,25 @@ __device__ __forceinline__ void load_b_kn(uint32_t (&b)[4], const __nv_bfloat16 
     ldsm_x4_t(b, smem_u32(base + k * ld + n));
 }
 
+// ---- swizzled [rows][128] bf16 tiles (256-byte rows, no padding): the 16-byte chunk c of
+//      row r is stored at chunk c ^ (r & 7), so the eight rows of an 8x8 ldmatrix always hit
+//      eight different bank groups
+__device__ __forceinline__ int swz128(int r, int c) {   // element offset of (row r, column c)
+    return r * 128 + ((((c >> 3) ^ (r & 7))) << 3) + (c & 7);
+}
+
+// load_b_nk on a swizzled [n][k] tile
+__device__ __forceinline__ void load_b_nk_swz(uint32_t (&b)[4], const __nv_bfloat16 *base, int n0, int k0, int lane) {
+    const int n = n0 + (lane & 7) + ((lane >> 4) << 3), k = k0 + ((lane >> 3) & 1) * 8;
+    ldsm_x4(b, smem_u32(base + swz128(n, k)));
+}
+
+// load_b_kn on a swizzled [k][n] tile
+__device__ __forceinline__ void load_b_kn_swz(uint32_t (&b)[4], const __nv_bfloat16 *base, int n0, int k0, int lane) {
+    const int k = k0 + (lane & 7) + (((lane >> 3) & 1) << 3), n = n0 + ((lane >> 4) << 3);
+    ldsm_x4_t(b, smem_u32(base + swz128(k, n)));
+}
+
 // ---- mbarrier + bulk copy (global -> shared through the TMA engine) ------------------------
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));

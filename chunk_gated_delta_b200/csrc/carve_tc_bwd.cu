@@ -40,7 +40,8 @@ struct BwdMaps {
 };
 
 struct __align__(16) TcBwdSmem {
-    __nv_bfloat16 rq[kBC * 128], rk[kBC * 128], rv[kBC * 128], rdo[kBC * 128];  // TMA tiles
+    // TMA tiles; after the gate recompute rq / rk hold the swizzled Qt / Kt of the chunk
+    __nv_bfloat16 rq[kBC * 128], rk[kBC * 128], rv[kBC * 128], rdo[kBC * 128];
     __nv_bfloat16 dop[kBC * kLdOp];
     __nv_bfloat16 qm[kBC * kLdOp], krm[kBC * kLdOp], kcm[kBC * kLdOp];
     __nv_bfloat16 s0b[128 * kLdOp], ds1b[128 * kLdOp];
@@ -298,6 +299,19 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             }
             sm.cij[tid] = sm.r15[tid] * sm.p7[128 + tid];   // e^{Lam_m(1) - Lam_m(0)}
         }
+        {   // decayed operands Kt = Krm Em, Qt = Qm Em into the (now free) raw q / k tiles,
+            // swizzled: one (channel, 16-token block) item per thread, own prefix of decays
+            const int ch = tid & 127, i = tid >> 7;
+            float em = sm.p7[i * 128 + ch];
+            for (int j = 0; j < i; ++j) em *= sm.p7[j * 128 + ch] * sm.r15[j * 128 + ch];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const int row = 16 * i + t;
+                sm.rq[swz128(row, ch)] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
+                sm.rk[swz128(row, ch)] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+            }
+            fence_proxy_async_smem();   // the next chunk's tile copy overwrites these
+        }
         if (!mbar_wait(&sm.bar_s0, phase)) atomicOr(&g_tc_bwd_timeout, 2);
         phase ^= 1u;
         colsum_partial();   // for gamma * dgamma
@@ -308,11 +322,13 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             for (int w = 0; w < 8; ++w) x += sm.xp[w * 128 + tid];
             sm.s0ds[tid] = x;
         }
-        // ---- Gram blocks (warps 0-3: type x row block), T_ii on the Akk warps
-        if (warp < 4) {
-            const int type = warp >> 1, i = warp & 1;
+        // ---- Gram blocks (warps 0-5: one (type, i, j) block each), T_ii on the diagonal Akk warps
+        if (warp < 6) {
+            const int type = warp / 3, blk = warp % 3;
+            const int i = blk == 0 ? 0 : 1, jd = blk == 1 ? 0 : i;   // blocks (0,0), (1,0), (1,1)
             const __nv_bfloat16 *rowop = type ? sm.qm : sm.krm;
-            for (int j = 0; j <= i; ++j) {
+            {
+                const int j = jd;
                 float acc[2][4] = {};
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
@@ -346,7 +362,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                         }
                     }
             }
-            if (type == 0) {
+            if (type == 0 && jd == i) {
                 __syncwarp();
                 if (lane < 16) {
                     float col[16];
@@ -367,12 +383,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bfr[4];
-                load_b_nk(bfr, sm.krm, kLdOp, 16 * np, 16 * ks, lane);
-                const float *f = sm.em + np * 128 + 16 * ks + 2 * c4;
-                bfr[0] = scale_bf16x2(bfr[0], f[0], f[1]);
-                bfr[1] = scale_bf16x2(bfr[1], f[8], f[9]);
-                bfr[2] = scale_bf16x2(bfr[2], f[0], f[1]);
-                bfr[3] = scale_bf16x2(bfr[3], f[8], f[9]);
+                load_b_nk_swz(bfr, sm.rk, 16 * np, 16 * ks, lane);   // Kt
                 mma_bf16(rr[2 * np], af, bfr[0], bfr[1]);
                 mma_bf16(rr[2 * np + 1], af, bfr[2], bfr[3]);
             }
@@ -386,7 +397,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             rr[j][3] = bf(sm.rv[(t + 1) * 128 + v1]) - rr[j][3];
         }
         __syncthreads();
-        if (cc > 0) issue(cc - 1);   // q, k, v and dO of this chunk are no longer read
         // ---- U (blocked WY solve), E = R - Akk U, U -> shared tile
         float ga[4][4];
 #pragma unroll
@@ -561,17 +571,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 #pragma unroll
             for (int np = 0; np < 8; ++np) {
                 uint32_t bq[4], bk[4];
-                load_b_kn(bq, sm.qm, kLdOp, 16 * np, 16 * kt, lane);
-                load_b_kn(bk, sm.krm, kLdOp, 16 * np, 16 * kt, lane);
-                const float f0 = sm.em[kt * 128 + 16 * np + g], f1 = sm.em[kt * 128 + 16 * np + 8 + g];
-                bq[0] = scale_bf16x2(bq[0], f0, f0);
-                bq[1] = scale_bf16x2(bq[1], f0, f0);
-                bq[2] = scale_bf16x2(bq[2], f1, f1);
-                bq[3] = scale_bf16x2(bq[3], f1, f1);
-                bk[0] = scale_bf16x2(bk[0], f0, f0);
-                bk[1] = scale_bf16x2(bk[1], f0, f0);
-                bk[2] = scale_bf16x2(bk[2], f1, f1);
-                bk[3] = scale_bf16x2(bk[3], f1, f1);
+                load_b_kn_swz(bq, sm.rq, 16 * np, 16 * kt, lane);   // Qt
+                load_b_kn_swz(bk, sm.rk, 16 * np, 16 * kt, lane);   // Kt
                 mma_bf16(ds[2 * np], ao, bq[0], bq[1]);
                 mma_bf16(ds[2 * np + 1], ao, bq[2], bq[3]);
                 mma_bf16(ds[2 * np], ar, bk[0], bk[1]);
@@ -579,6 +580,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             }
         }
         __syncthreads();
+        if (cc > 0) issue(cc - 1);   // q, k, v, dO and the Qt / Kt tiles of this chunk are read
         // ---- dAqk = dO U^T (s <= t), dAkk = -dR U^T (s < t): reductions over v, six 16x16 tiles
         if (warp < 6) {
             const int type = warp / 3, blk = warp % 3;

@@ -338,12 +338,18 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             }
         }
         __syncthreads();
-        // ---- Gram blocks (warp = type x row block); T_ii on the Akk warps
-        {
-            const int type = warp >> 2, i = warp & 3;
-            if (i < NB) {
+        // ---- Gram blocks: the NB (NB + 1) / 2 blocks (i, j <= i) of each type dealt round-robin
+        //      over the warps; T_ii after a diagonal Akk block, by the warp that formed it
+        constexpr int NBLK = NB * (NB + 1) / 2;
+        for (int q = warp; q < 2 * NBLK; q += 8) {
+            const int type = q / NBLK, bq = q % NBLK;
+            int i = 0;
+            while ((i + 1) * (i + 2) / 2 <= bq) ++i;
+            const int jd = bq - i * (i + 1) / 2;
+            {
                 const __nv_bfloat16 *rowop = type ? sm.qm : sm.krm;
-                for (int j = 0; j <= i; ++j) {
+                {
+                    const int j = jd;
                     float acc[2][4] = {};
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
@@ -376,7 +382,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                             }
                         }
                 }
-                if (type == 0) {
+                if (type == 0 && jd == i) {
                     __syncwarp();
                     if (lane < 16) {   // column `lane` of T_ii = (I + Diag(w) A_ii)^-1
                         float col[16];
