@@ -53,7 +53,7 @@ struct __align__(16) TcBwdSmem {
     float p7[kBNB * 128], r15[kBNB * 128], em[kBNB * 128], fm[kBNB * 128], cij[128];
     float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], htot[2 * kBNB * 128], pdd[2 * kBNB * 128];
     float bpart[kBNB * 128];
-    float delta[128], ddelta[128], mvec[128], zvec[64], dzv[64], dmv[128], dox[128], vecK[128], qbar[128];
+    float delta[128], ddelta[128], dzv[64], dmv[128], dox[128], qbar[128];
     uint64_t bar, bar_s0;
 };
 
@@ -173,15 +173,13 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     load_gates(NCC - 1);
     // the saved record of the next gate chunk and the write logits of the next compute chunk,
     // loaded one iteration ahead
-    float pm = 0.f, pd = 0.f, pq = 0.f, pz = 0.f, pw = 0.f;
-    auto load_aux = [&](int gc) {
+    float pd = 0.f, pq = 0.f, pw = 0.f;
+    auto load_aux = [&](int gc) {   // Delta and the mean q of a gate chunk
         const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (384 + R);
         if (tid < 128) {
-            pm = aux[tid];
             pd = aux[128 + R + tid];
             pq = aux[256 + R + tid];
         }
-        if (tid < R) pz = aux[128 + tid];
     };
     auto load_w = [&](int cc) {
         if (tid < C) pw = a.w_logit[((size_t)b * T + (size_t)cc * C + tid) * H + h];
@@ -196,12 +194,10 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         const int n = min(L, T - gc * L);
         if (gate_end) {
             if (tid < 128) {
-                sm.mvec[tid] = pm;
                 sm.delta[tid] = pd;
                 sm.qbar[tid] = pq;
                 sm.ddelta[tid] = 0.f;
             }
-            if (tid < R) sm.zvec[tid] = pz;
         }
         {   // the carried gradient as a bf16 tile
 #pragma unroll
@@ -299,19 +295,35 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             }
             sm.cij[tid] = sm.r15[tid] * sm.p7[128 + tid];   // e^{Lam_m(1) - Lam_m(0)}
         }
-        {   // decayed operands Kt = Krm Em, Qt = Qm Em into the (now free) raw q / k tiles,
-            // swizzled: one (channel, 16-token block) item per thread, own prefix of decays
-            const int ch = tid & 127, i = tid >> 7;
-            float em = sm.p7[i * 128 + ch];
-            for (int j = 0; j < i; ++j) em *= sm.p7[j * 128 + ch] * sm.r15[j * 128 + ch];
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const int row = 16 * i + t;
-                sm.rq[swz128(row, ch)] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
-                sm.rk[swz128(row, ch)] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+        // decayed operands Qt = Qm Em, Kt = Krm Em into the (now free) raw q / k tiles, swizzled:
+        // items of 8 channels of one token row, each forming its block's decay prefix
+        for (int it = tid; it < 2 * C * 16; it += 256) {
+            const int tile = it / (C * 16), t = (it >> 4) % C, c8 = it & 15, i = t >> 4;
+            const float4 *p7v = reinterpret_cast<const float4 *>(sm.p7 + i * 128 + 8 * c8);
+            float em[8];
+            {
+                const float4 a0 = p7v[0], a1 = p7v[1];
+                em[0] = a0.x; em[1] = a0.y; em[2] = a0.z; em[3] = a0.w;
+                em[4] = a1.x; em[5] = a1.y; em[6] = a1.z; em[7] = a1.w;
             }
-            fence_proxy_async_smem();   // the next chunk's tile copy overwrites these
+            for (int j = 0; j < i; ++j) {   // times the decay of each earlier block
+                const float4 *pj = reinterpret_cast<const float4 *>(sm.p7 + j * 128 + 8 * c8);
+                const float4 *rj = reinterpret_cast<const float4 *>(sm.r15 + j * 128 + 8 * c8);
+                const float4 p0 = pj[0], p1 = pj[1], r0 = rj[0], r1 = rj[1];
+                em[0] *= p0.x * r0.x; em[1] *= p0.y * r0.y; em[2] *= p0.z * r0.z; em[3] *= p0.w * r0.w;
+                em[4] *= p1.x * r1.x; em[5] *= p1.y * r1.y; em[6] *= p1.z * r1.z; em[7] *= p1.w * r1.w;
+            }
+            const __nv_bfloat16 *src = (tile ? sm.krm : sm.qm) + t * kLdOp + 8 * c8;
+            const uint4 x = *reinterpret_cast<const uint4 *>(src);
+            const __nv_bfloat162 *xv = reinterpret_cast<const __nv_bfloat162 *>(&x);
+            uint4 y;
+            uint32_t *yv = reinterpret_cast<uint32_t *>(&y);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) yv[e] = pack_bf16(bf(xv[e].x) * em[2 * e], bf(xv[e].y) * em[2 * e + 1]);
+            __nv_bfloat16 *dst = tile ? sm.rk : sm.rq;
+            *reinterpret_cast<uint4 *>(dst + t * 128 + ((c8 ^ (t & 7)) << 3)) = y;
         }
+        fence_proxy_async_smem();   // the next chunk's tile copy overwrites these
         if (!mbar_wait(&sm.bar_s0, phase)) atomicOr(&g_tc_bwd_timeout, 2);
         phase ^= 1u;
         colsum_partial();   // for gamma * dgamma
@@ -629,22 +641,27 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     uint32_t bs[4], bd[4];
                     load_b_kn(bs, sm.s0b, kLdOp, n0, 16 * ks, lane);
                     load_b_kn(bd, sm.ds1b, kLdOp, n0, 16 * ks, lane);
-                    const float e0 = sm.em[ib2 * 128 + n0 + g], e1 = sm.em[ib2 * 128 + n0 + 8 + g];
-                    const float f0 = sm.fm[ib2 * 128 + n0 + g], f1 = sm.fm[ib2 * 128 + n0 + 8 + g];
-                    bs[0] = scale_bf16x2(bs[0], e0, e0);
-                    bs[1] = scale_bf16x2(bs[1], e0, e0);
-                    bs[2] = scale_bf16x2(bs[2], e1, e1);
-                    bs[3] = scale_bf16x2(bs[3], e1, e1);
-                    bd[0] = scale_bf16x2(bd[0], f0, f0);
-                    bd[1] = scale_bf16x2(bd[1], f0, f0);
-                    bd[2] = scale_bf16x2(bd[2], f1, f1);
-                    bd[3] = scale_bf16x2(bd[3], f1, f1);
                     mma_bf16(gq[2 * np2], ao, bs[0], bs[1]);
                     mma_bf16(gq[2 * np2 + 1], ao, bs[2], bs[3]);
                     mma_bf16(gkr[2 * np2], ar, bs[0], bs[1]);
                     mma_bf16(gkr[2 * np2 + 1], ar, bs[2], bs[3]);
                     mma_bf16(gkb[2 * np2], au, bd[0], bd[1]);
                     mma_bf16(gkb[2 * np2 + 1], au, bd[2], bd[3]);
+                }
+            }
+            // the decays of S0 (Em) and dS1 (Fm) scale output columns, fixed for this token
+            // block: applied to the fp32 sums
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int ch = ch0 + 8 * nt + 2 * c4;
+                const float2 e2 = *reinterpret_cast<const float2 *>(sm.em + ib2 * 128 + ch);
+                const float2 f2 = *reinterpret_cast<const float2 *>(sm.fm + ib2 * 128 + ch);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float ev = (e & 1) ? e2.y : e2.x, fv = (e & 1) ? f2.y : f2.x;
+                    gq[nt][e] *= ev;
+                    gkr[nt][e] *= ev;
+                    gkb[nt][e] *= fv;
                 }
             }
             // Gram blocks: rows t of this block against columns s of block j (row side) and
