@@ -758,6 +758,10 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 }
         }
         __syncthreads();
+        // the S0 tile is read for the last time above unless this chunk closes a gate chunk
+        // with the boundary-state readout: the next chunk's state can come in now
+        const bool s0_early = !(gate_start && a.mc_mode == 0);
+        if (cc > 0 && s0_early) issue_s0(cc - 1);
         // ---- reverse cumulative sum of dLam within the chunk, gate gradients.  Half-block
         //      totals first (the chunk's last-token term xl joins the last half), then each
         //      thread scans its 8 tokens from the total of everything after them.
@@ -829,6 +833,10 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 *reinterpret_cast<float2 *>(&sm.rfac[row * kLdF + c0]) = make_float2(db[0], db[1]);
             }
             *reinterpret_cast<float2 *>(&sm.pdd[hb * 128 + c0]) = make_float2(pdd[0], pdd[1]);
+        }
+        if (cc > 0) {   // the gate logits were read for the last time in the scan above
+            load_gates(cc - 1);
+            load_w(cc - 1);
         }
         __syncthreads();
         if (tid < 128) {
@@ -905,9 +913,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         }
         __syncthreads();
         if (cc > 0) {
-            issue_s0(cc - 1);
-            load_gates(cc - 1);
-            load_w(cc - 1);
+            if (!s0_early) issue_s0(cc - 1);
             if (gate_start) load_aux((cc - 1) / CPG);   // chunk cc - 1 ends the previous gate chunk
         }
     }
