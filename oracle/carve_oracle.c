@@ -12,11 +12,14 @@
  *                                                   CARVE paperdance abstract)
  *           | (1/n_{c-1}) sum_{t in c-1} o_t      (mc_mode 1: previous chunk's mean output;
  *                                                   CARVE blog, section 2.2; m_0 = m_prev_in or 0)
- *     Delta = A (B m_c)                            (U_b = A.B, low rank; blog section 2.2)
+ *     z_c   = B m_c ;  Delta = A z_c                (U_b = A.B, low rank; blog section 2.2)
+ *     dw_c  = Aw . z_c  (optional content term of the write gate: the same zero-initialised
+ *                       low-rank projection of m_c yields the erase bias and the write bias,
+ *                       blog section 2.2, Figure 1; dw_c = 0 when Aw is absent)
  *     for t in c:
  *       g_t = exp(-softplus(g_logit_t))           key-axis decay (blog section 2.3, decay gate)
  *       b_t = sigmoid(bx_t + Delta)               key-axis content-aware erase (blog section 2.2)
- *       a_t = g_t * b_t ;  w_t = sigmoid(w_logit_t)  scalar write per head (blog section 2.3)
+ *       a_t = g_t * b_t ;  w_t = sigmoid(w_logit_t + dw_c)  scalar write per head (blog 2.3)
  *       P   = S Diag(a_t) ; e_t = v_t - P k_t ; S = P + w_t e_t k_t^T      (blog section 2.1)
  *       o_t = S q_t
  *
@@ -30,7 +33,7 @@
  *
  * Layouts (all contiguous, row-major):
  *   q, k, g_logit, bx : [B,T,H,K]    v, o : [B,T,H,V]    w_logit : [B,T,H]
- *   A : [H,K,R]   Bm : [H,R,V]   S0, S_final, dS : [B,H,V,K]   m vectors : [B,H,V]
+ *   A : [H,K,R]   Bm : [H,R,V]   Aw : [H,R]   S0, S_final, dS : [B,H,V,K]   m vectors : [B,H,V]
  * Units (b,h) are independent and run under OpenMP; dA and dB are summed over b in a
  * fixed order afterwards, so results do not depend on the thread count.
  */
@@ -51,14 +54,22 @@ static double sigm(double x) { return 1.0 / (1.0 + exp(-x)); }
 
 /* gate activations of one token (b,t,h): a, g, bgate over K; returns w */
 static double gates(const orc_dims *d, int b, int t, int h, const double *gl, const double *bx,
-                    const double *wl, const double *delta, double *a, double *g, double *bg) {
+                    const double *wl, const double *delta, double dwc, double *a, double *g, double *bg) {
     for (int i = 0; i < d->K; ++i) {
         size_t ix = IX_TK(d, b, t, h, i, d->K);
         g[i] = exp(-softplus(gl[ix]));
         bg[i] = d->content_off ? sigm(bx[ix]) : sigm(bx[ix] + delta[i]);
         a[i] = g[i] * bg[i];
     }
-    return sigm(wl[((size_t)b * d->T + t) * d->H + h]);
+    return sigm(wl[((size_t)b * d->T + t) * d->H + h] + dwc);
+}
+
+/* dw = Aw[h] . z (0 without the write-gate content term) */
+static double write_bias(const orc_dims *d, int h, const double *Aw, const double *z) {
+    if (!Aw || d->content_off) return 0.0;
+    double s = 0.0;
+    for (int j = 0; j < d->R; ++j) s += Aw[(size_t)h * d->R + j] * z[j];
+    return s;
 }
 
 /* Delta = A (B m); z = B m is returned too */
@@ -103,10 +114,10 @@ static int check_dims(const orc_dims *d) {
     return 0;
 }
 
-/* Forward.  S0, m_prev_in, m_prev_out may be NULL.  Returns 0 or -1 on bad dims. */
+/* Forward.  Aw, S0, m_prev_in, m_prev_out may be NULL.  Returns 0 or -1 on bad dims. */
 int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v,
             const double *gl, const double *bx, const double *wl, const double *A,
-            const double *Bm, const double *S0, const double *m_prev_in, double *o,
+            const double *Bm, const double *Aw, const double *S0, const double *m_prev_in, double *o,
             double *S_final, double *m_prev_out) {
     if (check_dims(d)) return -1;
     const int K = d->K, V = d->V, R = d->R, T = d->T, L = d->L, H = d->H;
@@ -141,9 +152,10 @@ int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v
                 }
                 content_delta(d, h, A, Bm, m, z, delta);
             }
+            const double dwc = write_bias(d, h, Aw, z);
             for (int j = 0; j < V; ++j) osum[j] = 0.0;
             for (int t = t0; t < t1; ++t) {
-                double w = gates(d, b, t, h, gl, bx, wl, delta, a, g, bg);
+                double w = gates(d, b, t, h, gl, bx, wl, delta, dwc, a, g, bg);
                 gather_tok(d, q, b, t, h, K, qt);
                 gather_tok(d, k, b, t, h, K, kt);
                 gather_tok(d, v, b, t, h, V, vt);
@@ -164,14 +176,15 @@ int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v
 /*
  * Backward by back-propagation through time.  Given dO (and optionally dS_final, and
  * dm_prev_out in mc_mode 1), returns the gradient of sum(dO*o) + sum(dS_final*S_final)
- * + sum(dm_prev_out*m_prev_out) with respect to every input.  dA, dB are overwritten.
+ * + sum(dm_prev_out*m_prev_out) with respect to every input.  dA, dB (and dAw when given)
+ * are overwritten; Aw and dAw may be NULL.
  * dS0 and dm_prev_in may be NULL.
  */
 int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v,
             const double *gl, const double *bx, const double *wl, const double *A,
-            const double *Bm, const double *S0, const double *m_prev_in, const double *dO,
+            const double *Bm, const double *Aw, const double *S0, const double *m_prev_in, const double *dO,
             const double *dS_final, const double *dm_prev_out, double *dq, double *dk,
-            double *dv, double *dgl, double *dbx, double *dwl, double *dA, double *dB,
+            double *dv, double *dgl, double *dbx, double *dwl, double *dA, double *dB, double *dAw,
             double *dS0, double *dm_prev_in) {
     if (check_dims(d)) return -1;
     const int K = d->K, V = d->V, R = d->R, T = d->T, L = d->L, H = d->H;
@@ -180,6 +193,7 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
     const size_t VK = (size_t)V * K;
     double *dA_u = calloc((size_t)units * K * R, sizeof(double));
     double *dB_u = calloc((size_t)units * R * V, sizeof(double));
+    double *dAw_u = calloc((size_t)units * R, sizeof(double));
 #pragma omp parallel for schedule(dynamic, 1)
     for (int u = 0; u < units; ++u) {
         const int b = u / H, h = u % H;
@@ -199,7 +213,7 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
         double *dox = calloc(V, sizeof(double)), *dot = calloc(V, sizeof(double));
         double *de = calloc(V, sizeof(double)), *dd = calloc(K, sizeof(double));
         double *dz = calloc(R, sizeof(double)), *dm = calloc(V, sizeof(double)), *tmp = calloc(K, sizeof(double));
-        double *dAu = dA_u + (size_t)u * K * R, *dBu = dB_u + (size_t)u * R * V;
+        double *dAu = dA_u + (size_t)u * K * R, *dBu = dB_u + (size_t)u * R * V, *dAwu = dAw_u + (size_t)u * R;
 
         /* forward pass: chunk-start states and content signals */
         if (S0) memcpy(S, S0 + (size_t)u * VK, sizeof(double) * VK);
@@ -225,8 +239,9 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                 content_delta(d, h, A, Bm, m, zc + (size_t)c * R, dc + (size_t)c * K);
             }
             for (int j = 0; j < V; ++j) osum[j] = 0.0;
+            const double dwc = write_bias(d, h, Aw, zc + (size_t)c * R);
             for (int t = t0; t < t1; ++t) {
-                double w = gates(d, b, t, h, gl, bx, wl, dc + (size_t)c * K, at, gt, bt);
+                double w = gates(d, b, t, h, gl, bx, wl, dc + (size_t)c * K, dwc, at, gt, bt);
                 gather_tok(d, q, b, t, h, K, qt);
                 gather_tok(d, k, b, t, h, K, kt);
                 gather_tok(d, v, b, t, h, V, vt);
@@ -246,11 +261,13 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
         for (int c = N - 1; c >= 0; --c) {
             const int t0 = c * L, t1 = t0 + L < T ? t0 + L : T, n = t1 - t0;
             const double *delta = dc + (size_t)c * K;
+            const double dwc = write_bias(d, h, Aw, zc + (size_t)c * R);
+            double ddw = 0.0;   /* gradient of dw_c: sum of the chunk's write-logit gradients */
             /* recompute the chunk's per-token states St[0..n] and gates */
             memcpy(St, Sb + (size_t)c * VK, sizeof(double) * VK);
             for (int tau = 0; tau < n; ++tau) {
                 const int t = t0 + tau;
-                wt[tau] = gates(d, b, t, h, gl, bx, wl, delta, at + (size_t)tau * K,
+                wt[tau] = gates(d, b, t, h, gl, bx, wl, delta, dwc, at + (size_t)tau * K,
                                 gt + (size_t)tau * K, bt + (size_t)tau * K);
                 memcpy(St + (size_t)(tau + 1) * VK, St + (size_t)tau * VK, sizeof(double) * VK);
                 gather_tok(d, q, b, t, h, K, qt);
@@ -309,6 +326,7 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                 for (int j = 0; j < V; ++j)
                     for (int i = 0; i < K; ++i) dS[(size_t)j * K + i] = dP[(size_t)j * K + i] * a[i];
                 dwl[((size_t)b * T + t) * H + h] = dw * w * (1.0 - w);
+                ddw += dw * w * (1.0 - w);
             }
             /* chunk start: Delta = A z, z = B m */
             for (int j = 0; j < V; ++j) dox[j] = 0.0;
@@ -317,8 +335,11 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                 for (int j = 0; j < R; ++j) {
                     double s = 0.0;
                     for (int i = 0; i < K; ++i) s += A[((size_t)h * K + i) * R + j] * dd[i];
+                    if (Aw) s += Aw[(size_t)h * R + j] * ddw;   /* dw_c = Aw . z */
                     dz[j] = s;
                 }
+                if (Aw)
+                    for (int j = 0; j < R; ++j) dAwu[j] += ddw * z[j];
                 for (int i = 0; i < K; ++i)
                     for (int j = 0; j < R; ++j) dAu[(size_t)i * R + j] += dd[i] * z[j];
                 for (int vv = 0; vv < V; ++vv) {
@@ -357,12 +378,15 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
     /* dA, dB: per-head sums over the batch in a fixed order */
     memset(dA, 0, sizeof(double) * (size_t)H * K * R);
     memset(dB, 0, sizeof(double) * (size_t)H * R * V);
+    if (dAw) memset(dAw, 0, sizeof(double) * (size_t)H * R);
     for (int u = 0; u < units; ++u) {
         const int h = u % H;
         for (size_t x = 0; x < (size_t)K * R; ++x) dA[(size_t)h * K * R + x] += dA_u[(size_t)u * K * R + x];
         for (size_t x = 0; x < (size_t)R * V; ++x) dB[(size_t)h * R * V + x] += dB_u[(size_t)u * R * V + x];
+        if (dAw)
+            for (int j = 0; j < R; ++j) dAw[(size_t)h * R + j] += dAw_u[(size_t)u * R + j];
     }
-    free(dA_u); free(dB_u);
+    free(dA_u); free(dB_u); free(dAw_u);
     return 0;
 }
 
@@ -374,12 +398,12 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
  *   mc_mode 1: the content signal is the mean output of the previous complete block of
  *              L tokens.  mstate [B,H,2,V] holds (running sum of o in the current block,
  *              mean of the previous block); pos [B,H] counts tokens consumed.
- * Inputs q, k, g_logit, bx: [B,H,K]; v: [B,H,V]; w_logit: [B,H]; S [B,H,V,K] in/out;
- * o: [B,H,V].
+ * Inputs q, k, g_logit, bx: [B,H,K]; v: [B,H,V]; w_logit: [B,H]; Aw [H,R] or NULL;
+ * S [B,H,V,K] in/out; o: [B,H,V].
  */
 int orc_step(const orc_dims *d, const double *q, const double *k, const double *v,
              const double *gl, const double *bx, const double *wl, const double *A,
-             const double *Bm, double *S, double *mstate, int *pos, double *o) {
+             const double *Bm, const double *Aw, double *S, double *mstate, int *pos, double *o) {
     if (check_dims(d)) return -1;
     const int K = d->K, V = d->V, R = d->R, H = d->H, L = d->L;
     const int units = d->B * H;
@@ -411,7 +435,7 @@ int orc_step(const orc_dims *d, const double *q, const double *k, const double *
             const double bb = d->content_off ? sigm(bx[(size_t)u * K + i]) : sigm(bx[(size_t)u * K + i] + delta[i]);
             a[i] = g * bb;
         }
-        const double w = sigm(wl[u]);
+        const double w = sigm(wl[u] + write_bias(d, h, Aw, z));
         token_update(d, Su, a, w, ku, v + (size_t)u * V, qu, e, o + (size_t)u * V);
         if (d->mc_mode == 1) {
             double *msum = mstate + (size_t)u * 2 * V;

@@ -67,19 +67,21 @@ def _content(S, qbar, mprev, A, Bm, mc_mode):
     return m, z, A @ z
 
 
-def fwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, mc_mode=0):
+def fwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, mc_mode=0, aw=None):
     """One (batch, head) unit: q, k, gl, bx [T,K]; v [T,V]; wl [T]; A [K,R]; Bm [R,V];
-    S0 [V,K]; m_prev [V].  Returns o [T,V], S_final, m_prev_out."""
+    S0 [V,K]; m_prev [V]; aw [R] or None (the write gate's content term: the chunk's write
+    logits are shifted by aw . z).  Returns o [T,V], S_final, m_prev_out."""
     T = q.shape[0]
     S = S0.copy()
     mprev = m_prev.copy()
     o = np.zeros((T, v.shape[1]))
     for t0 in range(0, T, L):
         t1 = min(t0 + L, T)
-        _, _, delta = _content(S, q[t0:t1].mean(axis=0), mprev, A, Bm, mc_mode)
+        _, z, delta = _content(S, q[t0:t1].mean(axis=0), mprev, A, Bm, mc_mode)
+        wls = wl + (0.0 if aw is None else float(aw @ z))
         for s0 in range(t0, t1, Lc):
             s1 = min(s0 + Lc, t1)
-            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wl[s0:s1], delta)
+            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta)
             o[s0:s1] = O
         mprev = o[t0:t1].mean(axis=0)
     return o, S, mprev
@@ -123,29 +125,32 @@ def _sub_bwd(S0, q, k, gl, it, dO, dS1):
     return dq, dk, dv, dgl, dbeta, dwl, dS0
 
 
-def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_prev_out, mc_mode=0):
+def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_prev_out, mc_mode=0, aw=None):
     """Reverse sweep over chunks (and compute sub-chunks inside each chunk).
-    Returns dq, dk, dv, dgl, dbx, dwl, dA, dB, dS0, dm_prev_in for one unit."""
+    Returns dq, dk, dv, dgl, dbx, dwl, dA, dB, dS0, dm_prev_in, daw for one unit."""
     T, K = q.shape
     V = v.shape[1]
     # forward: chunk-start states, content signals
     S = S0.copy()
     mprev = m_prev.copy()
-    starts, ms, zs, deltas, qbars = [], [], [], [], []
+    starts, ms, zs, deltas, qbars, wlss = [], [], [], [], [], []
     o = np.zeros((T, V))
     for t0 in range(0, T, L):
         t1 = min(t0 + L, T)
         qbar = q[t0:t1].mean(axis=0)
         m, z, delta = _content(S, qbar, mprev, A, Bm, mc_mode)
+        wls = wl + (0.0 if aw is None else float(aw @ z))
         starts.append(S.copy()); ms.append(m); zs.append(z); deltas.append(delta); qbars.append(qbar)
+        wlss.append(wls)
         for s0 in range(t0, t1, Lc):
             s1 = min(s0 + Lc, t1)
-            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wl[s0:s1], delta)
+            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta)
             o[s0:s1] = O
         mprev = o[t0:t1].mean(axis=0)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     dgl, dbx, dwl = np.zeros_like(gl), np.zeros_like(bx), np.zeros_like(wl)
     dA, dB = np.zeros_like(A), np.zeros_like(Bm)
+    daw = np.zeros(A.shape[1])
     dS = dS_final.copy()
     dO = dO.copy()
     nch = len(starts)
@@ -155,14 +160,14 @@ def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_pre
     dm_prev_in = np.zeros(V)
     for c in range(nch - 1, -1, -1):
         t0, t1 = c * L, min(c * L + L, T)
-        delta = deltas[c]
+        delta, wls = deltas[c], wlss[c]
         subs = list(range(t0, t1, Lc))
         sub_states, its = [], []
         Sx = starts[c]
         for s0 in subs:
             s1 = min(s0 + Lc, t1)
             sub_states.append(Sx)
-            _, Sx, it = _sub_fwd(Sx, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wl[s0:s1], delta)
+            _, Sx, it = _sub_fwd(Sx, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta)
             its.append(it)
         ddelta = np.zeros(K)
         for j in range(len(subs) - 1, -1, -1):
@@ -172,6 +177,10 @@ def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_pre
             dq[s0:s1], dk[s0:s1], dv[s0:s1], dgl[s0:s1], dbx[s0:s1], dwl[s0:s1], dS = r
             ddelta += r[4].sum(axis=0)
         dz = A.T @ ddelta
+        if aw is not None:   # the chunk's write logits were shifted by aw . z
+            ddw = dwl[t0:t1].sum()
+            dz = dz + aw * ddw
+            daw += ddw * zs[c]
         dA += np.outer(ddelta, zs[c])
         dm = Bm.T @ dz
         dB += np.outer(dz, ms[c])
@@ -182,7 +191,7 @@ def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_pre
             dO[(c - 1) * L:c * L] += dm[None, :] / L
         else:
             dm_prev_in = dm
-    return dq, dk, dv, dgl, dbx, dwl, dA, dB, dS, dm_prev_in
+    return dq, dk, dv, dgl, dbx, dwl, dA, dB, dS, dm_prev_in, daw
 
 
 def _units(inp):
@@ -204,7 +213,8 @@ def fwd(inp, L, Lc=None, mc_mode=0, S0=None, m_prev=None):
         mp = np.zeros(V) if m_prev is None else np.asarray(m_prev[b, h], dtype=np.float64)
         o[b, :, h], Sf[b, h], mo[b, h] = fwd_unit(
             f["q"][b, :, h], f["k"][b, :, h], f["v"][b, :, h], f["g_logit"][b, :, h], f["bx"][b, :, h],
-            f["w_logit"][b, :, h], f["A"][h], f["B"][h], s0, mp, L, Lc, mc_mode)
+            f["w_logit"][b, :, h], f["A"][h], f["B"][h], s0, mp, L, Lc, mc_mode,
+            None if "Aw" not in f else f["Aw"][h])
     return dict(o=o, S_final=Sf, m_prev_out=mo)
 
 
@@ -215,8 +225,8 @@ def bwd(inp, L, dO, Lc=None, mc_mode=0, S0=None, m_prev=None, dS_final=None, dm_
     f = {k: np.asarray(inp[k], dtype=np.float64) for k in inp}
     out = dict(dq=np.zeros((B, T, H, K)), dk=np.zeros((B, T, H, K)), dv=np.zeros((B, T, H, V)),
                dg_logit=np.zeros((B, T, H, K)), dbx=np.zeros((B, T, H, K)), dw_logit=np.zeros((B, T, H)),
-               dA=np.zeros_like(f["A"]), dB=np.zeros_like(f["B"]), dS0=np.zeros((B, H, V, K)),
-               dm_prev_in=np.zeros((B, H, V)))
+               dA=np.zeros_like(f["A"]), dB=np.zeros_like(f["B"]), dAw=np.zeros(f["A"].shape[::2]),
+               dS0=np.zeros((B, H, V, K)), dm_prev_in=np.zeros((B, H, V)))
     for b, h in _units(inp):
         s0 = np.zeros((V, K)) if S0 is None else np.asarray(S0[b, h], dtype=np.float64)
         mp = np.zeros(V) if m_prev is None else np.asarray(m_prev[b, h], dtype=np.float64)
@@ -224,11 +234,13 @@ def bwd(inp, L, dO, Lc=None, mc_mode=0, S0=None, m_prev=None, dS_final=None, dm_
         dmo = np.zeros(V) if dm_prev_out is None else np.asarray(dm_prev_out[b, h], dtype=np.float64)
         r = bwd_unit(f["q"][b, :, h], f["k"][b, :, h], f["v"][b, :, h], f["g_logit"][b, :, h],
                      f["bx"][b, :, h], f["w_logit"][b, :, h], f["A"][h], f["B"][h], s0, mp, L, Lc,
-                     np.asarray(dO[b, :, h], dtype=np.float64), dsf, dmo, mc_mode)
+                     np.asarray(dO[b, :, h], dtype=np.float64), dsf, dmo, mc_mode,
+                     None if "Aw" not in f else f["Aw"][h])
         (out["dq"][b, :, h], out["dk"][b, :, h], out["dv"][b, :, h], out["dg_logit"][b, :, h],
          out["dbx"][b, :, h], out["dw_logit"][b, :, h]) = r[:6]
         out["dA"][h] += r[6]
         out["dB"][h] += r[7]
         out["dS0"][b, h] = r[8]
         out["dm_prev_in"][b, h] = r[9]
+        out["dAw"][h] += r[10]
     return out

@@ -44,6 +44,13 @@ MUTANTS = {
     "bwd_dwl_no_sigmoid_prime": ("= dw * w * (1.0 - w);", "= dw;"),
     # backward: prediction term of dk dropped
     "bwd_dk_missing_prediction": ("dkt[i] -= p * de[j];", "(void)p;"),
+    # write gate's content term ignored in the forward
+    "write_bias_ignored": ("return sigm(wl[((size_t)b * d->T + t) * d->H + h] + dwc);",
+                           "return sigm(wl[((size_t)b * d->T + t) * d->H + h]);"),
+    # write gate's content term built from the wrong component of z
+    "write_bias_wrong_z": ("s += Aw[(size_t)h * d->R + j] * z[j];", "s += Aw[(size_t)h * d->R + j] * z[0];"),
+    # backward: the write bias's gradient not fed back into dz
+    "bwd_write_bias_not_in_dz": ("if (Aw) s += Aw[(size_t)h * R + j] * ddw;", "(void)ddw;"),
 }
 
 # the mutant that changes nothing observable must survive: it guards the harness itself
@@ -56,8 +63,10 @@ PIN_TESTS = [
     pins.test_write_zero_is_pure_decay,
     pins.test_exact_write_with_unit_keys,
     pins.test_orthogonal_keys_give_linear_attention,
-    lambda: pins.test_content_signal_closed_form(0),
-    lambda: pins.test_content_signal_closed_form(1),
+    lambda: pins.test_content_signal_closed_form(0, False),
+    lambda: pins.test_content_signal_closed_form(1, False),
+    lambda: pins.test_content_signal_closed_form(0, True),
+    lambda: pins.test_content_signal_closed_form(1, True),
     pins.test_state_norm_bound_every_token,
     lambda: pins.test_gradients_central_differences(0),
     lambda: pins.test_gradients_central_differences(1),

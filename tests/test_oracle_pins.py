@@ -162,6 +162,27 @@ def test_zero_projection_is_bit_identical(mc_mode, zero):
     assert np.array_equal(r["S_final"], base["S_final"])
 
 
+@pytest.mark.parametrize("mc_mode", [0, 1])
+def test_zero_write_projection_is_bit_identical(mc_mode):
+    """Aw = 0 (zero-initialised, like U_b): sigmoid(w_logit + 0) = sigmoid(w_logit) exactly, so
+    the forward and every backward output equal those without the write term, bit for bit,
+    and d(Aw) is still the true gradient (compared against finite differences elsewhere)."""
+    w, d = tiny(T=13, L=4)
+    d["A"] *= 30.0
+    d["B"] *= 30.0
+    S0 = I.make_state(w, 0.2).astype(np.float64)
+    dO = I.normal(8, 1, (w.B, w.T, w.H, w.V))
+    dz = dict(d, Aw=np.zeros((w.H, w.R)))
+    r, base = oracle.fwd(dz, L=4, mc_mode=mc_mode, S0=S0), oracle.fwd(d, L=4, mc_mode=mc_mode, S0=S0)
+    for key in r:
+        assert np.array_equal(r[key], base[key]), key
+    g, gb = oracle.bwd(dz, 4, dO, mc_mode=mc_mode, S0=S0), oracle.bwd(d, 4, dO, mc_mode=mc_mode, S0=S0)
+    for key in g:
+        if key != "dAw":
+            assert np.array_equal(g[key], gb[key]), key
+    assert np.all(gb["dAw"] == 0.0) and np.abs(g["dAw"]).max() > 0.0
+
+
 def test_chunk_size_enters_only_through_the_content_signal():
     """With U_b = 0 the gate grouping is irrelevant: every L gives the same bits."""
     w, d = tiny(T=16)
@@ -179,16 +200,21 @@ def test_chunk_size_enters_only_through_the_content_signal():
 # 4. The content signal in closed form (which state, which mean, which factor order)
 # ---------------------------------------------------------------------------------------
 @pytest.mark.parametrize("mc_mode", [0, 1])
-def test_content_signal_closed_form(mc_mode):
+@pytest.mark.parametrize("write_term", [False, True])
+def test_content_signal_closed_form(mc_mode, write_term):
     """Chunk 0 (L = 4 tokens) with a == 1, w == 1 and keys e_0..e_3 gives
     S_[0] = sum_t v_t e_t^T and o_t = sum_{s<=t} v_s q_t[s] in closed form.  The first token
     of chunk 1 (ragged: 3 tokens) then sees m_1 = S_[0] mean(q over chunk 1) (mode 0:
     boundary state, mean over the CURRENT chunk incl. later tokens; paperdance abstract)
-    or m_1 = mean(o over chunk 0) (mode 1; CARVE blog section 2.2), Delta = A (B m_1)."""
+    or m_1 = mean(o over chunk 0) (mode 1; CARVE blog section 2.2), Delta = A (B m_1), and
+    with the write gate's content term w = sigmoid(w_logit + Aw . (B m_1)) (the same
+    low-rank projection of m_1 gives the erase and the write bias, blog section 2.2)."""
     K = V = 5
     w, d = tiny(B=1, H=1, T=7, K=K, V=V, R=2, L=4)
     d["A"] *= 60.0
     d["B"] *= 60.0
+    if write_term:
+        d["Aw"] = np.array([[25.0, -40.0]])
     d["w_logit"][:, :4] = BIG
     d["g_logit"][:, :4] = -BIG
     d["bx"][:, :4] = BIG
@@ -200,10 +226,13 @@ def test_content_signal_closed_form(mc_mode):
     o0 = np.array([sum(vv[s] * qq[t][s] for s in range(t + 1)) for t in range(4)])
     assert np.abs(r["o"][0, :4, 0] - o0).max() < 1e-13
     m = S0 @ qq[4:7].mean(axis=0) if mc_mode == 0 else o0.mean(axis=0)
-    delta = d["A"][0] @ (d["B"][0] @ m)
+    z = d["B"][0] @ m
+    delta = d["A"][0] @ z
     k, t = d["k"][0, 4, 0], 4
     a = sig(-d["g_logit"][0, t, 0]) * sig(d["bx"][0, t, 0] + delta)
-    wt = sig(d["w_logit"][0, t, 0])
+    wt = sig(d["w_logit"][0, t, 0] + (d["Aw"][0] @ z if write_term else 0.0))
+    if write_term:   # the term matters in this construction
+        assert abs(wt - sig(d["w_logit"][0, t, 0])) > 1e-3
     e = vv[t] - S0 @ (a * k)
     S1 = S0 * a[None, :] + wt * np.outer(e, k)
     assert np.abs(r["o"][0, 4, 0] - S1 @ qq[4]).max() < 1e-13
@@ -267,6 +296,7 @@ def test_gradients_central_differences(mc_mode):
     w, d = tiny(B=2, H=1, T=7, K=3, V=3, R=2, L=3, seed=21)
     d["A"] *= 30.0
     d["B"] *= 30.0
+    d["Aw"] = I.normal(21, 9, (w.H, w.R), 0.0, 3.0)
     S0 = I.make_state(w, 0.4).astype(np.float64)
     mp = I.normal(3, 3, (w.B, w.H, w.V))
     dO = I.normal(4, 4, (w.B, w.T, w.H, w.V))
@@ -280,7 +310,8 @@ def test_gradients_central_differences(mc_mode):
     g = oracle.bwd(d, 3, dO, mc_mode=mc_mode, S0=S0, m_prev=mp, dS_final=dSf, dm_prev_out=dmo)
     eps = 1e-6
     names = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("g_logit", "dg_logit"), ("bx", "dbx"),
-             ("w_logit", "dw_logit"), ("A", "dA"), ("B", "dB"), ("S0", "dS0"), ("m_prev", "dm_prev_in")]
+             ("w_logit", "dw_logit"), ("A", "dA"), ("B", "dB"), ("Aw", "dAw"), ("S0", "dS0"),
+             ("m_prev", "dm_prev_in")]
     for x, gx in names:
         base = S0 if x == "S0" else mp if x == "m_prev" else d[x]
         num = np.zeros_like(base)
