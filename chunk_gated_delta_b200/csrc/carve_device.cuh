@@ -64,9 +64,15 @@ __device__ __forceinline__ void content_signal(const float *Bh, const float *Ah,
 // Host: raise `kern`'s dynamic shared-memory limit to `bytes` on the current device, once.
 cudaError_t set_smem_once(const void *kern, int bytes);
 
+// Records of the tensor-core path, per (unit, gate chunk), in floats:
+//   saved by the forward: m (128), z (R), Delta (128), mean q (128), dw (1), 3 pad
+//   written by the backward for the dA / dB / dAw reduction: dDelta (128), dz (32), d(dw) (1), 3 pad
+constexpr int kTcAuxFixed = 388;   // + R
+constexpr int kTcGradRec = 164;
+
 struct FwdArgs {
     const void *q, *k, *v;
-    const float *g_logit, *bx, *w_logit, *A, *Bm, *S0, *m_prev_in;
+    const float *g_logit, *bx, *w_logit, *A, *Bm, *Aw, *S0, *m_prev_in;
     void *o;
     float *S_final, *m_prev_out;
     float *saved_states;  // [B,H,T/16,V,K] or null
@@ -76,13 +82,13 @@ struct FwdArgs {
 
 struct BwdArgs {
     const void *q, *k, *v;
-    const float *g_logit, *bx, *w_logit, *A, *Bm;
+    const float *g_logit, *bx, *w_logit, *A, *Bm, *Aw;   // Aw [H,R] or null: write gate content term
     const float *saved_states, *saved_aux;
     const void *dO;
     const float *dS_final, *dm_prev_out;
     void *dq, *dk, *dv;
-    float *dg_logit, *dbx, *dw_logit, *dS0, *dm_prev_in;
-    float *ws;  // [B,H,K*R + R*V] per-unit dA/dB partials
+    float *dg_logit, *dbx, *dw_logit, *dS0, *dm_prev_in, *dAw;
+    float *ws;  // scratch: per-unit dA/dB(/dAw) partials or per-gate-chunk gradient records
     int B, H, T, R, L, mc_mode;
 };
 

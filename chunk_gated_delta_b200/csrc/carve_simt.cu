@@ -29,7 +29,7 @@ template <int K, int V>
 struct FwdSmem {
     static constexpr int KP = K + 1, VP = V + 1;
     static constexpr int floats = V * KP + 3 * kSub * KP + 3 * kSub * K + 3 * kSub * VP +
-                                  2 * kSub * 17 + kSub + 3 * K + 3 * V + 64;
+                                  2 * kSub * 17 + kSub + 3 * K + 3 * V + 64 + 4;
     static constexpr size_t bytes = sizeof(float) * floats;
 };
 
@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
     float *osum = mvec + V;          // [V]
     float *mprev = osum + V;         // [V]
     float *zvec = mprev + V;         // [64]
+    float *wsc = zvec + 64;          // [4]: the write gate's content term dw_c
 
     const int tid = threadIdx.x;
     const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
@@ -96,6 +97,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
         __syncthreads();
         content_signal<K, V>(a.Bm + (size_t)h * R * V, a.A + (size_t)h * K * R, mvec, zvec, delta, R);
         if (tid < V) osum[tid] = 0.f;
+        if (tid == 0) {   // dw_c = Aw . z (the same projection of m_c biases the write gate)
+            float s = 0.f;
+            if (a.Aw)
+                for (int j = 0; j < R; ++j) s += a.Aw[(size_t)h * R + j] * zvec[j];
+            wsc[0] = s;
+        }
         __syncthreads();
         if (a.saved_aux) {
             float *aux = a.saved_aux + ((size_t)u * NC + c) * (V + R + K);
@@ -121,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
                 const int t = idx / V, r = idx % V;
                 vs[t * VP + r] = ld_io(vv + tk(b, s0 + t, h, r, T, H, V));
             }
-            if (tid < kSub) wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + s0 + tid) * H + h]);
+            if (tid < kSub) wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + s0 + tid) * H + h] + wsc[0]);
             __syncthreads();
             if (tid < K) {
                 float run = 0.f;
@@ -222,7 +229,7 @@ template <int K, int V>
 struct BwdSmem {
     static constexpr int KP = K + 1, VP = V + 1;
     static constexpr int floats = V * KP + 6 * kSub * KP + 3 * kSub * K + 4 * kSub * VP +
-                                  4 * kSub * 17 + 2 * kSub + 5 * K + 3 * V + 2 * 64;
+                                  4 * kSub * 17 + 2 * kSub + 5 * K + 3 * V + 2 * 64 + 4;
     static constexpr size_t bytes = sizeof(float) * floats;
 };
 
@@ -261,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
     float *dox = dmv + V;            // [V] extra output gradient of the chunk (mc_mode 1)
     float *zvec = dox + V;           // [64]
     float *dzv = zvec + 64;          // [64]
+    float *wsc = dzv + 64;           // [4]: dw_c and the gradient accumulated for it
 
     const int tid = threadIdx.x;
     const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
@@ -269,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
     const IO *q = static_cast<const IO *>(a.q), *kk = static_cast<const IO *>(a.k);
     const IO *vv = static_cast<const IO *>(a.v), *dO = static_cast<const IO *>(a.dO);
     IO *dq = static_cast<IO *>(a.dq), *dk = static_cast<IO *>(a.dk), *dv = static_cast<IO *>(a.dv);
-    float *wsu = a.ws + (size_t)u * (K * R + R * V);
+    float *wsu = a.ws + (size_t)u * (K * R + R * V + R);   // dA, dB, dAw partials of the unit
 
     for (int idx = tid; idx < V * K; idx += kThreads)
         dS[(idx / K) * KP + idx % K] = a.dS_final ? a.dS_final[(size_t)u * V * K + idx] : 0.f;
@@ -277,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
         const int nl = T - (NC - 1) * L;
         dox[tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * V + tid] / (float)nl : 0.f;
     }
-    for (int idx = tid; idx < K * R + R * V; idx += kThreads) wsu[idx] = 0.f;
+    for (int idx = tid; idx < K * R + R * V + R; idx += kThreads) wsu[idx] = 0.f;
     __syncthreads();
 
     for (int c = NC - 1; c >= 0; --c) {
@@ -290,6 +298,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
                 delta[tid] = aux[V + R + tid];
                 ddelta[tid] = 0.f;
             }
+        }
+        __syncthreads();
+        if (tid == 0) {   // dw_c = Aw . z, and its gradient starts at 0
+            float s = 0.f;
+            if (a.Aw)
+                for (int j = 0; j < R; ++j) s += a.Aw[(size_t)h * R + j] * zvec[j];
+            wsc[0] = s;
+            wsc[1] = 0.f;
         }
         __syncthreads();
         for (int jj = nsub - 1; jj >= 0; --jj) {
@@ -308,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
                 Rs[t * VP + r] = ld_io(vv + tk(b, s0 + t, h, r, T, H, V));
                 dOs[t * VP + r] = ld_io(dO + tk(b, s0 + t, h, r, T, H, V)) + dox[r];
             }
-            if (tid < kSub) wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + s0 + tid) * H + h]);
+            if (tid < kSub) wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + s0 + tid) * H + h] + wsc[0]);
             __syncthreads();
             if (tid < K) {
                 float run = 0.f;
@@ -411,9 +427,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
                 if (s == 0) dwv[t] = cw;
             }
             __syncthreads();
-            if (tid < kSub) {
-                const float w = wv[tid];
-                a.dw_logit[((size_t)b * T + s0 + tid) * H + h] = dwv[tid] * w * (1.f - w);
+            if (tid < 32) {   // d w_logit, and its sum over the sub-chunk for dw_c
+                float x = 0.f;
+                if (tid < kSub) {
+                    const float w = wv[tid];
+                    x = dwv[tid] * w * (1.f - w);
+                    a.dw_logit[((size_t)b * T + s0 + tid) * H + h] = x;
+                }
+#pragma unroll
+                for (int off = 8; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+                if (tid == 0) wsc[1] += x;
             }
             // [dQt; dKt] = [dO; -dR] S0,  dKb = U dS1,  dgamma = colsum(S0 * dS1)
             {
@@ -524,9 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
             s += __shfl_xor_sync(0xffffffffu, s, 4);
             s += __shfl_xor_sync(0xffffffffu, s, 2);
             s += __shfl_xor_sync(0xffffffffu, s, 1);
-            if (j < R && part == 0) dzv[j] = s;
+            if (j < R && part == 0) dzv[j] = s + (a.Aw ? a.Aw[(size_t)h * R + j] * wsc[1] : 0.f);
         }
         __syncthreads();
+        if (a.Aw && tid < R) wsu[K * R + R * V + tid] += wsc[1] * zvec[tid];
         for (int idx = tid; idx < K * R; idx += kThreads) wsu[idx] += ddelta[idx / R] * zvec[idx % R];
         for (int idx = tid; idx < R * V; idx += kThreads) wsu[K * R + idx] += dzv[idx / V] * mvec[idx % V];
         if (tid < V) {
@@ -572,15 +596,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
     if (a.mc_mode == 0 && a.dm_prev_in && tid < V) a.dm_prev_in[(size_t)u * V + tid] = 0.f;
 }
 
-// dA[h] = sum_b ws[b,h][:K*R],  dB[h] = sum_b ws[b,h][K*R:]   (fixed order over b)
-__global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, int B, int H, int KR, int RV) {
+// dA[h] = sum_b ws[b,h][:K*R],  dB[h] = sum_b ws[b,h][K*R : K*R+R*V],  dAw[h] = the last R
+// (fixed order over b)
+__global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, float *dAw, int B, int H, int KR, int RV,
+                                   int R) {
     const int h = blockIdx.y;
     const int x = blockIdx.x * blockDim.x + threadIdx.x;
-    if (x >= KR + RV) return;
+    if (x >= KR + RV + R) return;
     float s = 0.f;
-    for (int b = 0; b < B; ++b) s += ws[((size_t)b * H + h) * (KR + RV) + x];
+    for (int b = 0; b < B; ++b) s += ws[((size_t)b * H + h) * (KR + RV + R) + x];
     if (x < KR) dA[(size_t)h * KR + x] = s;
-    else dB[(size_t)h * RV + (x - KR)] = s;
+    else if (x < KR + RV) dB[(size_t)h * RV + (x - KR)] = s;
+    else if (dAw) dAw[(size_t)h * R + (x - KR - RV)] = s;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -602,8 +629,8 @@ cudaError_t launch_bwd_simt_t(const BwdArgs &a, float *dA, float *dB, cudaStream
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int KR = K * a.R, RV = a.R * V;
-    dim3 grid((KR + RV + 255) / 256, a.H);
-    reduce_dAdB_kernel<<<grid, 256, 0, st>>>(a.ws, dA, dB, a.B, a.H, KR, RV);
+    dim3 grid((KR + RV + a.R + 255) / 256, a.H);
+    reduce_dAdB_kernel<<<grid, 256, 0, st>>>(a.ws, dA, dB, a.dAw, a.B, a.H, KR, RV, a.R);
     return cudaGetLastError();
 }
 

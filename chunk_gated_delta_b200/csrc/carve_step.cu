@@ -3,7 +3,7 @@
 // With P = S Diag(a) the token's update and output expand to matrix-vector products over the
 // same state rows, so each (batch, head) state is read once and written once:
 //   m  = S q                     (mc_mode 0: content signal from the state before the token)
-//   a  = exp(-softplus(g_logit)) * sigmoid(bx + A (Bm m)),  w = sigmoid(w_logit)
+//   z  = Bm m,  a = exp(-softplus(g_logit)) * sigmoid(bx + A z),  w = sigmoid(w_logit + Aw . z)
 //   p  = S (a*k),  e = v - p
 //   o  = S (a*q) + w e (k.q)     (= S' q)
 //   S' = S Diag(a) + w e k^T
@@ -28,7 +28,7 @@ namespace carve {
 
 struct StepArgs {
     const void *q, *k, *v;
-    const float *g_logit, *bx, *w_logit, *A, *Bm;
+    const float *g_logit, *bx, *w_logit, *A, *Bm, *Aw;
     float *S, *mstate;
     int *pos;
     void *o;
@@ -176,7 +176,6 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
                 sm.bxv[tid] = t.bx[tid];
             }
             if (tid < V) sm.vv[tid] = ld_io(t.v + tid);
-            if (tid == 0) sm.w = sigmoid_f(t.wl[0]);
         }
         fetch_tokens(i + 1);   // tok[(i + 1) & 1] was last read before the barrier above
         if (tid < V) {
@@ -272,6 +271,12 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
                 if (part + TPK * x < R) acc += pA[x] * sm.zv[part + TPK * x];
 #pragma unroll
             for (int off = TPK / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (tid == 0) {   // w = sigmoid(w_logit + Aw . z): the same projection biases the write gate
+                float dw = 0.f;
+                if (a.Aw)
+                    for (int j = 0; j < R; ++j) dw += a.Aw[(size_t)h * R + j] * sm.zv[j];
+                sm.w = sigmoid_f(sm.tok[i & 1].wl[0] + dw);
+            }
             if (part == 0) {
                 // a = sigma(-g_logit) sigma(bx + Delta) = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)}))
                 const float e1 = __expf(sm.glv[kk]), e2 = __expf(-(sm.bxv[kk] + acc));
@@ -402,9 +407,9 @@ cudaError_t dispatch_step(int K, int V, const StepArgs &a, cudaStream_t st) {
 
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit, const float *A,
-                        const float *Bm, float *S, float *mstate, int *pos, void *o, int B, int H,
-                        int R, int L, int mc_mode, cudaStream_t st) {
-    StepArgs a{q, k, v, g_logit, bx, w_logit, A, Bm, S, mstate, pos, o, B, H, R, L, mc_mode};
+                        const float *Bm, const float *Aw, float *S, float *mstate, int *pos, void *o, int B,
+                        int H, int R, int L, int mc_mode, cudaStream_t st) {
+    StepArgs a{q, k, v, g_logit, bx, w_logit, A, Bm, Aw, S, mstate, pos, o, B, H, R, L, mc_mode};
     return bf16 ? dispatch_step<__nv_bfloat16>(K, V, a, st) : dispatch_step<float>(K, V, a, st);
 }
 

@@ -54,6 +54,7 @@ struct __align__(16) TcBwdSmem {
     float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], htot[2 * kBNB * 128], pdd[2 * kBNB * 128];
     float bpart[kBNB * 128];
     float delta[128], ddelta[128], dzv[64], dmv[128], dox[128], qbar[128];
+    float dwc, ddw;   // the write gate's content term of the gate chunk and its gradient
     uint64_t bar, bar_s0;
 };
 
@@ -76,8 +77,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     const __nv_bfloat16 *states = reinterpret_cast<const __nv_bfloat16 *>(a.saved_states) + (size_t)u * NCC * 128 * kLdOp;
     // workspace: per gate chunk dDelta (128) and dz (32) for the dA / dB reduction, then the
     // readout vectors of dq (128 per gate chunk)
-    float *wsg = a.ws + (size_t)u * NG * 160;
-    float *wsv = a.ws + (size_t)a.B * a.H * NG * 160 + (size_t)u * NG * 128;
+    float *wsg = a.ws + (size_t)u * NG * kTcGradRec;
+    float *wsv = a.ws + (size_t)a.B * a.H * NG * kTcGradRec + (size_t)u * NG * 128;
     // gate phases: channel pair c0 = 2 cp, 2 cp + 1 over tokens 8 hf + [0, 8) of 16-token block ib
     const int cp = tid & 63, hf = (tid >> 6) & 1, ib = tid >> 7, c0 = 2 * cp;
 
@@ -173,13 +174,14 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     load_gates(NCC - 1);
     // the saved record of the next gate chunk and the write logits of the next compute chunk,
     // loaded one iteration ahead
-    float pd = 0.f, pq = 0.f, pw = 0.f;
-    auto load_aux = [&](int gc) {   // Delta and the mean q of a gate chunk
-        const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (384 + R);
+    float pd = 0.f, pq = 0.f, pw = 0.f, pdw = 0.f;
+    auto load_aux = [&](int gc) {   // Delta, the mean q and the write-gate term of a gate chunk
+        const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (kTcAuxFixed + R);
         if (tid < 128) {
             pd = aux[128 + R + tid];
             pq = aux[256 + R + tid];
         }
+        if (tid == 0) pdw = aux[384 + R];
     };
     auto load_w = [&](int cc) {
         if (tid < C) pw = a.w_logit[((size_t)b * T + (size_t)cc * C + tid) * H + h];
@@ -197,6 +199,10 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 sm.delta[tid] = pd;
                 sm.qbar[tid] = pq;
                 sm.ddelta[tid] = 0.f;
+            }
+            if (tid == 0) {
+                sm.dwc = pdw;
+                sm.ddw = 0.f;
             }
         }
         {   // the carried gradient as a bf16 tile
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 *reinterpret_cast<float2 *>(&sm.rfac[row * kLdF + c0]) = make_float2(rf[0][t], rf[1][t]);
             }
         }
-        if (tid < C) sm.wv[tid] = sigmoid_f(pw);
+        if (tid < C) sm.wv[tid] = sigmoid_f(pw + sm.dwc);
         __syncthreads();
         if (tid < 128) {
             float dblk[NB];   // decay over each 16-token block
@@ -786,12 +792,16 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             }
             *reinterpret_cast<float2 *>(&sm.htot[hb * 128 + c0]) = make_float2(t0s, t1s);
         }
-        if (tid < C) {
+        if (tid < C) {   // d w_logit (warp 0: C = 32), and its sum for the write-gate term
             float dw = 0.f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) dw += sm.dwp[w * C + tid];
             const float w = sm.wv[tid];
-            a.dw_logit[((size_t)b * T + t0 + tid) * H + h] = dw * w * (1.f - w);
+            float x = dw * w * (1.f - w);
+            a.dw_logit[((size_t)b * T + t0 + tid) * H + h] = x;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+            if (tid == 0) sm.ddw += x;
         }
         for (int idx = tid; idx < C * 16; idx += 256) {   // dv = dR
             const int t = idx >> 4, part = idx & 15;
@@ -864,11 +874,12 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 s += __shfl_xor_sync(0xffffffffu, s, 4);
                 s += __shfl_xor_sync(0xffffffffu, s, 2);
                 s += __shfl_xor_sync(0xffffffffu, s, 1);
-                if (j < R && part == 0) sm.dzv[j] = s;
+                if (j < R && part == 0) sm.dzv[j] = s + (a.Aw ? a.Aw[(size_t)h * R + j] * sm.ddw : 0.f);
             }
             __syncthreads();
-            if (tid < 128) wsg[(size_t)gc * 160 + tid] = sm.ddelta[tid];
-            if (tid < R) wsg[(size_t)gc * 160 + 128 + tid] = sm.dzv[tid];
+            if (tid < 128) wsg[(size_t)gc * kTcGradRec + tid] = sm.ddelta[tid];
+            if (tid < R) wsg[(size_t)gc * kTcGradRec + 128 + tid] = sm.dzv[tid];
+            if (tid == 0) wsg[(size_t)gc * kTcGradRec + 160] = sm.ddw;
             {   // dm = B^T dz, two threads per output
                 const int vv = tid >> 1, half = tid & 1;
                 float sacc = 0.f;
@@ -939,9 +950,10 @@ constexpr int kRedRec = 32, kRedSlice = 64;
 __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *wsg, const float *aux, float *part,
                                                                   int B, int H, int NG, int R) {
     __shared__ __align__(16) float gd[kRedRec][128], rm[kRedRec][128], gz[kRedRec][kTcMaxRankBwd],
-        rz[kRedRec][kTcMaxRankBwd];
+        rz[kRedRec][kTcMaxRankBwd], gw[kRedRec];
     const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x, NR = B * NG;
     const int r0 = sl * kRedSlice, r1 = min(NR, r0 + kRedSlice);
+    float accW = 0.f;   // dAw[h][tid] for tid < R
     // each thread: a 4x4 tile of dA (rows k = 4 ka + a, columns j = 4 ja + b) and of dB
     // (rows j = 4 jb + a, columns v = 4 vb + b); the operands of a record are float4 reads
     const int ka = tid >> 3, ja = tid & 7, jb = tid >> 5, vb = tid & 31;
@@ -953,9 +965,9 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
             const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
             if (part4 < 32) {
                 *reinterpret_cast<float4 *>(&gd[i][4 * part4]) =
-                    *reinterpret_cast<const float4 *>(wsg + (u * NG + gc) * 160 + 4 * part4);
+                    *reinterpret_cast<const float4 *>(wsg + (u * NG + gc) * kTcGradRec + 4 * part4);
             } else {
-                const float *r = aux + (u * NG + gc) * (384 + R) + 4 * (part4 - 32);
+                const float *r = aux + (u * NG + gc) * (kTcAuxFixed + R) + 4 * (part4 - 32);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) rm[i][4 * (part4 - 32) + e] = r[e];
             }
@@ -963,10 +975,13 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
         for (int idx = tid; idx < nr * kTcMaxRankBwd; idx += 256) {   // dz and z (zero beyond R)
             const int i = idx / kTcMaxRankBwd, j = idx % kTcMaxRankBwd, rec = i0 + i;
             const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
-            gz[i][j] = j < R ? wsg[(u * NG + gc) * 160 + 128 + j] : 0.f;
-            rz[i][j] = j < R ? aux[(u * NG + gc) * (384 + R) + 128 + j] : 0.f;
+            gz[i][j] = j < R ? wsg[(u * NG + gc) * kTcGradRec + 128 + j] : 0.f;
+            rz[i][j] = j < R ? aux[(u * NG + gc) * (kTcAuxFixed + R) + 128 + j] : 0.f;
+            if (j == 0) gw[i] = wsg[(u * NG + gc) * kTcGradRec + 160];
         }
         __syncthreads();
+        if (tid < R)
+            for (int i = 0; i < nr; ++i) accW += gw[i] * rz[i][tid];
         for (int i = 0; i < nr; ++i) {
             const float4 g4 = *reinterpret_cast<const float4 *>(&gd[i][4 * ka]);
             const float4 z4 = *reinterpret_cast<const float4 *>(&rz[i][4 * ja]);
@@ -984,8 +999,10 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
         }
         __syncthreads();
     }
-    // partial sums in output order: dA (k, j) at k R + j, then dB (j, v) at 128 R + 128 j + v
-    float *dst = part + ((size_t)sl * H + h) * 256 * R;
+    // partial sums in output order: dA (k, j) at k R + j, dB (j, v) at 128 R + 128 j + v, then
+    // dAw (j) at 256 R + j
+    float *dst = part + ((size_t)sl * H + h) * 257 * R;
+    if (tid < R) dst[256 * R + tid] = accW;
 #pragma unroll
     for (int x = 0; x < 4; ++x)
 #pragma unroll
@@ -997,15 +1014,16 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
         }
 }
 
-__global__ void __launch_bounds__(256) reduce_dAdB_final_kernel(const float *part, float *dA, float *dB, int H,
-                                                                int R, int S) {
+__global__ void __launch_bounds__(256) reduce_dAdB_final_kernel(const float *part, float *dA, float *dB,
+                                                                float *dAw, int H, int R, int S) {
     const int idx = blockIdx.x * 256 + threadIdx.x;
-    if (idx >= H * 256 * R) return;
-    const int h = idx / (256 * R), o = idx % (256 * R);
+    if (idx >= H * 257 * R) return;
+    const int h = idx / (257 * R), o = idx % (257 * R);
     float acc = 0.f;
-    for (int sl = 0; sl < S; ++sl) acc += part[((size_t)sl * H + h) * 256 * R + o];
+    for (int sl = 0; sl < S; ++sl) acc += part[((size_t)sl * H + h) * 257 * R + o];
     if (o < 128 * R) dA[(size_t)h * 128 * R + o] = acc;
-    else dB[(size_t)h * R * 128 + (o - 128 * R)] = acc;
+    else if (o < 256 * R) dB[(size_t)h * R * 128 + (o - 128 * R)] = acc;
+    else if (dAw) dAw[(size_t)h * R + (o - 256 * R)] = acc;
 }
 
 // Record slices of the dA / dB reduction (B * NG records per head, kRedSlice per slice).
@@ -1047,16 +1065,16 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.mc_mode == 0) {
         const size_t rows = (size_t)a.B * a.T * a.H;
-        const float *vec = a.ws + (size_t)a.B * a.H * ((a.T + a.L - 1) / a.L) * 160;
+        const float *vec = a.ws + (size_t)a.B * a.H * ((a.T + a.L - 1) / a.L) * kTcGradRec;
         dq_readout_kernel<<<(unsigned)((rows * 16 + 255) / 256), 256, 0, st>>>(static_cast<__nv_bfloat16 *>(a.dq), vec,
                                                                               a.H, a.T, a.L, rows);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int NG = (a.T + a.L - 1) / a.L, S = tc_reduce_slices(a.B, NG);
-    float *part = a.ws + (size_t)a.B * a.H * NG * (160 + 128);
+    float *part = a.ws + (size_t)a.B * a.H * NG * (kTcGradRec + 128);
     reduce_dAdB_partial_kernel<<<dim3(a.H, S), 256, 0, st>>>(a.ws, a.saved_aux, part, a.B, a.H, NG, a.R);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    reduce_dAdB_final_kernel<<<(a.H * 256 * a.R + 255) / 256, 256, 0, st>>>(part, dA, dB, a.H, a.R, S);
+    reduce_dAdB_final_kernel<<<(a.H * 257 * a.R + 255) / 256, 256, 0, st>>>(part, dA, dB, a.dAw, a.H, a.R, S);
     return cudaGetLastError();
 }
 

@@ -131,11 +131,12 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     issue(0, 0);
     if (SM::ST == 1) issue(0, 1);
     uint32_t phase_bits = 0u;   // bit st: parity to wait for on stage st
+    float dwc = 0.f;            // write-gate content term of the current gate chunk
     float wnext = tid < C ? a.w_logit[((size_t)b * T + tid) * H + h] : 0.f;
     // mean q of the next gate chunk from the saved record (mode 0 with saving), one chunk ahead
     auto load_qbar = [&](int gc) {
         return (a.saved_aux && a.mc_mode == 0 && tid < 128 && gc < NG)
-                   ? a.saved_aux[((size_t)u * NG + gc) * (384 + R) + 256 + R + tid]
+                   ? a.saved_aux[((size_t)u * NG + gc) * (kTcAuxFixed + R) + 256 + R + tid]
                    : 0.f;
     };
     float pqb = load_qbar(0);
@@ -218,13 +219,21 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             __syncthreads();
             content_signal<128, 128>(sm.Bh, sm.Ah, sm.mvec, sm.zvec, sm.delta, R);
             if (tid < 128) sm.osum[tid] = 0.f;
+            {   // dw_c = Aw . z: the same projection of m_c biases the write gate (every warp forms
+                // it, so each write-gate thread holds it in a register for the whole gate chunk)
+                float x = (a.Aw && lane < R) ? a.Aw[(size_t)h * R + lane] * sm.zvec[lane] : 0.f;
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+                dwc = x;
+            }
             if (a.saved_aux) {
-                float *aux = a.saved_aux + ((size_t)u * NG + gc) * (384 + R);
+                float *aux = a.saved_aux + ((size_t)u * NG + gc) * (kTcAuxFixed + R);
                 if (tid < 128) {
                     aux[tid] = sm.mvec[tid];
                     aux[128 + R + tid] = sm.delta[tid];
                 }
                 if (tid < R) aux[128 + tid] = sm.zvec[tid];
+                if (tid == 0) aux[384 + R] = dwc;
             }
         }
         // ---- gates and mid-block referenced operands: per work item, two channels over half a
@@ -293,7 +302,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 }
             }
         }
-        if (tid < C) sm.wv[tid] = sigmoid_f(wcur);
+        if (tid < C) sm.wv[tid] = sigmoid_f(wcur + dwc);
         __syncthreads();
         // ---- decayed operands Qt = Qm Em, Kt = Krm Em: one (channel, 16-token block) item per
         //      thread, each forming its own prefix of block decays; chunk-level factors per
@@ -544,7 +553,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 }
 
 // Per (batch, gate chunk): mean of q over the gate chunk's tokens for every head, into the saved
-// aux records (offset 256 + R of each 384 + R floats).  A token's H*128 channels are one
+// aux records (offset 256 + R of each kTcAuxFixed + R floats).  A token's H*128 channels are one
 // contiguous row; each thread owns 8 consecutive channels (one 16-byte load per token).
 __global__ void __launch_bounds__(256) qbar_kernel(const __nv_bfloat16 *q, float *aux, int H, int T, int L, int R) {
     const int NG = (T + L - 1) / L, b = blockIdx.x / NG, gc = blockIdx.x % NG;
@@ -575,7 +584,7 @@ __global__ void __launch_bounds__(256) qbar_kernel(const __nv_bfloat16 *q, float
             }
         }
         const int h = c8 / 16, ch = (c8 % 16) * 8;
-        float *dst = aux + (((size_t)b * H + h) * NG + gc) * (384 + R) + 256 + R + ch;
+        float *dst = aux + (((size_t)b * H + h) * NG + gc) * (kTcAuxFixed + R) + 256 + R + ch;
 #pragma unroll
         for (int e = 0; e < 8; ++e) dst[e] = (acc[0][e] + acc[1][e]) / (float)n;
     }
@@ -612,7 +621,7 @@ int tc_compute_chunk(int L) { return L == 32 ? 32 : (L == 64 || L == 128) ? 64 :
 
 // C = 32 or 64 tokens per compute chunk.  With a.saved_states set (32-token chunks), a bf16
 // copy of the state at every compute-chunk start ([T/32][128][136] per unit, rows padded) and
-// per gate chunk the record (m, z, Delta, mean q) of 384 + R floats are written for the
+// per gate chunk the record (m, z, Delta, mean q, dw) of kTcAuxFixed + R floats are written for the
 // backward.
 cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st) {
     return C == 32 ? launch_tc_fwd_t<2>(a, st) : launch_tc_fwd_t<4>(a, st);

@@ -11,10 +11,13 @@
  *                                                     paperdance abstract)
  *           | mean_{t in c-1} o_t                     (mc_mode 1, previous-chunk mean output,
  *                                                     CARVE blog section 2.2)
- *     Delta = A (Bm m_c)                              (U_b = A.Bm, zero-initialisable low rank)
+ *     z_c   = Bm m_c ;  Delta = A z_c                 (U_b = A.Bm, zero-initialisable low rank)
+ *     dw_c  = Aw . z_c                                (optional, Aw may be NULL: the same projection
+ *                                                     of m_c also biases the write gate, CARVE
+ *                                                     blog section 2.2, Figure 1)
  *     for t in c:
  *       a_t = exp(-softplus(g_logit_t)) * sigmoid(bx_t + Delta)      (key axis, length dk)
- *       w_t = sigmoid(w_logit_t)                                      (one scalar per head)
+ *       w_t = sigmoid(w_logit_t + dw_c)                               (one scalar per head)
  *       S_t = S_{t-1} Diag(a_t) + w_t (v_t - S_{t-1} Diag(a_t) k_t) k_t^T
  *       o_t = S_t q_t
  *
@@ -33,6 +36,7 @@
  *   q, k           [B, T, H, dk]  io        v, o           [B, T, H, dv]  io
  *   g_logit, bx    [B, T, H, dk]  float     w_logit        [B, T, H]      float
  *   A              [H, dk, rank]  float     Bm             [H, rank, dv]  float
+ *   Aw             [H, rank]      float (nullable: no content term on the write gate)
  *   S0, S_final    [B, H, dv, dk] float     m vectors      [B, H, dv]     float
  * Gradients have the layout and dtype of the tensor they belong to.  Every device pointer
  * must be 16-byte aligned.
@@ -86,6 +90,7 @@ size_t carve_bwd_workspace_bytes(const carve_dims *d);
 /*
  * carve_fwd -- the forward recurrence over T tokens (the chunked WY evaluation of the
  * definition above; CARVE blog sections 2.1-2.3, paperdance abstract).
+ *   Aw          nullable: the write gate's content factor (dw_c = 0 when NULL)
  *   S0          nullable: initial state (treated as 0 when NULL)
  *   m_prev_in   nullable: mc_mode 1 content signal for the first chunk (0 when NULL)
  *   o           out: outputs
@@ -96,7 +101,7 @@ size_t carve_bwd_workspace_bytes(const carve_dims *d);
  */
 carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
                        const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *S0,
+                       const float *A, const float *Bm, const float *Aw, const float *S0,
                        const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
                        void *saved, void *stream);
 
@@ -107,16 +112,18 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
  * the matching carve_fwd call must be passed unchanged.  dA and dB are overwritten (summed
  * over the batch), not accumulated.
  *   dS_final, dm_prev_out   nullable (0 when NULL)
+ *   Aw, dAw                 both NULL (no write-gate content term) or both given; dAw is
+ *                           overwritten with the gradient summed over the batch
  *   dS0, dm_prev_in         nullable outputs
  *   workspace               carve_bwd_workspace_bytes(d) bytes of scratch
  */
 carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const void *v,
                        const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *S0,
+                       const float *A, const float *Bm, const float *Aw, const float *S0,
                        const float *m_prev_in, const void *saved, const void *dO,
                        const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
                        void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
-                       float *dB, float *dS0, float *dm_prev_in, void *workspace,
+                       float *dB, float *dAw, float *dS0, float *dm_prev_in, void *workspace,
                        void *stream);
 
 /*
@@ -129,8 +136,8 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
  * Arguments, layouts, results and errors are those of carve_bwd.  The scratch is a 4 MiB
  * array inside the library, present on every GPU that loads it until the process exits, so
  * the call allocates nothing.  Limit: carve_bwd_workspace_bytes(d) <= 4 MiB, that is
- * B*H*(dk*rank + rank*dv) floats, or, when the tensor-core kernels run (bf16,
- * dk = dv = 128, rank <= 32), B*H*NG*288 + ceil(B*NG/64)*H*256*rank floats with
+ * B*H*(dk*rank + rank*dv + rank) floats, or, when the tensor-core kernels run (bf16,
+ * dk = dv = 128, rank <= 32), B*H*NG*292 + ceil(B*NG/64)*H*257*rank floats with
  * NG = ceil(T/chunk); larger problems return
  * CARVE_ERR_UNSUPPORTED without launching anything.
  * The first call on each device looks up the array's device address (with that device
@@ -140,11 +147,11 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
  */
 carve_status carve_bwd_noalloc(const carve_dims *d, const void *q, const void *k, const void *v,
                                const float *g_logit, const float *bx, const float *w_logit,
-                               const float *A, const float *Bm, const float *S0,
+                               const float *A, const float *Bm, const float *Aw, const float *S0,
                                const float *m_prev_in, const void *saved, const void *dO,
                                const float *dS_final, const float *dm_prev_out, void *dq,
                                void *dk, void *dv, float *dg_logit, float *dbx,
-                               float *dw_logit, float *dA, float *dB, float *dS0,
+                               float *dw_logit, float *dA, float *dB, float *dAw, float *dS0,
                                float *dm_prev_in, void *stream);
 
 /*
@@ -162,8 +169,8 @@ carve_status carve_bwd_noalloc(const carve_dims *d, const void *q, const void *k
  */
 carve_status carve_step(const carve_dims *d, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit,
-                        const float *A, const float *Bm, float *S, float *mstate, int32_t *pos,
-                        void *o, void *stream);
+                        const float *A, const float *Bm, const float *Aw, float *S, float *mstate,
+                        int32_t *pos, void *o, void *stream);
 
 /*
  * carve_check -- blocks the host until the work queued on `stream` has finished, then

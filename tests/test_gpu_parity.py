@@ -298,3 +298,92 @@ def test_decode_shapes_all_units(cuda_device, K, V, io):
         if mode == 1:
             check("mstate", host(mstate), ms, TOL[io])
             assert torch.all(pos == steps)
+
+
+# ---------------------------------------------------------------------------------------
+# content term of the write gate: w = sigmoid(w_logit + Aw . z_c) (both kernel paths, decode)
+# ---------------------------------------------------------------------------------------
+def _write_term_case(cuda_device, w, L, mode):
+    import torch
+    d = I.make_inputs(w)
+    d["A"] *= 10.0
+    d["B"] *= 10.0
+    d["Aw"] = I.normal(w.seed, 97, (w.H, w.R), 0.0, 2.0)
+    dO = I.make_grad_out(w)
+    S0 = I.make_state(w, 0.05)
+    mp = I.normal(3, 2, (w.B, w.H, w.V)).astype(np.float32)
+    dSf = I.normal(3, 3, (w.B, w.H, w.V, w.K)).astype(np.float32)
+    dd = to_dev(dict(d, dO=dO), w.io, cuda_device)
+    Aw = torch.from_numpy(d["Aw"].astype(np.float32)).to(cuda_device)
+    tS0, tmp, tdS = (torch.from_numpy(x).to(cuda_device) for x in (S0, mp, dSf))
+    args = (dd["q"], dd["k"], dd["v"], dd["g_logit"], dd["bx"], dd["w_logit"], dd["A"], dd["B"])
+    out = carve.carve_fwd(*args, chunk=L, mc_mode=mode, S0=tS0, m_prev_in=tmp, Aw=Aw)
+    g = carve.carve_bwd(*args, out["saved"], dd["dO"], chunk=L, mc_mode=mode, S0=tS0, m_prev_in=tmp,
+                        dS_final=tdS, Aw=Aw)
+    torch.cuda.synchronize()
+    r = oracle.fwd(d, L=L, mc_mode=mode, S0=S0, m_prev=mp)
+    rg = oracle.bwd(d, L, dO, mc_mode=mode, S0=S0, m_prev=mp, dS_final=dSf)
+    tol = TOL[w.io]
+    check("o", host(out["o"]), r["o"], tol)
+    check("S_final", host(out["S_final"]), r["S_final"], tol)
+    for key in GRADS + ("dAw", "dS0"):
+        check(key, host(g[key]), rg[key], tol)
+    return d, dd, args, tS0, tmp, tdS
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("path", ["tensor_core", "simt"])
+def test_write_gate_term(cuda_device, path, mode):
+    if path == "tensor_core":
+        w = dataclasses.replace(I.FWD_1P3B, B=1, H=3, T=256, L=64, seed=61 + mode)
+    else:
+        w = dataclasses.replace(I.TINY_FP32, B=2, H=2, T=96, L=32, seed=63 + mode)
+    _write_term_case(cuda_device, w, w.L, mode)
+
+
+def test_zero_write_factor_is_bit_identical(cuda_device):
+    """Aw = 0 on the tensor-core path: every output equals the run without the term, bit for bit."""
+    import torch
+    w = dataclasses.replace(I.FWD_1P3B, B=1, H=2, T=128, L=64, seed=65)
+    d = I.make_inputs(w)
+    d["A"] *= 10.0
+    d["B"] *= 10.0
+    dd = to_dev(dict(d, dO=I.make_grad_out(w)), w.io, cuda_device)
+    args = (dd["q"], dd["k"], dd["v"], dd["g_logit"], dd["bx"], dd["w_logit"], dd["A"], dd["B"])
+    zero = torch.zeros((w.H, w.R), dtype=torch.float32, device=cuda_device)
+    f0 = carve.carve_fwd(*args, chunk=w.L)
+    f1 = carve.carve_fwd(*args, chunk=w.L, Aw=zero)
+    g0 = carve.carve_bwd(*args, f0["saved"], dd["dO"], chunk=w.L)
+    g1 = carve.carve_bwd(*args, f1["saved"], dd["dO"], chunk=w.L, Aw=zero)
+    torch.cuda.synchronize()
+    assert torch.equal(f0["o"], f1["o"]) and torch.equal(f0["S_final"], f1["S_final"])
+    for key in GRADS:
+        assert torch.equal(g0[key], g1[key]), key
+
+
+@pytest.mark.parametrize("K,V,io", [(128, 128, "bf16"), (64, 64, "fp32")])
+def test_decode_write_gate_term(cuda_device, K, V, io):
+    import torch
+    w = dataclasses.replace(I.DECODE, B=4, H=8, K=K, V=V, R=16, io=io, seed=700 + K)
+    steps, L = 12, 4
+    pool = I.make_decode_pool(w, pool=steps)
+    Aw_np = I.normal(w.seed, 96, (w.H, w.R), 0.0, 3.0)
+    for mode in (0, 1):
+        S_np = I.make_state(w, 0.05)
+        tp = to_dev({k: pool[k] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}, io, cuda_device)
+        A = torch.from_numpy(pool["A"]).to(cuda_device)
+        Bm = torch.from_numpy(pool["B"]).to(cuda_device)
+        Aw = torch.from_numpy(Aw_np.astype(np.float32)).to(cuda_device)
+        S = torch.from_numpy(S_np).to(cuda_device)
+        mstate = torch.zeros((w.B, w.H, 2, V), dtype=torch.float32, device=cuda_device)
+        pos = torch.zeros((w.B, w.H), dtype=torch.int32, device=cuda_device)
+        outs = [host(carve.carve_step(tp["q"][j], tp["k"][j], tp["v"][j], tp["g_logit"][j], tp["bx"][j],
+                                      tp["w_logit"][j], A, Bm, S, mc_mode=mode, chunk=L, mstate=mstate, pos=pos,
+                                      Aw=Aw)) for j in range(steps)]
+        Sr = S_np.astype(np.float64).copy()
+        ms = np.zeros((w.B, w.H, 2, V))
+        ps = np.zeros((w.B, w.H), dtype=np.int32)
+        ref = [oracle.step({k: pool[k][j] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}, pool["A"],
+                           pool["B"], Sr, L=L, mc_mode=mode, mstate=ms, pos=ps, Aw=Aw_np) for j in range(steps)]
+        check(f"o mode {mode}", np.stack(outs), np.stack(ref), TOL[io])
+        check(f"S mode {mode}", host(S), Sr, TOL[io])
