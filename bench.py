@@ -258,15 +258,18 @@ def run_train(args, w, fwd_only=False):
     dv_ = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
     torch.cuda.synchronize()
     L, mode = w.L, w.mc_mode
+    Aw = None
+    if args.write_gate:   # a seeded content factor of the write gate, N(0, 0.02^2) like A and B
+        Aw = torch.from_numpy(I.normal(w.seed, 95, (w.H, w.R), 0.0, 0.02).astype(np.float32)).to(dev)
     fwd_out = carve.carve_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
-                              dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only)
+                              dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only, Aw=Aw)
     bwd_out = None
     if not fwd_only:   # dA and dB as views of one flat buffer: the step's only collective
         from chunk_gated_delta_b200 import dist as cdist
         dAB, dA_, dB_ = cdist.grad_buffer(w.H, w.K, w.V, w.R, dev)
         bwd_out = carve.carve_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
                                   dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode,
-                                  out={"dA": dA_, "dB": dB_})
+                                  out={"dA": dA_, "dB": dB_}, Aw=Aw)
     workspace = torch.empty(carve.bwd_workspace_bytes(carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode)),
                             dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -275,7 +278,7 @@ def run_train(args, w, fwd_only=False):
         if ev is not None:
             ev[0].record(stream)
         carve.carve_fwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"], chunk=L,
-                        mc_mode=mode, out=fwd_out, save_for_bwd=not fwd_only)
+                        mc_mode=mode, out=fwd_out, save_for_bwd=not fwd_only, Aw=Aw)
         if ev is not None:
             ev[1].record(stream)
         if fwd_only:
@@ -283,7 +286,7 @@ def run_train(args, w, fwd_only=False):
                 ev[2].record(stream)
             return
         carve.carve_bwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"],
-                        fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace)
+                        fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace, Aw=Aw)
         if ev is not None:
             ev[2].record(stream)
         if ws > 1:
@@ -332,6 +335,7 @@ def run_train(args, w, fwd_only=False):
         "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "heads": w.H, "d": w.K,
                    "chunk": L, "rank": w.R, "mc_mode": mode, "parallelism": f"dp{ws}",
+                   "write_gate_term": bool(args.write_gate),
                    "l2": "no flush: step working set ~3 GB >> 126 MB L2"},
         "tensor_frac": tensor_frac,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
@@ -550,6 +554,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
     ap.add_argument("--seq-len", type=int, default=None, help="override T (smaller cases for profiling)")
+    ap.add_argument("--write-gate", action="store_true",
+                    help="train/fwd with the write gate's content term (a seeded non-zero Aw [H, rank])")
     args = ap.parse_args()
     w = {"fwd": I.FWD_1P3B, "decode": I.DECODE}.get(args.workload, I.TRAIN_1P3B)
     if args.batch:
