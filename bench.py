@@ -320,7 +320,7 @@ def run_train(args, w, fwd_only=False):
     achieved = dbytes / (dms * 1e-3) / 1e9
     flops = (fwd_flops(dd, L, w.R) + (0 if fwd_only else bwd_flops(dd, L, w.R))) * th * ws
     tensor_frac = flops / (ms * 1e-3) / (peaks["bf16"] * 1e12 * ws)
-    traffic = load_traffic(dom)
+    traffic = None if args.write_gate else load_traffic(w.name, dom)
 
     e2e = None
     if not args.no_e2e:
@@ -455,7 +455,7 @@ def run_decode(args, w):
                    "launch": "one CUDA graph per token-pool slot (one kernel each), replayed in order",
                    "l2": "no flush: 256 MB state and 470 MB token pool >> 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "carve_step", "achieved": achieved, "peak": peaks["hbm"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm"], "traffic": load_traffic("carve_step"),
+                     "unit": "GB/s", "frac": achieved / peaks["hbm"], "traffic": load_traffic(w.name, "carve_step"),
                      "peak_source": peaks["source"]},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk.summary(),
     }
@@ -466,13 +466,13 @@ def run_decode(args, w):
         dist.destroy_process_group()
 
 
-def load_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it is current."""
+def load_traffic(workload, call):
+    """DRAM bytes of one `call` on `workload` from the committed ncu summary (None when that
+    workload was not captured)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    j = json.load(open(p))
-    return j.get(kernel)
+    return json.load(open(p)).get(f"{workload}/{call}")
 
 
 def pipelined_e2e(n, stream, h2d, compute, d2h):

@@ -68,7 +68,9 @@ cudaError_t set_smem_once(const void *kern, int bytes);
 //   saved by the forward: m (128), z (R), Delta (128), mean q (128), dw (1), 3 pad
 //   written by the backward for the dA / dB / dAw reduction: dDelta (128), dz (32), d(dw) (1), 3 pad
 constexpr int kTcAuxFixed = 388;   // + R
+constexpr int kTcAuxDw = 384;      // + R: offset of dw in the saved record
 constexpr int kTcGradRec = 164;
+constexpr int kTcGradDw = 160;     // offset of d(dw) in the gradient record
 
 struct FwdArgs {
     const void *q, *k, *v;

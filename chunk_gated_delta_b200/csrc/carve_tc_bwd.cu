@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             pd = aux[128 + R + tid];
             pq = aux[256 + R + tid];
         }
-        if (tid == 0) pdw = aux[384 + R];
+        if (tid == 0) pdw = aux[kTcAuxDw + R];
     };
     auto load_w = [&](int cc) {
         if (tid < C) pw = a.w_logit[((size_t)b * T + (size_t)cc * C + tid) * H + h];
@@ -879,7 +879,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             __syncthreads();
             if (tid < 128) wsg[(size_t)gc * kTcGradRec + tid] = sm.ddelta[tid];
             if (tid < R) wsg[(size_t)gc * kTcGradRec + 128 + tid] = sm.dzv[tid];
-            if (tid == 0) wsg[(size_t)gc * kTcGradRec + 160] = sm.ddw;
+            if (tid == 0) wsg[(size_t)gc * kTcGradRec + kTcGradDw] = sm.ddw;
             {   // dm = B^T dz, two threads per output
                 const int vv = tid >> 1, half = tid & 1;
                 float sacc = 0.f;
@@ -977,7 +977,7 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
             const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
             gz[i][j] = j < R ? wsg[(u * NG + gc) * kTcGradRec + 128 + j] : 0.f;
             rz[i][j] = j < R ? aux[(u * NG + gc) * (kTcAuxFixed + R) + 128 + j] : 0.f;
-            if (j == 0) gw[i] = wsg[(u * NG + gc) * kTcGradRec + 160];
+            if (j == 0) gw[i] = wsg[(u * NG + gc) * kTcGradRec + kTcGradDw];
         }
         __syncthreads();
         if (tid < R)

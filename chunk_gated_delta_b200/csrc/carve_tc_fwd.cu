@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                     aux[128 + R + tid] = sm.delta[tid];
                 }
                 if (tid < R) aux[128 + tid] = sm.zvec[tid];
-                if (tid == 0) aux[384 + R] = dwc;
+                if (tid == 0) aux[kTcAuxDw + R] = dwc;
             }
         }
         // ---- gates and mid-block referenced operands: per work item, two channels over half a
