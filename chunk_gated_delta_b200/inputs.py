@@ -14,6 +14,8 @@ Recipe (the pages' 1.3B setting: 16 heads, d = 128; CARVE gist.science summary, 
   v ~ N(0,1);  g_logit ~ N(-3, 0.5^2)  (so g = exp(-softplus(g_logit)) ~ 0.953)
   bx ~ N(0,1); w_logit ~ N(0,1);  A, B (the low-rank factors of U_b) ~ N(0, 0.02^2)
   S0 = 0 for sequence workloads; decode state S ~ N(0, 0.05^2).
+  Decay parameters, when a workload uses them: A_dec (the log-amplitude, per head)
+  = log U(0.5, 2), tau (the bias, per head and key channel) ~ N(0, 0.5^2).
 bf16 workloads round q, k, v to bfloat16 (round-to-nearest-even) after normalisation;
 the oracle then reads exactly those rounded values.
 """
@@ -116,7 +118,7 @@ DECODE = Workload("decode_B256_H16_d128_1000steps", 256, 16, 1, 128, 128, 32, 1,
                   BASE_SEED + 4, steps=1000)
 
 # stream ids (fixed forever: changing one changes every stored expectation)
-_S_Q, _S_K, _S_V, _S_GL, _S_BX, _S_WL, _S_A, _S_B, _S_DO, _S_S0, _S_DS = range(1, 12)
+_S_Q, _S_K, _S_V, _S_GL, _S_BX, _S_WL, _S_A, _S_B, _S_DO, _S_S0, _S_DS, _S_ADEC, _S_TAU = range(1, 14)
 
 
 def _l2norm_last(x: np.ndarray) -> np.ndarray:
@@ -143,6 +145,15 @@ def make_inputs(w: Workload, seed: int | None = None, T: int | None = None) -> d
         A=normal(s, _S_A, (H, K, R), 0.0, 0.02).astype(np.float32),
         B=normal(s, _S_B, (H, R, V), 0.0, 0.02).astype(np.float32),
     )
+
+
+def make_decay(w: Workload, seed: int | None = None) -> dict:
+    """The decay's per-head parameters: A_dec [H] = log U(0.5, 2) and tau [H,K] ~ N(0, 0.5^2),
+    float32."""
+    s = w.seed if seed is None else seed
+    amp = 0.5 + 1.5 * uniform01(s, _S_ADEC, w.H)
+    return dict(A_dec=np.log(amp).astype(np.float32),
+                tau=normal(s, _S_TAU, (w.H, w.K), 0.0, 0.5).astype(np.float32))
 
 
 def make_grad_out(w: Workload, seed: int | None = None, T: int | None = None) -> np.ndarray:

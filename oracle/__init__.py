@@ -41,9 +41,9 @@ def bind(path: str):
     """Load a compiled oracle library and declare its entry points."""
     lib = ctypes.CDLL(path)
     P = ctypes.c_void_p
-    lib.orc_fwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 14
-    lib.orc_bwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 25
-    lib.orc_step.argtypes = [ctypes.POINTER(_Dims)] + [P] * 13
+    lib.orc_fwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 16
+    lib.orc_bwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 29
+    lib.orc_step.argtypes = [ctypes.POINTER(_Dims)] + [P] * 15
     for f in (lib.orc_fwd, lib.orc_bwd, lib.orc_step):
         f.restype = ctypes.c_int
     return lib
@@ -78,16 +78,19 @@ _KEYS = ("q", "k", "v", "g_logit", "bx", "w_logit", "A", "B")
 
 
 def fwd(inp: dict, L: int, mc_mode: int = 0, S0=None, m_prev=None, content_off: bool = False):
-    """Forward over [B,T,H,*] inputs (inp["Aw"], optional [H,R]: the write gate's content
-    term).  Returns dict(o, S_final, m_prev_out) in fp64."""
+    """Forward over [B,T,H,*] inputs.  Optional entries: inp["Aw"] [H,R], the write gate's
+    content term; inp["A_dec"] [H] and inp["tau"] [H,K], the decay's log-amplitude and bias.
+    Returns dict(o, S_final, m_prev_out) in fp64."""
     lib = _load()
     d = _dims(inp, L, mc_mode, content_off)
     a = [_f64(inp[k]) for k in _KEYS]
     Aw, S0, m_prev = _f64(inp.get("Aw")), _f64(S0), _f64(m_prev)
+    A_dec, tau = _f64(inp.get("A_dec")), _f64(inp.get("tau"))
     o = np.zeros((d.B, d.T, d.H, d.V))
     S = np.zeros((d.B, d.H, d.V, d.K))
     m = np.zeros((d.B, d.H, d.V))
-    rc = lib.orc_fwd(ctypes.byref(d), *[_p(x) for x in a], _p(Aw), _p(S0), _p(m_prev), _p(o), _p(S), _p(m))
+    rc = lib.orc_fwd(ctypes.byref(d), *[_p(x) for x in a], _p(Aw), _p(A_dec), _p(tau), _p(S0), _p(m_prev), _p(o),
+                     _p(S), _p(m))
     if rc:
         raise ValueError("oracle fwd: bad dims")
     return dict(o=o, S_final=S, m_prev_out=m)
@@ -96,21 +99,23 @@ def fwd(inp: dict, L: int, mc_mode: int = 0, S0=None, m_prev=None, content_off: 
 def bwd(inp: dict, L: int, dO, mc_mode: int = 0, S0=None, m_prev=None, dS_final=None,
         dm_prev_out=None, content_off: bool = False):
     """Gradients of sum(dO*o) + sum(dS_final*S_final) + sum(dm_prev_out*m_prev_out).
-    Returns dict(dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dS0, dm_prev_in) in fp64
-    (dAw is zero when inp has no "Aw")."""
+    Returns dict(dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dA_dec, dtau, dS0,
+    dm_prev_in) in fp64 (dAw, dA_dec, dtau are zero when inp lacks "Aw", "A_dec", "tau")."""
     lib = _load()
     d = _dims(inp, L, mc_mode, content_off)
     a = [_f64(inp[k]) for k in _KEYS]
-    Aw = _f64(inp.get("Aw"))
+    Aw, A_dec, tau = _f64(inp.get("Aw")), _f64(inp.get("A_dec")), _f64(inp.get("tau"))
     S0, m_prev, dO = _f64(S0), _f64(m_prev), _f64(dO)
     dS_final, dm_prev_out = _f64(dS_final), _f64(dm_prev_out)
     B, T, H, K, V, R = d.B, d.T, d.H, d.K, d.V, d.R
     out = dict(dq=np.zeros((B, T, H, K)), dk=np.zeros((B, T, H, K)), dv=np.zeros((B, T, H, V)),
                dg_logit=np.zeros((B, T, H, K)), dbx=np.zeros((B, T, H, K)), dw_logit=np.zeros((B, T, H)),
                dA=np.zeros((H, K, R)), dB=np.zeros((H, R, V)), dAw=np.zeros((H, R)),
-               dS0=np.zeros((B, H, V, K)), dm_prev_in=np.zeros((B, H, V)))
-    order = ("dq", "dk", "dv", "dg_logit", "dbx", "dw_logit", "dA", "dB", "dAw", "dS0", "dm_prev_in")
-    rc = lib.orc_bwd(ctypes.byref(d), *[_p(x) for x in a], _p(Aw), _p(S0), _p(m_prev), _p(dO), _p(dS_final),
+               dA_dec=np.zeros(H), dtau=np.zeros((H, K)), dS0=np.zeros((B, H, V, K)), dm_prev_in=np.zeros((B, H, V)))
+    order = ("dq", "dk", "dv", "dg_logit", "dbx", "dw_logit", "dA", "dB", "dAw", "dA_dec", "dtau", "dS0",
+             "dm_prev_in")
+    rc = lib.orc_bwd(ctypes.byref(d), *[_p(x) for x in a], _p(Aw), _p(A_dec), _p(tau), _p(S0), _p(m_prev),
+                     _p(dO), _p(dS_final),
                      _p(dm_prev_out), *[_p(out[k]) for k in order])
     if rc:
         raise ValueError("oracle bwd: bad dims")
@@ -118,9 +123,10 @@ def bwd(inp: dict, L: int, dO, mc_mode: int = 0, S0=None, m_prev=None, dS_final=
 
 
 def step(tok: dict, A, Bm, S, L: int = 1, mc_mode: int = 0, mstate=None, pos=None,
-         content_off: bool = False, Aw=None):
+         content_off: bool = False, Aw=None, A_dec=None, tau=None):
     """One decode step.  tok holds q, k, g_logit, bx [B,H,K], v [B,H,V], w_logit [B,H]; Aw
-    [H,R] optional (the write gate's content term).
+    [H,R] (the write gate's content term), A_dec [H] and tau [H,K] (the decay's log-amplitude
+    and bias) are optional.
     S [B,H,V,K] (fp64) is updated in place; mstate [B,H,2,V] and pos [B,H] (int32) too in
     mc_mode 1.  Returns o [B,H,V]."""
     lib = _load()
@@ -135,10 +141,11 @@ def step(tok: dict, A, Bm, S, L: int = 1, mc_mode: int = 0, mstate=None, pos=Non
         pos = np.zeros((B, H), dtype=np.int32)
     assert mstate.dtype == np.float64 and pos.dtype == np.int32
     t = {k: _f64(tok[k]) for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}
-    A, Bm, Aw = _f64(A), _f64(Bm), _f64(Aw)
+    A, Bm, Aw, A_dec, tau = _f64(A), _f64(Bm), _f64(Aw), _f64(A_dec), _f64(tau)
     o = np.zeros((B, H, V))
     rc = lib.orc_step(ctypes.byref(d), _p(t["q"]), _p(t["k"]), _p(t["v"]), _p(t["g_logit"]), _p(t["bx"]),
-                      _p(t["w_logit"]), _p(A), _p(Bm), _p(Aw), _p(S), _p(mstate), _p(pos), _p(o))
+                      _p(t["w_logit"]), _p(A), _p(Bm), _p(Aw), _p(A_dec), _p(tau), _p(S), _p(mstate),
+                      _p(pos), _p(o))
     if rc:
         raise ValueError("oracle step: bad dims")
     return o

@@ -17,7 +17,10 @@
  *                       low-rank projection of m_c yields the erase bias and the write bias,
  *                       blog section 2.2, Figure 1; dw_c = 0 when Aw is absent)
  *     for t in c:
- *       g_t = exp(-softplus(g_logit_t))           key-axis decay (blog section 2.3, decay gate)
+ *       g_t = exp(-e^{A_dec} softplus(g_logit_t + tau))  key-axis decay (blog section 2.3, the
+ *                                                 fused decay: A_dec [H] the learned log-decay
+ *                                                 amplitude, tau [H,K] the bias; A_dec = 0 and
+ *                                                 tau = 0 when absent)
  *       b_t = sigmoid(bx_t + Delta)               key-axis content-aware erase (blog section 2.2)
  *       a_t = g_t * b_t ;  w_t = sigmoid(w_logit_t + dw_c)  scalar write per head (blog 2.3)
  *       P   = S Diag(a_t) ; e_t = v_t - P k_t ; S = P + w_t e_t k_t^T      (blog section 2.1)
@@ -33,9 +36,10 @@
  *
  * Layouts (all contiguous, row-major):
  *   q, k, g_logit, bx : [B,T,H,K]    v, o : [B,T,H,V]    w_logit : [B,T,H]
- *   A : [H,K,R]   Bm : [H,R,V]   Aw : [H,R]   S0, S_final, dS : [B,H,V,K]   m vectors : [B,H,V]
- * Units (b,h) are independent and run under OpenMP; dA and dB are summed over b in a
- * fixed order afterwards, so results do not depend on the thread count.
+ *   A : [H,K,R]   Bm : [H,R,V]   Aw : [H,R]   A_dec : [H]   tau : [H,K]
+ *   S0, S_final, dS : [B,H,V,K]   m vectors : [B,H,V]
+ * Units (b,h) are independent and run under OpenMP; the per-head parameter gradients are
+ * summed over b in a fixed order afterwards, so results do not depend on the thread count.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -52,12 +56,20 @@ static double sigm(double x) { return 1.0 / (1.0 + exp(-x)); }
 
 #define IX_TK(d, b, t, h, i, W) ((((size_t)(b) * (d)->T + (t)) * (d)->H + (h)) * (W) + (i))
 
+/* the decay's parameters of head h: amplitude e^{A_dec} and the bias of channel i */
+static double decay_amp(const double *A_dec, int h) { return A_dec ? exp(A_dec[h]) : 1.0; }
+static double decay_bias(const orc_dims *d, const double *tau, int h, int i) {
+    return tau ? tau[(size_t)h * d->K + i] : 0.0;
+}
+
 /* gate activations of one token (b,t,h): a, g, bgate over K; returns w */
 static double gates(const orc_dims *d, int b, int t, int h, const double *gl, const double *bx,
-                    const double *wl, const double *delta, double dwc, double *a, double *g, double *bg) {
+                    const double *wl, const double *A_dec, const double *tau, const double *delta,
+                    double dwc, double *a, double *g, double *bg) {
+    const double amp = decay_amp(A_dec, h);
     for (int i = 0; i < d->K; ++i) {
         size_t ix = IX_TK(d, b, t, h, i, d->K);
-        g[i] = exp(-softplus(gl[ix]));
+        g[i] = exp(-amp * softplus(gl[ix] + decay_bias(d, tau, h, i)));
         bg[i] = d->content_off ? sigm(bx[ix]) : sigm(bx[ix] + delta[i]);
         a[i] = g[i] * bg[i];
     }
@@ -114,10 +126,12 @@ static int check_dims(const orc_dims *d) {
     return 0;
 }
 
-/* Forward.  Aw, S0, m_prev_in, m_prev_out may be NULL.  Returns 0 or -1 on bad dims. */
+/* Forward.  Aw, A_dec, tau, S0, m_prev_in, m_prev_out may be NULL.  Returns 0 or -1 on bad
+   dims. */
 int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v,
             const double *gl, const double *bx, const double *wl, const double *A,
-            const double *Bm, const double *Aw, const double *S0, const double *m_prev_in, double *o,
+            const double *Bm, const double *Aw, const double *A_dec, const double *tau,
+            const double *S0, const double *m_prev_in, double *o,
             double *S_final, double *m_prev_out) {
     if (check_dims(d)) return -1;
     const int K = d->K, V = d->V, R = d->R, T = d->T, L = d->L, H = d->H;
@@ -155,7 +169,7 @@ int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v
             const double dwc = write_bias(d, h, Aw, z);
             for (int j = 0; j < V; ++j) osum[j] = 0.0;
             for (int t = t0; t < t1; ++t) {
-                double w = gates(d, b, t, h, gl, bx, wl, delta, dwc, a, g, bg);
+                double w = gates(d, b, t, h, gl, bx, wl, A_dec, tau, delta, dwc, a, g, bg);
                 gather_tok(d, q, b, t, h, K, qt);
                 gather_tok(d, k, b, t, h, K, kt);
                 gather_tok(d, v, b, t, h, V, vt);
@@ -176,16 +190,17 @@ int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v
 /*
  * Backward by back-propagation through time.  Given dO (and optionally dS_final, and
  * dm_prev_out in mc_mode 1), returns the gradient of sum(dO*o) + sum(dS_final*S_final)
- * + sum(dm_prev_out*m_prev_out) with respect to every input.  dA, dB (and dAw when given)
- * are overwritten; Aw and dAw may be NULL.
+ * + sum(dm_prev_out*m_prev_out) with respect to every input.  dA, dB (and dAw, dA_dec,
+ * dtau when given) are overwritten; Aw, A_dec, tau and their gradients may be NULL.
  * dS0 and dm_prev_in may be NULL.
  */
 int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v,
             const double *gl, const double *bx, const double *wl, const double *A,
-            const double *Bm, const double *Aw, const double *S0, const double *m_prev_in, const double *dO,
+            const double *Bm, const double *Aw, const double *A_dec, const double *tau,
+            const double *S0, const double *m_prev_in, const double *dO,
             const double *dS_final, const double *dm_prev_out, double *dq, double *dk,
             double *dv, double *dgl, double *dbx, double *dwl, double *dA, double *dB, double *dAw,
-            double *dS0, double *dm_prev_in) {
+            double *dA_dec, double *dtau, double *dS0, double *dm_prev_in) {
     if (check_dims(d)) return -1;
     const int K = d->K, V = d->V, R = d->R, T = d->T, L = d->L, H = d->H;
     const int units = d->B * H;
@@ -194,6 +209,8 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
     double *dA_u = calloc((size_t)units * K * R, sizeof(double));
     double *dB_u = calloc((size_t)units * R * V, sizeof(double));
     double *dAw_u = calloc((size_t)units * R, sizeof(double));
+    double *dAdec_u = calloc((size_t)units, sizeof(double));
+    double *dtau_u = calloc((size_t)units * K, sizeof(double));
 #pragma omp parallel for schedule(dynamic, 1)
     for (int u = 0; u < units; ++u) {
         const int b = u / H, h = u % H;
@@ -214,6 +231,8 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
         double *de = calloc(V, sizeof(double)), *dd = calloc(K, sizeof(double));
         double *dz = calloc(R, sizeof(double)), *dm = calloc(V, sizeof(double)), *tmp = calloc(K, sizeof(double));
         double *dAu = dA_u + (size_t)u * K * R, *dBu = dB_u + (size_t)u * R * V, *dAwu = dAw_u + (size_t)u * R;
+        double *dtauu = dtau_u + (size_t)u * K;
+        const double amp = decay_amp(A_dec, h);
 
         /* forward pass: chunk-start states and content signals */
         if (S0) memcpy(S, S0 + (size_t)u * VK, sizeof(double) * VK);
@@ -241,7 +260,7 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
             for (int j = 0; j < V; ++j) osum[j] = 0.0;
             const double dwc = write_bias(d, h, Aw, zc + (size_t)c * R);
             for (int t = t0; t < t1; ++t) {
-                double w = gates(d, b, t, h, gl, bx, wl, dc + (size_t)c * K, dwc, at, gt, bt);
+                double w = gates(d, b, t, h, gl, bx, wl, A_dec, tau, dc + (size_t)c * K, dwc, at, gt, bt);
                 gather_tok(d, q, b, t, h, K, qt);
                 gather_tok(d, k, b, t, h, K, kt);
                 gather_tok(d, v, b, t, h, V, vt);
@@ -265,23 +284,23 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
             double ddw = 0.0;   /* gradient of dw_c: sum of the chunk's write-logit gradients */
             /* recompute the chunk's per-token states St[0..n] and gates */
             memcpy(St, Sb + (size_t)c * VK, sizeof(double) * VK);
-            for (int tau = 0; tau < n; ++tau) {
-                const int t = t0 + tau;
-                wt[tau] = gates(d, b, t, h, gl, bx, wl, delta, dwc, at + (size_t)tau * K,
-                                gt + (size_t)tau * K, bt + (size_t)tau * K);
-                memcpy(St + (size_t)(tau + 1) * VK, St + (size_t)tau * VK, sizeof(double) * VK);
+            for (int ti = 0; ti < n; ++ti) {
+                const int t = t0 + ti;
+                wt[ti] = gates(d, b, t, h, gl, bx, wl, A_dec, tau, delta, dwc, at + (size_t)ti * K,
+                                gt + (size_t)ti * K, bt + (size_t)ti * K);
+                memcpy(St + (size_t)(ti + 1) * VK, St + (size_t)ti * VK, sizeof(double) * VK);
                 gather_tok(d, q, b, t, h, K, qt);
                 gather_tok(d, k, b, t, h, K, kt);
                 gather_tok(d, v, b, t, h, V, vt);
-                token_update(d, St + (size_t)(tau + 1) * VK, at + (size_t)tau * K, wt[tau], kt, vt,
-                             qt, et + (size_t)tau * V, ot);
+                token_update(d, St + (size_t)(ti + 1) * VK, at + (size_t)ti * K, wt[ti], kt, vt,
+                             qt, et + (size_t)ti * V, ot);
             }
             for (int i = 0; i < K; ++i) dd[i] = 0.0;
-            for (int tau = n - 1; tau >= 0; --tau) {
-                const int t = t0 + tau;
-                const double *a = at + (size_t)tau * K, *g = gt + (size_t)tau * K, *bg = bt + (size_t)tau * K;
-                const double *e = et + (size_t)tau * V, w = wt[tau];
-                const double *Sprev = St + (size_t)tau * VK, *Scur = St + (size_t)(tau + 1) * VK;
+            for (int ti = n - 1; ti >= 0; --ti) {
+                const int t = t0 + ti;
+                const double *a = at + (size_t)ti * K, *g = gt + (size_t)ti * K, *bg = bt + (size_t)ti * K;
+                const double *e = et + (size_t)ti * V, w = wt[ti];
+                const double *Sprev = St + (size_t)ti * VK, *Scur = St + (size_t)(ti + 1) * VK;
                 gather_tok(d, q, b, t, h, K, qt);
                 gather_tok(d, k, b, t, h, K, kt);
                 for (int j = 0; j < V; ++j) dot[j] = dO[IX_TK(d, b, t, h, j, V)] + dox[j];
@@ -317,8 +336,12 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                     double da = 0.0;
                     for (int j = 0; j < V; ++j) da += Sprev[(size_t)j * K + i] * dP[(size_t)j * K + i];
                     const size_t ix = IX_TK(d, b, t, h, i, K);
-                    /* a = g b, g = exp(-softplus(gl)) => dg/dgl = -g sigmoid(gl) */
-                    dglt[i] = -da * a[i] * sigm(gl[ix]);
+                    /* a = g b, log g = -amp softplus(gl + tau) => dg/dgl = dg/dtau
+                       = -g amp sigmoid(gl + tau), dg/dA_dec = g log g */
+                    const double x = gl[ix] + decay_bias(d, tau, h, i);
+                    dglt[i] = -da * a[i] * amp * sigm(x);
+                    if (tau) dtauu[i] += dglt[i];
+                    if (A_dec) dAdec_u[u] += da * a[i] * (-amp * softplus(x));   /* log g, finite where g underflows */
                     const double dbeta = da * g[i] * bg[i] * (1.0 - bg[i]);
                     dbxt[i] = dbeta;
                     dd[i] += dbeta;
@@ -379,14 +402,19 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
     memset(dA, 0, sizeof(double) * (size_t)H * K * R);
     memset(dB, 0, sizeof(double) * (size_t)H * R * V);
     if (dAw) memset(dAw, 0, sizeof(double) * (size_t)H * R);
+    if (dA_dec) memset(dA_dec, 0, sizeof(double) * (size_t)H);
+    if (dtau) memset(dtau, 0, sizeof(double) * (size_t)H * K);
     for (int u = 0; u < units; ++u) {
         const int h = u % H;
+        if (dA_dec) dA_dec[h] += dAdec_u[u];
+        if (dtau)
+            for (int i = 0; i < K; ++i) dtau[(size_t)h * K + i] += dtau_u[(size_t)u * K + i];
         for (size_t x = 0; x < (size_t)K * R; ++x) dA[(size_t)h * K * R + x] += dA_u[(size_t)u * K * R + x];
         for (size_t x = 0; x < (size_t)R * V; ++x) dB[(size_t)h * R * V + x] += dB_u[(size_t)u * R * V + x];
         if (dAw)
             for (int j = 0; j < R; ++j) dAw[(size_t)h * R + j] += dAw_u[(size_t)u * R + j];
     }
-    free(dA_u); free(dB_u); free(dAw_u);
+    free(dA_u); free(dB_u); free(dAw_u); free(dAdec_u); free(dtau_u);
     return 0;
 }
 
@@ -398,12 +426,14 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
  *   mc_mode 1: the content signal is the mean output of the previous complete block of
  *              L tokens.  mstate [B,H,2,V] holds (running sum of o in the current block,
  *              mean of the previous block); pos [B,H] counts tokens consumed.
- * Inputs q, k, g_logit, bx: [B,H,K]; v: [B,H,V]; w_logit: [B,H]; Aw [H,R] or NULL;
+ * Inputs q, k, g_logit, bx: [B,H,K]; v: [B,H,V]; w_logit: [B,H]; Aw [H,R], A_dec [H] and
+ * ti [H,K] or NULL;
  * S [B,H,V,K] in/out; o: [B,H,V].
  */
 int orc_step(const orc_dims *d, const double *q, const double *k, const double *v,
              const double *gl, const double *bx, const double *wl, const double *A,
-             const double *Bm, const double *Aw, double *S, double *mstate, int *pos, double *o) {
+             const double *Bm, const double *Aw, const double *A_dec, const double *tau, double *S,
+             double *mstate, int *pos, double *o) {
     if (check_dims(d)) return -1;
     const int K = d->K, V = d->V, R = d->R, H = d->H, L = d->L;
     const int units = d->B * H;
@@ -431,7 +461,7 @@ int orc_step(const orc_dims *d, const double *q, const double *k, const double *
             content_delta(d, h, A, Bm, m, z, delta);
         }
         for (int i = 0; i < K; ++i) {
-            const double g = exp(-softplus(gl[(size_t)u * K + i]));
+            const double g = exp(-decay_amp(A_dec, h) * softplus(gl[(size_t)u * K + i] + decay_bias(d, tau, h, i)));
             const double bb = d->content_off ? sigm(bx[(size_t)u * K + i]) : sigm(bx[(size_t)u * K + i] + delta[i]);
             a[i] = g * bb;
         }

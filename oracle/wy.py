@@ -8,7 +8,8 @@ serves them all; paperdance abstract: "one unmodified WY-form solve").
 
 Notation per chunk of n tokens with start state S0 (V x K), everything relative to the
 chunk (or compute sub-chunk) start:
-  l_t      = log a_t = -softplus(g_logit_t) - softplus(-(bx_t + Delta))     (key axis)
+  l_t      = log a_t = -e^{A_dec} softplus(g_logit_t + tau) - softplus(-(bx_t + Delta))   (key axis;
+             A_dec = 0, tau = 0 unless the decay's amplitude and bias are given)
   Lam_t    = sum_{s<=t} l_s            (inclusive cumulative log-retention)
   D[t,s,i] = exp(Lam_t,i - Lam_s,i) for s <= t   (decay from token s to token t)
   Akk[t,s] = sum_i k_t,i k_s,i D[t,s,i]   (s < t)        Aqk[t,s] = sum_i q_t,i k_s,i D[t,s,i]  (s <= t)
@@ -35,11 +36,13 @@ def _sigmoid(x):
     return 0.5 * (1.0 + np.tanh(0.5 * x))
 
 
-def _sub_fwd(S0, q, k, v, gl, bx, wl, delta):
-    """One compute sub-chunk.  Returns O, S1 and the intermediates the backward needs."""
+def _sub_fwd(S0, q, k, v, gl, bx, wl, delta, dec):
+    """One compute sub-chunk (dec = (A_dec, tau [K]) of the head).  Returns O, S1 and the
+    intermediates the backward needs."""
     n = q.shape[0]
     beta = bx + delta[None, :]
-    ell = -_softplus(gl) - _softplus(-beta)
+    log_g = -np.exp(dec[0]) * _softplus(gl + dec[1][None, :])
+    ell = log_g - _softplus(-beta)
     Lam = np.cumsum(ell, axis=0)
     w = _sigmoid(wl)
     diff = Lam[:, None, :] - Lam[None, :, :]                 # [t,s,i]
@@ -57,7 +60,7 @@ def _sub_fwd(S0, q, k, v, gl, bx, wl, delta):
     O = Qt @ S0.T + Aqk @ U
     gam = np.exp(Lam[-1])
     S1 = S0 * gam[None, :] + U.T @ Kb
-    return O, S1, dict(beta=beta, Lam=Lam, w=w, D=D, Akk=Akk, Aqk=Aqk, Qt=Qt, Kt=Kt, Kb=Kb,
+    return O, S1, dict(beta=beta, log_g=log_g, Lam=Lam, w=w, D=D, Akk=Akk, Aqk=Aqk, Qt=Qt, Kt=Kt, Kb=Kb,
                        M=M, R=R, U=U, gam=gam)
 
 
@@ -67,11 +70,17 @@ def _content(S, qbar, mprev, A, Bm, mc_mode):
     return m, z, A @ z
 
 
-def fwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, mc_mode=0, aw=None):
+def _decay(dec, K):
+    return (0.0, np.zeros(K)) if dec is None else (float(dec[0]), np.asarray(dec[1], dtype=np.float64))
+
+
+def fwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, mc_mode=0, aw=None, dec=None):
     """One (batch, head) unit: q, k, gl, bx [T,K]; v [T,V]; wl [T]; A [K,R]; Bm [R,V];
     S0 [V,K]; m_prev [V]; aw [R] or None (the write gate's content term: the chunk's write
-    logits are shifted by aw . z).  Returns o [T,V], S_final, m_prev_out."""
+    logits are shifted by aw . z); dec = (A_dec, tau [K]) or None (the decay's log-amplitude
+    and bias).  Returns o [T,V], S_final, m_prev_out."""
     T = q.shape[0]
+    dec = _decay(dec, q.shape[1])
     S = S0.copy()
     mprev = m_prev.copy()
     o = np.zeros((T, v.shape[1]))
@@ -81,14 +90,15 @@ def fwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, mc_mode=0, aw=None):
         wls = wl + (0.0 if aw is None else float(aw @ z))
         for s0 in range(t0, t1, Lc):
             s1 = min(s0 + Lc, t1)
-            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta)
+            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta, dec)
             o[s0:s1] = O
         mprev = o[t0:t1].mean(axis=0)
     return o, S, mprev
 
 
-def _sub_bwd(S0, q, k, gl, it, dO, dS1):
-    """Backward of one compute sub-chunk.  Returns dq, dk, dv, dgl, dbeta, dw_logit, dS0."""
+def _sub_bwd(S0, q, k, gl, it, dO, dS1, dec):
+    """Backward of one compute sub-chunk.  Returns dq, dk, dv, dgl, dbeta, dw_logit, dS0 and
+    the sub-chunk's contribution to the gradient of A_dec."""
     Lam, w, D, Akk, Aqk = it["Lam"], it["w"], it["D"], it["Akk"], it["Aqk"]
     Qt, Kt, Kb, M, R, U, gam = it["Qt"], it["Kt"], it["Kb"], it["M"], it["R"], it["U"], it["gam"]
     n = q.shape[0]
@@ -119,16 +129,20 @@ def _sub_bwd(S0, q, k, gl, it, dO, dS1):
     dLam = q * dq_a + k * dk_row - k * dk_col + dQt * Qt + dKt * Kt - dKb * Kb
     dLam[-1] += np.sum(dKb * Kb, axis=0) + dgam * gam
     dell = np.cumsum(dLam[::-1], axis=0)[::-1]
-    dgl = -_sigmoid(gl) * dell
+    # log g = -e^{A_dec} softplus(gl + tau): d/dgl = d/dtau = -e^{A_dec} sigmoid(gl + tau),
+    # d/dA_dec = log g
+    dgl = -np.exp(dec[0]) * _sigmoid(gl + dec[1][None, :]) * dell
     dbeta = _sigmoid(-it["beta"]) * dell
     dwl = dw * w * (1.0 - w)
-    return dq, dk, dv, dgl, dbeta, dwl, dS0
+    return dq, dk, dv, dgl, dbeta, dwl, dS0, float(np.sum(dell * it["log_g"]))
 
 
-def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_prev_out, mc_mode=0, aw=None):
+def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_prev_out, mc_mode=0, aw=None,
+             dec=None):
     """Reverse sweep over chunks (and compute sub-chunks inside each chunk).
-    Returns dq, dk, dv, dgl, dbx, dwl, dA, dB, dS0, dm_prev_in, daw for one unit."""
+    Returns dq, dk, dv, dgl, dbx, dwl, dA, dB, dS0, dm_prev_in, daw, dA_dec, dtau for one unit."""
     T, K = q.shape
+    dec = _decay(dec, K)
     V = v.shape[1]
     # forward: chunk-start states, content signals
     S = S0.copy()
@@ -144,13 +158,14 @@ def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_pre
         wlss.append(wls)
         for s0 in range(t0, t1, Lc):
             s1 = min(s0 + Lc, t1)
-            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta)
+            O, S, _ = _sub_fwd(S, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta, dec)
             o[s0:s1] = O
         mprev = o[t0:t1].mean(axis=0)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     dgl, dbx, dwl = np.zeros_like(gl), np.zeros_like(bx), np.zeros_like(wl)
     dA, dB = np.zeros_like(A), np.zeros_like(Bm)
     daw = np.zeros(A.shape[1])
+    da_dec = 0.0
     dS = dS_final.copy()
     dO = dO.copy()
     nch = len(starts)
@@ -167,14 +182,15 @@ def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_pre
         for s0 in subs:
             s1 = min(s0 + Lc, t1)
             sub_states.append(Sx)
-            _, Sx, it = _sub_fwd(Sx, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta)
+            _, Sx, it = _sub_fwd(Sx, q[s0:s1], k[s0:s1], v[s0:s1], gl[s0:s1], bx[s0:s1], wls[s0:s1], delta, dec)
             its.append(it)
         ddelta = np.zeros(K)
         for j in range(len(subs) - 1, -1, -1):
             s0 = subs[j]
             s1 = min(s0 + Lc, t1)
-            r = _sub_bwd(sub_states[j], q[s0:s1], k[s0:s1], gl[s0:s1], its[j], dO[s0:s1], dS)
-            dq[s0:s1], dk[s0:s1], dv[s0:s1], dgl[s0:s1], dbx[s0:s1], dwl[s0:s1], dS = r
+            r = _sub_bwd(sub_states[j], q[s0:s1], k[s0:s1], gl[s0:s1], its[j], dO[s0:s1], dS, dec)
+            dq[s0:s1], dk[s0:s1], dv[s0:s1], dgl[s0:s1], dbx[s0:s1], dwl[s0:s1], dS = r[:7]
+            da_dec += r[7]
             ddelta += r[4].sum(axis=0)
         dz = A.T @ ddelta
         if aw is not None:   # the chunk's write logits were shifted by aw . z
@@ -191,7 +207,7 @@ def bwd_unit(q, k, v, gl, bx, wl, A, Bm, S0, m_prev, L, Lc, dO, dS_final, dm_pre
             dO[(c - 1) * L:c * L] += dm[None, :] / L
         else:
             dm_prev_in = dm
-    return dq, dk, dv, dgl, dbx, dwl, dA, dB, dS, dm_prev_in, daw
+    return dq, dk, dv, dgl, dbx, dwl, dA, dB, dS, dm_prev_in, daw, da_dec, dgl.sum(axis=0)
 
 
 def _units(inp):
@@ -199,6 +215,12 @@ def _units(inp):
     for b in range(B):
         for h in range(H):
             yield b, h
+
+
+def _head_decay(f, h, K):
+    if "A_dec" not in f and "tau" not in f:
+        return None
+    return (f["A_dec"][h] if "A_dec" in f else 0.0, f["tau"][h] if "tau" in f else np.zeros(K))
 
 
 def fwd(inp, L, Lc=None, mc_mode=0, S0=None, m_prev=None):
@@ -214,7 +236,7 @@ def fwd(inp, L, Lc=None, mc_mode=0, S0=None, m_prev=None):
         o[b, :, h], Sf[b, h], mo[b, h] = fwd_unit(
             f["q"][b, :, h], f["k"][b, :, h], f["v"][b, :, h], f["g_logit"][b, :, h], f["bx"][b, :, h],
             f["w_logit"][b, :, h], f["A"][h], f["B"][h], s0, mp, L, Lc, mc_mode,
-            None if "Aw" not in f else f["Aw"][h])
+            None if "Aw" not in f else f["Aw"][h], _head_decay(f, h, K))
     return dict(o=o, S_final=Sf, m_prev_out=mo)
 
 
@@ -226,7 +248,7 @@ def bwd(inp, L, dO, Lc=None, mc_mode=0, S0=None, m_prev=None, dS_final=None, dm_
     out = dict(dq=np.zeros((B, T, H, K)), dk=np.zeros((B, T, H, K)), dv=np.zeros((B, T, H, V)),
                dg_logit=np.zeros((B, T, H, K)), dbx=np.zeros((B, T, H, K)), dw_logit=np.zeros((B, T, H)),
                dA=np.zeros_like(f["A"]), dB=np.zeros_like(f["B"]), dAw=np.zeros(f["A"].shape[::2]),
-               dS0=np.zeros((B, H, V, K)), dm_prev_in=np.zeros((B, H, V)))
+               dA_dec=np.zeros(H), dtau=np.zeros((H, K)), dS0=np.zeros((B, H, V, K)), dm_prev_in=np.zeros((B, H, V)))
     for b, h in _units(inp):
         s0 = np.zeros((V, K)) if S0 is None else np.asarray(S0[b, h], dtype=np.float64)
         mp = np.zeros(V) if m_prev is None else np.asarray(m_prev[b, h], dtype=np.float64)
@@ -235,7 +257,7 @@ def bwd(inp, L, dO, Lc=None, mc_mode=0, S0=None, m_prev=None, dS_final=None, dm_
         r = bwd_unit(f["q"][b, :, h], f["k"][b, :, h], f["v"][b, :, h], f["g_logit"][b, :, h],
                      f["bx"][b, :, h], f["w_logit"][b, :, h], f["A"][h], f["B"][h], s0, mp, L, Lc,
                      np.asarray(dO[b, :, h], dtype=np.float64), dsf, dmo, mc_mode,
-                     None if "Aw" not in f else f["Aw"][h])
+                     None if "Aw" not in f else f["Aw"][h], _head_decay(f, h, K))
         (out["dq"][b, :, h], out["dk"][b, :, h], out["dv"][b, :, h], out["dg_logit"][b, :, h],
          out["dbx"][b, :, h], out["dw_logit"][b, :, h]) = r[:6]
         out["dA"][h] += r[6]
@@ -243,4 +265,8 @@ def bwd(inp, L, dO, Lc=None, mc_mode=0, S0=None, m_prev=None, dS_final=None, dm_
         out["dS0"][b, h] = r[8]
         out["dm_prev_in"][b, h] = r[9]
         out["dAw"][h] += r[10]
+        if "A_dec" in f:
+            out["dA_dec"][h] += r[11]
+        if "tau" in f:
+            out["dtau"][h] += r[12]
     return out

@@ -4,8 +4,8 @@
    recurrence is written out again as eager float64 torch operations on the CPU and
    torch.autograd produces the gradients of sum(dO*o) + sum(dS_final*S_final) +
    sum(dm_prev_out*m_prev_out) for every input (q, k, v, both gate logits, the write logit,
-   the low-rank factors A and B, the write gate's content factor Aw, the initial state and
-   the carried content signal), in
+   the low-rank factors A and B, the write gate's content factor Aw, the decay's
+   log-amplitude A_dec and bias tau, the initial state and the carried content signal), in
    both readout modes, with a ragged last chunk.  The gradient arithmetic comes from
    autograd, not from the oracle's derivation, so a slip in any adjoint fails here.
 2. The precision of the oracle's fp64 evaluation: the same definition evaluated in 50-digit
@@ -34,8 +34,8 @@ def _case(seed, B=2, H=2, T=7, K=4, V=3, R=2, L=3):
 
 def _torch_forward(torch, x, L, mc_mode):
     """The recurrence as written in the definition (per unit, token-sequential)."""
-    q, k, v, gl, bx, wl, A, Bm, Aw, S0, mp = (x[n] for n in ("q", "k", "v", "g_logit", "bx", "w_logit", "A",
-                                                             "B", "Aw", "S0", "m_prev"))
+    q, k, v, gl, bx, wl, A, Bm, Aw, A_dec, tau, S0, mp = (
+        x[n] for n in ("q", "k", "v", "g_logit", "bx", "w_logit", "A", "B", "Aw", "A_dec", "tau", "S0", "m_prev"))
     B, T, H, K = q.shape
     V = v.shape[-1]
     sp = torch.nn.functional.softplus
@@ -57,7 +57,8 @@ def _torch_forward(torch, x, L, mc_mode):
                 dw = Aw[h] @ z   # the write gate's content term
                 o_chunk = []
                 for t in range(t0, t1):
-                    a = torch.exp(-sp(gl[b, t, h])) * torch.sigmoid(bx[b, t, h] + delta)
+                    decay = torch.exp(-torch.exp(A_dec[h]) * sp(gl[b, t, h] + tau[h]))
+                    a = decay * torch.sigmoid(bx[b, t, h] + delta)
                     wt = torch.sigmoid(wl[b, t, h] + dw)
                     P = S * a[None, :]
                     e = v[b, t, h] - P @ k[b, t, h]
@@ -80,11 +81,13 @@ def test_backward_matches_autograd(mc_mode):
     torch = pytest.importorskip("torch")
     w, d, S0, mp = _case(31 + mc_mode)
     d["Aw"] = I.normal(31, 8, (w.H, w.R), 0.0, 3.0)
+    d["A_dec"] = I.normal(31, 9, (w.H,), 0.0, 0.7)
+    d["tau"] = I.normal(31, 10, (w.H, w.K), 0.0, 1.0)
     dO = I.normal(5, 1, (w.B, w.T, w.H, w.V))
     dSf = I.normal(5, 2, (w.B, w.H, w.V, w.K))
     dmo = I.normal(5, 3, (w.B, w.H, w.V))
     x = {n: torch.tensor(d[n], dtype=torch.float64, requires_grad=True) for n in
-         ("q", "k", "v", "g_logit", "bx", "w_logit", "A", "B", "Aw")}
+         ("q", "k", "v", "g_logit", "bx", "w_logit", "A", "B", "Aw", "A_dec", "tau")}
     x["S0"] = torch.tensor(S0, dtype=torch.float64, requires_grad=True)
     x["m_prev"] = torch.tensor(mp, dtype=torch.float64, requires_grad=True)
     o, Sf, mo = _torch_forward(torch, x, w.L, mc_mode)
@@ -93,10 +96,11 @@ def test_backward_matches_autograd(mc_mode):
     np.testing.assert_allclose(Sf.detach().numpy(), ref["S_final"], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(mo.detach().numpy(), ref["m_prev_out"], rtol=1e-12, atol=1e-13)
     loss = (o * torch.from_numpy(dO)).sum() + (Sf * torch.from_numpy(dSf)).sum() + (mo * torch.from_numpy(dmo)).sum()
-    names = ["q", "k", "v", "g_logit", "bx", "w_logit", "A", "B", "Aw", "S0", "m_prev"]
+    names = ["q", "k", "v", "g_logit", "bx", "w_logit", "A", "B", "Aw", "A_dec", "tau", "S0", "m_prev"]
     grads = torch.autograd.grad(loss, [x[n] for n in names], allow_unused=True)   # m_prev: mode 1 only
     g = oracle.bwd(d, w.L, dO, mc_mode=mc_mode, S0=S0, m_prev=mp, dS_final=dSf, dm_prev_out=dmo)
-    keys = ["dq", "dk", "dv", "dg_logit", "dbx", "dw_logit", "dA", "dB", "dAw", "dS0", "dm_prev_in"]
+    keys = ["dq", "dk", "dv", "dg_logit", "dbx", "dw_logit", "dA", "dB", "dAw", "dA_dec", "dtau", "dS0",
+            "dm_prev_in"]
     for n, gk, ga in zip(names, keys, grads):
         if ga is None:   # the input does not reach the loss: the oracle must report zeros
             assert np.all(g[gk] == 0.0), gk

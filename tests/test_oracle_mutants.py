@@ -23,7 +23,15 @@ MUTANTS = {
     # wrong sign of the delta correction
     "correction_sign": ("row[i] = row[i] * a[i] + w * e[j] * k[i];", "row[i] = row[i] * a[i] - w * e[j] * k[i];"),
     # decay gate with the wrong sign of its logit
-    "decay_logit_sign": ("g[i] = exp(-softplus(gl[ix]));", "g[i] = exp(-softplus(-gl[ix]));"),
+    "decay_logit_sign": ("g[i] = exp(-amp * softplus(gl[ix] + decay_bias(d, tau, h, i)));",
+                         "g[i] = exp(-amp * softplus(-(gl[ix] + decay_bias(d, tau, h, i))));"),
+    # decay amplitude e^{-A_dec} instead of e^{A_dec}
+    "decay_amp_sign": ("return A_dec ? exp(A_dec[h]) : 1.0;", "return A_dec ? exp(-A_dec[h]) : 1.0;"),
+    # decay bias added outside the softplus
+    "decay_bias_outside_softplus": ("g[i] = exp(-amp * softplus(gl[ix] + decay_bias(d, tau, h, i)));",
+                                    "g[i] = exp(-amp * softplus(gl[ix]) - decay_bias(d, tau, h, i));"),
+    # decay bias of head 0 used for every head
+    "decay_bias_wrong_head": ("return tau ? tau[(size_t)h * d->K + i] : 0.0;", "return tau ? tau[i] : 0.0;"),
     # erase gate ignoring the content signal
     "erase_without_content": ("sigm(bx[ix] + delta[i]);", "sigm(bx[ix]);"),
     # chunk mean over L instead of the chunk's actual length
@@ -37,7 +45,12 @@ MUTANTS = {
     "noop_guard": ("static double sigm(double x) { return 1.0 / (1.0 + exp(-x)); }",
                    "static double sigm(double x) { return 1.0 / (exp(-x) + 1.0); }"),
     # backward: decay-gate gradient with the wrong sign
-    "bwd_dgl_sign": ("dglt[i] = -da * a[i] * sigm(gl[ix]);", "dglt[i] = da * a[i] * sigm(gl[ix]);"),
+    "bwd_dgl_sign": ("dglt[i] = -da * a[i] * amp * sigm(x);", "dglt[i] = da * a[i] * amp * sigm(x);"),
+    # backward: decay-logit gradient without the amplitude
+    "bwd_dgl_missing_amp": ("dglt[i] = -da * a[i] * amp * sigm(x);", "dglt[i] = -da * a[i] * sigm(x);"),
+    # backward: amplitude gradient without the amplitude factor of log g
+    "bwd_dA_dec_missing_amp": ("if (A_dec) dAdec_u[u] += da * a[i] * (-amp * softplus(x));",
+                               "if (A_dec) dAdec_u[u] += da * a[i] * (-softplus(x));"),
     # backward: readout path into dq dropped
     "bwd_no_readout_dq": ("for (int i = 0; i < K; ++i) dq[IX_TK(d, b, t, h, i, K)] += tmp[i];", "(void)tmp;"),
     # backward: write-gate gradient without the sigmoid derivative
@@ -62,6 +75,7 @@ PIN_TESTS = [
     pins.test_retention_one_is_plain_delta_rule,
     pins.test_write_zero_is_pure_decay,
     pins.test_exact_write_with_unit_keys,
+    pins.test_decay_amplitude_and_bias_closed_form,
     pins.test_orthogonal_keys_give_linear_attention,
     lambda: pins.test_content_signal_closed_form(0, False),
     lambda: pins.test_content_signal_closed_form(1, False),

@@ -114,6 +114,31 @@ def test_write_zero_is_pure_decay():
     assert np.allclose(r["S_final"], S0 * np.exp(cum[:, -1])[:, :, None, :], rtol=1e-12, atol=1e-14)
 
 
+def test_decay_amplitude_and_bias_closed_form():
+    """The fused decay (CARVE blog section 2.3: log-decay amplitude A_dec per head, bias tau,
+    g <= 0 in the log domain): with w == 0 and U_b = 0,
+    S_t = S0 Diag(prod_{s<=t} a_s), log a = -e^{A_dec[h]} log(1 + e^{g_logit + tau[h]}) - log(1 + e^{-bx}).
+    Two heads with different amplitudes and biases pin the sign of the amplitude, the bias
+    inside the softplus and the head index of both."""
+    w, d = tiny(T=9)
+    d["w_logit"][:] = -BIG
+    d["A"][:] = 0.0
+    d["A_dec"] = np.array([np.log(0.5), np.log(3.0)])
+    d["tau"] = I.normal(5, 77, (w.H, w.K), 0.0, 1.5)
+    S0 = I.make_state(w, 0.5).astype(np.float64)
+    r = oracle.fwd(d, L=4, S0=S0)
+    amp = np.exp(d["A_dec"])[None, None, :, None]
+    loga = -amp * np.log1p(np.exp(d["g_logit"] + d["tau"][None, None])) - np.log1p(np.exp(-d["bx"]))
+    cum = np.cumsum(loga, axis=1)
+    for t in range(w.T):
+        St = S0 * np.exp(cum[:, t])[:, :, None, :]
+        assert np.allclose(r["o"][:, t], np.einsum("bhvk,bhk->bhv", St, d["q"][:, t]), rtol=1e-12, atol=1e-14)
+    assert np.allclose(r["S_final"], S0 * np.exp(cum[:, -1])[:, :, None, :], rtol=1e-12, atol=1e-14)
+    # the parameters matter in this construction
+    base = oracle.fwd({k: v for k, v in d.items() if k not in ("A_dec", "tau")}, L=4, S0=S0)
+    assert np.abs(base["S_final"] - r["S_final"]).max() > 1e-3
+
+
 def test_exact_write_with_unit_keys():
     """w == 1, a == 1, ||k|| = 1: the delta rule stores v_t exactly under k_t, S_t k_t = v_t."""
     w, d = tiny(T=7, V=4)
@@ -181,6 +206,30 @@ def test_zero_write_projection_is_bit_identical(mc_mode):
         if key != "dAw":
             assert np.array_equal(g[key], gb[key]), key
     assert np.all(gb["dAw"] == 0.0) and np.abs(g["dAw"]).max() > 0.0
+
+
+@pytest.mark.parametrize("mc_mode", [0, 1])
+def test_zero_decay_parameters_are_bit_identical(mc_mode):
+    """A_dec = 0 and tau = 0: e^0 softplus(g_logit + 0) is exactly softplus(g_logit), so every
+    output equals the run without the parameters bit for bit; their gradients are the true
+    ones (finite differences elsewhere), and d tau = sum over batch and tokens of d g_logit
+    because tau enters only through g_logit + tau."""
+    w, d = tiny(B=2, T=13, L=4)
+    d["A"] *= 30.0
+    d["B"] *= 30.0
+    S0 = I.make_state(w, 0.2).astype(np.float64)
+    dO = I.normal(8, 2, (w.B, w.T, w.H, w.V))
+    dz = dict(d, A_dec=np.zeros(w.H), tau=np.zeros((w.H, w.K)))
+    r, base = oracle.fwd(dz, L=4, mc_mode=mc_mode, S0=S0), oracle.fwd(d, L=4, mc_mode=mc_mode, S0=S0)
+    for key in r:
+        assert np.array_equal(r[key], base[key]), key
+    g, gb = oracle.bwd(dz, 4, dO, mc_mode=mc_mode, S0=S0), oracle.bwd(d, 4, dO, mc_mode=mc_mode, S0=S0)
+    for key in g:
+        if key not in ("dA_dec", "dtau"):
+            assert np.array_equal(g[key], gb[key]), key
+    assert np.all(gb["dA_dec"] == 0.0) and np.all(gb["dtau"] == 0.0)
+    assert np.abs(g["dA_dec"]).min() > 0.0
+    np.testing.assert_allclose(g["dtau"], g["dg_logit"].sum(axis=(0, 1)), rtol=1e-12, atol=1e-15)
 
 
 def test_chunk_size_enters_only_through_the_content_signal():
@@ -269,10 +318,15 @@ def test_state_norm_bound_every_token():
 # 6. Decode step == sequence forward (L = 1 readout in mode 0; running block mean in mode 1)
 # ---------------------------------------------------------------------------------------
 @pytest.mark.parametrize("mc_mode,L", [(0, 1), (1, 3)])
-def test_step_equals_sequence(mc_mode, L):
+@pytest.mark.parametrize("decay", [False, True])
+def test_step_equals_sequence(mc_mode, L, decay):
     w, d = tiny(T=11, L=L)
     d["A"] *= 40.0
     d["B"] *= 40.0
+    dec = {}
+    if decay:
+        dec = {k: np.asarray(v, dtype=np.float64) for k, v in I.make_decay(w).items()}
+        d.update(dec)
     S0 = I.make_state(w, 0.3).astype(np.float64)
     mp = I.normal(9, 1, (w.B, w.H, w.V))
     r = oracle.fwd(d, L=L, mc_mode=mc_mode, S0=S0, m_prev=mp)
@@ -282,7 +336,7 @@ def test_step_equals_sequence(mc_mode, L):
     pos = np.zeros((w.B, w.H), dtype=np.int32)
     for t in range(w.T):
         tok = {k: d[k][:, t] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}
-        o = oracle.step(tok, d["A"], d["B"], S, L=L, mc_mode=mc_mode, mstate=ms, pos=pos)
+        o = oracle.step(tok, d["A"], d["B"], S, L=L, mc_mode=mc_mode, mstate=ms, pos=pos, **dec)
         assert np.abs(o - r["o"][:, t]).max() < 1e-12
     assert np.abs(S - r["S_final"]).max() < 1e-12
     assert np.all(pos == w.T)
@@ -297,6 +351,8 @@ def test_gradients_central_differences(mc_mode):
     d["A"] *= 30.0
     d["B"] *= 30.0
     d["Aw"] = I.normal(21, 9, (w.H, w.R), 0.0, 3.0)
+    d["A_dec"] = np.array([0.7])
+    d["tau"] = I.normal(21, 10, (w.H, w.K), 0.0, 1.0)
     S0 = I.make_state(w, 0.4).astype(np.float64)
     mp = I.normal(3, 3, (w.B, w.H, w.V))
     dO = I.normal(4, 4, (w.B, w.T, w.H, w.V))
@@ -310,7 +366,8 @@ def test_gradients_central_differences(mc_mode):
     g = oracle.bwd(d, 3, dO, mc_mode=mc_mode, S0=S0, m_prev=mp, dS_final=dSf, dm_prev_out=dmo)
     eps = 1e-6
     names = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("g_logit", "dg_logit"), ("bx", "dbx"),
-             ("w_logit", "dw_logit"), ("A", "dA"), ("B", "dB"), ("Aw", "dAw"), ("S0", "dS0"),
+             ("w_logit", "dw_logit"), ("A", "dA"), ("B", "dB"), ("Aw", "dAw"), ("A_dec", "dA_dec"),
+             ("tau", "dtau"), ("S0", "dS0"),
              ("m_prev", "dm_prev_in")]
     for x, gx in names:
         base = S0 if x == "S0" else mp if x == "m_prev" else d[x]

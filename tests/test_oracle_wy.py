@@ -29,19 +29,24 @@ def rel(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def with_write_term(w, d):
+def with_terms(w, d, terms):
+    """Optional terms: the write gate's content term ("write") and the decay's amplitude and
+    bias ("decay", scaled up so they matter at these sizes)."""
     d = dict(d)
-    d["Aw"] = I.normal(w.seed, 98, (w.H, w.R), 0.0, 40.0 * 0.02)
+    if "write" in terms:
+        d["Aw"] = I.normal(w.seed, 98, (w.H, w.R), 0.0, 40.0 * 0.02)
+    if "decay" in terms:
+        d["A_dec"] = I.normal(w.seed, 97, (w.H,), 0.5, 0.5)
+        d["tau"] = I.normal(w.seed, 96, (w.H, w.K), 1.0, 1.0)
     return d
 
 
 @pytest.mark.parametrize("mc_mode", [0, 1])
 @pytest.mark.parametrize("L,Lc", [(16, 16), (16, 8), (16, 4), (16, 1), (12, 4), (1, 1)])
-@pytest.mark.parametrize("write_term", [False, True])
-def test_wy_forward_matches_sequential(mc_mode, L, Lc, write_term):
+@pytest.mark.parametrize("terms", ["", "write", "decay"])
+def test_wy_forward_matches_sequential(mc_mode, L, Lc, terms):
     w, d, S0, mp = case()
-    if write_term:
-        d = with_write_term(w, d)
+    d = with_terms(w, d, terms)
     r = oracle.fwd(d, L=L, mc_mode=mc_mode, S0=S0, m_prev=mp)
     q = wy.fwd(d, L, Lc, mc_mode, S0=S0, m_prev=mp)
     for key in r:
@@ -50,18 +55,18 @@ def test_wy_forward_matches_sequential(mc_mode, L, Lc, write_term):
 
 @pytest.mark.parametrize("mc_mode", [0, 1])
 @pytest.mark.parametrize("L,Lc", [(16, 16), (16, 4), (12, 6), (1, 1)])
-@pytest.mark.parametrize("write_term", [False, True])
-def test_wy_backward_matches_bptt(mc_mode, L, Lc, write_term):
+@pytest.mark.parametrize("terms", ["", "write", "decay"])
+def test_wy_backward_matches_bptt(mc_mode, L, Lc, terms):
     w, d, S0, mp = case(T=29)
-    if write_term:
-        d = with_write_term(w, d)
+    d = with_terms(w, d, terms)
     dO = I.normal(1, 2, (w.B, w.T, w.H, w.V))
     dSf = I.normal(1, 3, (w.B, w.H, w.V, w.K))
     dmo = I.normal(1, 4, (w.B, w.H, w.V))
     g = oracle.bwd(d, L, dO, mc_mode=mc_mode, S0=S0, m_prev=mp, dS_final=dSf, dm_prev_out=dmo)
     h = wy.bwd(d, L, dO, Lc, mc_mode, S0=S0, m_prev=mp, dS_final=dSf, dm_prev_out=dmo)
     for key in g:
-        if (mc_mode == 0 and key == "dm_prev_in") or (not write_term and key == "dAw"):
+        absent = (key == "dAw" and "write" not in terms) or (key in ("dA_dec", "dtau") and "decay" not in terms)
+        if (mc_mode == 0 and key == "dm_prev_in") or absent:
             assert np.all(g[key] == 0) and np.all(h[key] == 0)
             continue
         assert rel(h[key], g[key]) < 1e-11, key
