@@ -56,13 +56,14 @@ def bwd_flops(d, L, r):
     return 14 * L * d + 14 * d * d + L * L
 
 
-def launches_per_step(w, fwd_only):
+def launches_per_step(w, fwd_only, decay=False):
     """Kernels one step launches on the tensor-core path (bf16, d = 128): the forward (plus the
     chunk-mean prologue when it saves for the backward in mode 0); the backward, the dq
-    readout pass (mode 0) and the dA/dB reduction."""
+    readout pass (mode 0), the dA/dB reduction and (with the decay's parameters) the d tau /
+    d A_dec reduction."""
     if fwd_only:
         return 1
-    return (2 if w.mc_mode == 0 else 1) + (3 if w.mc_mode == 0 else 2)
+    return (2 if w.mc_mode == 0 else 1) + (3 if w.mc_mode == 0 else 2) + (1 if decay else 0)
 
 
 def load_peaks():
@@ -258,18 +259,20 @@ def run_train(args, w, fwd_only=False):
     dv_ = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
     torch.cuda.synchronize()
     L, mode = w.L, w.mc_mode
-    Aw = None
+    opt = {}   # the optional terms of the recurrence
     if args.write_gate:   # a seeded content factor of the write gate, N(0, 0.02^2) like A and B
-        Aw = torch.from_numpy(I.normal(w.seed, 95, (w.H, w.R), 0.0, 0.02).astype(np.float32)).to(dev)
+        opt["Aw"] = torch.from_numpy(I.normal(w.seed, 95, (w.H, w.R), 0.0, 0.02).astype(np.float32)).to(dev)
+    if args.decay:        # the decay's log-amplitude [H] and bias [H, dk]
+        opt.update({k: torch.from_numpy(v).to(dev) for k, v in I.make_decay(w).items()})
     fwd_out = carve.carve_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
-                              dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only, Aw=Aw)
+                              dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only, **opt)
     bwd_out = None
     if not fwd_only:   # dA and dB as views of one flat buffer: the step's only collective
         from chunk_gated_delta_b200 import dist as cdist
         dAB, dA_, dB_ = cdist.grad_buffer(w.H, w.K, w.V, w.R, dev)
         bwd_out = carve.carve_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
                                   dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode,
-                                  out={"dA": dA_, "dB": dB_}, Aw=Aw)
+                                  out={"dA": dA_, "dB": dB_}, **opt)
     workspace = torch.empty(carve.bwd_workspace_bytes(carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode)),
                             dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -278,7 +281,7 @@ def run_train(args, w, fwd_only=False):
         if ev is not None:
             ev[0].record(stream)
         carve.carve_fwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"], chunk=L,
-                        mc_mode=mode, out=fwd_out, save_for_bwd=not fwd_only, Aw=Aw)
+                        mc_mode=mode, out=fwd_out, save_for_bwd=not fwd_only, **opt)
         if ev is not None:
             ev[1].record(stream)
         if fwd_only:
@@ -286,7 +289,7 @@ def run_train(args, w, fwd_only=False):
                 ev[2].record(stream)
             return
         carve.carve_bwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"],
-                        fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace, Aw=Aw)
+                        fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace, **opt)
         if ev is not None:
             ev[2].record(stream)
         if ws > 1:
@@ -320,7 +323,7 @@ def run_train(args, w, fwd_only=False):
     achieved = dbytes / (dms * 1e-3) / 1e9
     flops = (fwd_flops(dd, L, w.R) + (0 if fwd_only else bwd_flops(dd, L, w.R))) * th * ws
     tensor_frac = flops / (ms * 1e-3) / (peaks["bf16"] * 1e12 * ws)
-    traffic = None if args.write_gate else load_traffic(w.name, dom)
+    traffic = None if opt else load_traffic(w.name, dom)
 
     e2e = None
     if not args.no_e2e:
@@ -335,13 +338,13 @@ def run_train(args, w, fwd_only=False):
         "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "heads": w.H, "d": w.K,
                    "chunk": L, "rank": w.R, "mc_mode": mode, "parallelism": f"dp{ws}",
-                   "write_gate_term": bool(args.write_gate),
+                   "write_gate_term": bool(args.write_gate), "decay_parameters": bool(args.decay),
                    "l2": "no flush: step working set ~3 GB >> 126 MB L2"},
         "tensor_frac": tensor_frac,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm"], "traffic": traffic, "peak_source": peaks["source"]},
         "kernels_ms": {"carve_fwd": fwd_ms, "carve_bwd": bwd_ms},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, fwd_only) * args.steps,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, fwd_only, args.decay) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0:
@@ -380,9 +383,11 @@ def run_decode(args, w):
     keys = ("q", "k", "v", "g_logit", "bx", "w_logit")
     stream = torch.cuda.current_stream()
 
+    dec = {k: torch.from_numpy(v).to(dev) for k, v in I.make_decay(w).items()} if args.decay else {}
+
     def step(x):
         carve.carve_step(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], dp["A"], dp["B"], S,
-                         mc_mode=w.mc_mode, chunk=1, o=o)
+                         mc_mode=w.mc_mode, chunk=1, o=o, **dec)
 
     # One step is one short kernel, so the loop is launch-bound from Python: each pool slot's
     # step is captured once in a CUDA graph and the timed loop replays them in order.
@@ -452,10 +457,12 @@ def run_decode(args, w):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * ws, "heads": w.H, "d": w.K, "rank": w.R,
                    "mc_mode": w.mc_mode, "parallelism": f"dp{ws}", "tokens_per_s": value * w.B,
+                   "decay_parameters": bool(args.decay),
                    "launch": "one CUDA graph per token-pool slot (one kernel each), replayed in order",
                    "l2": "no flush: 256 MB state and 470 MB token pool >> 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": "carve_step", "achieved": achieved, "peak": peaks["hbm"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm"], "traffic": load_traffic(w.name, "carve_step"),
+                     "unit": "GB/s", "frac": achieved / peaks["hbm"],
+                     "traffic": None if args.decay else load_traffic(w.name, "carve_step"),
                      "peak_source": peaks["source"]},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk.summary(),
     }
@@ -556,6 +563,8 @@ def main():
     ap.add_argument("--seq-len", type=int, default=None, help="override T (smaller cases for profiling)")
     ap.add_argument("--write-gate", action="store_true",
                     help="train/fwd with the write gate's content term (a seeded non-zero Aw [H, rank])")
+    ap.add_argument("--decay", action="store_true",
+                    help="train/fwd/decode with the decay's log-amplitude A_dec [H] and bias tau [H, dk] (seeded)")
     args = ap.parse_args()
     w = {"fwd": I.FWD_1P3B, "decode": I.DECODE}.get(args.workload, I.TRAIN_1P3B)
     if args.batch:

@@ -54,9 +54,9 @@ def load():
     for f in (lib.carve_saved_bytes, lib.carve_bwd_workspace_bytes):
         f.argtypes = [D]
         f.restype = ctypes.c_size_t
-    lib.carve_fwd.argtypes = [D] + [P] * 16
-    lib.carve_bwd.argtypes = [D] + [P] * 27
-    lib.carve_step.argtypes = [D] + [P] * 14
+    lib.carve_fwd.argtypes = [D] + [P] * 18
+    lib.carve_bwd.argtypes = [D] + [P] * 32
+    lib.carve_step.argtypes = [D] + [P] * 16
     lib.carve_check.argtypes = [P]
     lib.carve_selftest_timeout.argtypes = [ctypes.c_uint32, P]
     for f in (lib.carve_fwd, lib.carve_bwd, lib.carve_step, lib.carve_check, lib.carve_selftest_timeout):
@@ -121,10 +121,11 @@ def carve_check(stream=None) -> int:
 
 
 def carve_fwd(q, k, v, g_logit, bx, w_logit, A, B, chunk: int, mc_mode: int = 0, S0=None, m_prev_in=None,
-              save_for_bwd: bool = True, out: dict | None = None, stream=None, Aw=None) -> dict:
-    """Forward over [B,T,H,*] device tensors (Aw [H,rank] optional: the write gate's content
-    term).  Returns dict(o, S_final, m_prev_out, saved); `out` may supply preallocated
-    buffers under the same keys."""
+              save_for_bwd: bool = True, out: dict | None = None, stream=None, Aw=None, A_dec=None,
+              tau=None) -> dict:
+    """Forward over [B,T,H,*] device tensors.  Optional: Aw [H,rank], the write gate's content
+    term; A_dec [H] and tau [H,dk], the decay's log-amplitude and bias.  Returns dict(o,
+    S_final, m_prev_out, saved); `out` may supply preallocated buffers under the same keys."""
     torch = _torch()
     lib = load()
     d = dims_of(q, v, A, chunk, mc_mode)
@@ -142,17 +143,18 @@ def carve_fwd(q, k, v, g_logit, bx, w_logit, A, B, chunk: int, mc_mode: int = 0,
             raise CarveError("carve_saved_bytes", 1)
         out["saved"] = torch.empty(n, dtype=torch.uint8, device=dev)
     rc = lib.carve_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g_logit), _ptr(bx), _ptr(w_logit),
-                       _ptr(A), _ptr(B), _ptr(Aw), _ptr(S0), _ptr(m_prev_in), _ptr(out["o"]), _ptr(out["S_final"]),
-                       _ptr(out["m_prev_out"]), _ptr(out.get("saved") if save_for_bwd else None), _stream(stream))
+                       _ptr(A), _ptr(B), _ptr(Aw), _ptr(A_dec), _ptr(tau), _ptr(S0), _ptr(m_prev_in), _ptr(out["o"]),
+                       _ptr(out["S_final"]), _ptr(out["m_prev_out"]), _ptr(out.get("saved") if save_for_bwd else None),
+                       _stream(stream))
     _check("carve_fwd", rc)
     return out
 
 
 def carve_bwd(q, k, v, g_logit, bx, w_logit, A, B, saved, dO, chunk: int, mc_mode: int = 0, S0=None,
               m_prev_in=None, dS_final=None, dm_prev_out=None, want_dS0: bool = True, out: dict | None = None,
-              workspace=None, stream=None, Aw=None) -> dict:
+              workspace=None, stream=None, Aw=None, A_dec=None, tau=None) -> dict:
     """Reverse sweep.  Returns dict(dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dS0, dm_prev_in),
-    plus dAw when the forward had the write gate's content term (Aw)."""
+    plus dAw, dA_dec, dtau when the forward had Aw, A_dec, tau."""
     torch = _torch()
     lib = load()
     d = dims_of(q, v, A, chunk, mc_mode)
@@ -164,27 +166,30 @@ def carve_bwd(q, k, v, g_logit, bx, w_logit, A, B, saved, dO, chunk: int, mc_mod
                   dm_prev_in=((d.B, d.H, d.dv), torch.float32))
     if want_dS0:
         shapes["dS0"] = ((d.B, d.H, d.dv, d.dk), torch.float32)
-    if Aw is not None:
-        shapes["dAw"] = (Aw.shape, torch.float32)
+    for name, x in (("dAw", Aw), ("dA_dec", A_dec), ("dtau", tau)):
+        if x is not None:
+            shapes[name] = (x.shape, torch.float32)
     for key, (shp, dt) in shapes.items():
         if key not in out:
             out[key] = torch.empty(shp, dtype=dt, device=dev)
     if workspace is None:
         workspace = torch.empty(bwd_workspace_bytes(d), dtype=torch.uint8, device=dev)
     rc = lib.carve_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g_logit), _ptr(bx), _ptr(w_logit), _ptr(A),
-                       _ptr(B), _ptr(Aw), _ptr(S0), _ptr(m_prev_in), _ptr(saved), _ptr(dO), _ptr(dS_final),
-                       _ptr(dm_prev_out), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg_logit"]),
-                       _ptr(out["dbx"]), _ptr(out["dw_logit"]), _ptr(out["dA"]), _ptr(out["dB"]),
-                       _ptr(out.get("dAw") if Aw is not None else None), _ptr(out.get("dS0")),
+                       _ptr(B), _ptr(Aw), _ptr(A_dec), _ptr(tau), _ptr(S0), _ptr(m_prev_in), _ptr(saved), _ptr(dO),
+                       _ptr(dS_final), _ptr(dm_prev_out), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                       _ptr(out["dg_logit"]), _ptr(out["dbx"]), _ptr(out["dw_logit"]), _ptr(out["dA"]), _ptr(out["dB"]),
+                       _ptr(out.get("dAw") if Aw is not None else None),
+                       _ptr(out.get("dA_dec") if A_dec is not None else None),
+                       _ptr(out.get("dtau") if tau is not None else None), _ptr(out.get("dS0")),
                        _ptr(out["dm_prev_in"]), _ptr(workspace), _stream(stream))
     _check("carve_bwd", rc)
     return out
 
 
 def carve_step(q, k, v, g_logit, bx, w_logit, A, B, S, mc_mode: int = 0, chunk: int = 1, mstate=None, pos=None,
-               o=None, stream=None, Aw=None):
+               o=None, stream=None, Aw=None, A_dec=None, tau=None):
     """One decode token for every (b,h): q, k, g_logit, bx [B,H,dk]; v [B,H,dv]; w_logit [B,H];
-    Aw [H,rank] optional; S [B,H,dv,dk] float32 updated in place (mstate/pos too in mc_mode 1).
+    Aw [H,rank], A_dec [H], tau [H,dk] optional; S [B,H,dv,dk] float32 updated in place (mstate/pos too in mc_mode 1).
     Returns o [B,H,dv]."""
     torch = _torch()
     lib = load()
@@ -193,6 +198,7 @@ def carve_step(q, k, v, g_logit, bx, w_logit, A, B, S, mc_mode: int = 0, chunk: 
     if o is None:
         o = torch.empty((Bn, H, d.dv), dtype=q.dtype, device=q.device)
     rc = lib.carve_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g_logit), _ptr(bx), _ptr(w_logit), _ptr(A),
-                        _ptr(B), _ptr(Aw), _ptr(S), _ptr(mstate), _ptr(pos), _ptr(o), _stream(stream))
+                        _ptr(B), _ptr(Aw), _ptr(A_dec), _ptr(tau), _ptr(S), _ptr(mstate), _ptr(pos), _ptr(o),
+                        _stream(stream))
     _check("carve_step", rc)
     return o

@@ -18,8 +18,8 @@ cudaError_t launch_selftest_timeout(uint32_t iterations, cudaStream_t st);
 cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit, const float *A,
-                        const float *Bm, const float *Aw, float *S, float *mstate, int *pos, void *o, int B,
-                        int H, int R, int L, int mc_mode, cudaStream_t st);
+                        const float *Bm, const float *Aw, const float *A_dec, const float *tau, float *S,
+                        float *mstate, int *pos, void *o, int B, int H, int R, int L, int mc_mode, cudaStream_t st);
 }  // namespace carve
 
 namespace {
@@ -102,26 +102,30 @@ size_t carve_bwd_workspace_bytes(const carve_dims *d) {
     if (check_dims(d, true) != CARVE_OK) return 0;
     const size_t units = (size_t)d->B * d->H;
     if (use_tc_bwd(d))   // per gate chunk: the gradient record and the readout vector of dq;
-                         // then the per-slice partial sums of dA, dB and dAw
+                         // then the per-slice partial sums of dA, dB and dAw; then per unit the
+                         // decay parameters' partial sums
         return sizeof(float) * (units * n_chunks(d) * (carve::kTcGradRec + (size_t)d->dk) +
-                                (size_t)carve::tc_reduce_slices(d->B, (int)n_chunks(d)) * d->H * 257 * d->rank);
-    return sizeof(float) * units * ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv + d->rank);
+                                (size_t)carve::tc_reduce_slices(d->B, (int)n_chunks(d)) * d->H * 257 * d->rank +
+                                units * carve::kTcDecayRec);
+    // per unit: dA, dB, dAw, dtau and dA_dec partial sums
+    return sizeof(float) * units *
+           ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv + d->rank + (size_t)d->dk + 1);
 }
 
 carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
                        const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *Aw, const float *S0,
-                       const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
-                       void *saved, void *stream) {
+                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                       const float *tau, const float *S0, const float *m_prev_in, void *o,
+                       float *S_final, float *m_prev_out, void *saved, void *stream) {
     carve_status st = check_dims(d, true);
     if (st != CARVE_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
-        !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(Aw) || !ok_ptr(o) || !ok_opt(S0) || !ok_opt(m_prev_in) ||
-        !ok_opt(S_final) || !ok_opt(m_prev_out) || !ok_opt(saved))
+        !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(Aw) || !ok_opt(A_dec) || !ok_opt(tau) || !ok_ptr(o) ||
+        !ok_opt(S0) || !ok_opt(m_prev_in) || !ok_opt(S_final) || !ok_opt(m_prev_out) || !ok_opt(saved))
         return CARVE_ERR_INVALID_ARG;
     carve::FwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
-    a.Aw = Aw; a.S0 = S0; a.m_prev_in = m_prev_in; a.o = o; a.S_final = S_final; a.m_prev_out = m_prev_out;
+    a.Aw = Aw; a.A_dec = A_dec; a.tau = tau; a.S0 = S0; a.m_prev_in = m_prev_in; a.o = o; a.S_final = S_final; a.m_prev_out = m_prev_out;
     const bool tc_saved = use_tc_bwd(d);
     if (saved) {
         a.saved_states = static_cast<float *>(saved);
@@ -141,25 +145,27 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
 
 carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const void *v,
                        const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *Aw, const float *S0,
-                       const float *m_prev_in, const void *saved, const void *dO,
-                       const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
-                       void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
-                       float *dB, float *dAw, float *dS0, float *dm_prev_in, void *workspace,
-                       void *stream) {
+                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                       const float *tau, const float *S0, const float *m_prev_in, const void *saved,
+                       const void *dO, const float *dS_final, const float *dm_prev_out, void *dq,
+                       void *dk, void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
+                       float *dB, float *dAw, float *dA_dec, float *dtau, float *dS0,
+                       float *dm_prev_in, void *workspace, void *stream) {
     carve_status st = check_dims(d, true);
     if (st != CARVE_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
         !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(S0) || !ok_opt(m_prev_in) || !ok_ptr(saved) || !ok_ptr(dO) ||
         !ok_opt(dS_final) || !ok_opt(dm_prev_out) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
         !ok_ptr(dg_logit) || !ok_ptr(dbx) || !ok_ptr(dw_logit) || !ok_ptr(dA) || !ok_ptr(dB) || !ok_opt(dS0) ||
-        !ok_opt(dm_prev_in) || !ok_ptr(workspace) || !ok_opt(Aw) || (Aw ? !ok_ptr(dAw) : dAw != nullptr))
+        !ok_opt(dm_prev_in) || !ok_ptr(workspace) || !ok_opt(Aw) || (Aw ? !ok_ptr(dAw) : dAw != nullptr) ||
+        !ok_opt(A_dec) || (A_dec ? !ok_ptr(dA_dec) : dA_dec != nullptr) || !ok_opt(tau) ||
+        (tau ? !ok_ptr(dtau) : dtau != nullptr))
         return CARVE_ERR_INVALID_ARG;
     (void)S0;
     (void)m_prev_in;  // their effect is captured by the saved states and content signals
     carve::BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.g_logit = g_logit; a.bx = bx; a.w_logit = w_logit; a.A = A; a.Bm = Bm;
-    a.Aw = Aw; a.dAw = dAw;
+    a.Aw = Aw; a.dAw = dAw; a.A_dec = A_dec; a.tau = tau; a.dA_dec = dA_dec; a.dtau = dtau;
     const bool tc = use_tc_bwd(d);
     a.saved_states = static_cast<const float *>(saved);
     a.saved_aux = reinterpret_cast<const float *>(static_cast<const char *>(saved) + saved_states_bytes(d));
@@ -175,17 +181,17 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
 
 carve_status carve_step(const carve_dims *d, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit,
-                        const float *A, const float *Bm, const float *Aw, float *S, float *mstate,
-                        int32_t *pos, void *o, void *stream) {
+                        const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                        const float *tau, float *S, float *mstate, int32_t *pos, void *o, void *stream) {
     carve_status st = check_dims(d, false);
     if (st != CARVE_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
-        !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(Aw) || !ok_ptr(S) || !ok_ptr(o))
+        !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(Aw) || !ok_opt(A_dec) || !ok_opt(tau) || !ok_ptr(S) || !ok_ptr(o))
         return CARVE_ERR_INVALID_ARG;
     if (d->mc_mode == CARVE_MC_PREV_MEAN_O && (!ok_ptr(mstate) || !ok_ptr(pos))) return CARVE_ERR_INVALID_ARG;
     cudaError_t e = carve::launch_step(d->dk, d->dv, d->io == CARVE_IO_BF16, q, k, v, g_logit, bx, w_logit, A, Bm, Aw,
-                                       S, mstate, pos, o, d->B, d->H, d->rank, d->chunk, d->mc_mode,
-                                       static_cast<cudaStream_t>(stream));
+                                       A_dec, tau, S, mstate, pos, o, d->B, d->H, d->rank, d->chunk,
+                                       d->mc_mode, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 

@@ -19,10 +19,19 @@ __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + lo
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
 
 // log-retention of one key channel: log a = log g + log b
-//   g = exp(-softplus(g_logit))        (key-axis decay gate)
+//   g = exp(-amp softplus(g_logit + tau))   (key-axis decay gate; amp = e^{A_dec} is the head's
+//                                             decay amplitude, tau the channel's bias; 1 and 0
+//                                             without them, which leaves every bit unchanged)
 //   b = sigmoid(bx + Delta) = exp(-softplus(-(bx + Delta)))  (content-aware erase gate)
-__device__ __forceinline__ float log_retention(float g_logit, float beta) {
-    return -softplus_f(g_logit) - softplus_f(-beta);
+__device__ __forceinline__ float log_retention(float g_logit, float beta, float amp = 1.f, float tau = 0.f) {
+    return -amp * softplus_f(g_logit + tau) - softplus_f(-beta);
+}
+
+// The decay's parameters of head h: amplitude e^{A_dec[h]} (1 without A_dec) and the bias of
+// channel i of K (0 without tau).
+__device__ __forceinline__ float decay_amp(const float *A_dec, int h) { return A_dec ? expf(A_dec[h]) : 1.f; }
+__device__ __forceinline__ float decay_bias(const float *tau, int h, int i, int K) {
+    return tau ? tau[(size_t)h * K + i] : 0.f;
 }
 
 // Content signal of a chunk: z = Bh m (R outputs, dot products over V) then
@@ -71,10 +80,13 @@ constexpr int kTcAuxFixed = 388;   // + R
 constexpr int kTcAuxDw = 384;      // + R: offset of dw in the saved record
 constexpr int kTcGradRec = 164;
 constexpr int kTcGradDw = 160;     // offset of d(dw) in the gradient record
+//   per unit, after the sweep, when the decay has parameters: d tau (128), d A_dec (1), 3 pad
+constexpr int kTcDecayRec = 132;
 
 struct FwdArgs {
     const void *q, *k, *v;
     const float *g_logit, *bx, *w_logit, *A, *Bm, *Aw, *S0, *m_prev_in;
+    const float *A_dec, *tau;   // [H], [H,K] or null: the decay's log-amplitude and bias
     void *o;
     float *S_final, *m_prev_out;
     float *saved_states;  // [B,H,T/16,V,K] or null
@@ -85,11 +97,12 @@ struct FwdArgs {
 struct BwdArgs {
     const void *q, *k, *v;
     const float *g_logit, *bx, *w_logit, *A, *Bm, *Aw;   // Aw [H,R] or null: write gate content term
+    const float *A_dec, *tau;                            // [H], [H,K] or null: decay amplitude, bias
     const float *saved_states, *saved_aux;
     const void *dO;
     const float *dS_final, *dm_prev_out;
     void *dq, *dk, *dv;
-    float *dg_logit, *dbx, *dw_logit, *dS0, *dm_prev_in, *dAw;
+    float *dg_logit, *dbx, *dw_logit, *dS0, *dm_prev_in, *dAw, *dA_dec, *dtau;
     float *ws;  // scratch: per-unit dA/dB(/dAw) partials or per-gate-chunk gradient records
     int B, H, T, R, L, mc_mode;
 };

@@ -48,20 +48,24 @@ cudaError_t scratch_for_current_device(void **out) {
 
 extern "C" carve_status carve_bwd_noalloc(const carve_dims *d, const void *q, const void *k, const void *v,
                                           const float *g_logit, const float *bx, const float *w_logit,
-                                          const float *A, const float *Bm, const float *Aw, const float *S0,
-                                          const float *m_prev_in, const void *saved, const void *dO,
-                                          const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
-                                          void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
-                                          float *dB, float *dAw, float *dS0, float *dm_prev_in, void *stream) {
+                                          const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                                          const float *tau, const float *S0, const float *m_prev_in,
+                                          const void *saved, const void *dO, const float *dS_final,
+                                          const float *dm_prev_out, void *dq, void *dk, void *dv, float *dg_logit,
+                                          float *dbx, float *dw_logit, float *dA, float *dB, float *dAw,
+                                          float *dA_dec, float *dtau, float *dS0, float *dm_prev_in,
+                                          void *stream) {
     const size_t need = carve_bwd_workspace_bytes(d);
     if (need == 0)  // malformed dims: carve_bwd rejects them on the host, before any launch
-        return carve_bwd(d, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, S0, m_prev_in, saved, dO, dS_final, dm_prev_out,
-                         dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dS0, dm_prev_in, nullptr, stream);
+        return carve_bwd(d, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, A_dec, tau, S0, m_prev_in, saved, dO, dS_final,
+                         dm_prev_out, dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dA_dec, dtau, dS0, dm_prev_in,
+                         nullptr, stream);
     if (need > kScratchBytes) return CARVE_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     if (scratch_for_current_device(&scratch) != cudaSuccess) return CARVE_ERR_CUDA;
     // The backward kernel zeroes the part of the scratch it accumulates into before using it,
     // so the contents left by an earlier call do not leak into this one.
-    return carve_bwd(d, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, S0, m_prev_in, saved, dO, dS_final, dm_prev_out, dq,
-                     dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dS0, dm_prev_in, scratch, stream);
+    return carve_bwd(d, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, A_dec, tau, S0, m_prev_in, saved, dO, dS_final,
+                     dm_prev_out, dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dA_dec, dtau, dS0, dm_prev_in,
+                     scratch, stream);
 }

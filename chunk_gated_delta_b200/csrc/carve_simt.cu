@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
     const int tid = threadIdx.x;
     const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
     const int b = u / H, h = u % H;
+    const float amp = decay_amp(a.A_dec, h);   // e^{A_dec[h]}, 1 without the decay amplitude
     const int NC = (T + L - 1) / L, NS = T / kSub;
     const IO *q = static_cast<const IO *>(a.q), *kk = static_cast<const IO *>(a.k);
     const IO *vv = static_cast<const IO *>(a.v);
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
                 const size_t g = tk(b, s0 + t, h, i, T, H, K);
                 qs[t * KP + i] = ld_io(q + g);
                 ks[t * KP + i] = ld_io(kk + g);
-                lam[t * KP + i] = log_retention(a.g_logit[g], a.bx[g] + delta[i]);
+                lam[t * KP + i] = log_retention(a.g_logit[g], a.bx[g] + delta[i], amp, decay_bias(a.tau, h, i, K));
             }
             for (int idx = tid; idx < kSub * V; idx += kThreads) {
                 const int t = idx / V, r = idx % V;
@@ -277,7 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
     const IO *q = static_cast<const IO *>(a.q), *kk = static_cast<const IO *>(a.k);
     const IO *vv = static_cast<const IO *>(a.v), *dO = static_cast<const IO *>(a.dO);
     IO *dq = static_cast<IO *>(a.dq), *dk = static_cast<IO *>(a.dk), *dv = static_cast<IO *>(a.dv);
-    float *wsu = a.ws + (size_t)u * (K * R + R * V + R);   // dA, dB, dAw partials of the unit
+    // per-unit partials: dA [K*R], dB [R*V], dAw [R], dtau [K], dA_dec [1]
+    const int rec = K * R + R * V + R + K + 1;
+    float *wsu = a.ws + (size_t)u * rec;
+    const float amp = decay_amp(a.A_dec, h);
+    float dtau_acc = 0.f, dadec_acc = 0.f;   // this thread's channel (tid < K), over the sweep
 
     for (int idx = tid; idx < V * K; idx += kThreads)
         dS[(idx / K) * KP + idx % K] = a.dS_final ? a.dS_final[(size_t)u * V * K + idx] : 0.f;
@@ -285,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
         const int nl = T - (NC - 1) * L;
         dox[tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * V + tid] / (float)nl : 0.f;
     }
-    for (int idx = tid; idx < K * R + R * V + R; idx += kThreads) wsu[idx] = 0.f;
+    for (int idx = tid; idx < rec; idx += kThreads) wsu[idx] = 0.f;
     __syncthreads();
 
     for (int c = NC - 1; c >= 0; --c) {
@@ -317,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
                 const size_t g = tk(b, s0 + t, h, i, T, H, K);
                 qs[t * KP + i] = ld_io(q + g);
                 ks[t * KP + i] = ld_io(kk + g);
-                lam[t * KP + i] = log_retention(a.g_logit[g], a.bx[g] + delta[i]);
+                lam[t * KP + i] = log_retention(a.g_logit[g], a.bx[g] + delta[i], amp, decay_bias(a.tau, h, i, K));
             }
             for (int idx = tid; idx < kSub * V; idx += kThreads) {
                 const int t = idx / V, r = idx % V;
@@ -523,7 +528,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
                     run += dls[t * KP + tid];
                     const size_t g = tk(b, s0 + t, h, tid, T, H, K);
                     const float beta = a.bx[g] + delta[tid];
-                    a.dg_logit[g] = -sigmoid_f(a.g_logit[g]) * run;
+                    // log g = -amp softplus(g_logit + tau): d/dg_logit = d/dtau = -amp sigmoid(.),
+                    // d/dA_dec = log g
+                    const float x = a.g_logit[g] + decay_bias(a.tau, h, tid, K);
+                    const float dgl = -amp * sigmoid_f(x) * run;
+                    a.dg_logit[g] = dgl;
+                    dtau_acc += dgl;
+                    dadec_acc += run * (-amp * softplus_f(x));
                     const float dbeta = sigmoid_f(-beta) * run;
                     a.dbx[g] = dbeta;
                     ddelta[tid] += dbeta;
@@ -594,20 +605,38 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
     if (a.dS0)
         for (int idx = tid; idx < V * K; idx += kThreads) a.dS0[(size_t)u * V * K + idx] = dS[(idx / K) * KP + idx % K];
     if (a.mc_mode == 0 && a.dm_prev_in && tid < V) a.dm_prev_in[(size_t)u * V + tid] = 0.f;
+    if (a.A_dec || a.tau) {   // the decay parameters' partials of this unit (fixed-order sum)
+        if (tid < K) {
+            wsu[K * R + R * V + R + tid] = dtau_acc;
+            vecK[tid] = dadec_acc;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float s = 0.f;
+            for (int i = 0; i < K; ++i) s += vecK[i];
+            wsu[K * R + R * V + R + K] = s;
+        }
+    }
 }
 
-// dA[h] = sum_b ws[b,h][:K*R],  dB[h] = sum_b ws[b,h][K*R : K*R+R*V],  dAw[h] = the last R
-// (fixed order over b)
-__global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, float *dAw, int B, int H, int KR, int RV,
-                                   int R) {
+// Per-head sums over b (fixed order) of the unit records [dA K*R | dB R*V | dAw R | dtau K | dA_dec 1]
+__global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, float *dAw, float *dtau, float *dA_dec,
+                                   int B, int H, int KR, int RV, int R, int K) {
     const int h = blockIdx.y;
     const int x = blockIdx.x * blockDim.x + threadIdx.x;
-    if (x >= KR + RV + R) return;
+    const int rec = KR + RV + R + K + 1;
+    if (x >= rec) return;
     float s = 0.f;
-    for (int b = 0; b < B; ++b) s += ws[((size_t)b * H + h) * (KR + RV + R) + x];
+    for (int b = 0; b < B; ++b) s += ws[((size_t)b * H + h) * rec + x];
     if (x < KR) dA[(size_t)h * KR + x] = s;
     else if (x < KR + RV) dB[(size_t)h * RV + (x - KR)] = s;
-    else if (dAw) dAw[(size_t)h * R + (x - KR - RV)] = s;
+    else if (x < KR + RV + R) {
+        if (dAw) dAw[(size_t)h * R + (x - KR - RV)] = s;
+    } else if (x < rec - 1) {
+        if (dtau) dtau[(size_t)h * K + (x - KR - RV - R)] = s;
+    } else if (dA_dec) {
+        dA_dec[h] = s;
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -629,8 +658,8 @@ cudaError_t launch_bwd_simt_t(const BwdArgs &a, float *dA, float *dB, cudaStream
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int KR = K * a.R, RV = a.R * V;
-    dim3 grid((KR + RV + a.R + 255) / 256, a.H);
-    reduce_dAdB_kernel<<<grid, 256, 0, st>>>(a.ws, dA, dB, a.dAw, a.B, a.H, KR, RV, a.R);
+    dim3 grid((KR + RV + a.R + K + 1 + 255) / 256, a.H);
+    reduce_dAdB_kernel<<<grid, 256, 0, st>>>(a.ws, dA, dB, a.dAw, a.dtau, a.dA_dec, a.B, a.H, KR, RV, a.R, K);
     return cudaGetLastError();
 }
 

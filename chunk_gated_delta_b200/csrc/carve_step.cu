@@ -29,6 +29,7 @@ namespace carve {
 struct StepArgs {
     const void *q, *k, *v;
     const float *g_logit, *bx, *w_logit, *A, *Bm, *Aw;
+    const float *A_dec, *tau;   // [H], [H,K] or null: the decay's log-amplitude and bias
     float *S, *mstate;
     int *pos;
     void *o;
@@ -191,6 +192,8 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
                 sm.msum[tid] = msum;
             }
         }
+        // the decay's log-amplitude and this thread's channel bias, used in the gate phase
+        const float pAdec = a.A_dec ? a.A_dec[h] : 0.f, ptau = a.tau ? a.tau[(size_t)h * K + tid / TPK] : 0.f;
         float pB[ZP][VP], pA[AP];
 #pragma unroll
         for (int zp = 0; zp < ZP; ++zp) {
@@ -278,10 +281,15 @@ __global__ void __launch_bounds__(kGroupThreads *NGRP, 1) step_kernel(StepArgs a
                 sm.w = sigmoid_f(sm.tok[i & 1].wl[0] + dw);
             }
             if (part == 0) {
-                // a = sigma(-g_logit) sigma(bx + Delta) = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)}))
-                const float e1 = __expf(sm.glv[kk]), e2 = __expf(-(sm.bxv[kk] + acc));
-                const float av = __fdividef(1.f, (1.f + e1) * (1.f + e2));
-                sm.av[kk] = av;
+                // a = sigma(-g_logit) sigma(bx + Delta) = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)}));
+                // with the decay's amplitude and bias, 1 / g = e^{amp softplus(g_logit + tau)}
+                const float e2 = __expf(-(sm.bxv[kk] + acc));
+                float ig;
+                if (a.A_dec || a.tau)
+                    ig = __expf(expf(pAdec) * softplus_f(sm.glv[kk] + ptau));
+                else
+                    ig = 1.f + __expf(sm.glv[kk]);
+                sm.av[kk] = __fdividef(1.f, ig * (1.f + e2));
             }
         }
         group_sync(grp);
@@ -407,9 +415,9 @@ cudaError_t dispatch_step(int K, int V, const StepArgs &a, cudaStream_t st) {
 
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit, const float *A,
-                        const float *Bm, const float *Aw, float *S, float *mstate, int *pos, void *o, int B,
-                        int H, int R, int L, int mc_mode, cudaStream_t st) {
-    StepArgs a{q, k, v, g_logit, bx, w_logit, A, Bm, Aw, S, mstate, pos, o, B, H, R, L, mc_mode};
+                        const float *Bm, const float *Aw, const float *A_dec, const float *tau, float *S,
+                        float *mstate, int *pos, void *o, int B, int H, int R, int L, int mc_mode, cudaStream_t st) {
+    StepArgs a{q, k, v, g_logit, bx, w_logit, A, Bm, Aw, A_dec, tau, S, mstate, pos, o, B, H, R, L, mc_mode};
     return bf16 ? dispatch_step<__nv_bfloat16>(K, V, a, st) : dispatch_step<float>(K, V, a, st);
 }
 

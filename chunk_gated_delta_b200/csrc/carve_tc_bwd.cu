@@ -16,7 +16,9 @@
 //                Gkb = U (dS1 Fm)                          (the Kbar part of Gkc)
 //                dLam = Qm Gq + Krm Gkr - Kcm (Gkc + Gkb)
 //                       (+ sum_s Kbar_s dKbar_s + gamma colsum(S0 * dS1) at the chunk's last token)
-//   gates      dl = reverse cumsum of dLam; d g_logit = -sigma(g_logit) dl; dbx = sigma(-beta) dl
+//   gates      dl = reverse cumsum of dLam; d g_logit = -amp sigma(g_logit + tau) dl (amp = 1,
+//              tau = 0 without the decay parameters; d tau sums it, d A_dec sums dl log g);
+//              dbx = sigma(-beta) dl
 // (Qm, Krm, Kcm: mid-block referenced operands; Em, Fm, C: the block-level decay factors of the
 // forward.)  The content path (dz = A^T dDelta, dm = B^T dz) closes each gate chunk; with the
 // boundary-state readout its term in dq (S0^T dm / n for every token of the gate chunk) is
@@ -60,6 +62,8 @@ struct __align__(16) TcBwdSmem {
 
 __device__ int g_tc_bwd_timeout;
 
+// DEC: the decay has its amplitude and bias (a.A_dec or a.tau given)
+template <bool DEC>
 __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_constant__ BwdMaps maps) {
     constexpr int C = kBC, NB = kBNB;
     extern __shared__ __align__(128) unsigned char smraw[];
@@ -81,6 +85,11 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     float *wsv = a.ws + (size_t)a.B * a.H * NG * kTcGradRec + (size_t)u * NG * 128;
     // gate phases: channel pair c0 = 2 cp, 2 cp + 1 over tokens 8 hf + [0, 8) of 16-token block ib
     const int cp = tid & 63, hf = (tid >> 6) & 1, ib = tid >> 7, c0 = 2 * cp;
+    // the decay's amplitude and this thread's channel biases; its partial sums of d tau (two
+    // channels) and d A_dec over the sweep
+    const float amp = DEC ? decay_amp(a.A_dec, h) : 1.f;
+    const float tb[2] = {DEC ? decay_bias(a.tau, h, c0, 128) : 0.f, DEC ? decay_bias(a.tau, h, c0 + 1, 128) : 0.f};
+    float dtp[2] = {0.f, 0.f}, dap = 0.f;
 
     float ds[16][4];
 #pragma unroll
@@ -235,8 +244,13 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             float av[2][8], ia[2][8], rf[2][8], cf[2][8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-                retention(glr[t].x, bxr[t].x + dl0, av[0][t], ia[0][t]);
-                retention(glr[t].y, bxr[t].y + dl1, av[1][t], ia[1][t]);
+                if constexpr (DEC) {
+                    retention_dec(glr[t].x + tb[0], amp, bxr[t].x + dl0, av[0][t], ia[0][t]);
+                    retention_dec(glr[t].y + tb[1], amp, bxr[t].y + dl1, av[1][t], ia[1][t]);
+                } else {
+                    retention(glr[t].x, bxr[t].x + dl0, av[0][t], ia[0][t]);
+                    retention(glr[t].y, bxr[t].y + dl1, av[1][t], ia[1][t]);
+                }
             }
             if (hf == 0) {
 #pragma unroll
@@ -831,11 +845,21 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 for (int e = 0; e < 2; ++e) {
                     run[e] += e ? d2.y : d2.x;
                     if (t == 7) run[e] += xl[e];
-                    const float e1 = __expf(e ? glr[t].y : glr[t].x), e2 = __expf(-((e ? bxr[t].y : bxr[t].x) + dl[e]));
-                    const float D = (1.f + e1) * (1.f + e2);
-                    const bool floor = !(__fdividef(1.f, D) >= kAMin);
-                    dg[e] = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run[e];
-                    db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
+                    const float gx = e ? glr[t].y : glr[t].x, e2 = __expf(-((e ? bxr[t].y : bxr[t].x) + dl[e]));
+                    if constexpr (DEC) {   // log g = -amp softplus(x), x = g_logit + tau: d/dx = -amp sigmoid(x)
+                        const float x = gx + tb[e], e1 = __expf(x), sp = softplus_fast(x, e1);
+                        const bool floor = !(__fdividef(1.f, __expf(amp * sp) * (1.f + e2)) >= kAMin);
+                        dg[e] = floor ? 0.f : -amp * sigmoid_fast(x, e1) * run[e];
+                        db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
+                        dtp[e] += dg[e];
+                        dap += floor ? 0.f : run[e] * (-amp * sp);   // d A_dec = dlog a . log g
+                    } else {
+                        const float e1 = __expf(gx);
+                        const float D = (1.f + e1) * (1.f + e2);
+                        const bool floor = !(__fdividef(1.f, D) >= kAMin);
+                        dg[e] = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run[e];
+                        db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
+                    }
                     pdd[e] += db[e];
                 }
                 // staged in this thread's own positions for the vectorised stores below
@@ -938,6 +962,38 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         }
     }
     if (a.mc_mode == 0 && a.dm_prev_in && tid < 128) a.dm_prev_in[(size_t)u * 128 + tid] = 0.f;
+    if constexpr (DEC) {   // this unit's d tau (the four threads of each channel pair) and d A_dec, fixed order
+        float *red = sm.xp;   // free after the sweep: [256][2] channel partials, then [256] amplitude
+        *reinterpret_cast<float2 *>(&red[2 * tid]) = make_float2(dtp[0], dtp[1]);
+        red[512 + tid] = dap;
+        __syncthreads();
+        float *dst = a.ws + (size_t)a.B * a.H * NG * (kTcGradRec + 128) + (size_t)u * kTcDecayRec;
+        if (tid < 128) {
+            const int pr = tid >> 1, e = tid & 1;
+            dst[tid] = ((red[2 * pr + e] + red[2 * (pr + 64) + e]) + red[2 * (pr + 128) + e]) + red[2 * (pr + 192) + e];
+        }
+        if (warp == 0) {
+            float x = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x += red[512 + 8 * lane + j];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+            if (lane == 0) dst[128] = x;
+        }
+    }
+}
+
+// d tau [H,128] and d A_dec [H]: sums over b (fixed order) of the units' decay records
+__global__ void reduce_decay_kernel(const float *part, float *dtau, float *dA_dec, int B, int H) {
+    const int h = blockIdx.x, i = threadIdx.x;   // 128 threads
+    float s = 0.f, s2 = 0.f;
+    for (int b = 0; b < B; ++b) {
+        const float *r = part + ((size_t)b * H + h) * kTcDecayRec;
+        s += r[i];
+        if (i == 0) s2 += r[128];
+    }
+    if (dtau) dtau[(size_t)h * 128 + i] = s;
+    if (i == 0 && dA_dec) dA_dec[h] = s2;
 }
 
 
@@ -1053,7 +1109,9 @@ __global__ void dq_readout_kernel(__nv_bfloat16 *dq, const float *vec, int H, in
 
 cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st) {
     const int bytes = (int)sizeof(TcBwdSmem);
-    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(tc_bwd_kernel), bytes);
+    const bool dec = a.A_dec || a.tau;
+    auto kern = dec ? tc_bwd_kernel<true> : tc_bwd_kernel<false>;
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), bytes);
     if (e != cudaSuccess) return e;
     const long long rows = (long long)a.B * a.T;
     BwdMaps maps;
@@ -1061,7 +1119,7 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
     if ((e = make_token_tile_map(&maps.k, a.k, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
     if ((e = make_token_tile_map(&maps.v, a.v, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
     if ((e = make_token_tile_map(&maps.dO, a.dO, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
-    tc_bwd_kernel<<<a.B * a.H, 256, bytes, st>>>(a, maps);
+    kern<<<a.B * a.H, 256, bytes, st>>>(a, maps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.mc_mode == 0) {
         const size_t rows = (size_t)a.B * a.T * a.H;
@@ -1071,7 +1129,12 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int NG = (a.T + a.L - 1) / a.L, S = tc_reduce_slices(a.B, NG);
-    float *part = a.ws + (size_t)a.B * a.H * NG * (kTcGradRec + 128);
+    const float *dec_part = a.ws + (size_t)a.B * a.H * NG * (kTcGradRec + 128);
+    float *part = const_cast<float *>(dec_part) + (size_t)a.B * a.H * kTcDecayRec;
+    if (dec) {
+        reduce_decay_kernel<<<a.H, 128, 0, st>>>(dec_part, a.dtau, a.dA_dec, a.B, a.H);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     reduce_dAdB_partial_kernel<<<dim3(a.H, S), 256, 0, st>>>(a.ws, a.saved_aux, part, a.B, a.H, NG, a.R);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     reduce_dAdB_final_kernel<<<(a.H * 257 * a.R + 255) / 256, 256, 0, st>>>(part, dA, dB, a.dAw, a.H, a.R, S);

@@ -22,6 +22,21 @@ __device__ __forceinline__ void retention(float g_logit, float beta, float &a, f
     inv_a = floor ? kInvAMin : D;
 }
 
+// softplus(x) and sigmoid(x) from one fast exponential; beyond x = 15, log(1 + e^x) is x and
+// sigmoid(x) is 1 to fp32 rounding (and e^x may overflow), so both take those values there
+__device__ __forceinline__ float softplus_fast(float x, float e1) { return x > 15.f ? x : __logf(1.f + e1); }
+__device__ __forceinline__ float sigmoid_fast(float x, float e1) { return x > 15.f ? 1.f : __fdividef(e1, 1.f + e1); }
+
+// The same with the decay's amplitude and bias: 1 / g = e^{amp softplus(x)}, x = g_logit + tau
+// (the product form above is its amp = 1, tau = 0 case, evaluated with fewer operations).
+__device__ __forceinline__ void retention_dec(float x, float amp, float beta, float &a, float &inv_a) {
+    const float D = __expf(amp * softplus_fast(x, __expf(x))) * (1.f + __expf(-beta));
+    const float r = __fdividef(1.f, D);
+    const bool floor = !(r >= kAMin);
+    a = floor ? kAMin : r;
+    inv_a = floor ? kInvAMin : D;
+}
+
 // Mid-block references of one 16-token block from its retentions av (and reciprocals ia):
 // rf[t] = e^{Lam_t - Lam_7}, cf[t] = 1 / rf[t], both as running products from token 7.
 __device__ __forceinline__ void mid_reference(const float (&av)[16], const float (&ia)[16], float (&rf)[16],

@@ -7,7 +7,8 @@
 // state never round-trips through memory except when it is saved for the backward.
 //
 // Per compute chunk (CARVE blog section 2.3: one WY solve shared by all value channels):
-//   gates      a_t = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)})), floored at e^-10, and its
+//   gates      a_t = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)})) (with the decay amplitude and
+//              bias: 1 / g = e^{amp softplus(g_logit + tau)}), floored at e^-10, and its
 //              reciprocal (free), per key channel
 //   operands   mid-block referenced q*e^{Lam_t - Lam_m}, k*e^{Lam_t - Lam_m}, k*e^{Lam_m - Lam_s}
 //              (m = middle of the token's 16-block) built from running products of a and 1/a,
@@ -56,7 +57,8 @@ struct TileMaps {
     CUtensorMap q, k, v, gl, bx;
 };
 
-template <int NB>
+// DEC: the decay has its amplitude and bias (a.A_dec or a.tau given)
+template <int NB, bool DEC>
 __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_constant__ TileMaps maps) {
     using SM = TcFwdSmem<NB>;
     constexpr int C = SM::C, LDA = SM::LDA;
@@ -72,6 +74,10 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     const size_t tstride = (size_t)H * 128;
     const size_t base_bh = (size_t)b * T * tstride + (size_t)h * 128;   // token 0 of this unit
     const int v0 = 16 * warp + g, v1 = v0 + 8;
+    // the decay's amplitude and the biases of this thread's gate channels 2 (tid & 63) + {0, 1}
+    const float amp = DEC ? decay_amp(a.A_dec, h) : 1.f;
+    const float tb0 = DEC ? decay_bias(a.tau, h, 2 * (tid & 63), 128) : 0.f;
+    const float tb1 = DEC ? decay_bias(a.tau, h, 2 * (tid & 63) + 1, 128) : 0.f;
 
     float s[16][4];
 #pragma unroll
@@ -256,8 +262,13 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                         gv = glr[x][t];
                         bv = bxr[x][t];
                     }
-                    retention(gv.x, bv.x + dl0, av[0][t], ia[0][t]);
-                    retention(gv.y, bv.y + dl1, av[1][t], ia[1][t]);
+                    if constexpr (DEC) {
+                        retention_dec(gv.x + tb0, amp, bv.x + dl0, av[0][t], ia[0][t]);
+                        retention_dec(gv.y + tb1, amp, bv.y + dl1, av[1][t], ia[1][t]);
+                    } else {
+                        retention(gv.x, bv.x + dl0, av[0][t], ia[0][t]);
+                        retention(gv.y, bv.y + dl1, av[1][t], ia[1][t]);
+                    }
                 }
                 float rf[2][8], cf[2][8];
                 if (hf == 0) {
@@ -592,7 +603,7 @@ __global__ void __launch_bounds__(256) qbar_kernel(const __nv_bfloat16 *q, float
 
 template <int NB>
 cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
-    auto kern = tc_fwd_kernel<NB>;
+    auto kern = (a.A_dec || a.tau) ? tc_fwd_kernel<NB, true> : tc_fwd_kernel<NB, false>;
     const int bytes = (int)sizeof(TcFwdSmem<NB>);
     cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), bytes);
     if (e != cudaSuccess) return e;

@@ -16,7 +16,9 @@
  *                                                     of m_c also biases the write gate, CARVE
  *                                                     blog section 2.2, Figure 1)
  *     for t in c:
- *       a_t = exp(-softplus(g_logit_t)) * sigmoid(bx_t + Delta)      (key axis, length dk)
+ *       a_t = exp(-e^{A_dec} softplus(g_logit_t + tau)) * sigmoid(bx_t + Delta)   (key axis, length dk;
+ *             A_dec, the head's log-decay amplitude, and tau, the per-channel bias, are optional
+ *             (0 when NULL): the fused decay of CARVE blog section 2.3)
  *       w_t = sigmoid(w_logit_t + dw_c)                               (one scalar per head)
  *       S_t = S_{t-1} Diag(a_t) + w_t (v_t - S_{t-1} Diag(a_t) k_t) k_t^T
  *       o_t = S_t q_t
@@ -37,6 +39,8 @@
  *   g_logit, bx    [B, T, H, dk]  float     w_logit        [B, T, H]      float
  *   A              [H, dk, rank]  float     Bm             [H, rank, dv]  float
  *   Aw             [H, rank]      float (nullable: no content term on the write gate)
+ *   A_dec          [H]            float (nullable: decay amplitude e^0 = 1)
+ *   tau            [H, dk]        float (nullable: decay bias 0)
  *   S0, S_final    [B, H, dv, dk] float     m vectors      [B, H, dv]     float
  * Gradients have the layout and dtype of the tensor they belong to.  Every device pointer
  * must be 16-byte aligned.
@@ -91,6 +95,7 @@ size_t carve_bwd_workspace_bytes(const carve_dims *d);
  * carve_fwd -- the forward recurrence over T tokens (the chunked WY evaluation of the
  * definition above; CARVE blog sections 2.1-2.3, paperdance abstract).
  *   Aw          nullable: the write gate's content factor (dw_c = 0 when NULL)
+ *   A_dec, tau  nullable, independently: the decay's log-amplitude and bias (0 when NULL)
  *   S0          nullable: initial state (treated as 0 when NULL)
  *   m_prev_in   nullable: mc_mode 1 content signal for the first chunk (0 when NULL)
  *   o           out: outputs
@@ -101,9 +106,9 @@ size_t carve_bwd_workspace_bytes(const carve_dims *d);
  */
 carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
                        const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *Aw, const float *S0,
-                       const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
-                       void *saved, void *stream);
+                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                       const float *tau, const float *S0, const float *m_prev_in, void *o,
+                       float *S_final, float *m_prev_out, void *saved, void *stream);
 
 /*
  * carve_bwd -- reverse sweep over the chunks: gradients of
@@ -114,17 +119,19 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
  *   dS_final, dm_prev_out   nullable (0 when NULL)
  *   Aw, dAw                 both NULL (no write-gate content term) or both given; dAw is
  *                           overwritten with the gradient summed over the batch
+ *   A_dec, dA_dec; tau, dtau  each pair both NULL or both given; dA_dec [H] and dtau [H, dk]
+ *                           are overwritten with the gradients summed over the batch
  *   dS0, dm_prev_in         nullable outputs
  *   workspace               carve_bwd_workspace_bytes(d) bytes of scratch
  */
 carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const void *v,
                        const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *Aw, const float *S0,
-                       const float *m_prev_in, const void *saved, const void *dO,
-                       const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
-                       void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
-                       float *dB, float *dAw, float *dS0, float *dm_prev_in, void *workspace,
-                       void *stream);
+                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                       const float *tau, const float *S0, const float *m_prev_in, const void *saved,
+                       const void *dO, const float *dS_final, const float *dm_prev_out, void *dq,
+                       void *dk, void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
+                       float *dB, float *dAw, float *dA_dec, float *dtau, float *dS0,
+                       float *dm_prev_in, void *workspace, void *stream);
 
 /*
  * carve_bwd_noalloc -- carve_bwd without a workspace argument, for callers that cannot
@@ -136,8 +143,8 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
  * Arguments, layouts, results and errors are those of carve_bwd.  The scratch is a 4 MiB
  * array inside the library, present on every GPU that loads it until the process exits, so
  * the call allocates nothing.  Limit: carve_bwd_workspace_bytes(d) <= 4 MiB, that is
- * B*H*(dk*rank + rank*dv + rank) floats, or, when the tensor-core kernels run (bf16,
- * dk = dv = 128, rank <= 32), B*H*NG*292 + ceil(B*NG/64)*H*257*rank floats with
+ * B*H*(dk*rank + rank*dv + rank + dk + 1) floats, or, when the tensor-core kernels run (bf16,
+ * dk = dv = 128, rank <= 32), B*H*(NG*292 + 132) + ceil(B*NG/64)*H*257*rank floats with
  * NG = ceil(T/chunk); larger problems return
  * CARVE_ERR_UNSUPPORTED without launching anything.
  * The first call on each device looks up the array's device address (with that device
@@ -147,11 +154,12 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
  */
 carve_status carve_bwd_noalloc(const carve_dims *d, const void *q, const void *k, const void *v,
                                const float *g_logit, const float *bx, const float *w_logit,
-                               const float *A, const float *Bm, const float *Aw, const float *S0,
-                               const float *m_prev_in, const void *saved, const void *dO,
-                               const float *dS_final, const float *dm_prev_out, void *dq,
-                               void *dk, void *dv, float *dg_logit, float *dbx,
-                               float *dw_logit, float *dA, float *dB, float *dAw, float *dS0,
+                               const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                               const float *tau, const float *S0, const float *m_prev_in,
+                               const void *saved, const void *dO, const float *dS_final,
+                               const float *dm_prev_out, void *dq, void *dk, void *dv,
+                               float *dg_logit, float *dbx, float *dw_logit, float *dA, float *dB,
+                               float *dAw, float *dA_dec, float *dtau, float *dS0,
                                float *dm_prev_in, void *stream);
 
 /*
@@ -165,12 +173,14 @@ carve_status carve_bwd_noalloc(const carve_dims *d, const void *q, const void *k
  *              of the previous block) and pos [B,H] int32 the tokens consumed so far; both
  *              are updated in place.  Unused (may be NULL) in mc_mode 0.
  * Inputs: q, k [B,H,dk] io; v [B,H,dv] io; g_logit, bx [B,H,dk] float; w_logit [B,H]
- * float.  S [B,H,dv,dk] float is read and written in place; o [B,H,dv] io.
+ * float; Aw, A_dec, tau nullable as in carve_fwd.  S [B,H,dv,dk] float is read and written
+ * in place; o [B,H,dv] io.
  */
 carve_status carve_step(const carve_dims *d, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit,
-                        const float *A, const float *Bm, const float *Aw, float *S, float *mstate,
-                        int32_t *pos, void *o, void *stream);
+                        const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                        const float *tau, float *S, float *mstate, int32_t *pos, void *o,
+                        void *stream);
 
 /*
  * carve_check -- blocks the host until the work queued on `stream` has finished, then

@@ -56,7 +56,7 @@ def test_buffer_sizes(lib):
     states = units * (128 // 16) * 64 * 128
     aux = units * 2 * (64 + 8 + 128)
     assert carve.saved_bytes(d) == 4 * (states + aux)
-    assert carve.bwd_workspace_bytes(d) == 4 * units * (128 * 8 + 8 * 64 + 8)
+    assert carve.bwd_workspace_bytes(d) == 4 * units * (128 * 8 + 8 * 64 + 8 + 128 + 1)
     for bad in (dict(dk=96), dict(T=100), dict(chunk=48), dict(rank=65), dict(io=3), dict(mc_mode=2), dict(B=0),
                 dict(T=0)):
         assert carve.saved_bytes(good_dims(**bad)) == 0, bad
@@ -70,11 +70,29 @@ def test_bad_dims_rejected(lib, bad, code):
     """Dimension checks run first, so the (fake) pointers below are never dereferenced."""
     d = good_dims(**bad)
     P = ctypes.c_void_p(4096)
-    assert lib.carve_fwd(ctypes.byref(d), *([P] * 8), None, None, None, P, None, None, None, None) == code
-    assert lib.carve_bwd(ctypes.byref(d), *([P] * 8), None, None, None, P, P, None, None, *([P] * 8), None, None,
-                         None, P, None) == code
+    assert lib.carve_fwd(ctypes.byref(d), *fwd_args(P)) == code
+    assert lib.carve_bwd(ctypes.byref(d), *bwd_args(P)) == code
     if "T" not in bad and "chunk" not in bad:       # decode ignores T and (in mode 0) chunk
-        assert lib.carve_step(ctypes.byref(d), *([P] * 8), None, P, None, None, P, None) == code
+        assert lib.carve_step(ctypes.byref(d), *step_args(P)) == code
+
+
+# Valid argument lists (P: a 16-byte aligned placeholder; None where a pointer is optional).
+# fwd: 8 inputs 0-7, Aw 8, A_dec 9, tau 10, S0 11, m_prev_in 12, o 13, S_final 14,
+#      m_prev_out 15, saved 16, stream 17
+def fwd_args(P):
+    return [P] * 8 + [None] * 5 + [P, None, None, None, None]
+
+
+# bwd: 8 inputs 0-7, Aw 8, A_dec 9, tau 10, S0 11, m_prev_in 12, saved 13, dO 14, dS_final 15,
+#      dm_prev_out 16, dq..dB 17-24, dAw 25, dA_dec 26, dtau 27, dS0 28, dm_prev_in 29,
+#      workspace 30, stream 31
+def bwd_args(P):
+    return [P] * 8 + [None] * 5 + [P, P, None, None] + [P] * 8 + [None] * 5 + [P, None]
+
+
+# step: 8 inputs 0-7, Aw 8, A_dec 9, tau 10, S 11, mstate 12, pos 13, o 14, stream 15
+def step_args(P):
+    return [P] * 8 + [None] * 3 + [P, None, None, P, None]
 
 
 def test_null_and_misaligned_pointers_rejected(lib):
@@ -82,34 +100,38 @@ def test_null_and_misaligned_pointers_rejected(lib):
     the host with CARVE_ERR_INVALID_ARG before any launch."""
     d = good_dims()
     P = ctypes.c_void_p(4096)
-    fwd_ok = [P] * 8 + [None, None, None, P, None, None, None, None]
-    for j in (0, 1, 2, 3, 4, 5, 6, 7, 11):              # each required forward pointer
+    fwd_ok = fwd_args(P)
+    for j in (0, 1, 2, 3, 4, 5, 6, 7, 13):              # each required forward pointer
         args = list(fwd_ok)
         args[j] = None
         assert lib.carve_fwd(ctypes.byref(d), *args) == 1, j
         args[j] = ctypes.c_void_p(4100)                 # misaligned
         assert lib.carve_fwd(ctypes.byref(d), *args) == 1, j
-    for j in (8, 9, 10, 12, 13, 14):                    # optional pointers: misaligned is rejected
+    for j in (8, 9, 10, 11, 12, 14, 15, 16):            # optional pointers: misaligned is rejected
         args = list(fwd_ok)
         args[j] = ctypes.c_void_p(4104)
         assert lib.carve_fwd(ctypes.byref(d), *args) == 1, j
-    # bwd: 8 inputs, Aw 8, S0 9, m_prev_in 10, saved 11, dO 12, dS_final 13, dm_prev_out 14,
-    #      dq..dB 15-22, dAw 23, dS0 24, dm_prev_in 25, workspace 26, stream 27
-    bwd_ok = [P] * 8 + [None, None, None, P, P, None, None] + [P] * 8 + [None, None, None, P, None]
-    for j in (11, 12, 15, 16, 17, 18, 19, 20, 21, 22, 26):
+    bwd_ok = bwd_args(P)
+    for j in (13, 14, 17, 18, 19, 20, 21, 22, 23, 24, 30):
         args = list(bwd_ok)
         args[j] = None
         assert lib.carve_bwd(ctypes.byref(d), *args) == 1, j
-    args = list(bwd_ok)
-    args[8] = P                                         # Aw without dAw
-    assert lib.carve_bwd(ctypes.byref(d), *args) == 1
-    args = list(bwd_ok)
-    args[23] = P                                        # dAw without Aw
-    assert lib.carve_bwd(ctypes.byref(d), *args) == 1
+    for x, dx in ((8, 25), (9, 26), (10, 27)):          # Aw / A_dec / tau and their gradients come in pairs
+        args = list(bwd_ok)
+        args[x] = P
+        assert lib.carve_bwd(ctypes.byref(d), *args) == 1, (x, "without its gradient")
+        args = list(bwd_ok)
+        args[dx] = P
+        assert lib.carve_bwd(ctypes.byref(d), *args) == 1, (dx, "without its parameter")
     ds = good_dims(mc_mode=1)
-    assert lib.carve_step(ctypes.byref(ds), *([P] * 8), None, P, None, None, P, None) == 1   # needs mstate, pos
-    assert lib.carve_step(ctypes.byref(d), *([P] * 8), None, None, None, None, P, None) == 1  # S missing
-    assert lib.carve_step(ctypes.byref(d), *([P] * 8), ctypes.c_void_p(4104), P, None, None, P, None) == 1
+    assert lib.carve_step(ctypes.byref(ds), *step_args(P)) == 1   # needs mstate, pos
+    args = step_args(P)
+    args[11] = None                                     # S missing
+    assert lib.carve_step(ctypes.byref(d), *args) == 1
+    for j in (8, 9, 10):                                # misaligned Aw, A_dec, tau
+        args = step_args(P)
+        args[j] = ctypes.c_void_p(4104)
+        assert lib.carve_step(ctypes.byref(d), *args) == 1, j
     assert lib.carve_fwd(None, *fwd_ok) == 1
 
 

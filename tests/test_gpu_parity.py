@@ -301,33 +301,46 @@ def test_decode_shapes_all_units(cuda_device, K, V, io):
 
 
 # ---------------------------------------------------------------------------------------
-# content term of the write gate: w = sigmoid(w_logit + Aw . z_c) (both kernel paths, decode)
+# content term of the write gate: w = sigmoid(w_logit + Aw . z_c), and the decay's amplitude
+# and bias: g = exp(-e^{A_dec} softplus(g_logit + tau))  (both kernel paths, decode)
 # ---------------------------------------------------------------------------------------
-def _write_term_case(cuda_device, w, L, mode):
+def _terms_case(cuda_device, w, L, mode, write=True, decay=False):
     import torch
     d = I.make_inputs(w)
     d["A"] *= 10.0
     d["B"] *= 10.0
-    d["Aw"] = I.normal(w.seed, 97, (w.H, w.R), 0.0, 2.0)
+    extra, grads = {}, ()
+    if write:
+        d["Aw"] = I.normal(w.seed, 97, (w.H, w.R), 0.0, 2.0)
+        grads += ("dAw",)
+    if decay:
+        d.update(I.make_decay(w))
+        grads += ("dA_dec", "dtau")
     dO = I.make_grad_out(w)
     S0 = I.make_state(w, 0.05)
     mp = I.normal(3, 2, (w.B, w.H, w.V)).astype(np.float32)
     dSf = I.normal(3, 3, (w.B, w.H, w.V, w.K)).astype(np.float32)
     dd = to_dev(dict(d, dO=dO), w.io, cuda_device)
-    Aw = torch.from_numpy(d["Aw"].astype(np.float32)).to(cuda_device)
+    for key in ("Aw", "A_dec", "tau"):
+        if key in d:
+            extra[key] = torch.from_numpy(np.asarray(d[key], dtype=np.float32)).to(cuda_device)
     tS0, tmp, tdS = (torch.from_numpy(x).to(cuda_device) for x in (S0, mp, dSf))
     args = (dd["q"], dd["k"], dd["v"], dd["g_logit"], dd["bx"], dd["w_logit"], dd["A"], dd["B"])
-    out = carve.carve_fwd(*args, chunk=L, mc_mode=mode, S0=tS0, m_prev_in=tmp, Aw=Aw)
+    out = carve.carve_fwd(*args, chunk=L, mc_mode=mode, S0=tS0, m_prev_in=tmp, **extra)
     g = carve.carve_bwd(*args, out["saved"], dd["dO"], chunk=L, mc_mode=mode, S0=tS0, m_prev_in=tmp,
-                        dS_final=tdS, Aw=Aw)
+                        dS_final=tdS, **extra)
     torch.cuda.synchronize()
     r = oracle.fwd(d, L=L, mc_mode=mode, S0=S0, m_prev=mp)
     rg = oracle.bwd(d, L, dO, mc_mode=mode, S0=S0, m_prev=mp, dS_final=dSf)
     tol = TOL[w.io]
     check("o", host(out["o"]), r["o"], tol)
     check("S_final", host(out["S_final"]), r["S_final"], tol)
-    for key in GRADS + ("dAw", "dS0"):
+    for key in GRADS + grads + ("dS0",):
         check(key, host(g[key]), rg[key], tol)
+    if decay and mode == 0:   # the forward-only path (64-token compute chunks on the tensor cores)
+        f = carve.carve_fwd(*args, chunk=L, mc_mode=mode, S0=tS0, m_prev_in=tmp, save_for_bwd=False, **extra)
+        torch.cuda.synchronize()
+        check("o (forward only)", host(f["o"]), r["o"], tol)
     return d, dd, args, tS0, tmp, tdS
 
 
@@ -338,7 +351,23 @@ def test_write_gate_term(cuda_device, path, mode):
         w = dataclasses.replace(I.FWD_1P3B, B=1, H=3, T=256, L=64, seed=61 + mode)
     else:
         w = dataclasses.replace(I.TINY_FP32, B=2, H=2, T=96, L=32, seed=63 + mode)
-    _write_term_case(cuda_device, w, w.L, mode)
+    _terms_case(cuda_device, w, w.L, mode)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("path", ["tensor_core", "simt"])
+def test_decay_amplitude_and_bias(cuda_device, path, mode):
+    if path == "tensor_core":
+        w = dataclasses.replace(I.FWD_1P3B, B=2, H=3, T=256, L=64, seed=71 + mode)
+    else:
+        w = dataclasses.replace(I.TINY_FP32, B=2, H=2, T=96, L=32, seed=73 + mode)
+    _terms_case(cuda_device, w, w.L, mode, write=False, decay=True)
+
+
+def test_decay_with_write_gate_term(cuda_device):
+    """Both optional terms at once on the tensor-core path, with a ragged last gate chunk."""
+    w = dataclasses.replace(I.FWD_1P3B, B=2, H=2, T=224, L=64, seed=75)
+    _terms_case(cuda_device, w, w.L, 0, write=True, decay=True)
 
 
 def test_zero_write_factor_is_bit_identical(cuda_device):
@@ -362,12 +391,17 @@ def test_zero_write_factor_is_bit_identical(cuda_device):
 
 
 @pytest.mark.parametrize("K,V,io", [(128, 128, "bf16"), (64, 64, "fp32")])
-def test_decode_write_gate_term(cuda_device, K, V, io):
+@pytest.mark.parametrize("decay", [False, True])
+def test_decode_write_gate_term(cuda_device, K, V, io, decay):
+    """The decode step with the write gate's content term, and (decay) also the decay's
+    amplitude and bias."""
     import torch
     w = dataclasses.replace(I.DECODE, B=4, H=8, K=K, V=V, R=16, io=io, seed=700 + K)
     steps, L = 12, 4
     pool = I.make_decode_pool(w, pool=steps)
     Aw_np = I.normal(w.seed, 96, (w.H, w.R), 0.0, 3.0)
+    dec_np = I.make_decay(w) if decay else {}
+    dec = {k: torch.from_numpy(v).to(cuda_device) for k, v in dec_np.items()}
     for mode in (0, 1):
         S_np = I.make_state(w, 0.05)
         tp = to_dev({k: pool[k] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}, io, cuda_device)
@@ -379,11 +413,12 @@ def test_decode_write_gate_term(cuda_device, K, V, io):
         pos = torch.zeros((w.B, w.H), dtype=torch.int32, device=cuda_device)
         outs = [host(carve.carve_step(tp["q"][j], tp["k"][j], tp["v"][j], tp["g_logit"][j], tp["bx"][j],
                                       tp["w_logit"][j], A, Bm, S, mc_mode=mode, chunk=L, mstate=mstate, pos=pos,
-                                      Aw=Aw)) for j in range(steps)]
+                                      Aw=Aw, **dec)) for j in range(steps)]
         Sr = S_np.astype(np.float64).copy()
         ms = np.zeros((w.B, w.H, 2, V))
         ps = np.zeros((w.B, w.H), dtype=np.int32)
         ref = [oracle.step({k: pool[k][j] for k in ("q", "k", "v", "g_logit", "bx", "w_logit")}, pool["A"],
-                           pool["B"], Sr, L=L, mc_mode=mode, mstate=ms, pos=ps, Aw=Aw_np) for j in range(steps)]
+                           pool["B"], Sr, L=L, mc_mode=mode, mstate=ms, pos=ps, Aw=Aw_np,
+                           **{k: v.astype(np.float64) for k, v in dec_np.items()}) for j in range(steps)]
         check(f"o mode {mode}", np.stack(outs), np.stack(ref), TOL[io])
         check(f"S mode {mode}", host(S), Sr, TOL[io])

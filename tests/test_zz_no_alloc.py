@@ -25,20 +25,20 @@ def _lib():
     build.build()
     lib = carve.load()
     f = lib.carve_bwd_noalloc
-    f.argtypes = [ctypes.POINTER(carve.Dims)] + [ctypes.c_void_p] * 27
+    f.argtypes = [ctypes.POINTER(carve.Dims)] + [ctypes.c_void_p] * 31
     f.restype = ctypes.c_int
     return lib
 
 
 def test_too_large_for_the_array_is_refused_before_any_launch():
-    """B*H*(dk*rank + rank*dv + rank) above 1,048,576 floats (4 MiB) returns
+    """B*H*(dk*rank + rank*dv + rank + dk + 1) above 1,048,576 floats (4 MiB) returns
     CARVE_ERR_UNSUPPORTED.  The size check comes first, so the placeholder pointers are never
     used."""
     lib = _lib()
     d = carve.Dims(B=5, H=16, T=64, dk=128, dv=128, rank=64, chunk=64, io=1, mc_mode=0)
     assert carve.bwd_workspace_bytes(d) > 4 << 20
     P = ctypes.c_void_p(4096)
-    args = [P] * 8 + [None, None, None, P, P, None, None] + [P] * 8 + [None, None, None, None]
+    args = [P] * 8 + [None] * 5 + [P, P, None, None] + [P] * 8 + [None] * 5 + [None]
     assert lib.carve_bwd_noalloc(ctypes.byref(d), *args) == 2
     fits = carve.Dims(B=3, H=16, T=64, dk=128, dv=128, rank=64, chunk=64, io=1, mc_mode=0)
     assert carve.bwd_workspace_bytes(fits) <= 4 << 20
@@ -65,9 +65,10 @@ def test_noalloc_backward_matches_carve_bwd_twice(cuda_device, io, mode):
     p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())   # noqa: E731
     for call in range(2):
         out = {k: torch.full_like(ref[k], float("nan")) for k in GRADS}
-        grads = [p(out[k]) for k in GRADS]   # ... dA, dB, (dAw: none), dS0, dm_prev_in
-        rc = lib.carve_bwd_noalloc(ctypes.byref(dims), *[p(t) for t in args], None, None, None, p(fwd["saved"]),
-                                   p(dd["dO"]), p(dSf), None, *grads[:8], None, *grads[8:], stream)
+        grads = [p(out[k]) for k in GRADS]   # ... dA, dB, (dAw, dA_dec, dtau: none), dS0, dm_prev_in
+        rc = lib.carve_bwd_noalloc(ctypes.byref(dims), *[p(t) for t in args], None, None, None, None, None,
+                                   p(fwd["saved"]), p(dd["dO"]), p(dSf), None, *grads[:8], None, None, None,
+                                   *grads[8:], stream)
         assert rc == 0, carve.STATUS.get(rc, rc)
         torch.cuda.synchronize()
         for k in GRADS:
