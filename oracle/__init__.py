@@ -41,8 +41,8 @@ def bind(path: str):
     """Load a compiled oracle library and declare its entry points."""
     lib = ctypes.CDLL(path)
     P = ctypes.c_void_p
-    lib.orc_fwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 16
-    lib.orc_bwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 29
+    lib.orc_fwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 17
+    lib.orc_bwd.argtypes = [ctypes.POINTER(_Dims)] + [P] * 30
     lib.orc_step.argtypes = [ctypes.POINTER(_Dims)] + [P] * 15
     for f in (lib.orc_fwd, lib.orc_bwd, lib.orc_step):
         f.restype = ctypes.c_int
@@ -67,56 +67,68 @@ def _p(x):
     return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
 
 
-def _dims(inp, L, mc_mode, content_off, T=None):
-    B, T_, H, K = inp["q"].shape
+def _dims(inp, L, mc_mode, content_off, cu=None):
+    B, T, H, K = inp["q"].shape
     V = inp["v"].shape[-1]
     R = inp["A"].shape[-1]
-    return _Dims(B, H, T_ if T is None else T, K, V, R, L, mc_mode, int(content_off))
+    if cu is not None:   # packed sequences: [1, T, H, *] tensors, len(cu) - 1 sequences
+        assert B == 1, "packed sequences use a leading dimension of 1"
+        B = len(cu) - 1
+    return _Dims(B, H, T, K, V, R, L, mc_mode, int(content_off))
+
+
+def _cu(cu_seqlens):
+    return None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
 
 
 _KEYS = ("q", "k", "v", "g_logit", "bx", "w_logit", "A", "B")
 
 
-def fwd(inp: dict, L: int, mc_mode: int = 0, S0=None, m_prev=None, content_off: bool = False):
+def fwd(inp: dict, L: int, mc_mode: int = 0, S0=None, m_prev=None, content_off: bool = False, cu_seqlens=None):
     """Forward over [B,T,H,*] inputs.  Optional entries: inp["Aw"] [H,R], the write gate's
     content term; inp["A_dec"] [H] and inp["tau"] [H,K], the decay's log-amplitude and bias.
+    cu_seqlens ([N+1] ints): N sequences packed along the token axis of [1,T,H,*] inputs;
+    S0, m_prev and the per-sequence outputs are then [N,H,...].
     Returns dict(o, S_final, m_prev_out) in fp64."""
     lib = _load()
-    d = _dims(inp, L, mc_mode, content_off)
+    cu = _cu(cu_seqlens)
+    d = _dims(inp, L, mc_mode, content_off, cu)
     a = [_f64(inp[k]) for k in _KEYS]
     Aw, S0, m_prev = _f64(inp.get("Aw")), _f64(S0), _f64(m_prev)
     A_dec, tau = _f64(inp.get("A_dec")), _f64(inp.get("tau"))
-    o = np.zeros((d.B, d.T, d.H, d.V))
+    o = np.zeros((1 if cu is not None else d.B, d.T, d.H, d.V))
     S = np.zeros((d.B, d.H, d.V, d.K))
     m = np.zeros((d.B, d.H, d.V))
     rc = lib.orc_fwd(ctypes.byref(d), *[_p(x) for x in a], _p(Aw), _p(A_dec), _p(tau), _p(S0), _p(m_prev), _p(o),
-                     _p(S), _p(m))
+                     _p(S), _p(m), _p(cu))
     if rc:
         raise ValueError("oracle fwd: bad dims")
     return dict(o=o, S_final=S, m_prev_out=m)
 
 
 def bwd(inp: dict, L: int, dO, mc_mode: int = 0, S0=None, m_prev=None, dS_final=None,
-        dm_prev_out=None, content_off: bool = False):
+        dm_prev_out=None, content_off: bool = False, cu_seqlens=None):
     """Gradients of sum(dO*o) + sum(dS_final*S_final) + sum(dm_prev_out*m_prev_out).
     Returns dict(dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dA_dec, dtau, dS0,
     dm_prev_in) in fp64 (dAw, dA_dec, dtau are zero when inp lacks "Aw", "A_dec", "tau")."""
     lib = _load()
-    d = _dims(inp, L, mc_mode, content_off)
+    cu = _cu(cu_seqlens)
+    d = _dims(inp, L, mc_mode, content_off, cu)
     a = [_f64(inp[k]) for k in _KEYS]
     Aw, A_dec, tau = _f64(inp.get("Aw")), _f64(inp.get("A_dec")), _f64(inp.get("tau"))
     S0, m_prev, dO = _f64(S0), _f64(m_prev), _f64(dO)
     dS_final, dm_prev_out = _f64(dS_final), _f64(dm_prev_out)
     B, T, H, K, V, R = d.B, d.T, d.H, d.K, d.V, d.R
-    out = dict(dq=np.zeros((B, T, H, K)), dk=np.zeros((B, T, H, K)), dv=np.zeros((B, T, H, V)),
-               dg_logit=np.zeros((B, T, H, K)), dbx=np.zeros((B, T, H, K)), dw_logit=np.zeros((B, T, H)),
+    Bt = 1 if cu is not None else B   # leading dimension of the token tensors
+    out = dict(dq=np.zeros((Bt, T, H, K)), dk=np.zeros((Bt, T, H, K)), dv=np.zeros((Bt, T, H, V)),
+               dg_logit=np.zeros((Bt, T, H, K)), dbx=np.zeros((Bt, T, H, K)), dw_logit=np.zeros((Bt, T, H)),
                dA=np.zeros((H, K, R)), dB=np.zeros((H, R, V)), dAw=np.zeros((H, R)),
                dA_dec=np.zeros(H), dtau=np.zeros((H, K)), dS0=np.zeros((B, H, V, K)), dm_prev_in=np.zeros((B, H, V)))
     order = ("dq", "dk", "dv", "dg_logit", "dbx", "dw_logit", "dA", "dB", "dAw", "dA_dec", "dtau", "dS0",
              "dm_prev_in")
     rc = lib.orc_bwd(ctypes.byref(d), *[_p(x) for x in a], _p(Aw), _p(A_dec), _p(tau), _p(S0), _p(m_prev),
                      _p(dO), _p(dS_final),
-                     _p(dm_prev_out), *[_p(out[k]) for k in order])
+                     _p(dm_prev_out), *[_p(out[k]) for k in order], _p(cu))
     if rc:
         raise ValueError("oracle bwd: bad dims")
     return out

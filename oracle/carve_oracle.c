@@ -36,6 +36,7 @@
  *
  * Layouts (all contiguous, row-major):
  *   q, k, g_logit, bx : [B,T,H,K]    v, o : [B,T,H,V]    w_logit : [B,T,H]
+ *   (varlen: B sequences packed as [1,T,H,*] and delimited by cu_seqlens, see unit_tokens)
  *   A : [H,K,R]   Bm : [H,R,V]   Aw : [H,R]   A_dec : [H]   tau : [H,K]
  *   S0, S_final, dS : [B,H,V,K]   m vectors : [B,H,V]
  * Units (b,h) are independent and run under OpenMP; the per-head parameter gradients are
@@ -120,25 +121,45 @@ static void gather_tok(const orc_dims *d, const double *x, int b, int t, int h, 
     memcpy(out, x + IX_TK(d, b, t, h, 0, W), sizeof(double) * (size_t)W);
 }
 
+/* Tokens of sequence b.  Without cu_seqlens: batch element b of [B,T,H,*] tensors, all T
+ * tokens.  With cu_seqlens ([B+1], non-decreasing, cu[0] = 0, cu[B] <= T): the B sequences are
+ * packed along the token axis of [1,T,H,*] tensors and sequence b is rows [cu[b], cu[b+1]);
+ * each has its own state, content signal and chunk grid (chunks restart at its first token). */
+static void unit_tokens(const orc_dims *d, const int *cu, int b, int *bb, int *toff, int *Tn) {
+    *bb = cu ? 0 : b;
+    *toff = cu ? cu[b] : 0;
+    *Tn = cu ? cu[b + 1] - cu[b] : d->T;
+}
+
+static int check_seqlens(const orc_dims *d, const int *cu) {
+    if (!cu) return 0;
+    if (cu[0] != 0 || cu[d->B] > d->T) return -1;
+    for (int b = 0; b < d->B; ++b)
+        if (cu[b + 1] < cu[b]) return -1;
+    return 0;
+}
+
 static int check_dims(const orc_dims *d) {
     if (d->B < 1 || d->H < 1 || d->T < 0 || d->K < 1 || d->V < 1 || d->R < 1 || d->L < 1) return -1;
     if (d->mc_mode != 0 && d->mc_mode != 1) return -1;
     return 0;
 }
 
-/* Forward.  Aw, A_dec, tau, S0, m_prev_in, m_prev_out may be NULL.  Returns 0 or -1 on bad
-   dims. */
+/* Forward.  Aw, A_dec, tau, S0, m_prev_in, m_prev_out may be NULL; so may cu_seqlens (see
+   unit_tokens).  Returns 0 or -1 on bad dims. */
 int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v,
             const double *gl, const double *bx, const double *wl, const double *A,
             const double *Bm, const double *Aw, const double *A_dec, const double *tau,
             const double *S0, const double *m_prev_in, double *o,
-            double *S_final, double *m_prev_out) {
-    if (check_dims(d)) return -1;
-    const int K = d->K, V = d->V, R = d->R, T = d->T, L = d->L, H = d->H;
+            double *S_final, double *m_prev_out, const int *cu_seqlens) {
+    if (check_dims(d) || check_seqlens(d, cu_seqlens)) return -1;
+    const int K = d->K, V = d->V, R = d->R, L = d->L, H = d->H;
     const int units = d->B * H;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int u = 0; u < units; ++u) {
         const int b = u / H, h = u % H;
+        int bb, toff, Tn;
+        unit_tokens(d, cu_seqlens, b, &bb, &toff, &Tn);
         double *S = (double *)calloc((size_t)V * K, sizeof(double));
         double *m = calloc(V, sizeof(double)), *z = calloc(R, sizeof(double));
         double *delta = calloc(K, sizeof(double)), *qbar = calloc(K, sizeof(double));
@@ -148,13 +169,13 @@ int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v
         double *mprev = calloc(V, sizeof(double)), *osum = calloc(V, sizeof(double));
         if (S0) memcpy(S, S0 + (size_t)u * V * K, sizeof(double) * (size_t)V * K);
         if (m_prev_in) memcpy(mprev, m_prev_in + (size_t)u * V, sizeof(double) * (size_t)V);
-        for (int t0 = 0; t0 < T; t0 += L) {
-            const int t1 = t0 + L < T ? t0 + L : T, n = t1 - t0;
+        for (int t0 = 0; t0 < Tn; t0 += L) {
+            const int t1 = t0 + L < Tn ? t0 + L : Tn, n = t1 - t0;
             if (!d->content_off) {
                 if (d->mc_mode == 0) {
                     for (int i = 0; i < K; ++i) qbar[i] = 0.0;
                     for (int t = t0; t < t1; ++t)
-                        for (int i = 0; i < K; ++i) qbar[i] += q[IX_TK(d, b, t, h, i, K)];
+                        for (int i = 0; i < K; ++i) qbar[i] += q[IX_TK(d, bb, toff + t, h, i, K)];
                     for (int i = 0; i < K; ++i) qbar[i] /= n;
                     for (int j = 0; j < V; ++j) {
                         double s = 0.0;
@@ -169,12 +190,12 @@ int orc_fwd(const orc_dims *d, const double *q, const double *k, const double *v
             const double dwc = write_bias(d, h, Aw, z);
             for (int j = 0; j < V; ++j) osum[j] = 0.0;
             for (int t = t0; t < t1; ++t) {
-                double w = gates(d, b, t, h, gl, bx, wl, A_dec, tau, delta, dwc, a, g, bg);
-                gather_tok(d, q, b, t, h, K, qt);
-                gather_tok(d, k, b, t, h, K, kt);
-                gather_tok(d, v, b, t, h, V, vt);
+                double w = gates(d, bb, toff + t, h, gl, bx, wl, A_dec, tau, delta, dwc, a, g, bg);
+                gather_tok(d, q, bb, toff + t, h, K, qt);
+                gather_tok(d, k, bb, toff + t, h, K, kt);
+                gather_tok(d, v, bb, toff + t, h, V, vt);
                 token_update(d, S, a, w, kt, vt, qt, e, ot);
-                memcpy(o + IX_TK(d, b, t, h, 0, V), ot, sizeof(double) * (size_t)V);
+                memcpy(o + IX_TK(d, bb, toff + t, h, 0, V), ot, sizeof(double) * (size_t)V);
                 for (int j = 0; j < V; ++j) osum[j] += ot[j];
             }
             for (int j = 0; j < V; ++j) mprev[j] = osum[j] / n;
@@ -200,11 +221,10 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
             const double *S0, const double *m_prev_in, const double *dO,
             const double *dS_final, const double *dm_prev_out, double *dq, double *dk,
             double *dv, double *dgl, double *dbx, double *dwl, double *dA, double *dB, double *dAw,
-            double *dA_dec, double *dtau, double *dS0, double *dm_prev_in) {
-    if (check_dims(d)) return -1;
+            double *dA_dec, double *dtau, double *dS0, double *dm_prev_in, const int *cu_seqlens) {
+    if (check_dims(d) || check_seqlens(d, cu_seqlens)) return -1;
     const int K = d->K, V = d->V, R = d->R, T = d->T, L = d->L, H = d->H;
     const int units = d->B * H;
-    const int N = (T + L - 1) / L;
     const size_t VK = (size_t)V * K;
     double *dA_u = calloc((size_t)units * K * R, sizeof(double));
     double *dB_u = calloc((size_t)units * R * V, sizeof(double));
@@ -214,6 +234,9 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
 #pragma omp parallel for schedule(dynamic, 1)
     for (int u = 0; u < units; ++u) {
         const int b = u / H, h = u % H;
+        int bb, toff, Tn;
+        unit_tokens(d, cu_seqlens, b, &bb, &toff, &Tn);
+        const int N = (Tn + L - 1) / L;
         double *Sb = calloc((size_t)(N > 0 ? N : 1) * VK, sizeof(double)); /* chunk-start states */
         double *mc = calloc((size_t)(N > 0 ? N : 1) * V, sizeof(double));
         double *zc = calloc((size_t)(N > 0 ? N : 1) * R, sizeof(double));
@@ -238,12 +261,12 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
         if (S0) memcpy(S, S0 + (size_t)u * VK, sizeof(double) * VK);
         if (m_prev_in) memcpy(mprev, m_prev_in + (size_t)u * V, sizeof(double) * (size_t)V);
         for (int c = 0; c < N; ++c) {
-            const int t0 = c * L, t1 = t0 + L < T ? t0 + L : T, n = t1 - t0;
+            const int t0 = c * L, t1 = t0 + L < Tn ? t0 + L : Tn, n = t1 - t0;
             memcpy(Sb + (size_t)c * VK, S, sizeof(double) * VK);
             double *m = mc + (size_t)c * V, *qbar = qb + (size_t)c * K;
             for (int i = 0; i < K; ++i) qbar[i] = 0.0;
             for (int t = t0; t < t1; ++t)
-                for (int i = 0; i < K; ++i) qbar[i] += q[IX_TK(d, b, t, h, i, K)];
+                for (int i = 0; i < K; ++i) qbar[i] += q[IX_TK(d, bb, toff + t, h, i, K)];
             for (int i = 0; i < K; ++i) qbar[i] /= n;
             if (!d->content_off) {
                 if (d->mc_mode == 0) {
@@ -260,10 +283,10 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
             for (int j = 0; j < V; ++j) osum[j] = 0.0;
             const double dwc = write_bias(d, h, Aw, zc + (size_t)c * R);
             for (int t = t0; t < t1; ++t) {
-                double w = gates(d, b, t, h, gl, bx, wl, A_dec, tau, dc + (size_t)c * K, dwc, at, gt, bt);
-                gather_tok(d, q, b, t, h, K, qt);
-                gather_tok(d, k, b, t, h, K, kt);
-                gather_tok(d, v, b, t, h, V, vt);
+                double w = gates(d, bb, toff + t, h, gl, bx, wl, A_dec, tau, dc + (size_t)c * K, dwc, at, gt, bt);
+                gather_tok(d, q, bb, toff + t, h, K, qt);
+                gather_tok(d, k, bb, toff + t, h, K, kt);
+                gather_tok(d, v, bb, toff + t, h, V, vt);
                 token_update(d, S, at, w, kt, vt, qt, et, ot);
                 for (int j = 0; j < V; ++j) osum[j] += ot[j];
             }
@@ -274,11 +297,11 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
         if (dS_final) memcpy(dS, dS_final + (size_t)u * VK, sizeof(double) * VK);
         for (int j = 0; j < V; ++j) dox[j] = 0.0;
         if (dm_prev_out && N > 0) {
-            const int nl = T - (N - 1) * L;
+            const int nl = Tn - (N - 1) * L;
             for (int j = 0; j < V; ++j) dox[j] = dm_prev_out[(size_t)u * V + j] / nl;
         }
         for (int c = N - 1; c >= 0; --c) {
-            const int t0 = c * L, t1 = t0 + L < T ? t0 + L : T, n = t1 - t0;
+            const int t0 = c * L, t1 = t0 + L < Tn ? t0 + L : Tn, n = t1 - t0;
             const double *delta = dc + (size_t)c * K;
             const double dwc = write_bias(d, h, Aw, zc + (size_t)c * R);
             double ddw = 0.0;   /* gradient of dw_c: sum of the chunk's write-logit gradients */
@@ -286,12 +309,12 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
             memcpy(St, Sb + (size_t)c * VK, sizeof(double) * VK);
             for (int ti = 0; ti < n; ++ti) {
                 const int t = t0 + ti;
-                wt[ti] = gates(d, b, t, h, gl, bx, wl, A_dec, tau, delta, dwc, at + (size_t)ti * K,
+                wt[ti] = gates(d, bb, toff + t, h, gl, bx, wl, A_dec, tau, delta, dwc, at + (size_t)ti * K,
                                 gt + (size_t)ti * K, bt + (size_t)ti * K);
                 memcpy(St + (size_t)(ti + 1) * VK, St + (size_t)ti * VK, sizeof(double) * VK);
-                gather_tok(d, q, b, t, h, K, qt);
-                gather_tok(d, k, b, t, h, K, kt);
-                gather_tok(d, v, b, t, h, V, vt);
+                gather_tok(d, q, bb, toff + t, h, K, qt);
+                gather_tok(d, k, bb, toff + t, h, K, kt);
+                gather_tok(d, v, bb, toff + t, h, V, vt);
                 token_update(d, St + (size_t)(ti + 1) * VK, at + (size_t)ti * K, wt[ti], kt, vt,
                              qt, et + (size_t)ti * V, ot);
             }
@@ -301,11 +324,11 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                 const double *a = at + (size_t)ti * K, *g = gt + (size_t)ti * K, *bg = bt + (size_t)ti * K;
                 const double *e = et + (size_t)ti * V, w = wt[ti];
                 const double *Sprev = St + (size_t)ti * VK, *Scur = St + (size_t)(ti + 1) * VK;
-                gather_tok(d, q, b, t, h, K, qt);
-                gather_tok(d, k, b, t, h, K, kt);
-                for (int j = 0; j < V; ++j) dot[j] = dO[IX_TK(d, b, t, h, j, V)] + dox[j];
+                gather_tok(d, q, bb, toff + t, h, K, qt);
+                gather_tok(d, k, bb, toff + t, h, K, kt);
+                for (int j = 0; j < V; ++j) dot[j] = dO[IX_TK(d, bb, toff + t, h, j, V)] + dox[j];
                 /* o_t = S_t q_t */
-                double *dqt = dq + IX_TK(d, b, t, h, 0, K);
+                double *dqt = dq + IX_TK(d, bb, toff + t, h, 0, K);
                 for (int i = 0; i < K; ++i) dqt[i] = 0.0;
                 for (int j = 0; j < V; ++j)
                     for (int i = 0; i < K; ++i) {
@@ -314,7 +337,7 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                     }
                 /* S_t = P + w e k^T */
                 double dw = 0.0;
-                double *dkt = dk + IX_TK(d, b, t, h, 0, K);
+                double *dkt = dk + IX_TK(d, bb, toff + t, h, 0, K);
                 for (int i = 0; i < K; ++i) dkt[i] = 0.0;
                 for (int j = 0; j < V; ++j) {
                     double s = 0.0;
@@ -324,18 +347,18 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                     for (int i = 0; i < K; ++i) dkt[i] += w * dS[(size_t)j * K + i] * e[j];
                 }
                 /* e = v - P k, P = S_{t-1} Diag(a) */
-                for (int j = 0; j < V; ++j) dv[IX_TK(d, b, t, h, j, V)] = de[j];
+                for (int j = 0; j < V; ++j) dv[IX_TK(d, bb, toff + t, h, j, V)] = de[j];
                 for (int j = 0; j < V; ++j)
                     for (int i = 0; i < K; ++i) {
                         double p = Sprev[(size_t)j * K + i] * a[i];
                         dP[(size_t)j * K + i] = dS[(size_t)j * K + i] - de[j] * kt[i];
                         dkt[i] -= p * de[j];
                     }
-                double *dglt = dgl + IX_TK(d, b, t, h, 0, K), *dbxt = dbx + IX_TK(d, b, t, h, 0, K);
+                double *dglt = dgl + IX_TK(d, bb, toff + t, h, 0, K), *dbxt = dbx + IX_TK(d, bb, toff + t, h, 0, K);
                 for (int i = 0; i < K; ++i) {
                     double da = 0.0;
                     for (int j = 0; j < V; ++j) da += Sprev[(size_t)j * K + i] * dP[(size_t)j * K + i];
-                    const size_t ix = IX_TK(d, b, t, h, i, K);
+                    const size_t ix = IX_TK(d, bb, toff + t, h, i, K);
                     /* a = g b, log g = -amp softplus(gl + tau) => dg/dgl = dg/dtau
                        = -g amp sigmoid(gl + tau), dg/dA_dec = g log g */
                     const double x = gl[ix] + decay_bias(d, tau, h, i);
@@ -348,7 +371,7 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                 }
                 for (int j = 0; j < V; ++j)
                     for (int i = 0; i < K; ++i) dS[(size_t)j * K + i] = dP[(size_t)j * K + i] * a[i];
-                dwl[((size_t)b * T + t) * H + h] = dw * w * (1.0 - w);
+                dwl[((size_t)bb * T + toff + t) * H + h] = dw * w * (1.0 - w);
                 ddw += dw * w * (1.0 - w);
             }
             /* chunk start: Delta = A z, z = B m */
@@ -382,7 +405,7 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                         tmp[i] = s / n;
                     }
                     for (int t = t0; t < t1; ++t)
-                        for (int i = 0; i < K; ++i) dq[IX_TK(d, b, t, h, i, K)] += tmp[i];
+                        for (int i = 0; i < K; ++i) dq[IX_TK(d, bb, toff + t, h, i, K)] += tmp[i];
                 } else if (c > 0) {
                     const int np = L; /* every chunk before the last is complete */
                     for (int j = 0; j < V; ++j) dox[j] = dm[j] / np;
@@ -391,8 +414,11 @@ int orc_bwd(const orc_dims *d, const double *q, const double *k, const double *v
                 }
             }
         }
-        if (d->content_off || d->mc_mode == 0 || N == 0)
-            if (dm_prev_in) memset(dm_prev_in + (size_t)u * V, 0, sizeof(double) * (size_t)V);
+        if (dm_prev_in && N == 0) {   /* no token: m_prev_out is m_prev_in passed through */
+            for (int j = 0; j < V; ++j) dm_prev_in[(size_t)u * V + j] = dm_prev_out ? dm_prev_out[(size_t)u * V + j] : 0.0;
+        } else if (dm_prev_in && (d->content_off || d->mc_mode == 0)) {
+            memset(dm_prev_in + (size_t)u * V, 0, sizeof(double) * (size_t)V);
+        }
         if (dS0) memcpy(dS0 + (size_t)u * VK, dS, sizeof(double) * VK);
         free(Sb); free(mc); free(zc); free(dc); free(qb); free(St); free(S); free(dS); free(dP);
         free(at); free(gt); free(bt); free(wt); free(et); free(qt); free(kt); free(vt); free(ot);

@@ -52,7 +52,7 @@ MUTANTS = {
     "bwd_dA_dec_missing_amp": ("if (A_dec) dAdec_u[u] += da * a[i] * (-amp * softplus(x));",
                                "if (A_dec) dAdec_u[u] += da * a[i] * (-softplus(x));"),
     # backward: readout path into dq dropped
-    "bwd_no_readout_dq": ("for (int i = 0; i < K; ++i) dq[IX_TK(d, b, t, h, i, K)] += tmp[i];", "(void)tmp;"),
+    "bwd_no_readout_dq": ("for (int i = 0; i < K; ++i) dq[IX_TK(d, bb, toff + t, h, i, K)] += tmp[i];", "(void)tmp;"),
     # backward: write-gate gradient without the sigmoid derivative
     "bwd_dwl_no_sigmoid_prime": ("= dw * w * (1.0 - w);", "= dw;"),
     # backward: prediction term of dk dropped
@@ -62,6 +62,11 @@ MUTANTS = {
                            "return sigm(wl[((size_t)b * d->T + t) * d->H + h]);"),
     # write gate's content term built from the wrong component of z
     "write_bias_wrong_z": ("s += Aw[(size_t)h * d->R + j] * z[j];", "s += Aw[(size_t)h * d->R + j] * z[0];"),
+    # packed sequences: a sequence's gate logits read from the first rows of the packed tensor
+    "varlen_gate_rows": ("double w = gates(d, bb, toff + t, h, gl, bx, wl, A_dec, tau, delta, dwc, a, g, bg);",
+                         "double w = gates(d, bb, t, h, gl, bx, wl, A_dec, tau, delta, dwc, a, g, bg);"),
+    # packed sequences: the chunk-mean of q read from the first rows of the packed tensor
+    "varlen_qbar_rows": ("qbar[i] += q[IX_TK(d, bb, toff + t, h, i, K)];", "qbar[i] += q[IX_TK(d, bb, t, h, i, K)];"),
     # backward: the write bias's gradient not fed back into dz
     "bwd_write_bias_not_in_dz": ("if (Aw) s += Aw[(size_t)h * R + j] * ddw;", "(void)ddw;"),
 }
@@ -82,6 +87,7 @@ PIN_TESTS = [
     lambda: pins.test_content_signal_closed_form(0, True),
     lambda: pins.test_content_signal_closed_form(1, True),
     pins.test_state_norm_bound_every_token,
+    lambda: pins.test_packed_sequences_equal_separate_calls(0),
     lambda: pins.test_gradients_central_differences(0),
     lambda: pins.test_gradients_central_differences(1),
 ]

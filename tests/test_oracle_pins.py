@@ -390,3 +390,74 @@ def test_gradients_central_differences(mc_mode):
         assert err < 1e-6, (x, err)
     if mc_mode == 0:
         assert np.all(g["dm_prev_in"] == 0.0)
+
+
+# ---------------------------------------------------------------------------------------
+# 8. Packed variable-length sequences: each sequence is an independent recurrence with its own
+#    state, content signal and chunk grid (chunks restart at its first token)
+# ---------------------------------------------------------------------------------------
+def packed_case(lens, seed, H=2, K=6, V=5, R=3):
+    """Sequences of the given lengths, drawn separately, and their packing along the token axis."""
+    seqs = []
+    for n, T in enumerate(lens):
+        w = dataclasses.replace(I.TINY_FP32, B=1, H=H, T=T, K=K, V=V, R=R, L=4, seed=seed + n)
+        d = {k: np.asarray(v, dtype=np.float64) for k, v in I.make_inputs(w).items()}
+        seqs.append(d)
+    shared = {k: seqs[0][k] * 40.0 for k in ("A", "B")}
+    for d in seqs:
+        d.update(shared)
+    Ttot = sum(lens) + 3   # three trailing rows that belong to no sequence
+    packed = dict(shared)
+    for k in ("q", "k", "v", "g_logit", "bx", "w_logit"):
+        tail = np.full((1, 3) + seqs[0][k].shape[2:], 7.0)
+        packed[k] = np.concatenate([d[k] for d in seqs] + [tail], axis=1)
+        assert packed[k].shape[1] == Ttot
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return seqs, packed, cu
+
+
+@pytest.mark.parametrize("mc_mode", [0, 1])
+def test_packed_sequences_equal_separate_calls(mc_mode):
+    """Forward and backward over packed sequences (lengths with an empty one, a one-token one,
+    ragged last chunks) give, bit for bit, what separate calls give per sequence; dA and dB
+    are the per-sequence sums in order; rows past the last sequence stay zero."""
+    lens = [7, 0, 13, 1, 8]
+    seqs, packed, cu = packed_case(lens, 300 + mc_mode)
+    N, H, K, V = len(lens), 2, 6, 5
+    S0 = I.normal(9, 10, (N, H, V, K), 0.0, 0.3)
+    mp = I.normal(9, 11, (N, H, V))
+    dO = I.normal(9, 12, (1, cu[-1] + 3, H, V))
+    dSf = I.normal(9, 13, (N, H, V, K))
+    dmo = I.normal(9, 14, (N, H, V))
+    r = oracle.fwd(packed, L=4, mc_mode=mc_mode, S0=S0, m_prev=mp, cu_seqlens=cu)
+    g = oracle.bwd(packed, 4, dO, mc_mode=mc_mode, S0=S0, m_prev=mp, dS_final=dSf, dm_prev_out=dmo, cu_seqlens=cu)
+    dA = np.zeros_like(packed["A"])
+    dB = np.zeros_like(packed["B"])
+    for n, d in enumerate(seqs):
+        a, b = cu[n], cu[n + 1]
+        if b == a:   # an empty sequence passes its state and content signal through
+            assert np.array_equal(r["S_final"][n], S0[n]) and np.array_equal(r["m_prev_out"][n], mp[n])
+            assert np.array_equal(g["dS0"][n], dSf[n])
+            assert np.array_equal(g["dm_prev_in"][n], dmo[n])
+            continue
+        rs = oracle.fwd(d, L=4, mc_mode=mc_mode, S0=S0[n:n + 1], m_prev=mp[n:n + 1])
+        gs = oracle.bwd(d, 4, dO[:, a:b], mc_mode=mc_mode, S0=S0[n:n + 1], m_prev=mp[n:n + 1],
+                        dS_final=dSf[n:n + 1], dm_prev_out=dmo[n:n + 1])
+        assert np.array_equal(r["o"][:, a:b], rs["o"])
+        assert np.array_equal(r["S_final"][n], rs["S_final"][0])
+        assert np.array_equal(r["m_prev_out"][n], rs["m_prev_out"][0])
+        for key in ("dq", "dk", "dv", "dg_logit", "dbx", "dw_logit"):
+            assert np.array_equal(g[key][:, a:b], gs[key]), key
+        for key in ("dS0", "dm_prev_in"):
+            assert np.array_equal(g[key][n], gs[key][0]), key
+        dA += gs["dA"]
+        dB += gs["dB"]
+    assert np.array_equal(g["dA"], dA) and np.array_equal(g["dB"], dB)
+    assert np.all(r["o"][:, cu[-1]:] == 0.0) and np.all(g["dq"][:, cu[-1]:] == 0.0)
+
+
+def test_packed_sequences_rejected_when_malformed():
+    _, packed, cu = packed_case([4, 4], 310)
+    for bad in ([1, 4, 8], [0, 5, 4], [0, 4, 100]):
+        with pytest.raises(ValueError):
+            oracle.fwd(packed, L=4, cu_seqlens=np.array(bad))
