@@ -57,9 +57,12 @@ def load():
     lib.carve_fwd.argtypes = [D] + [P] * 18
     lib.carve_bwd.argtypes = [D] + [P] * 32
     lib.carve_step.argtypes = [D] + [P] * 16
+    lib.carve_fwd_varlen.argtypes = [D, P, ctypes.c_int64] + [P] * 18
+    lib.carve_bwd_varlen.argtypes = [D, P, ctypes.c_int64] + [P] * 32
     lib.carve_check.argtypes = [P]
     lib.carve_selftest_timeout.argtypes = [ctypes.c_uint32, P]
-    for f in (lib.carve_fwd, lib.carve_bwd, lib.carve_step, lib.carve_check, lib.carve_selftest_timeout):
+    for f in (lib.carve_fwd, lib.carve_bwd, lib.carve_fwd_varlen, lib.carve_bwd_varlen, lib.carve_step,
+              lib.carve_check, lib.carve_selftest_timeout):
         f.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -101,6 +104,23 @@ def dims_of(q, v, A, chunk, mc_mode) -> Dims:
     return Dims(B, H, T, K, v.shape[-1], A.shape[-1], chunk, _io_of(q), mc_mode)
 
 
+def dims_varlen(q, v, A, cu_seqlens, max_len, chunk, mc_mode) -> Dims:
+    """Dims of a packed call: B = number of sequences, T = max_len rounded up to 16."""
+    T = max(16, (int(max_len) + 15) // 16 * 16)
+    return Dims(cu_seqlens.numel() - 1, q.shape[-2], T, q.shape[-1], v.shape[-1], A.shape[-1], chunk, _io_of(q),
+                mc_mode)
+
+
+def _packed(cu_seqlens, max_len, q):
+    """(cu pointer, row count) of a packed call; max_len None reads the lengths on the host."""
+    torch = _torch()
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != q.device:
+        raise TypeError("cu_seqlens must be an int32 tensor on the device of q")
+    if max_len is None:
+        max_len = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if cu_seqlens.numel() > 1 else 0
+    return [_ptr(cu_seqlens), ctypes.c_int64(q.shape[-3])], max_len
+
+
 def saved_bytes(d: Dims) -> int:
     return int(load().carve_saved_bytes(ctypes.byref(d)))
 
@@ -126,13 +146,30 @@ def carve_fwd(q, k, v, g_logit, bx, w_logit, A, B, chunk: int, mc_mode: int = 0,
     """Forward over [B,T,H,*] device tensors.  Optional: Aw [H,rank], the write gate's content
     term; A_dec [H] and tau [H,dk], the decay's log-amplitude and bias.  Returns dict(o,
     S_final, m_prev_out, saved); `out` may supply preallocated buffers under the same keys."""
+    return _fwd(dims_of(q, v, A, chunk, mc_mode), None, q, k, v, g_logit, bx, w_logit, A, B, S0, m_prev_in,
+                save_for_bwd, out, stream, Aw, A_dec, tau)
+
+
+def carve_fwd_varlen(q, k, v, g_logit, bx, w_logit, A, B, cu_seqlens, chunk: int, max_len=None, mc_mode: int = 0,
+                     S0=None, m_prev_in=None, save_for_bwd: bool = True, out: dict | None = None, stream=None,
+                     Aw=None, A_dec=None, tau=None) -> dict:
+    """Forward over variable-length sequences packed along the token axis: q, k, g_logit, bx
+    [total,H,dk]; v [total,H,dv]; w_logit [total,H]; cu_seqlens int32 [N+1] on the device
+    (sequence n = rows cu[n]..cu[n+1]); max_len >= every length (None: read from cu_seqlens on
+    the host).  S0, m_prev_in and the per-sequence outputs are [N,H,...]."""
+    pk, max_len = _packed(cu_seqlens, max_len, q)
+    d = dims_varlen(q, v, A, cu_seqlens, max_len, chunk, mc_mode)
+    return _fwd(d, pk, q, k, v, g_logit, bx, w_logit, A, B, S0, m_prev_in, save_for_bwd, out, stream, Aw, A_dec,
+                tau)
+
+
+def _fwd(d, pk, q, k, v, g_logit, bx, w_logit, A, B, S0, m_prev_in, save_for_bwd, out, stream, Aw, A_dec, tau):
     torch = _torch()
     lib = load()
-    d = dims_of(q, v, A, chunk, mc_mode)
     out = dict(out or {})
     dev = q.device
     if "o" not in out:
-        out["o"] = torch.empty((d.B, d.T, d.H, d.dv), dtype=q.dtype, device=dev)
+        out["o"] = torch.empty(v.shape, dtype=q.dtype, device=dev)
     if "S_final" not in out:
         out["S_final"] = torch.empty((d.B, d.H, d.dv, d.dk), dtype=torch.float32, device=dev)
     if "m_prev_out" not in out:
@@ -142,11 +179,12 @@ def carve_fwd(q, k, v, g_logit, bx, w_logit, A, B, chunk: int, mc_mode: int = 0,
         if n == 0:
             raise CarveError("carve_saved_bytes", 1)
         out["saved"] = torch.empty(n, dtype=torch.uint8, device=dev)
-    rc = lib.carve_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g_logit), _ptr(bx), _ptr(w_logit),
-                       _ptr(A), _ptr(B), _ptr(Aw), _ptr(A_dec), _ptr(tau), _ptr(S0), _ptr(m_prev_in), _ptr(out["o"]),
-                       _ptr(out["S_final"]), _ptr(out["m_prev_out"]), _ptr(out.get("saved") if save_for_bwd else None),
-                       _stream(stream))
-    _check("carve_fwd", rc)
+    fn = lib.carve_fwd if pk is None else lib.carve_fwd_varlen
+    rc = fn(ctypes.byref(d), *(pk or []), _ptr(q), _ptr(k), _ptr(v), _ptr(g_logit), _ptr(bx), _ptr(w_logit),
+            _ptr(A), _ptr(B), _ptr(Aw), _ptr(A_dec), _ptr(tau), _ptr(S0), _ptr(m_prev_in), _ptr(out["o"]),
+            _ptr(out["S_final"]), _ptr(out["m_prev_out"]), _ptr(out.get("saved") if save_for_bwd else None),
+            _stream(stream))
+    _check("carve_fwd" if pk is None else "carve_fwd_varlen", rc)
     return out
 
 
@@ -155,9 +193,25 @@ def carve_bwd(q, k, v, g_logit, bx, w_logit, A, B, saved, dO, chunk: int, mc_mod
               workspace=None, stream=None, Aw=None, A_dec=None, tau=None) -> dict:
     """Reverse sweep.  Returns dict(dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dS0, dm_prev_in),
     plus dAw, dA_dec, dtau when the forward had Aw, A_dec, tau."""
+    return _bwd(dims_of(q, v, A, chunk, mc_mode), None, q, k, v, g_logit, bx, w_logit, A, B, saved, dO, S0,
+                m_prev_in, dS_final, dm_prev_out, want_dS0, out, workspace, stream, Aw, A_dec, tau)
+
+
+def carve_bwd_varlen(q, k, v, g_logit, bx, w_logit, A, B, saved, dO, cu_seqlens, chunk: int, max_len=None,
+                     mc_mode: int = 0, S0=None, m_prev_in=None, dS_final=None, dm_prev_out=None,
+                     want_dS0: bool = True, out: dict | None = None, workspace=None, stream=None, Aw=None,
+                     A_dec=None, tau=None) -> dict:
+    """Reverse sweep of carve_fwd_varlen (same packed layouts and the same max_len)."""
+    pk, max_len = _packed(cu_seqlens, max_len, q)
+    d = dims_varlen(q, v, A, cu_seqlens, max_len, chunk, mc_mode)
+    return _bwd(d, pk, q, k, v, g_logit, bx, w_logit, A, B, saved, dO, S0, m_prev_in, dS_final, dm_prev_out,
+                want_dS0, out, workspace, stream, Aw, A_dec, tau)
+
+
+def _bwd(d, pk, q, k, v, g_logit, bx, w_logit, A, B, saved, dO, S0, m_prev_in, dS_final, dm_prev_out, want_dS0,
+         out, workspace, stream, Aw, A_dec, tau):
     torch = _torch()
     lib = load()
-    d = dims_of(q, v, A, chunk, mc_mode)
     dev = q.device
     out = dict(out or {})
     shapes = dict(dq=(q.shape, q.dtype), dk=(k.shape, k.dtype), dv=(v.shape, v.dtype),
@@ -174,15 +228,16 @@ def carve_bwd(q, k, v, g_logit, bx, w_logit, A, B, saved, dO, chunk: int, mc_mod
             out[key] = torch.empty(shp, dtype=dt, device=dev)
     if workspace is None:
         workspace = torch.empty(bwd_workspace_bytes(d), dtype=torch.uint8, device=dev)
-    rc = lib.carve_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(g_logit), _ptr(bx), _ptr(w_logit), _ptr(A),
-                       _ptr(B), _ptr(Aw), _ptr(A_dec), _ptr(tau), _ptr(S0), _ptr(m_prev_in), _ptr(saved), _ptr(dO),
-                       _ptr(dS_final), _ptr(dm_prev_out), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
-                       _ptr(out["dg_logit"]), _ptr(out["dbx"]), _ptr(out["dw_logit"]), _ptr(out["dA"]), _ptr(out["dB"]),
-                       _ptr(out.get("dAw") if Aw is not None else None),
-                       _ptr(out.get("dA_dec") if A_dec is not None else None),
-                       _ptr(out.get("dtau") if tau is not None else None), _ptr(out.get("dS0")),
-                       _ptr(out["dm_prev_in"]), _ptr(workspace), _stream(stream))
-    _check("carve_bwd", rc)
+    fn = lib.carve_bwd if pk is None else lib.carve_bwd_varlen
+    rc = fn(ctypes.byref(d), *(pk or []), _ptr(q), _ptr(k), _ptr(v), _ptr(g_logit), _ptr(bx), _ptr(w_logit), _ptr(A),
+            _ptr(B), _ptr(Aw), _ptr(A_dec), _ptr(tau), _ptr(S0), _ptr(m_prev_in), _ptr(saved), _ptr(dO),
+            _ptr(dS_final), _ptr(dm_prev_out), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+            _ptr(out["dg_logit"]), _ptr(out["dbx"]), _ptr(out["dw_logit"]), _ptr(out["dA"]), _ptr(out["dB"]),
+            _ptr(out.get("dAw") if Aw is not None else None),
+            _ptr(out.get("dA_dec") if A_dec is not None else None),
+            _ptr(out.get("dtau") if tau is not None else None), _ptr(out.get("dS0")),
+            _ptr(out["dm_prev_in"]), _ptr(workspace), _stream(stream))
+    _check("carve_bwd" if pk is None else "carve_bwd_varlen", rc)
     return out
 
 

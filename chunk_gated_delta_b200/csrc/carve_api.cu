@@ -14,6 +14,7 @@ int tc_reduce_slices(int B, int NG);
 int tc_fwd_take_timeout();
 int tc_bwd_take_timeout();
 int step_take_timeout();
+int simt_take_bad_seqlens();
 cudaError_t launch_selftest_timeout(uint32_t iterations, cudaStream_t st);
 cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
@@ -44,6 +45,13 @@ carve_status check_dims(const carve_dims *d, bool seq) {
         if (d->T % carve::kSub != 0) return CARVE_ERR_UNSUPPORTED;
         if ((long long)d->B * d->T * d->H * (d->dk > d->dv ? d->dk : d->dv) > (1LL << 40)) return CARVE_ERR_UNSUPPORTED;
     }
+    return CARVE_OK;
+}
+
+// packed sequences: `total` rows of [1, total, H, *] token tensors
+carve_status check_packed(const carve_dims *d, long long total) {
+    if (total < 0 || total > 0x7fffffffLL) return CARVE_ERR_INVALID_ARG;
+    if (total * d->H * (d->dk > d->dv ? d->dk : d->dv) > (1LL << 40)) return CARVE_ERR_UNSUPPORTED;
     return CARVE_OK;
 }
 
@@ -112,13 +120,15 @@ size_t carve_bwd_workspace_bytes(const carve_dims *d) {
            ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv + d->rank + (size_t)d->dk + 1);
 }
 
-carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
-                       const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
-                       const float *tau, const float *S0, const float *m_prev_in, void *o,
-                       float *S_final, float *m_prev_out, void *saved, void *stream) {
+// cu == nullptr: [B,T,H,*] batches; else B sequences packed in `total` rows (see carve_fwd_varlen)
+static carve_status fwd_impl(const carve_dims *d, const int32_t *cu, long long total, const void *q, const void *k,
+                             const void *v, const float *g_logit, const float *bx, const float *w_logit,
+                             const float *A, const float *Bm, const float *Aw, const float *A_dec, const float *tau,
+                             const float *S0, const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
+                             void *saved, void *stream) {
     carve_status st = check_dims(d, true);
     if (st != CARVE_OK) return st;
+    if (cu && (st = check_packed(d, total)) != CARVE_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
         !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(Aw) || !ok_opt(A_dec) || !ok_opt(tau) || !ok_ptr(o) ||
         !ok_opt(S0) || !ok_opt(m_prev_in) || !ok_opt(S_final) || !ok_opt(m_prev_out) || !ok_opt(saved))
@@ -132,8 +142,10 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
         a.saved_aux = reinterpret_cast<float *>(static_cast<char *>(saved) + saved_states_bytes(d));
     }
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
+    a.cu_seqlens = cu; a.total = total;
     cudaError_t e;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cu && tc_shape(d)) return CARVE_ERR_UNSUPPORTED;   // packed sequences: SIMT kernels only
     if (saved != nullptr && tc_saved)
         e = carve::launch_fwd_tc(a, 32, cs);
     else if (saved == nullptr && tc_fwd_chunk(d) > 0)
@@ -143,16 +155,17 @@ carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const 
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 
-carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const void *v,
-                       const float *g_logit, const float *bx, const float *w_logit,
-                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
-                       const float *tau, const float *S0, const float *m_prev_in, const void *saved,
-                       const void *dO, const float *dS_final, const float *dm_prev_out, void *dq,
-                       void *dk, void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
-                       float *dB, float *dAw, float *dA_dec, float *dtau, float *dS0,
-                       float *dm_prev_in, void *workspace, void *stream) {
+static carve_status bwd_impl(const carve_dims *d, const int32_t *cu, long long total, const void *q, const void *k,
+                             const void *v, const float *g_logit, const float *bx, const float *w_logit,
+                             const float *A, const float *Bm, const float *Aw, const float *A_dec, const float *tau,
+                             const float *S0, const float *m_prev_in, const void *saved, const void *dO,
+                             const float *dS_final, const float *dm_prev_out, void *dq, void *dk, void *dv,
+                             float *dg_logit, float *dbx, float *dw_logit, float *dA, float *dB, float *dAw,
+                             float *dA_dec, float *dtau, float *dS0, float *dm_prev_in, void *workspace,
+                             void *stream) {
     carve_status st = check_dims(d, true);
     if (st != CARVE_OK) return st;
+    if (cu && (st = check_packed(d, total)) != CARVE_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g_logit) || !ok_ptr(bx) || !ok_ptr(w_logit) ||
         !ok_ptr(A) || !ok_ptr(Bm) || !ok_opt(S0) || !ok_opt(m_prev_in) || !ok_ptr(saved) || !ok_ptr(dO) ||
         !ok_opt(dS_final) || !ok_opt(dm_prev_out) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
@@ -173,10 +186,60 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg_logit = dg_logit; a.dbx = dbx; a.dw_logit = dw_logit;
     a.dS0 = dS0; a.dm_prev_in = dm_prev_in; a.ws = static_cast<float *>(workspace);
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
+    a.cu_seqlens = cu; a.total = total;
+    if (cu && tc) return CARVE_ERR_UNSUPPORTED;   // packed sequences: SIMT kernels only
     cudaError_t e = tc ? carve::launch_bwd_tc(a, dA, dB, static_cast<cudaStream_t>(stream))
                        : carve::launch_bwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
                                                 static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_fwd(const carve_dims *d, const void *q, const void *k, const void *v,
+                       const float *g_logit, const float *bx, const float *w_logit,
+                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                       const float *tau, const float *S0, const float *m_prev_in, void *o,
+                       float *S_final, float *m_prev_out, void *saved, void *stream) {
+    return fwd_impl(d, nullptr, 0, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, A_dec, tau, S0, m_prev_in, o, S_final,
+                    m_prev_out, saved, stream);
+}
+
+carve_status carve_fwd_varlen(const carve_dims *d, const int32_t *cu_seqlens, int64_t total_tokens,
+                              const void *q, const void *k, const void *v, const float *g_logit,
+                              const float *bx, const float *w_logit, const float *A, const float *Bm,
+                              const float *Aw, const float *A_dec, const float *tau, const float *S0,
+                              const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
+                              void *saved, void *stream) {
+    if (!ok_ptr(cu_seqlens)) return CARVE_ERR_INVALID_ARG;
+    return fwd_impl(d, cu_seqlens, total_tokens, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, A_dec, tau, S0,
+                    m_prev_in, o, S_final, m_prev_out, saved, stream);
+}
+
+carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const void *v,
+                       const float *g_logit, const float *bx, const float *w_logit,
+                       const float *A, const float *Bm, const float *Aw, const float *A_dec,
+                       const float *tau, const float *S0, const float *m_prev_in, const void *saved,
+                       const void *dO, const float *dS_final, const float *dm_prev_out, void *dq,
+                       void *dk, void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
+                       float *dB, float *dAw, float *dA_dec, float *dtau, float *dS0,
+                       float *dm_prev_in, void *workspace, void *stream) {
+    return bwd_impl(d, nullptr, 0, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, A_dec, tau, S0, m_prev_in, saved, dO,
+                    dS_final, dm_prev_out, dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw, dA_dec, dtau, dS0,
+                    dm_prev_in, workspace, stream);
+}
+
+carve_status carve_bwd_varlen(const carve_dims *d, const int32_t *cu_seqlens, int64_t total_tokens,
+                              const void *q, const void *k, const void *v, const float *g_logit,
+                              const float *bx, const float *w_logit, const float *A, const float *Bm,
+                              const float *Aw, const float *A_dec, const float *tau, const float *S0,
+                              const float *m_prev_in, const void *saved, const void *dO,
+                              const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
+                              void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
+                              float *dB, float *dAw, float *dA_dec, float *dtau, float *dS0,
+                              float *dm_prev_in, void *workspace, void *stream) {
+    if (!ok_ptr(cu_seqlens)) return CARVE_ERR_INVALID_ARG;
+    return bwd_impl(d, cu_seqlens, total_tokens, q, k, v, g_logit, bx, w_logit, A, Bm, Aw, A_dec, tau, S0,
+                    m_prev_in, saved, dO, dS_final, dm_prev_out, dq, dk, dv, dg_logit, dbx, dw_logit, dA, dB, dAw,
+                    dA_dec, dtau, dS0, dm_prev_in, workspace, stream);
 }
 
 carve_status carve_step(const carve_dims *d, const void *q, const void *k, const void *v,
@@ -198,7 +261,8 @@ carve_status carve_step(const carve_dims *d, const void *q, const void *k, const
 carve_status carve_check(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CARVE_ERR_CUDA;
     const int t = carve::tc_fwd_take_timeout() | carve::tc_bwd_take_timeout() | carve::step_take_timeout();
-    return t ? CARVE_ERR_TIMEOUT : CARVE_OK;
+    const int bad = carve::simt_take_bad_seqlens();
+    return t ? CARVE_ERR_TIMEOUT : bad ? CARVE_ERR_INVALID_ARG : CARVE_OK;
 }
 
 carve_status carve_selftest_timeout(uint32_t iterations, void *stream) {

@@ -91,6 +91,8 @@ struct FwdArgs {
     float *S_final, *m_prev_out;
     float *saved_states;  // [B,H,T/16,V,K] or null
     float *saved_aux;     // [B,H,NC,V+R+K] or null
+    const int *cu_seqlens;  // [B+1] or null: B sequences packed along the token axis
+    long long total;        // rows of the packed token tensors (with cu_seqlens)
     int B, H, T, R, L, mc_mode;
 };
 
@@ -104,7 +106,34 @@ struct BwdArgs {
     void *dq, *dk, *dv;
     float *dg_logit, *dbx, *dw_logit, *dS0, *dm_prev_in, *dAw, *dA_dec, *dtau;
     float *ws;  // scratch: per-unit dA/dB(/dAw) partials or per-gate-chunk gradient records
+    const int *cu_seqlens;  // [B+1] or null: B sequences packed along the token axis
+    long long total;        // rows of the packed token tensors (with cu_seqlens)
     int B, H, T, R, L, mc_mode;
 };
+
+// Tokens of sequence b: rows [toff, toff + Tn) of tensor batch bb.  Without cu_seqlens the
+// unit is batch element b with all T tokens; with it, the sequences are packed along the token
+// axis of [1, total, H, *] tensors and sequence b owns rows [cu[b], cu[b+1]), which must lie
+// in [0, total] and number at most T (else the sequence is treated as empty and *bad, the
+// calling file's device status word, records it).
+__device__ __forceinline__ void seq_tokens(const int *cu, long long total, int T, int b, int &bb, int &toff,
+                                           int &Tn, int *bad) {
+    if (!cu) {
+        bb = b;
+        toff = 0;
+        Tn = T;
+        return;
+    }
+    const int c0 = cu[b], c1 = cu[b + 1];
+    bb = 0;
+    toff = 0;
+    Tn = 0;
+    if (c0 < 0 || c1 < c0 || (long long)c1 > total || c1 - c0 > T) {
+        if (threadIdx.x == 0) atomicOr(bad, 1);
+        return;
+    }
+    toff = c0;
+    Tn = c1 - c0;
+}
 
 }  // namespace carve

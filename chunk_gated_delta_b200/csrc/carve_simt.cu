@@ -21,6 +21,19 @@
 
 namespace carve {
 
+__device__ int g_simt_bad_seqlens;   // set when a sequence's offsets are out of range
+
+// Device status word of the sequence offsets (SIMT kernels): returns and clears it.
+int simt_take_bad_seqlens() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_simt_bad_seqlens, sizeof(int)) != cudaSuccess) return 0;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_simt_bad_seqlens, &z, sizeof(int));
+    }
+    return v;
+}
+
 __device__ __forceinline__ size_t tk(int b, int t, int h, int i, int T, int H, int W) {
     return (((size_t)b * T + t) * H + h) * W + i;
 }
@@ -64,7 +77,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
     const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
     const int b = u / H, h = u % H;
     const float amp = decay_amp(a.A_dec, h);   // e^{A_dec[h]}, 1 without the decay amplitude
-    const int NC = (T + L - 1) / L, NS = T / kSub;
+    const int NC = (T + L - 1) / L, NS = T / kSub;   // record strides (T bounds every sequence)
+    int bb, toff, Tn;   // this unit's tokens: rows [toff, toff + Tn) of tensor batch bb
+    seq_tokens(a.cu_seqlens, a.total, T, b, bb, toff, Tn, &g_simt_bad_seqlens);
+    const int NCn = (Tn + L - 1) / L;
     const IO *q = static_cast<const IO *>(a.q), *kk = static_cast<const IO *>(a.k);
     const IO *vv = static_cast<const IO *>(a.v);
     IO *o = static_cast<IO *>(a.o);
@@ -77,13 +93,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
     __syncthreads();
 
     int sidx = 0;
-    for (int c = 0; c < NC; ++c) {
-        const int t0 = c * L, n = min(L, T - t0);
+    for (int c = 0; c < NCn; ++c) {
+        const int t0 = c * L, n = min(L, Tn - t0);
         // ---- content signal of the chunk: m_c, z = Bm m_c, Delta = A z
         if (a.mc_mode == 0) {
             if (tid < K) {
                 float s = 0.f;
-                for (int t = t0; t < t0 + n; ++t) s += ld_io(q + tk(b, t, h, tid, T, H, K));
+                for (int t = t0; t < t0 + n; ++t) s += ld_io(q + tk(bb, toff + t, h, tid, T, H, K));
                 qbar[tid] = s / (float)n;
             }
             __syncthreads();
@@ -117,19 +133,24 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
                 float *st = a.saved_states + ((size_t)u * NS + sidx) * V * K;
                 for (int idx = tid; idx < V * K; idx += kThreads) st[idx] = S[(idx / K) * KP + idx % K];
             }
-            // ---- load the sub-chunk, gate activations
+            // ---- load the sub-chunk, gate activations; rows past the sequence's end (nv <= t) are
+            //      inert: q = k = v = 0, a = 1, w = 0, so they leave the state unchanged
+            const int nv = min(kSub, t0 + n - s0);
             for (int idx = tid; idx < kSub * K; idx += kThreads) {
                 const int t = idx / K, i = idx % K;
-                const size_t g = tk(b, s0 + t, h, i, T, H, K);
-                qs[t * KP + i] = ld_io(q + g);
-                ks[t * KP + i] = ld_io(kk + g);
-                lam[t * KP + i] = log_retention(a.g_logit[g], a.bx[g] + delta[i], amp, decay_bias(a.tau, h, i, K));
+                const size_t g = tk(bb, toff + s0 + t, h, i, T, H, K);
+                const bool in = t < nv;
+                qs[t * KP + i] = in ? ld_io(q + g) : 0.f;
+                ks[t * KP + i] = in ? ld_io(kk + g) : 0.f;
+                lam[t * KP + i] =
+                    in ? log_retention(a.g_logit[g], a.bx[g] + delta[i], amp, decay_bias(a.tau, h, i, K)) : 0.f;
             }
             for (int idx = tid; idx < kSub * V; idx += kThreads) {
                 const int t = idx / V, r = idx % V;
-                vs[t * VP + r] = ld_io(vv + tk(b, s0 + t, h, r, T, H, V));
+                vs[t * VP + r] = t < nv ? ld_io(vv + tk(bb, toff + s0 + t, h, r, T, H, V)) : 0.f;
             }
-            if (tid < kSub) wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + s0 + tid) * H + h] + wsc[0]);
+            if (tid < kSub)
+                wv[tid] = tid < nv ? sigmoid_f(a.w_logit[((size_t)bb * T + toff + s0 + tid) * H + h] + wsc[0]) : 0.f;
             __syncthreads();
             if (tid < K) {
                 float run = 0.f;
@@ -202,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_simt_kernel(FwdArgs a) {
                 float x = Oi[t * VP + r];
                 for (int s = 0; s <= t; ++s) x += Aqk[t * 17 + s] * Us[s * VP + r];
                 Oi[t * VP + r] = x;
-                st_io(o + tk(b, s0 + t, h, r, T, H, V), x);
+                if (t < nv) st_io(o + tk(bb, toff + s0 + t, h, r, T, H, V), x);
             }
             __syncthreads();
             if (tid < V)
@@ -281,20 +302,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
     // per-unit partials: dA [K*R], dB [R*V], dAw [R], dtau [K], dA_dec [1]
     const int rec = K * R + R * V + R + K + 1;
     float *wsu = a.ws + (size_t)u * rec;
+    int bb, toff, Tn;   // this unit's tokens: rows [toff, toff + Tn) of tensor batch bb
+    seq_tokens(a.cu_seqlens, a.total, T, b, bb, toff, Tn, &g_simt_bad_seqlens);
+    const int NCn = (Tn + L - 1) / L;
     const float amp = decay_amp(a.A_dec, h);
     float dtau_acc = 0.f, dadec_acc = 0.f;   // this thread's channel (tid < K), over the sweep
 
     for (int idx = tid; idx < V * K; idx += kThreads)
         dS[(idx / K) * KP + idx % K] = a.dS_final ? a.dS_final[(size_t)u * V * K + idx] : 0.f;
     if (tid < V) {
-        const int nl = T - (NC - 1) * L;
+        const int nl = Tn - (NCn - 1) * L;
         dox[tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * V + tid] / (float)nl : 0.f;
     }
     for (int idx = tid; idx < rec; idx += kThreads) wsu[idx] = 0.f;
     __syncthreads();
 
-    for (int c = NC - 1; c >= 0; --c) {
-        const int t0 = c * L, n = min(L, T - t0), nsub = n / kSub, sub0 = t0 / kSub;
+    for (int c = NCn - 1; c >= 0; --c) {
+        const int t0 = c * L, n = min(L, Tn - t0), nsub = (n + kSub - 1) / kSub, sub0 = t0 / kSub;
         {
             const float *aux = a.saved_aux + ((size_t)u * NC + c) * (V + R + K);
             if (tid < V) mvec[tid] = aux[tid];
@@ -316,20 +340,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
         for (int jj = nsub - 1; jj >= 0; --jj) {
             const int s0 = t0 + jj * kSub;
             const float *S0g = a.saved_states + ((size_t)u * NS + sub0 + jj) * V * K;
-            // ---- recompute the sub-chunk's forward quantities
+            // ---- recompute the sub-chunk's forward quantities (rows nv.. past the sequence's end
+            //      are inert, as in the forward, and carry no output gradient)
+            const int nv = min(kSub, t0 + n - s0);
             for (int idx = tid; idx < kSub * K; idx += kThreads) {
                 const int t = idx / K, i = idx % K;
-                const size_t g = tk(b, s0 + t, h, i, T, H, K);
-                qs[t * KP + i] = ld_io(q + g);
-                ks[t * KP + i] = ld_io(kk + g);
-                lam[t * KP + i] = log_retention(a.g_logit[g], a.bx[g] + delta[i], amp, decay_bias(a.tau, h, i, K));
+                const size_t g = tk(bb, toff + s0 + t, h, i, T, H, K);
+                const bool in = t < nv;
+                qs[t * KP + i] = in ? ld_io(q + g) : 0.f;
+                ks[t * KP + i] = in ? ld_io(kk + g) : 0.f;
+                lam[t * KP + i] =
+                    in ? log_retention(a.g_logit[g], a.bx[g] + delta[i], amp, decay_bias(a.tau, h, i, K)) : 0.f;
             }
             for (int idx = tid; idx < kSub * V; idx += kThreads) {
                 const int t = idx / V, r = idx % V;
-                Rs[t * VP + r] = ld_io(vv + tk(b, s0 + t, h, r, T, H, V));
-                dOs[t * VP + r] = ld_io(dO + tk(b, s0 + t, h, r, T, H, V)) + dox[r];
+                const bool in = t < nv;
+                Rs[t * VP + r] = in ? ld_io(vv + tk(bb, toff + s0 + t, h, r, T, H, V)) : 0.f;
+                dOs[t * VP + r] = in ? ld_io(dO + tk(bb, toff + s0 + t, h, r, T, H, V)) + dox[r] : 0.f;
             }
-            if (tid < kSub) wv[tid] = sigmoid_f(a.w_logit[((size_t)b * T + s0 + tid) * H + h] + wsc[0]);
+            if (tid < kSub)
+                wv[tid] = tid < nv ? sigmoid_f(a.w_logit[((size_t)bb * T + toff + s0 + tid) * H + h] + wsc[0]) : 0.f;
             __syncthreads();
             if (tid < K) {
                 float run = 0.f;
@@ -406,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
 #pragma unroll
                 for (int t = 0; t < kSub; ++t) {
                     dYs[t * VP + tid] = acc[t];
-                    st_io(dv + tk(b, s0 + t, h, tid, T, H, V), wv[t] * acc[t]);   // dv = dR = w dY
+                    if (t < nv) st_io(dv + tk(bb, toff + s0 + t, h, tid, T, H, V), wv[t] * acc[t]);   // dv = w dY
                 }
             }
             __syncthreads();
@@ -437,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
                 if (tid < kSub) {
                     const float w = wv[tid];
                     x = dwv[tid] * w * (1.f - w);
-                    a.dw_logit[((size_t)b * T + s0 + tid) * H + h] = x;
+                    if (tid < nv) a.dw_logit[((size_t)bb * T + toff + s0 + tid) * H + h] = x;
                 }
 #pragma unroll
                 for (int off = 8; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
@@ -525,8 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
             if (tid < K) {
                 float run = 0.f;
                 for (int t = kSub - 1; t >= 0; --t) {
-                    run += dls[t * KP + tid];
-                    const size_t g = tk(b, s0 + t, h, tid, T, H, K);
+                    run += dls[t * KP + tid];   // inert rows carry the chunk-decay term to the others
+                    if (t >= nv) continue;
+                    const size_t g = tk(bb, toff + s0 + t, h, tid, T, H, K);
                     const float beta = a.bx[g] + delta[tid];
                     // log g = -amp softplus(g_logit + tau): d/dg_logit = d/dtau = -amp sigmoid(.),
                     // d/dA_dec = log g
@@ -540,9 +571,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
                     ddelta[tid] += dbeta;
                 }
             }
-            for (int idx = tid; idx < kSub * K; idx += kThreads) {
+            for (int idx = tid; idx < nv * K; idx += kThreads) {
                 const int t = idx / K, i = idx % K;
-                const size_t g = tk(b, s0 + t, h, i, T, H, K);
+                const size_t g = tk(bb, toff + s0 + t, h, i, T, H, K);
                 st_io(dq + g, dqs[t * KP + i]);
                 st_io(dk + g, dks[t * KP + i]);
             }
@@ -575,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
             // m = S_[c-1] qbar:  dS_[c-1] += dm qbar^T,  dq_t += S_[c-1]^T dm / n  (t in chunk)
             if (tid < K) {
                 float s = 0.f;
-                for (int t = t0; t < t0 + n; ++t) s += ld_io(q + tk(b, t, h, tid, T, H, K));
+                for (int t = t0; t < t0 + n; ++t) s += ld_io(q + tk(bb, toff + t, h, tid, T, H, K));
                 vecK[tid] = s / (float)n;
             }
             __syncthreads();
@@ -592,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
             }
             __syncthreads();
             for (int idx = tid; idx < n * K; idx += kThreads) {
-                const size_t g = tk(b, t0 + idx / K, h, idx % K, T, H, K);
+                const size_t g = tk(bb, toff + t0 + idx / K, h, idx % K, T, H, K);
                 st_io(dq + g, ld_io(dq + g) + vecK[idx % K]);
             }
             if (tid < V) dox[tid] = 0.f;
@@ -604,7 +635,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_simt_kernel(BwdArgs a) {
     }
     if (a.dS0)
         for (int idx = tid; idx < V * K; idx += kThreads) a.dS0[(size_t)u * V * K + idx] = dS[(idx / K) * KP + idx % K];
-    if (a.mc_mode == 0 && a.dm_prev_in && tid < V) a.dm_prev_in[(size_t)u * V + tid] = 0.f;
+    if (a.dm_prev_in && tid < V) {
+        if (NCn == 0)   // no token: m_prev_out is m_prev_in passed through
+            a.dm_prev_in[(size_t)u * V + tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * V + tid] : 0.f;
+        else if (a.mc_mode == 0)
+            a.dm_prev_in[(size_t)u * V + tid] = 0.f;
+    }
     if (a.A_dec || a.tau) {   // the decay parameters' partials of this unit (fixed-order sum)
         if (tid < K) {
             wsu[K * R + R * V + R + tid] = dtau_acc;

@@ -134,6 +134,42 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
                        float *dm_prev_in, void *workspace, void *stream);
 
 /*
+ * carve_fwd_varlen, carve_bwd_varlen -- carve_fwd / carve_bwd over variable-length sequences
+ * packed along the token axis (no padding).  d->B is the number of sequences N and d->T an
+ * upper bound on every sequence's length (a multiple of 16, it sizes `saved` and `workspace`
+ * through carve_saved_bytes(d) and carve_bwd_workspace_bytes(d)); cu_seqlens is a DEVICE
+ * int32 array [N+1] of row offsets (cu_seqlens[0] = 0, non-decreasing), sequence n owning
+ * rows [cu_seqlens[n], cu_seqlens[n+1]) of the token tensors, and total_tokens is their row
+ * count: q, k, g_logit, bx [total_tokens, H, dk]; v, o [total_tokens, H, dv]; w_logit
+ * [total_tokens, H] (and the gradients alike).  S0, S_final, m vectors and their gradients
+ * are per sequence, [N, H, ...].  Every sequence runs the recurrence above on its own: its own
+ * state, content signal and chunk grid, which restarts at its first token; any length from 0
+ * to d->T is allowed (a ragged last chunk computes only its own tokens, and an empty sequence
+ * passes S0 and m_prev_in through).  Rows that belong to no sequence are not written.  The
+ * offsets live on the device, so the host cannot check them: a sequence whose rows fall
+ * outside [0, total_tokens] or number more than d->T is computed as empty and the next
+ * carve_check returns CARVE_ERR_INVALID_ARG.  Currently served by the SIMT kernels only (fp32
+ * or bf16 I/O, any supported shape except the tensor-core one: bf16 with dk = dv = 128 and
+ * rank <= 32 returns CARVE_ERR_UNSUPPORTED).
+ */
+carve_status carve_fwd_varlen(const carve_dims *d, const int32_t *cu_seqlens, int64_t total_tokens,
+                              const void *q, const void *k, const void *v, const float *g_logit,
+                              const float *bx, const float *w_logit, const float *A, const float *Bm,
+                              const float *Aw, const float *A_dec, const float *tau, const float *S0,
+                              const float *m_prev_in, void *o, float *S_final, float *m_prev_out,
+                              void *saved, void *stream);
+
+carve_status carve_bwd_varlen(const carve_dims *d, const int32_t *cu_seqlens, int64_t total_tokens,
+                              const void *q, const void *k, const void *v, const float *g_logit,
+                              const float *bx, const float *w_logit, const float *A, const float *Bm,
+                              const float *Aw, const float *A_dec, const float *tau, const float *S0,
+                              const float *m_prev_in, const void *saved, const void *dO,
+                              const float *dS_final, const float *dm_prev_out, void *dq, void *dk,
+                              void *dv, float *dg_logit, float *dbx, float *dw_logit, float *dA,
+                              float *dB, float *dAw, float *dA_dec, float *dtau, float *dS0,
+                              float *dm_prev_in, void *workspace, void *stream);
+
+/*
  * carve_bwd_noalloc -- carve_bwd without a workspace argument, for callers that cannot
  * allocate device memory when they run the backward (for example a plugin inside a host
  * framework that owns all device memory and passes in only input and output buffers, or a
@@ -186,7 +222,8 @@ carve_status carve_step(const carve_dims *d, const void *q, const void *k, const
  * carve_check -- blocks the host until the work queued on `stream` has finished, then
  * reports what the device saw: CARVE_ERR_CUDA if the stream reports an error,
  * CARVE_ERR_TIMEOUT if a bounded device-side wait of a carve kernel (a shared-memory
- * barrier waiting for a bulk copy) gave up since the previous carve_check, else CARVE_OK.
+ * barrier waiting for a bulk copy) gave up since the previous carve_check,
+ * CARVE_ERR_INVALID_ARG if a varlen call met out-of-range sequence offsets, else CARVE_OK.
  * The device status words are cleared by the call.  A kernel whose wait gives up records
  * it, stops its sweep, waits (again bounded) for its own copies in flight and returns, so
  * the CUDA context stays usable; the outputs of that call are undefined.  The pages have

@@ -26,9 +26,9 @@ def declared_functions():
 
 
 def test_header_declares_the_boundary():
-    assert declared_functions() == ["carve_bwd", "carve_bwd_noalloc", "carve_bwd_workspace_bytes", "carve_check",
-                                    "carve_fwd", "carve_saved_bytes", "carve_selftest_timeout",
-                                    "carve_status_string", "carve_step"]
+    assert declared_functions() == ["carve_bwd", "carve_bwd_noalloc", "carve_bwd_varlen", "carve_bwd_workspace_bytes",
+                                    "carve_check", "carve_fwd", "carve_fwd_varlen", "carve_saved_bytes",
+                                    "carve_selftest_timeout", "carve_status_string", "carve_step"]
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -139,3 +139,16 @@ def test_selftest_timeout_bounds_checked_on_host(lib):
     """Out-of-range poll counts are rejected before any launch."""
     assert lib.carve_selftest_timeout(0, None) == 1
     assert lib.carve_selftest_timeout(1_000_001, None) == 1
+
+
+def test_varlen_arguments_checked_on_host(lib):
+    """carve_fwd_varlen / carve_bwd_varlen: a missing or misaligned cu_seqlens, a negative row
+    count, and (for now) the tensor-core shape are rejected before any launch."""
+    P = ctypes.c_void_p(4096)
+    d = good_dims()
+    for cu, total, code in ((None, 64, 1), (ctypes.c_void_p(4100), 64, 1), (P, -1, 1), (P, 1 << 40, 1)):
+        assert lib.carve_fwd_varlen(ctypes.byref(d), cu, total, *fwd_args(P)) == code, (cu, total)
+        assert lib.carve_bwd_varlen(ctypes.byref(d), cu, total, *bwd_args(P)) == code, (cu, total)
+    tc = good_dims(dk=128, dv=128, rank=32, io=1, chunk=64)
+    assert lib.carve_fwd_varlen(ctypes.byref(tc), P, 64, *fwd_args(P)) == 2
+    assert lib.carve_bwd_varlen(ctypes.byref(tc), P, 64, *bwd_args(P)) == 2
