@@ -105,8 +105,9 @@ def dims_of(q, v, A, chunk, mc_mode) -> Dims:
 
 
 def dims_varlen(q, v, A, cu_seqlens, max_len, chunk, mc_mode) -> Dims:
-    """Dims of a packed call: B = number of sequences, T = max_len rounded up to 16."""
-    T = max(16, (int(max_len) + 15) // 16 * 16)
+    """Dims of a packed call: B = number of sequences, T = max_len rounded up to 64 (so that the
+    tensor-core kernels, which tile sequences by 32 or 64 tokens, serve their shapes)."""
+    T = max(64, (int(max_len) + 63) // 64 * 64)
     return Dims(cu_seqlens.numel() - 1, q.shape[-2], T, q.shape[-1], v.shape[-1], A.shape[-1], chunk, _io_of(q),
                 mc_mode)
 

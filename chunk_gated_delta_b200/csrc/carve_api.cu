@@ -15,6 +15,8 @@ int tc_fwd_take_timeout();
 int tc_bwd_take_timeout();
 int step_take_timeout();
 int simt_take_bad_seqlens();
+int tc_fwd_take_bad_seqlens();
+int tc_bwd_take_bad_seqlens();
 cudaError_t launch_selftest_timeout(uint32_t iterations, cudaStream_t st);
 cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
@@ -145,7 +147,6 @@ static carve_status fwd_impl(const carve_dims *d, const int32_t *cu, long long t
     a.cu_seqlens = cu; a.total = total;
     cudaError_t e;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (cu && tc_shape(d)) return CARVE_ERR_UNSUPPORTED;   // packed sequences: SIMT kernels only
     if (saved != nullptr && tc_saved)
         e = carve::launch_fwd_tc(a, 32, cs);
     else if (saved == nullptr && tc_fwd_chunk(d) > 0)
@@ -187,7 +188,6 @@ static carve_status bwd_impl(const carve_dims *d, const int32_t *cu, long long t
     a.dS0 = dS0; a.dm_prev_in = dm_prev_in; a.ws = static_cast<float *>(workspace);
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
     a.cu_seqlens = cu; a.total = total;
-    if (cu && tc) return CARVE_ERR_UNSUPPORTED;   // packed sequences: SIMT kernels only
     cudaError_t e = tc ? carve::launch_bwd_tc(a, dA, dB, static_cast<cudaStream_t>(stream))
                        : carve::launch_bwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
                                                 static_cast<cudaStream_t>(stream));
@@ -261,7 +261,7 @@ carve_status carve_step(const carve_dims *d, const void *q, const void *k, const
 carve_status carve_check(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CARVE_ERR_CUDA;
     const int t = carve::tc_fwd_take_timeout() | carve::tc_bwd_take_timeout() | carve::step_take_timeout();
-    const int bad = carve::simt_take_bad_seqlens();
+    const int bad = carve::simt_take_bad_seqlens() | carve::tc_fwd_take_bad_seqlens() | carve::tc_bwd_take_bad_seqlens();
     return t ? CARVE_ERR_TIMEOUT : bad ? CARVE_ERR_INVALID_ARG : CARVE_OK;
 }
 

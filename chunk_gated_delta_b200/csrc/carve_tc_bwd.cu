@@ -61,9 +61,12 @@ struct __align__(16) TcBwdSmem {
 };
 
 __device__ int g_tc_bwd_timeout;
+__device__ int g_tc_bwd_bad_seqlens;   // set when a packed sequence's offsets are out of range
 
-// DEC: the decay has its amplitude and bias (a.A_dec or a.tau given)
-template <bool DEC>
+// DEC: the decay has its amplitude and bias (a.A_dec or a.tau given).  VL: the units are
+// packed sequences (a.cu_seqlens); rows of a partial last chunk past the sequence's end are
+// inert, carry no output gradient and are never stored.
+template <bool DEC, bool VL>
 __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_constant__ BwdMaps maps) {
     constexpr int C = kBC, NB = kBNB;
     extern __shared__ __align__(128) unsigned char smraw[];
@@ -71,11 +74,14 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, c4 = lane & 3;
     const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
     const int b = u / H, h = u % H;
-    const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;
+    const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;   // record strides
+    int bb = b, toff = 0, Tn = T;   // this unit's tokens: rows [toff, toff + Tn) of tensor batch bb
+    if constexpr (VL) seq_tokens(a.cu_seqlens, a.total, T, b, bb, toff, Tn, &g_tc_bwd_bad_seqlens);
+    const int NCCn = VL ? (Tn + C - 1) / C : NCC, NGn = VL ? (Tn + L - 1) / L : NG;
     __nv_bfloat16 *dq = static_cast<__nv_bfloat16 *>(a.dq), *dk = static_cast<__nv_bfloat16 *>(a.dk);
     __nv_bfloat16 *dv = static_cast<__nv_bfloat16 *>(a.dv);
     const size_t tstride = (size_t)H * 128;
-    const size_t base_bh = (size_t)b * T * tstride + (size_t)h * 128;
+    const size_t base_bh = ((size_t)bb * T + toff) * tstride + (size_t)h * 128;
     const int v0 = 16 * warp + g, v1 = v0 + 8;
     // bf16 chunk-start states written by the forward, rows padded to kLdOp
     const __nv_bfloat16 *states = reinterpret_cast<const __nv_bfloat16 *>(a.saved_states) + (size_t)u * NCC * 128 * kLdOp;
@@ -149,12 +155,12 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         fence_mbar_init();
     }
     if (tid < 128) {
-        const int nl = T - (NG - 1) * L;
+        const int nl = Tn - (NGn - 1) * L;
         sm.dox[tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * 128 + tid] / (float)nl : 0.f;
     }
     auto issue = [&](int cc) {
         if (tid != 0) return;
-        const int row = b * T + cc * C;
+        const int row = bb * T + toff + cc * C;
         mbar_expect_tx(&sm.bar, 4u * C * 256u);
         tma_load_3d(sm.rq, &maps.q, 0, h, row, &sm.bar);
         tma_load_3d(sm.rk, &maps.k, 0, h, row, &sm.bar);
@@ -166,8 +172,10 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         mbar_expect_tx(&sm.bar_s0, 128u * kLdOp * 2u);
         bulk_g2s(sm.s0b, states + (size_t)cc * 128 * kLdOp, 128u * kLdOp * 2u, &sm.bar_s0);
     };
-    issue(NCC - 1);
-    issue_s0(NCC - 1);
+    if (!VL || NCCn > 0) {
+        issue(NCCn - 1);
+        issue_s0(NCCn - 1);
+    }
     uint32_t phase = 0;
     __syncthreads();
     // gate logits of the chunk about to be processed, loaded one chunk ahead
@@ -175,12 +183,14 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     auto load_gates = [&](int cc) {
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            const size_t gi = base_bh + (size_t)(cc * C + 16 * ib + 8 * hf + t) * tstride + c0;
-            glr[t] = *reinterpret_cast<const float2 *>(a.g_logit + gi);
-            bxr[t] = *reinterpret_cast<const float2 *>(a.bx + gi);
+            const int tt = cc * C + 16 * ib + 8 * hf + t;
+            const size_t gi = base_bh + (size_t)tt * tstride + c0;
+            const bool in = !VL || tt < Tn;
+            glr[t] = in ? *reinterpret_cast<const float2 *>(a.g_logit + gi) : make_float2(0.f, 0.f);
+            bxr[t] = in ? *reinterpret_cast<const float2 *>(a.bx + gi) : make_float2(0.f, 0.f);
         }
     };
-    load_gates(NCC - 1);
+    if (!VL || NCCn > 0) load_gates(NCCn - 1);
     // the saved record of the next gate chunk and the write logits of the next compute chunk,
     // loaded one iteration ahead
     float pd = 0.f, pq = 0.f, pw = 0.f, pdw = 0.f;
@@ -193,16 +203,19 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         if (tid == 0) pdw = aux[kTcAuxDw + R];
     };
     auto load_w = [&](int cc) {
-        if (tid < C) pw = a.w_logit[((size_t)b * T + (size_t)cc * C + tid) * H + h];
+        if (tid < C && (!VL || cc * C + tid < Tn)) pw = a.w_logit[((size_t)bb * T + toff + (size_t)cc * C + tid) * H + h];
     };
-    load_aux((NCC - 1) / CPG);
-    load_w(NCC - 1);
+    if (!VL || NCCn > 0) {
+        load_aux((NCCn - 1) / CPG);
+        load_w(NCCn - 1);
+    }
 
-    for (int cc = NCC - 1; cc >= 0; --cc) {
+    for (int cc = NCCn - 1; cc >= 0; --cc) {
         const int t0 = cc * C, gc = cc / CPG;
-        const bool gate_end = (cc % CPG) == CPG - 1 || cc == NCC - 1;
+        const int nv = VL ? min(C, Tn - t0) : C;   // tokens of this chunk inside the sequence
+        const bool gate_end = (cc % CPG) == CPG - 1 || cc == NCCn - 1;
         const bool gate_start = (cc % CPG) == 0;
-        const int n = min(L, T - gc * L);
+        const int n = min(L, Tn - gc * L);
         if (gate_end) {
             if (tid < 128) {
                 sm.delta[tid] = pd;
@@ -224,9 +237,28 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         }
         if (!mbar_wait(&sm.bar, phase)) atomicOr(&g_tc_bwd_timeout, 1);
         __syncthreads();
-        // dO plus the content-signal gradient carried from the next gate chunk, padded
+        if constexpr (VL) {
+            if (nv < C) {   // rows past the sequence's end (another sequence's, or zero fill): cleared;
+                            // the proxy fence after the Qt / Kt stores below orders these writes
+                            // before the next chunk's tile copies
+                for (int idx = tid; idx < (C - nv) * 16; idx += 256) {
+                    const int off = (nv + (idx >> 4)) * 128 + (idx & 15) * 8;
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4 *>(sm.rq + off) = z;
+                    *reinterpret_cast<uint4 *>(sm.rk + off) = z;
+                    *reinterpret_cast<uint4 *>(sm.rv + off) = z;
+                }
+                __syncthreads();
+            }
+        }
+        // dO plus the content-signal gradient carried from the next gate chunk, padded (inert
+        // rows: none)
         for (int idx = tid; idx < C * 16; idx += 256) {
             const int t = idx >> 4, part = idx & 15;
+            if (VL && t >= nv) {
+                *reinterpret_cast<uint4 *>(sm.dop + t * kLdOp + part * 8) = make_uint4(0u, 0u, 0u, 0u);
+                continue;
+            }
             const uint4 x = *reinterpret_cast<const uint4 *>(sm.rdo + t * 128 + part * 8);
             const __nv_bfloat16 *xv = reinterpret_cast<const __nv_bfloat16 *>(&x);
             const float *dx = sm.dox + part * 8;
@@ -250,6 +282,9 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 } else {
                     retention(glr[t].x, bxr[t].x + dl0, av[0][t], ia[0][t]);
                     retention(glr[t].y, bxr[t].y + dl1, av[1][t], ia[1][t]);
+                }
+                if constexpr (VL) {
+                    if (16 * ib + 8 * hf + t >= nv) av[0][t] = av[1][t] = ia[0][t] = ia[1][t] = 1.f;   // inert row
                 }
             }
             if (hf == 0) {
@@ -294,7 +329,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 *reinterpret_cast<float2 *>(&sm.rfac[row * kLdF + c0]) = make_float2(rf[0][t], rf[1][t]);
             }
         }
-        if (tid < C) sm.wv[tid] = sigmoid_f(pw + sm.dwc);
+        if (tid < C) sm.wv[tid] = (!VL || tid < nv) ? sigmoid_f(pw + sm.dwc) : 0.f;
         __syncthreads();
         if (tid < 128) {
             float dblk[NB];   // decay over each 16-token block
@@ -764,8 +799,10 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     }
                     *reinterpret_cast<float2 *>(sm.dlam + t * kLdF + ch) = make_float2(dlv[0], dlv[1]);
                     const size_t gi = base_bh + (size_t)(t0 + t) * tstride + ch;
-                    *reinterpret_cast<uint32_t *>(dq + gi) = pack_bf16(dqv[0], dqv[1]);
-                    *reinterpret_cast<uint32_t *>(dk + gi) = pack_bf16(dkv[0], dkv[1]);
+                    if (!VL || t < nv) {
+                        *reinterpret_cast<uint32_t *>(dq + gi) = pack_bf16(dqv[0], dqv[1]);
+                        *reinterpret_cast<uint32_t *>(dk + gi) = pack_bf16(dkv[0], dkv[1]);
+                    }
                 }
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
@@ -812,12 +849,12 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             for (int w = 0; w < 8; ++w) dw += sm.dwp[w * C + tid];
             const float w = sm.wv[tid];
             float x = dw * w * (1.f - w);
-            a.dw_logit[((size_t)b * T + t0 + tid) * H + h] = x;
+            if (!VL || tid < nv) a.dw_logit[((size_t)bb * T + toff + t0 + tid) * H + h] = x;
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
             if (tid == 0) sm.ddw += x;
         }
-        for (int idx = tid; idx < C * 16; idx += 256) {   // dv = dR
+        for (int idx = tid; idx < nv * 16; idx += 256) {   // dv = dR
             const int t = idx >> 4, part = idx & 15;
             *reinterpret_cast<uint4 *>(dv + base_bh + (size_t)(t0 + t) * tstride + part * 8) =
                 *reinterpret_cast<const uint4 *>(sm.drb + t * kLdOp + part * 8);
@@ -840,6 +877,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             for (int t = 7; t >= 0; --t) {
                 const int row = 16 * ib + 8 * hf + t;
                 const float2 d2 = *reinterpret_cast<const float2 *>(&sm.dlam[row * kLdF + c0]);
+                const bool inert = VL && row >= nv;   // passes the running sum on, has no gate gradient
                 float dg[2], db[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
@@ -848,7 +886,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     const float gx = e ? glr[t].y : glr[t].x, e2 = __expf(-((e ? bxr[t].y : bxr[t].x) + dl[e]));
                     if constexpr (DEC) {   // log g = -amp softplus(x), x = g_logit + tau: d/dx = -amp sigmoid(x)
                         const float x = gx + tb[e], e1 = __expf(x), sp = softplus_fast(x, e1);
-                        const bool floor = !(__fdividef(1.f, __expf(amp * sp) * (1.f + e2)) >= kAMin);
+                        const bool floor = !(__fdividef(1.f, __expf(amp * sp) * (1.f + e2)) >= kAMin) || inert;
                         dg[e] = floor ? 0.f : -amp * sigmoid_fast(x, e1) * run[e];
                         db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
                         dtp[e] += dg[e];
@@ -856,7 +894,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     } else {
                         const float e1 = __expf(gx);
                         const float D = (1.f + e1) * (1.f + e2);
-                        const bool floor = !(__fdividef(1.f, D) >= kAMin);
+                        const bool floor = !(__fdividef(1.f, D) >= kAMin) || inert;
                         dg[e] = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run[e];
                         db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
                     }
@@ -879,7 +917,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             for (int h2 = 0; h2 < 2 * NB; ++h2) x += sm.pdd[h2 * 128 + tid];
             sm.ddelta[tid] += x;
         }
-        for (int idx = tid; idx < C * 32; idx += 256) {   // d g_logit, dbx: four channels per store
+        for (int idx = tid; idx < nv * 32; idx += 256) {   // d g_logit, dbx: four channels per store
             const int t = idx >> 5, c = (idx & 31) * 4;
             const float *gsrc = sm.dlam + t * kLdF + c, *bsrc = sm.rfac + t * kLdF + c;
             const size_t gi = base_bh + (size_t)(t0 + t) * tstride + c;
@@ -961,7 +999,12 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             *reinterpret_cast<float2 *>(D + v1 * 128 + col) = make_float2(ds[j][2], ds[j][3]);
         }
     }
-    if (a.mc_mode == 0 && a.dm_prev_in && tid < 128) a.dm_prev_in[(size_t)u * 128 + tid] = 0.f;
+    if (a.dm_prev_in && tid < 128) {
+        if (VL && NCCn == 0)   // no token: m_prev_out is m_prev_in passed through
+            a.dm_prev_in[(size_t)u * 128 + tid] = a.dm_prev_out ? a.dm_prev_out[(size_t)u * 128 + tid] : 0.f;
+        else if (a.mc_mode == 0)
+            a.dm_prev_in[(size_t)u * 128 + tid] = 0.f;
+    }
     if constexpr (DEC) {   // this unit's d tau (the four threads of each channel pair) and d A_dec, fixed order
         float *red = sm.xp;   // free after the sweep: [256][2] channel partials, then [256] amplitude
         *reinterpret_cast<float2 *>(&red[2 * tid]) = make_float2(dtp[0], dtp[1]);
@@ -1003,8 +1046,11 @@ __global__ void reduce_decay_kernel(const float *part, float *dtau, float *dA_de
 // of the head's 256 R outputs; the partial sums go to the workspace.  Pass 2 adds the slices
 // in order.
 constexpr int kRedRec = 32, kRedSlice = 64;
+// With packed sequences (cu) the records of gate chunks past a sequence's end hold nothing
+// and count as zero.
 __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *wsg, const float *aux, float *part,
-                                                                  int B, int H, int NG, int R) {
+                                                                  int B, int H, int NG, int R, const int *cu,
+                                                                  long long total, int T, int L) {
     __shared__ __align__(16) float gd[kRedRec][128], rm[kRedRec][128], gz[kRedRec][kTcMaxRankBwd],
         rz[kRedRec][kTcMaxRankBwd], gw[kRedRec];
     const int h = blockIdx.x, sl = blockIdx.y, tid = threadIdx.x, NR = B * NG;
@@ -1014,26 +1060,35 @@ __global__ void __launch_bounds__(256) reduce_dAdB_partial_kernel(const float *w
     // (rows j = 4 jb + a, columns v = 4 vb + b); the operands of a record are float4 reads
     const int ka = tid >> 3, ja = tid & 7, jb = tid >> 5, vb = tid & 31;
     float accA[4][4] = {}, accB[4][4] = {};
+    auto live = [&](int rec) {
+        if (!cu) return true;
+        int bb, toff, Tn;
+        seq_tokens(cu, total, T, rec / NG, bb, toff, Tn, &g_tc_bwd_bad_seqlens);
+        return (rec % NG) * L < Tn;
+    };
     for (int i0 = r0; i0 < r1; i0 += kRedRec) {
         const int nr = min(kRedRec, r1 - i0);
         for (int idx = tid; idx < nr * 64; idx += 256) {   // dDelta and m, four floats per load
             const int i = idx >> 6, part4 = idx & 63, rec = i0 + i;
             const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
+            const bool lv = live(rec);
             if (part4 < 32) {
                 *reinterpret_cast<float4 *>(&gd[i][4 * part4]) =
-                    *reinterpret_cast<const float4 *>(wsg + (u * NG + gc) * kTcGradRec + 4 * part4);
+                    lv ? *reinterpret_cast<const float4 *>(wsg + (u * NG + gc) * kTcGradRec + 4 * part4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
             } else {
                 const float *r = aux + (u * NG + gc) * (kTcAuxFixed + R) + 4 * (part4 - 32);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) rm[i][4 * (part4 - 32) + e] = r[e];
+                for (int e = 0; e < 4; ++e) rm[i][4 * (part4 - 32) + e] = lv ? r[e] : 0.f;
             }
         }
         for (int idx = tid; idx < nr * kTcMaxRankBwd; idx += 256) {   // dz and z (zero beyond R)
             const int i = idx / kTcMaxRankBwd, j = idx % kTcMaxRankBwd, rec = i0 + i;
             const size_t u = (size_t)(rec / NG) * H + h, gc = rec % NG;
-            gz[i][j] = j < R ? wsg[(u * NG + gc) * kTcGradRec + 128 + j] : 0.f;
-            rz[i][j] = j < R ? aux[(u * NG + gc) * (kTcAuxFixed + R) + 128 + j] : 0.f;
-            if (j == 0) gw[i] = wsg[(u * NG + gc) * kTcGradRec + kTcGradDw];
+            const bool lv = live(rec);
+            gz[i][j] = (lv && j < R) ? wsg[(u * NG + gc) * kTcGradRec + 128 + j] : 0.f;
+            rz[i][j] = (lv && j < R) ? aux[(u * NG + gc) * (kTcAuxFixed + R) + 128 + j] : 0.f;
+            if (j == 0) gw[i] = lv ? wsg[(u * NG + gc) * kTcGradRec + kTcGradDw] : 0.f;
         }
         __syncthreads();
         if (tid < R)
@@ -1107,13 +1162,37 @@ __global__ void dq_readout_kernel(__nv_bfloat16 *dq, const float *vec, int H, in
     *p = x;
 }
 
+// The same for packed sequences: one block per (unit, gate chunk), over the chunk's rows
+__global__ void dq_readout_varlen_kernel(__nv_bfloat16 *dq, const float *vec, int H, int T, int L, const int *cu,
+                                         long long total) {
+    const int NG = (T + L - 1) / L, u = blockIdx.x / NG, gc = blockIdx.x % NG, h = u % H;
+    int bb, toff, Tn;
+    seq_tokens(cu, total, T, u / H, bb, toff, Tn, &g_tc_bwd_bad_seqlens);
+    const int t0 = gc * L, t1 = min(Tn, t0 + L);
+    const float *vk = vec + ((size_t)u * NG + gc) * 128;
+    for (int i = threadIdx.x; i < (t1 - t0) * 16; i += blockDim.x) {
+        const int t = t0 + (i >> 4), part = i & 15;
+        uint4 *p = reinterpret_cast<uint4 *>(dq + ((size_t)(toff + t) * H + h) * 128 + part * 8);
+        uint4 x = *p;
+        __nv_bfloat162 *xv = reinterpret_cast<__nv_bfloat162 *>(&x);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(xv[e]);
+            xv[e] = __floats2bfloat162_rn(f.x + vk[part * 8 + 2 * e], f.y + vk[part * 8 + 2 * e + 1]);
+        }
+        *p = x;
+    }
+}
+
 cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t st) {
     const int bytes = (int)sizeof(TcBwdSmem);
-    const bool dec = a.A_dec || a.tau;
-    auto kern = dec ? tc_bwd_kernel<true> : tc_bwd_kernel<false>;
+    const bool dec = a.A_dec || a.tau, vl = a.cu_seqlens != nullptr;
+    auto kern = vl ? (dec ? tc_bwd_kernel<true, true> : tc_bwd_kernel<false, true>)
+                   : (dec ? tc_bwd_kernel<true, false> : tc_bwd_kernel<false, false>);
     cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), bytes);
     if (e != cudaSuccess) return e;
-    const long long rows = (long long)a.B * a.T;
+    // token rows: B T, or the packed row count (at least 1 for a valid map)
+    const long long rows = vl ? (a.total > 0 ? a.total : 1) : (long long)a.B * a.T;
     BwdMaps maps;
     if ((e = make_token_tile_map(&maps.q, a.q, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
     if ((e = make_token_tile_map(&maps.k, a.k, 2, 128, a.H, rows, kBC)) != cudaSuccess) return e;
@@ -1124,8 +1203,12 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
     if (a.mc_mode == 0) {
         const size_t rows = (size_t)a.B * a.T * a.H;
         const float *vec = a.ws + (size_t)a.B * a.H * ((a.T + a.L - 1) / a.L) * kTcGradRec;
-        dq_readout_kernel<<<(unsigned)((rows * 16 + 255) / 256), 256, 0, st>>>(static_cast<__nv_bfloat16 *>(a.dq), vec,
-                                                                              a.H, a.T, a.L, rows);
+        if (vl)
+            dq_readout_varlen_kernel<<<a.B * a.H * ((a.T + a.L - 1) / a.L), 256, 0, st>>>(
+                static_cast<__nv_bfloat16 *>(a.dq), vec, a.H, a.T, a.L, a.cu_seqlens, a.total);
+        else
+            dq_readout_kernel<<<(unsigned)((rows * 16 + 255) / 256), 256, 0, st>>>(
+                static_cast<__nv_bfloat16 *>(a.dq), vec, a.H, a.T, a.L, rows);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int NG = (a.T + a.L - 1) / a.L, S = tc_reduce_slices(a.B, NG);
@@ -1135,13 +1218,25 @@ cudaError_t launch_bwd_tc(const BwdArgs &a, float *dA, float *dB, cudaStream_t s
         reduce_decay_kernel<<<a.H, 128, 0, st>>>(dec_part, a.dtau, a.dA_dec, a.B, a.H);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    reduce_dAdB_partial_kernel<<<dim3(a.H, S), 256, 0, st>>>(a.ws, a.saved_aux, part, a.B, a.H, NG, a.R);
+    reduce_dAdB_partial_kernel<<<dim3(a.H, S), 256, 0, st>>>(a.ws, a.saved_aux, part, a.B, a.H, NG, a.R,
+                                                              a.cu_seqlens, a.total, a.T, a.L);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     reduce_dAdB_final_kernel<<<(a.H * 257 * a.R + 255) / 256, 256, 0, st>>>(part, dA, dB, a.dAw, a.H, a.R, S);
     return cudaGetLastError();
 }
 
 size_t tc_bwd_smem() { return sizeof(TcBwdSmem); }
+
+// Device status word of the packed-sequence offsets (this file): returns and clears it.
+int tc_bwd_take_bad_seqlens() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_bwd_bad_seqlens, sizeof(int)) != cudaSuccess) return 0;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_tc_bwd_bad_seqlens, &z, sizeof(int));
+    }
+    return v;
+}
 
 // Device status word of this file: returns and clears it.
 int tc_bwd_take_timeout() {

@@ -29,6 +29,7 @@ namespace carve {
 constexpr int kTcMaxRank = 32;                        // low-rank factors staged in shared memory
 
 __device__ int g_tc_timeout;  // set when a bounded wait gives up (never expected)
+__device__ int g_tc_bad_seqlens;  // set when a packed sequence's offsets are out of range
 
 template <int NB>
 struct __align__(16) TcFwdSmem {
@@ -57,8 +58,10 @@ struct TileMaps {
     CUtensorMap q, k, v, gl, bx;
 };
 
-// DEC: the decay has its amplitude and bias (a.A_dec or a.tau given)
-template <int NB, bool DEC>
+// DEC: the decay has its amplitude and bias (a.A_dec or a.tau given).  VL: the units are
+// packed sequences (a.cu_seqlens); the last chunk of a sequence may be partial, its rows past
+// the sequence's end are made inert (q = k = v = 0, a = 1, w = 0) and never stored.
+template <int NB, bool DEC, bool VL>
 __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_constant__ TileMaps maps) {
     using SM = TcFwdSmem<NB>;
     constexpr int C = SM::C, LDA = SM::LDA;
@@ -68,11 +71,14 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, c4 = lane & 3;
     const int u = blockIdx.x, H = a.H, T = a.T, R = a.R, L = a.L;
     const int b = u / H, h = u % H;
-    const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;
+    const int NCC = T / C, CPG = L / C, NG = (T + L - 1) / L;   // record strides
+    int bb = b, toff = 0, Tn = T;   // this unit's tokens: rows [toff, toff + Tn) of tensor batch bb
+    if constexpr (VL) seq_tokens(a.cu_seqlens, a.total, T, b, bb, toff, Tn, &g_tc_bad_seqlens);
+    const int NCCn = VL ? (Tn + C - 1) / C : NCC;   // compute chunks of this unit
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
     const size_t tstride = (size_t)H * 128;
-    const size_t base_bh = (size_t)b * T * tstride + (size_t)h * 128;   // token 0 of this unit
+    const size_t base_bh = ((size_t)bb * T + toff) * tstride + (size_t)h * 128;   // token 0 of this unit
     const int v0 = 16 * warp + g, v1 = v0 + 8;
     // the decay's amplitude and the biases of this thread's gate channels 2 (tid & 63) + {0, 1}
     const float amp = DEC ? decay_amp(a.A_dec, h) : 1.f;
@@ -112,7 +118,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     // arming the barrier) go out mid-chunk and v (which = 1) at the end of the previous chunk.
     auto issue = [&](int cc, int which) {
         if (tid != 0) return;
-        const int row = b * T + cc * C, st = cc % SM::ST;
+        const int row = bb * T + toff + cc * C, st = cc % SM::ST;
         uint64_t *bar = &sm.bar[st];
         if (which == 0) {
             mbar_expect_tx(bar, 3u * C * 256u + (SM::GT ? 2u * C * 512u : 0u));
@@ -134,11 +140,13 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             tma_prefetch_desc(&maps.bx);
         }
     }
-    issue(0, 0);
-    if (SM::ST == 1) issue(0, 1);
+    if (!VL || NCCn > 0) {
+        issue(0, 0);
+        if (SM::ST == 1) issue(0, 1);
+    }
     uint32_t phase_bits = 0u;   // bit st: parity to wait for on stage st
     float dwc = 0.f;            // write-gate content term of the current gate chunk
-    float wnext = tid < C ? a.w_logit[((size_t)b * T + tid) * H + h] : 0.f;
+    float wnext = (tid < C && (!VL || tid < Tn)) ? a.w_logit[((size_t)bb * T + toff + tid) * H + h] : 0.f;
     // mean q of the next gate chunk from the saved record (mode 0 with saving), one chunk ahead
     auto load_qbar = [&](int gc) {
         return (a.saved_aux && a.mc_mode == 0 && tid < 128 && gc < NG)
@@ -147,10 +155,11 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     };
     float pqb = load_qbar(0);
 
-    for (int cc = 0; cc < NCC; ++cc) {
+    for (int cc = 0; cc < NCCn; ++cc) {
         const int t0 = cc * C, gc = cc / CPG;
-        const bool first = (cc % CPG) == 0, last = (cc % CPG) == CPG - 1 || cc == NCC - 1;
-        const int n = min(L, T - gc * L);
+        const bool first = (cc % CPG) == 0, last = (cc % CPG) == CPG - 1 || cc == NCCn - 1;
+        const int n = min(L, Tn - gc * L);
+        const int nv = VL ? min(C, Tn - t0) : C;   // tokens of this chunk inside the sequence
         const int st = cc % SM::ST;
         // gate inputs of this chunk, into registers (one-stage layout only; their latency
         // overlaps the readout)
@@ -164,19 +173,33 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 if (p < 128 * NB) {
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
-                        const size_t gi =
-                            ((size_t)b * T + t0 + 16 * i + 8 * hf + t) * tstride + (size_t)h * 128 + 2 * cp;
-                        glr[x][t] = *reinterpret_cast<const float2 *>(a.g_logit + gi);
-                        bxr[x][t] = *reinterpret_cast<const float2 *>(a.bx + gi);
+                        const int tt = t0 + 16 * i + 8 * hf + t;
+                        const size_t gi = ((size_t)bb * T + toff + tt) * tstride + (size_t)h * 128 + 2 * cp;
+                        const bool in = !VL || tt < Tn;
+                        glr[x][t] = in ? *reinterpret_cast<const float2 *>(a.g_logit + gi) : make_float2(0.f, 0.f);
+                        bxr[x][t] = in ? *reinterpret_cast<const float2 *>(a.bx + gi) : make_float2(0.f, 0.f);
                     }
                 }
             }
         }
         if (!mbar_wait(&sm.bar[st], (phase_bits >> st) & 1u)) atomicOr(&g_tc_timeout, 1);
         phase_bits ^= 1u << st;
-        if (SM::ST == 2 && cc + 1 < NCC) issue(cc + 1, 0);   // the other stage is free since last chunk
+        if (SM::ST == 2 && cc + 1 < NCCn) issue(cc + 1, 0);   // the other stage is free since last chunk
+        if constexpr (VL) {
+            if (nv < C) {   // rows past the sequence's end (another sequence's, or zero fill): cleared
+                for (int idx = tid; idx < (C - nv) * 16; idx += 256) {
+                    const int off = (nv + (idx >> 4)) * 128 + (idx & 15) * 8;
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4 *>(&sm.rq[st][off]) = z;
+                    *reinterpret_cast<uint4 *>(&sm.rk[st][off]) = z;
+                    *reinterpret_cast<uint4 *>(&sm.rv[st][off]) = z;
+                }
+                __syncthreads();
+            }
+        }
         const float wcur = wnext;
-        if (tid < C && cc + 1 < NCC) wnext = a.w_logit[((size_t)b * T + t0 + C + tid) * H + h];
+        if (tid < C && cc + 1 < NCCn && (!VL || t0 + C + tid < Tn))
+            wnext = a.w_logit[((size_t)bb * T + toff + t0 + C + tid) * H + h];
         if (a.saved_states) {   // bf16 copy of the chunk-start state, rows padded to 136
             __nv_bfloat16 *stb = reinterpret_cast<__nv_bfloat16 *>(a.saved_states) + ((size_t)u * NCC + cc) * 128 * kLdOp;
 #pragma unroll
@@ -269,6 +292,9 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                         retention(gv.x, bv.x + dl0, av[0][t], ia[0][t]);
                         retention(gv.y, bv.y + dl1, av[1][t], ia[1][t]);
                     }
+                    if constexpr (VL) {
+                        if (16 * i + 8 * hf + t >= nv) av[0][t] = av[1][t] = ia[0][t] = ia[1][t] = 1.f;   // inert row
+                    }
                 }
                 float rf[2][8], cf[2][8];
                 if (hf == 0) {
@@ -313,7 +339,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 }
             }
         }
-        if (tid < C) sm.wv[tid] = sigmoid_f(wcur + dwc);
+        if (tid < C) sm.wv[tid] = (!VL || tid < nv) ? sigmoid_f(wcur + dwc) : 0.f;
         __syncthreads();
         // ---- decayed operands Qt = Qm Em, Kt = Krm Em: one (channel, 16-token block) item per
         //      thread, each forming its own prefix of block decays; chunk-level factors per
@@ -433,7 +459,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             }
         }
         __syncthreads();
-        if (SM::ST == 1 && cc + 1 < NCC) issue(cc + 1, 0);
+        if (SM::ST == 1 && cc + 1 < NCCn) issue(cc + 1, 0);
         // ---- X = Diag(w)(V - Kt S0^T), as X^T (rows v, cols t)
 #pragma unroll
         for (int j = 0; j < 2 * NB; ++j) {
@@ -540,8 +566,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             }
         }
         __syncthreads();
-        if (SM::ST == 1 && cc + 1 < NCC) issue(cc + 1, 1);
-        for (int idx = tid; idx < C * 16; idx += 256) {
+        if (SM::ST == 1 && cc + 1 < NCCn) issue(cc + 1, 1);
+        for (int idx = tid; idx < nv * 16; idx += 256) {
             const int t = idx >> 4, part = idx & 15;
             *reinterpret_cast<uint4 *>(o + base_bh + (size_t)(t0 + t) * tstride + part * 8) =
                 *reinterpret_cast<const uint4 *>(sm.ost() + t * kLdOp + part * 8);
@@ -566,11 +592,15 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 // Per (batch, gate chunk): mean of q over the gate chunk's tokens for every head, into the saved
 // aux records (offset 256 + R of each kTcAuxFixed + R floats).  A token's H*128 channels are one
 // contiguous row; each thread owns 8 consecutive channels (one 16-byte load per token).
-__global__ void __launch_bounds__(256) qbar_kernel(const __nv_bfloat16 *q, float *aux, int H, int T, int L, int R) {
+__global__ void __launch_bounds__(256) qbar_kernel(const __nv_bfloat16 *q, float *aux, int H, int T, int L, int R,
+                                                   const int *cu, long long total) {
     const int NG = (T + L - 1) / L, b = blockIdx.x / NG, gc = blockIdx.x % NG;
-    const int n = min(L, T - gc * L);
+    int bb = b, toff = 0, Tn = T;   // cu: packed sequences
+    if (cu) seq_tokens(cu, total, T, b, bb, toff, Tn, &g_tc_bad_seqlens);
+    if (gc * L >= Tn) return;
+    const int n = min(L, Tn - gc * L);
     const size_t row = (size_t)H * 128;
-    const __nv_bfloat16 *src = q + ((size_t)b * T + (size_t)gc * L) * row;
+    const __nv_bfloat16 *src = q + ((size_t)bb * T + toff + (size_t)gc * L) * row;
     for (int c8 = threadIdx.x; c8 < H * 16; c8 += blockDim.x) {
         float acc[2][8] = {};
         int t = 0;
@@ -603,12 +633,16 @@ __global__ void __launch_bounds__(256) qbar_kernel(const __nv_bfloat16 *q, float
 
 template <int NB>
 cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
-    auto kern = (a.A_dec || a.tau) ? tc_fwd_kernel<NB, true> : tc_fwd_kernel<NB, false>;
+    const bool dec = a.A_dec || a.tau, vl = a.cu_seqlens != nullptr;
+    auto kern = vl ? (dec ? tc_fwd_kernel<NB, true, true> : tc_fwd_kernel<NB, false, true>)
+                   : (dec ? tc_fwd_kernel<NB, true, false> : tc_fwd_kernel<NB, false, false>);
     const int bytes = (int)sizeof(TcFwdSmem<NB>);
     cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), bytes);
     if (e != cudaSuccess) return e;
     const int C = 16 * NB;
-    const long long rows = (long long)a.B * a.T;
+    // token rows of the tensors: B T, or the packed row count (at least 1 for a valid map; no
+    // copy is issued for a sequence without tokens)
+    const long long rows = a.cu_seqlens ? (a.total > 0 ? a.total : 1) : (long long)a.B * a.T;
     TileMaps maps;
     if ((e = make_token_tile_map(&maps.q, a.q, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
     if ((e = make_token_tile_map(&maps.k, a.k, 2, 128, a.H, rows, C)) != cudaSuccess) return e;
@@ -620,7 +654,7 @@ cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
     if (a.saved_aux && a.mc_mode == 0) {
         const int NG = (a.T + a.L - 1) / a.L;
         qbar_kernel<<<a.B * NG, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.q), a.saved_aux, a.H, a.T, a.L,
-                                              a.R);
+                                              a.R, a.cu_seqlens, a.total);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     kern<<<a.B * a.H, 256, bytes, st>>>(a, maps);
@@ -639,6 +673,17 @@ cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st) {
 }
 
 size_t tc_fwd_smem(int L) { return tc_compute_chunk(L) == 32 ? sizeof(TcFwdSmem<2>) : sizeof(TcFwdSmem<4>); }
+
+// Device status word of the packed-sequence offsets (this file): returns and clears it.
+int tc_fwd_take_bad_seqlens() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_bad_seqlens, sizeof(int)) != cudaSuccess) return 0;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_tc_bad_seqlens, &z, sizeof(int));
+    }
+    return v;
+}
 
 // Device status word of this file: returns and clears it.
 int tc_fwd_take_timeout() {

@@ -148,9 +148,9 @@ carve_status carve_bwd(const carve_dims *d, const void *q, const void *k, const 
  * passes S0 and m_prev_in through).  Rows that belong to no sequence are not written.  The
  * offsets live on the device, so the host cannot check them: a sequence whose rows fall
  * outside [0, total_tokens] or number more than d->T is computed as empty and the next
- * carve_check returns CARVE_ERR_INVALID_ARG.  Currently served by the SIMT kernels only (fp32
- * or bf16 I/O, any supported shape except the tensor-core one: bf16 with dk = dv = 128 and
- * rank <= 32 returns CARVE_ERR_UNSUPPORTED).
+ * carve_check returns CARVE_ERR_INVALID_ARG.  The kernels are chosen as for carve_fwd /
+ * carve_bwd from d (the tensor-core ones for bf16, dk = dv = 128, rank <= 32, chunk >= 32
+ * and a bound T that is a multiple of 32).
  */
 carve_status carve_fwd_varlen(const carve_dims *d, const int32_t *cu_seqlens, int64_t total_tokens,
                               const void *q, const void *k, const void *v, const float *g_logit,

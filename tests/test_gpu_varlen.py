@@ -38,13 +38,16 @@ def packed_case(lens, K, V, R, H, io, seed, L):
     return packed, cu
 
 
-@pytest.mark.parametrize("io,K,V", [("fp32", 64, 64), ("bf16", 128, 64)])
+@pytest.mark.parametrize("io,K,V,L", [("fp32", 64, 64, 32), ("bf16", 128, 64, 32), ("bf16", 128, 128, 64),
+                                      ("bf16", 128, 128, 32)])
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("terms", [False, True])
-def test_packed_sequences_match_oracle(cuda_device, io, K, V, mode, terms):
+def test_packed_sequences_match_oracle(cuda_device, io, K, V, L, mode, terms):
+    """(bf16, 128, 128): the tensor-core kernels (32-token chunks saving for the backward, and
+    the forward-only kernel with 64-token chunks when L = 64); the others: the SIMT kernels."""
     import torch
-    lens = [37, 0, 64, 1, 100, 16, 45, 112]
-    L, H, R = 32, 2, 16
+    lens = [37, 0, 64, 1, 100, 16, 45, 128]
+    H, R = 2, 16
     packed, cu = packed_case(lens, K, V, R, H, io, 900 + 10 * mode + K, L)
     N = len(lens)
     extra = {}
@@ -89,6 +92,14 @@ def test_packed_sequences_match_oracle(cuda_device, io, K, V, mode, terms):
             x, ref = x[:, :n_rows], ref[:, :n_rows]
         e = rel_l2(x, ref)
         assert e <= tol, f"{key}: rel-L2 {e:.3e}"
+    if L == 64:   # the forward-only path (64-token compute chunks on the tensor cores)
+        f = carve.carve_fwd_varlen(*args, tcu, chunk=L, max_len=max(lens), mc_mode=mode, S0=tS0, m_prev_in=tmp,
+                                   save_for_bwd=False, **tex)
+        assert carve.carve_check() == 0
+        e = rel_l2(host(f["o"])[:, :n_rows], r["o"][:, :n_rows])
+        assert e <= tol, f"o (forward only): rel-L2 {e:.3e}"
+        e = rel_l2(host(f["S_final"]), r["S_final"])
+        assert e <= tol, f"S_final (forward only): rel-L2 {e:.3e}"
     # the empty sequence passes its state and content signal (and their gradients) through
     assert np.array_equal(host(out["S_final"])[1], S0[1].astype(np.float64))
     assert np.array_equal(host(g["dS0"])[1], dSf[1].astype(np.float64))
