@@ -29,6 +29,7 @@ import numpy as np  # noqa: E402
 
 from chunk_gated_delta_b200 import inputs as I  # noqa: E402
 
+VARLEN_LO, VARLEN_HI = 512, 8192   # lengths of the packed variable-length benchmark
 METRIC = "fwd+bwd tokens/s per layer (B200, 16 heads, d=128) & % bf16 tensor peak"
 
 # Algorithmic HBM bytes per (token, head) at d = 128 with bf16 q/k/v/o and fp32 gates:
@@ -264,32 +265,40 @@ def run_train(args, w, fwd_only=False):
         opt["Aw"] = torch.from_numpy(I.normal(w.seed, 95, (w.H, w.R), 0.0, 0.02).astype(np.float32)).to(dev)
     if args.decay:        # the decay's log-amplitude [H] and bias [H, dk]
         opt.update({k: torch.from_numpy(v).to(dev) for k, v in I.make_decay(w).items()})
-    fwd_out = carve.carve_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
-                              dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only, **opt)
+    packed, lens = {}, None   # packed variable-length sequences: the w.T tokens cut into sequences
+    if args.varlen:
+        lens = I.make_lengths(w.T, VARLEN_LO, VARLEN_HI, w.seed + 7919 * rank)
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        packed = dict(cu_seqlens=torch.from_numpy(cu).to(dev), max_len=int(lens.max()))
+    fwd_fn = carve.carve_fwd_varlen if packed else carve.carve_fwd
+    bwd_fn = carve.carve_bwd_varlen if packed else carve.carve_bwd
+    fwd_out = fwd_fn(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
+                     dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only, **opt, **packed)
     bwd_out = None
     if not fwd_only:   # dA and dB as views of one flat buffer: the step's only collective
         from chunk_gated_delta_b200 import dist as cdist
         dAB, dA_, dB_ = cdist.grad_buffer(w.H, w.K, w.V, w.R, dev)
-        bwd_out = carve.carve_bwd(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
-                                  dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode,
-                                  out={"dA": dA_, "dB": dB_}, **opt)
-    workspace = torch.empty(carve.bwd_workspace_bytes(carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode)),
-                            dtype=torch.uint8, device=dev)
+        bwd_out = bwd_fn(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
+                         dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode,
+                         out={"dA": dA_, "dB": dB_}, **opt, **packed)
+    dims = (carve.dims_varlen(dv_["q"], dv_["v"], dv_["A"], packed["cu_seqlens"], packed["max_len"], L, mode)
+            if packed else carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode))
+    workspace = torch.empty(carve.bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(x, ev=None):
         if ev is not None:
             ev[0].record(stream)
-        carve.carve_fwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"], chunk=L,
-                        mc_mode=mode, out=fwd_out, save_for_bwd=not fwd_only, **opt)
+        fwd_fn(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"], chunk=L,
+               mc_mode=mode, out=fwd_out, save_for_bwd=not fwd_only, **opt, **packed)
         if ev is not None:
             ev[1].record(stream)
         if fwd_only:
             if ev is not None:
                 ev[2].record(stream)
             return
-        carve.carve_bwd(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"],
-                        fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace, **opt)
+        bwd_fn(x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"], x["B"],
+               fwd_out["saved"], x["dO"], chunk=L, mc_mode=mode, out=bwd_out, workspace=workspace, **opt, **packed)
         if ev is not None:
             ev[2].record(stream)
         if ws > 1:
@@ -323,13 +332,13 @@ def run_train(args, w, fwd_only=False):
     achieved = dbytes / (dms * 1e-3) / 1e9
     flops = (fwd_flops(dd, L, w.R) + (0 if fwd_only else bwd_flops(dd, L, w.R))) * th * ws
     tensor_frac = flops / (ms * 1e-3) / (peaks["bf16"] * 1e12 * ws)
-    traffic = None if opt else load_traffic(w.name, dom)
+    traffic = None if (opt or packed) else load_traffic(w.name, dom)
 
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(args, host, dv_, step, stream, ws, w, {"o": fwd_out["o"]} if fwd_only else bwd_out)
     cpu = None
-    if not args.no_cpu_baseline and rank == 0 and ws == 1:
+    if not args.no_cpu_baseline and rank == 0 and ws == 1 and not packed:
         v, cores, sample = cpu_oracle_sample(w, d, dO, fwd_only=fwd_only)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
     line = {
@@ -339,6 +348,9 @@ def run_train(args, w, fwd_only=False):
         "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "heads": w.H, "d": w.K,
                    "chunk": L, "rank": w.R, "mc_mode": mode, "parallelism": f"dp{ws}",
                    "write_gate_term": bool(args.write_gate), "decay_parameters": bool(args.decay),
+                   "packed_sequences": None if lens is None else {
+                       "count": len(lens), "lengths": f"U{{{VARLEN_LO}..{VARLEN_HI}}} filling {w.T} tokens",
+                       "max_len": int(lens.max()), "min_len": int(lens.min())},
                    "l2": "no flush: step working set ~3 GB >> 126 MB L2"},
         "tensor_frac": tensor_frac,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
@@ -563,6 +575,9 @@ def main():
     ap.add_argument("--seq-len", type=int, default=None, help="override T (smaller cases for profiling)")
     ap.add_argument("--write-gate", action="store_true",
                     help="train/fwd with the write gate's content term (a seeded non-zero Aw [H, rank])")
+    ap.add_argument("--varlen", action="store_true",
+                    help="train/fwd on packed variable-length sequences: the step's tokens cut into seeded lengths "
+                         "U{512..8192} (carve_fwd_varlen / carve_bwd_varlen)")
     ap.add_argument("--decay", action="store_true",
                     help="train/fwd/decode with the decay's log-amplitude A_dec [H] and bias tau [H, dk] (seeded)")
     args = ap.parse_args()
@@ -571,6 +586,11 @@ def main():
         w = dataclasses.replace(w, B=args.batch, name=w.name.replace(f"_B{w.B}_", f"_B{args.batch}_"))
     if args.seq_len:
         w = dataclasses.replace(w, T=args.seq_len, name=w.name.replace(f"_T{w.T}_", f"_T{args.seq_len}_"))
+    if args.varlen:   # the same token count, packed: one row of B T tokens
+        if args.workload == "decode":
+            raise SystemExit("--varlen applies to the train and fwd workloads")
+        w = dataclasses.replace(w, B=1, T=w.B * w.T, name=w.name.replace(f"_B{w.B}_", "_varlen_").replace(
+            f"_T{w.T}_", f"_{w.B * w.T}tok_"))
     if args.impl == "reference":
         run_reference(args, w)
     elif args.workload == "decode":

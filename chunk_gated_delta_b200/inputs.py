@@ -16,6 +16,7 @@ Recipe (the pages' 1.3B setting: 16 heads, d = 128; CARVE gist.science summary, 
   S0 = 0 for sequence workloads; decode state S ~ N(0, 0.05^2).
   Decay parameters, when a workload uses them: A_dec (the log-amplitude, per head)
   = log U(0.5, 2), tau (the bias, per head and key channel) ~ N(0, 0.5^2).
+  Packed variable-length batches: lengths ~ U{lo..hi} drawn until they fill the token budget.
 bf16 workloads round q, k, v to bfloat16 (round-to-nearest-even) after normalisation;
 the oracle then reads exactly those rounded values.
 """
@@ -118,7 +119,7 @@ DECODE = Workload("decode_B256_H16_d128_1000steps", 256, 16, 1, 128, 128, 32, 1,
                   BASE_SEED + 4, steps=1000)
 
 # stream ids (fixed forever: changing one changes every stored expectation)
-_S_Q, _S_K, _S_V, _S_GL, _S_BX, _S_WL, _S_A, _S_B, _S_DO, _S_S0, _S_DS, _S_ADEC, _S_TAU = range(1, 14)
+_S_Q, _S_K, _S_V, _S_GL, _S_BX, _S_WL, _S_A, _S_B, _S_DO, _S_S0, _S_DS, _S_ADEC, _S_TAU, _S_LEN = range(1, 15)
 
 
 def _l2norm_last(x: np.ndarray) -> np.ndarray:
@@ -154,6 +155,22 @@ def make_decay(w: Workload, seed: int | None = None) -> dict:
     amp = 0.5 + 1.5 * uniform01(s, _S_ADEC, w.H)
     return dict(A_dec=np.log(amp).astype(np.float32),
                 tau=normal(s, _S_TAU, (w.H, w.K), 0.0, 0.5).astype(np.float32))
+
+
+def make_lengths(total: int, lo: int, hi: int, seed: int) -> np.ndarray:
+    """Sequence lengths for a packed batch of exactly `total` tokens: each drawn uniformly from
+    [lo, hi] (integers) until the sum reaches `total`; the last one is cut to fit."""
+    u = uniform01(seed, _S_LEN, max(1, 4 * total // max(lo, 1) + 4))
+    lens, acc = [], 0
+    for x in u:
+        n = lo + min(int(x * (hi - lo + 1)), hi - lo)
+        n = min(n, total - acc)
+        lens.append(n)
+        acc += n
+        if acc == total:
+            break
+    assert acc == total
+    return np.asarray(lens, dtype=np.int32)
 
 
 def make_grad_out(w: Workload, seed: int | None = None, T: int | None = None) -> np.ndarray:
