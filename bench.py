@@ -64,6 +64,8 @@ def launches_per_step(w, fwd_only, decay=False):
     d A_dec reduction."""
     if fwd_only:
         return 1
+    if w.L == 1:   # the exact recurrence: its forward, its backward and the per-unit reduction
+        return 3
     return (2 if w.mc_mode == 0 else 1) + (3 if w.mc_mode == 0 else 2) + (1 if decay else 0)
 
 
@@ -323,10 +325,13 @@ def run_train(args, w, fwd_only=False):
 
     th = w.B * w.T * w.H          # token-heads of one rank's launch
     dd = w.K
+    # bytes per token-head: the exact recurrence (L = 1) keeps its state on chip and saves it
+    # every 64 tokens, so its state term is that of a 64-token save interval
+    Lb = 64 if L == 1 else L
     if fwd_only:
         kern = {"carve_fwd": (fwd_ms, 2052 * th)}
     else:
-        kern = {"carve_fwd": (fwd_ms, fwd_bytes(dd, L) * th), "carve_bwd": (bwd_ms, bwd_bytes(dd, L) * th)}
+        kern = {"carve_fwd": (fwd_ms, fwd_bytes(dd, Lb) * th), "carve_bwd": (bwd_ms, bwd_bytes(dd, Lb) * th)}
     dom = max(kern, key=lambda k: kern[k][0])
     dms, dbytes = kern[dom]
     achieved = dbytes / (dms * 1e-3) / 1e9
@@ -568,7 +573,8 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="carve", choices=["carve", "reference"])
-    ap.add_argument("--workload", default="train", choices=["train", "fwd", "decode"])
+    ap.add_argument("--workload", default="train", choices=["train", "fwd", "decode", "exact"],
+                    help="exact: the training step of the exact content-aware recurrence (chunk = 1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
@@ -582,6 +588,8 @@ def main():
                     help="train/fwd/decode with the decay's log-amplitude A_dec [H] and bias tau [H, dk] (seeded)")
     args = ap.parse_args()
     w = {"fwd": I.FWD_1P3B, "decode": I.DECODE}.get(args.workload, I.TRAIN_1P3B)
+    if args.workload == "exact":   # the same step with the state read at every token (L = 1)
+        w = dataclasses.replace(w, L=1, name=w.name.replace("_layer_", "_layer_exact_").replace("_L64", "_L1"))
     if args.batch:
         w = dataclasses.replace(w, B=args.batch, name=w.name.replace(f"_B{w.B}_", f"_B{args.batch}_"))
     if args.seq_len:

@@ -19,6 +19,9 @@ int tc_fwd_take_bad_seqlens();
 int tc_bwd_take_bad_seqlens();
 cudaError_t launch_selftest_timeout(uint32_t iterations, cudaStream_t st);
 cudaError_t launch_bwd_simt(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
+cudaError_t launch_fwd_exact(int K, int V, bool bf16, const FwdArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_exact(int K, int V, bool bf16, const BwdArgs &a, float *dA, float *dB, cudaStream_t st);
+int exact_segment();
 cudaError_t launch_step(int K, int V, bool bf16, const void *q, const void *k, const void *v,
                         const float *g_logit, const float *bx, const float *w_logit, const float *A,
                         const float *Bm, const float *Aw, const float *A_dec, const float *tau, float *S,
@@ -43,7 +46,9 @@ carve_status check_dims(const carve_dims *d, bool seq) {
     if ((long long)d->B * d->H > (1LL << 30)) return CARVE_ERR_UNSUPPORTED;
     if (seq) {
         if (d->T < 1) return CARVE_ERR_INVALID_ARG;
-        if (d->chunk != 16 && d->chunk != 32 && d->chunk != 64 && d->chunk != 128) return CARVE_ERR_UNSUPPORTED;
+        if (d->chunk != 1 && d->chunk != 16 && d->chunk != 32 && d->chunk != 64 && d->chunk != 128)
+            return CARVE_ERR_UNSUPPORTED;
+        if (d->chunk == 1 && d->mc_mode != CARVE_MC_BOUNDARY_STATE) return CARVE_ERR_UNSUPPORTED;
         if (d->T % carve::kSub != 0) return CARVE_ERR_UNSUPPORTED;
         if ((long long)d->B * d->T * d->H * (d->dk > d->dv ? d->dk : d->dv) > (1LL << 40)) return CARVE_ERR_UNSUPPORTED;
     }
@@ -63,8 +68,14 @@ size_t n_chunks(const carve_dims *d) { return (size_t)((d->T + d->chunk - 1) / d
 // 64 or 128 tokens; everything else runs the SIMT kernels.  The forward alone uses compute
 // chunks of min(chunk, 64) tokens (32 when T is not a multiple of that); a forward that saves
 // for the backward, and the backward, use 32-token compute chunks (T a multiple of 32).
+// chunk = 1: the exact content-aware recurrence (token-sequential kernels)
+bool exact(const carve_dims *d) { return d->chunk == 1; }
+size_t exact_segments(const carve_dims *d) {
+    return (size_t)((d->T + carve::exact_segment() - 1) / carve::exact_segment());
+}
+
 bool tc_shape(const carve_dims *d) {
-    return d->io == CARVE_IO_BF16 && d->dk == 128 && d->dv == 128 && d->rank <= 32 &&
+    return d->chunk > 1 && d->io == CARVE_IO_BF16 && d->dk == 128 && d->dv == 128 && d->rank <= 32 &&
            carve::tc_compute_chunk(d->chunk) > 0;
 }
 
@@ -104,6 +115,8 @@ const char *carve_status_string(carve_status s) {
 size_t carve_saved_bytes(const carve_dims *d) {
     if (check_dims(d, true) != CARVE_OK) return 0;
     const size_t units = (size_t)d->B * d->H;
+    if (exact(d))   // the fp32 state every exact_segment() tokens
+        return sizeof(float) * units * exact_segments(d) * d->dv * d->dk;
     const size_t rec = use_tc_bwd(d) ? (size_t)(carve::kTcAuxFixed + d->rank) : (size_t)(d->dv + d->rank + d->dk);
     return saved_states_bytes(d) + sizeof(float) * units * n_chunks(d) * rec;
 }
@@ -111,6 +124,9 @@ size_t carve_saved_bytes(const carve_dims *d) {
 size_t carve_bwd_workspace_bytes(const carve_dims *d) {
     if (check_dims(d, true) != CARVE_OK) return 0;
     const size_t units = (size_t)d->B * d->H;
+    const size_t unit_rec = (size_t)d->dk * d->rank + (size_t)d->rank * d->dv + d->rank + (size_t)d->dk + 1;
+    if (exact(d))   // per unit: the partial-sum record, then the states of one segment
+        return sizeof(float) * units * (unit_rec + (size_t)carve::exact_segment() * d->dv * d->dk);
     if (use_tc_bwd(d))   // per gate chunk: the gradient record and the readout vector of dq;
                          // then the per-slice partial sums of dA, dB and dAw; then per unit the
                          // decay parameters' partial sums
@@ -118,8 +134,7 @@ size_t carve_bwd_workspace_bytes(const carve_dims *d) {
                                 (size_t)carve::tc_reduce_slices(d->B, (int)n_chunks(d)) * d->H * 257 * d->rank +
                                 units * carve::kTcDecayRec);
     // per unit: dA, dB, dAw, dtau and dA_dec partial sums
-    return sizeof(float) * units *
-           ((size_t)d->dk * d->rank + (size_t)d->rank * d->dv + d->rank + (size_t)d->dk + 1);
+    return sizeof(float) * units * unit_rec;
 }
 
 // cu == nullptr: [B,T,H,*] batches; else B sequences packed in `total` rows (see carve_fwd_varlen)
@@ -147,7 +162,10 @@ static carve_status fwd_impl(const carve_dims *d, const int32_t *cu, long long t
     a.cu_seqlens = cu; a.total = total;
     cudaError_t e;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (saved != nullptr && tc_saved)
+    if (exact(d)) {
+        if (cu) return CARVE_ERR_UNSUPPORTED;   // packed sequences: chunked kernels only
+        e = carve::launch_fwd_exact(d->dk, d->dv, d->io == CARVE_IO_BF16, a, cs);
+    } else if (saved != nullptr && tc_saved)
         e = carve::launch_fwd_tc(a, 32, cs);
     else if (saved == nullptr && tc_fwd_chunk(d) > 0)
         e = carve::launch_fwd_tc(a, tc_fwd_chunk(d), cs);
@@ -188,6 +206,12 @@ static carve_status bwd_impl(const carve_dims *d, const int32_t *cu, long long t
     a.dS0 = dS0; a.dm_prev_in = dm_prev_in; a.ws = static_cast<float *>(workspace);
     a.B = d->B; a.H = d->H; a.T = d->T; a.R = d->rank; a.L = d->chunk; a.mc_mode = d->mc_mode;
     a.cu_seqlens = cu; a.total = total;
+    if (exact(d)) {
+        if (cu) return CARVE_ERR_UNSUPPORTED;
+        const cudaError_t ex = carve::launch_bwd_exact(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
+                                                       static_cast<cudaStream_t>(stream));
+        return ex == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+    }
     cudaError_t e = tc ? carve::launch_bwd_tc(a, dA, dB, static_cast<cudaStream_t>(stream))
                        : carve::launch_bwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
                                                 static_cast<cudaStream_t>(stream));

@@ -675,6 +675,16 @@ __global__ void reduce_dAdB_kernel(const float *ws, float *dA, float *dB, float 
     }
 }
 
+// Host: the reduction above over per-unit records of K*R + R*V + R + K + 1 floats (also used
+// by the exact-recurrence backward).
+cudaError_t launch_reduce_units(const float *ws, float *dA, float *dB, float *dAw, float *dtau, float *dA_dec, int B,
+                                int H, int K, int V, int R, cudaStream_t st) {
+    const int KR = K * R, RV = R * V;
+    dim3 grid((KR + RV + R + K + 1 + 255) / 256, H);
+    reduce_dAdB_kernel<<<grid, 256, 0, st>>>(ws, dA, dB, dAw, dtau, dA_dec, B, H, KR, RV, R, K);
+    return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------------------
 template <int K, int V, typename IO>
 cudaError_t launch_fwd_simt_t(const FwdArgs &a, cudaStream_t st) {
