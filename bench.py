@@ -490,6 +490,42 @@ def run_decode(args, w):
         dist.destroy_process_group()
 
 
+def run_deviation(args, w):
+    """Chunk-aligned readout against the exact recurrence: the relative L2 deviation of the
+    outputs o of carve_fwd at gate chunks L = 16 .. 128 (both readouts) from those of the exact
+    content-aware recurrence (chunk = 1), on the same synthetic inputs, in fp32 I/O so that the
+    measured deviation is not bf16 rounding; with the recipe's low-rank projections and with
+    them scaled by 10 (a stronger content path).  One forward per configuration."""
+    import torch
+    import chunk_gated_delta_b200 as carve
+    ws, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = I.make_inputs(w)
+    x = {k: torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).to(dev) for k, v in d.items()}
+    out = {}
+    for scale in (1.0, 10.0):
+        args8 = (x["q"], x["k"], x["v"], x["g_logit"], x["bx"], x["w_logit"], x["A"] * scale, x["B"] * scale)
+        ref = carve.carve_fwd(*args8, chunk=1, mc_mode=0, save_for_bwd=False)["o"].double()
+        row = {}
+        for mode in (0, 1):
+            for L in (16, 32, 64, 128):
+                o = carve.carve_fwd(*args8, chunk=L, mc_mode=mode, save_for_bwd=False)["o"].double()
+                row[f"mode{mode}_L{L}"] = float(torch.linalg.vector_norm(o - ref) / torch.linalg.vector_norm(ref))
+        out[f"projection_scale_{scale:g}"] = row
+    assert carve.carve_check() == 0
+    line = {
+        "metric": "chunk-aligned readout deviation (relative L2 of o against the exact recurrence)",
+        "value": out["projection_scale_1"]["mode1_L64"], "unit": "relative", "n_gpus": ws, "steps": 1,
+        "warmup": 0, "higher_is_better": False, "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.B, "seq_len": w.T, "heads": w.H, "d": w.K, "rank": w.R,
+                   "io": "fp32"},
+        "by_chunk": out,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def load_traffic(workload, call):
     """DRAM bytes of one `call` on `workload` from the committed ncu summary (None when that
     workload was not captured)."""
@@ -573,8 +609,9 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="carve", choices=["carve", "reference"])
-    ap.add_argument("--workload", default="train", choices=["train", "fwd", "decode", "exact"],
-                    help="exact: the training step of the exact content-aware recurrence (chunk = 1)")
+    ap.add_argument("--workload", default="train", choices=["train", "fwd", "decode", "exact", "deviation"],
+                    help="exact: the training step of the exact content-aware recurrence (chunk = 1); deviation: "
+                         "the chunk-aligned readout's output deviation from the exact recurrence")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
@@ -599,7 +636,9 @@ def main():
             raise SystemExit("--varlen applies to the train and fwd workloads")
         w = dataclasses.replace(w, B=1, T=w.B * w.T, name=w.name.replace(f"_B{w.B}_", "_varlen_").replace(
             f"_T{w.T}_", f"_{w.B * w.T}tok_"))
-    if args.impl == "reference":
+    if args.workload == "deviation":
+        run_deviation(args, dataclasses.replace(w, io="fp32", name=w.name.replace("train_", "deviation_")))
+    elif args.impl == "reference":
         run_reference(args, w)
     elif args.workload == "decode":
         run_decode(args, w)
