@@ -277,12 +277,14 @@ def run_train(args, w, fwd_only=False):
     fwd_out = fwd_fn(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
                      dv_["B"], chunk=L, mc_mode=mode, save_for_bwd=not fwd_only, **opt, **packed)
     bwd_out = None
-    if not fwd_only:   # dA and dB as views of one flat buffer: the step's only collective
+    if not fwd_only:
         from chunk_gated_delta_b200 import dist as cdist
-        dAB, dA_, dB_ = cdist.grad_buffer(w.H, w.K, w.V, w.R, dev)
+        # every per-head parameter gradient in one flat buffer: the step's one all-reduce
+        dAB, pviews = cdist.param_grad_buffer(w.H, w.K, w.V, w.R, dev, write_term="Aw" in opt,
+                                              decay="A_dec" in opt)
         bwd_out = bwd_fn(dv_["q"], dv_["k"], dv_["v"], dv_["g_logit"], dv_["bx"], dv_["w_logit"], dv_["A"],
                          dv_["B"], fwd_out["saved"], dv_["dO"], chunk=L, mc_mode=mode,
-                         out={"dA": dA_, "dB": dB_}, **opt, **packed)
+                         out=dict(pviews), **opt, **packed)
     dims = (carve.dims_varlen(dv_["q"], dv_["v"], dv_["A"], packed["cu_seqlens"], packed["max_len"], L, mode)
             if packed else carve.dims_of(dv_["q"], dv_["v"], dv_["A"], L, mode))
     workspace = torch.empty(carve.bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)

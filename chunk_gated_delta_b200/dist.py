@@ -2,8 +2,9 @@
 
 The (batch, head) units are independent, so each rank runs the forward and backward on its
 own batch shard with no exchange.  The one collective of the path is the sum over ranks of
-the low-rank factor gradients dA [H,K,r] and dB [H,r,V], which every unit of a head adds to:
-both live in one flat fp32 buffer so that the sum is a single all-reduce.  The sequence axis
+the per-head parameter gradients, which every unit of a head adds to: the low-rank factor
+gradients dA [H,K,r] and dB [H,r,V], and with the optional terms dAw [H,r], dA_dec [H] and
+dtau [H,K]; all live in one flat fp32 buffer so that the sum is a single all-reduce.  The sequence axis
 does not shard: the erase gate depends on the state, so a chunk cannot start before the
 previous one has finished.
 """
@@ -46,6 +47,29 @@ def grad_buffer(H: int, K: int, V: int, R: int, device):
     import torch
     flat = torch.empty(H * R * (K + V), dtype=torch.float32, device=device)
     return flat, flat[:H * K * R].view(H, K, R), flat[H * K * R:].view(H, R, V)
+
+
+def param_grad_buffer(H: int, K: int, V: int, R: int, device, write_term: bool = False, decay: bool = False):
+    """One flat fp32 buffer for every per-head parameter gradient of a step: dA [H,K,R], dB
+    [H,R,V], and (write_term) dAw [H,R], (decay) dA_dec [H] and dtau [H,K].  Returns (flat,
+    views by name); each view starts on a 16-byte boundary (sections padded to 4 floats), as
+    the library requires of every pointer."""
+    import torch
+    shapes = {"dA": (H, K, R), "dB": (H, R, V)}
+    if write_term:
+        shapes["dAw"] = (H, R)
+    if decay:
+        shapes["dA_dec"] = (H,)
+        shapes["dtau"] = (H, K)
+    offs, n = {}, 0
+    for name, shp in shapes.items():
+        size = 1
+        for x in shp:
+            size *= x
+        offs[name] = (n, size)
+        n += (size + 3) // 4 * 4
+    flat = torch.zeros(n, dtype=torch.float32, device=device)
+    return flat, {name: flat[o:o + size].view(shapes[name]) for name, (o, size) in offs.items()}
 
 
 def allreduce_(flat, group=None):
