@@ -81,15 +81,18 @@ def load_peaks():
 # ---------------------------------------------------------------------------------------
 class ClockSampler:
     """SM clock, power and throttle reasons of this process's GPU, polled through NVML every
-    `period` seconds on a host thread during the timed region (read-only queries); the
-    samples are also written to gpurun_out/clocks_rank<i>.csv."""
+    `period` seconds on a host thread during the timed region (read-only queries); with
+    `--clocks-csv PATH` the samples are also written to PATH (rank i: PATH.rank<i>)."""
     NAMES = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
              ("sw_power_cap", 0x4))
+
+    csv_path = None   # set from --clocks-csv
 
     def __init__(self, index: int, period: float = 0.005):
         self.index, self.period = index, period
         self.rows, self.err = [], None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = None if self.csv_path is None else (
+            self.csv_path if index == 0 else f"{self.csv_path}.rank{index}")
 
     def _handle(self, nv):
         import torch
@@ -134,7 +137,9 @@ class ClockSampler:
         self.stop.set()
         self.thread.join(timeout=5)
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            if self.path is None:
+                raise OSError("no csv requested")
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             with open(self.path, "w") as f:
                 f.write("time,sm_mhz,sm_max_mhz,power_w,reasons_mask\n")
                 for t, mhz, pw, rs in self.rows:
@@ -620,12 +625,15 @@ def main():
     ap.add_argument("--seq-len", type=int, default=None, help="override T (smaller cases for profiling)")
     ap.add_argument("--write-gate", action="store_true",
                     help="train/fwd with the write gate's content term (a seeded non-zero Aw [H, rank])")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write the clock samples of the timed region to this CSV file")
     ap.add_argument("--varlen", action="store_true",
                     help="train/fwd on packed variable-length sequences: the step's tokens cut into seeded lengths "
                          "U{512..8192} (carve_fwd_varlen / carve_bwd_varlen)")
     ap.add_argument("--decay", action="store_true",
                     help="train/fwd/decode with the decay's log-amplitude A_dec [H] and bias tau [H, dk] (seeded)")
     args = ap.parse_args()
+    ClockSampler.csv_path = args.clocks_csv
     w = {"fwd": I.FWD_1P3B, "decode": I.DECODE}.get(args.workload, I.TRAIN_1P3B)
     if args.workload == "exact":   # the same step with the state read at every token (L = 1)
         w = dataclasses.replace(w, L=1, name=w.name.replace("_layer_", "_layer_exact_").replace("_L64", "_L1"))
