@@ -186,7 +186,7 @@ carve_status carve_bwd_varlen(const carve_dims *d, const int32_t *cu_seqlens, in
  * the call allocates nothing.  Limit: carve_bwd_workspace_bytes(d) <= 4 MiB, that is
  * B*H*(dk*rank + rank*dv + rank + dk + 1) floats, or, when the tensor-core kernels run (bf16,
  * dk = dv = 128, rank <= 32), B*H*(NG*292 + 132) + ceil(B*NG/64)*H*257*rank floats with
- * NG = ceil(T/chunk); larger problems return
+ * NG = ceil(T/chunk) (chunk = 1 adds 64*dv*dk floats per unit); larger problems return
  * CARVE_ERR_UNSUPPORTED without launching anything.
  * The first call on each device looks up the array's device address (with that device
  * current) and caches it; make that first call before any stream capture begins.
