@@ -51,6 +51,7 @@ carve_status check_dims(const carve_dims *d, bool seq) {
         if (d->chunk == 1 && d->mc_mode != CARVE_MC_BOUNDARY_STATE) return CARVE_ERR_UNSUPPORTED;
         if (d->T % carve::kSub != 0) return CARVE_ERR_UNSUPPORTED;
         if ((long long)d->B * d->T * d->H * (d->dk > d->dv ? d->dk : d->dv) > (1LL << 40)) return CARVE_ERR_UNSUPPORTED;
+        if ((long long)d->B * d->T > 0x7fffffffLL) return CARVE_ERR_UNSUPPORTED;   // token rows index as int
     }
     return CARVE_OK;
 }

@@ -46,7 +46,8 @@
  * must be 16-byte aligned.
  *
  * Supported shapes: dk, dv in {64, 128}; 1 <= rank <= 64; chunk in {16, 32, 64, 128};
- * T a multiple of 16 (a shorter last chunk is allowed: its mean runs over its own tokens).
+ * T a multiple of 16 (a shorter last chunk is allowed: its mean runs over its own tokens);
+ * B*T < 2^31 token rows.
  * chunk = 1 selects the exact content-aware recurrence, whose content signal is read from the
  * state right before every token (m_t = S_{t-1} q_t; the L = 1 case of the definition, CARVE
  * blog Tables 1 and 3): token-sequential kernels, mc_mode 0 only, no packed sequences.  Its

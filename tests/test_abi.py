@@ -65,7 +65,8 @@ def test_buffer_sizes(lib):
 
 @pytest.mark.parametrize("bad,code", [(dict(dk=96), 2), (dict(dv=32), 2), (dict(T=100), 2), (dict(chunk=48), 2),
                                       (dict(rank=65), 2), (dict(io=7), 1), (dict(mc_mode=5), 1), (dict(H=0), 1),
-                                      (dict(T=0), 1), (dict(chunk=1, mc_mode=1), 2)])
+                                      (dict(T=0), 1), (dict(chunk=1, mc_mode=1), 2),
+                                      (dict(B=1 << 20, H=1, T=1 << 11, dk=64, dv=64), 2)])
 def test_bad_dims_rejected(lib, bad, code):
     """Dimension checks run first, so the (fake) pointers below are never dereferenced."""
     d = good_dims(**bad)
