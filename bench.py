@@ -354,7 +354,8 @@ def run_train(args, w, fwd_only=False):
         v, cores, sample = cpu_oracle_sample(w, d, dO, fwd_only=fwd_only)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
     line = {
-        "metric": "fwd tokens/s per layer (B200, 16 heads, d=128)" if fwd_only else METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "metric": "fwd tokens/s per layer (B200, 16 heads, d=128)" if fwd_only else METRIC, "value": value,
+        "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T, "heads": w.H, "d": w.K,
