@@ -30,6 +30,18 @@ def compute():
     for mode in (0, 1):
         r = oracle.fwd(d, L=w.L, mc_mode=mode)
         out[f"mc{mode}"] = {"o": r["o"].ravel().tolist(), "S_final": r["S_final"].ravel().tolist()}
+    # the optional terms: the write gate's content factor and the decay's amplitude and bias
+    dt = dict(d, Aw=np.array([[2.0, -3.0]]), A_dec=np.array([0.4]), tau=np.array([[0.5, -1.0, 0.25]]))
+    r = oracle.fwd(dt, L=w.L, mc_mode=0)
+    g = oracle.bwd(dt, w.L, np.ones_like(r["o"]), mc_mode=0)
+    out["terms"] = {"o": r["o"].ravel().tolist(), "S_final": r["S_final"].ravel().tolist(),
+                    "dAw": g["dAw"].ravel().tolist(), "dA_dec": g["dA_dec"].ravel().tolist(),
+                    "dtau": g["dtau"].ravel().tolist()}
+    # the exact recurrence (L = 1) and two packed sequences (4 + 2 tokens)
+    r = oracle.fwd(d, L=1, mc_mode=0)
+    out["exact"] = {"o": r["o"].ravel().tolist(), "S_final": r["S_final"].ravel().tolist()}
+    r = oracle.fwd(d, L=w.L, mc_mode=1, cu_seqlens=np.array([0, 4, 6]))
+    out["packed"] = {"o": r["o"].ravel().tolist(), "S_final": r["S_final"].ravel().tolist()}
     return out
 
 

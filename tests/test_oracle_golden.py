@@ -13,6 +13,7 @@ def test_oracle_matches_stored_tiny_case():
     stored = json.load(open(path))
     now = make_golden.compute()
     assert stored["case"] == now["case"]
-    for mode in ("mc0", "mc1"):
-        for key in ("o", "S_final"):
-            assert np.allclose(np.array(stored[mode][key]), np.array(now[mode][key]), rtol=1e-13, atol=1e-15)
+    for case in ("mc0", "mc1", "terms", "exact", "packed"):
+        for key in now[case]:
+            assert np.allclose(np.array(stored[case][key]), np.array(now[case][key]), rtol=1e-13, atol=1e-15), \
+                (case, key)
