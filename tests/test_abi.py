@@ -151,3 +151,6 @@ def test_varlen_arguments_checked_on_host(lib):
     for cu, total, code in ((None, 64, 1), (ctypes.c_void_p(4100), 64, 1), (P, -1, 1), (P, 1 << 40, 1)):
         assert lib.carve_fwd_varlen(ctypes.byref(d), cu, total, *fwd_args(P)) == code, (cu, total)
         assert lib.carve_bwd_varlen(ctypes.byref(d), cu, total, *bwd_args(P)) == code, (cu, total)
+    exact = good_dims(chunk=1)   # the exact recurrence has no packed form
+    assert lib.carve_fwd_varlen(ctypes.byref(exact), P, 64, *fwd_args(P)) == 2
+    assert lib.carve_bwd_varlen(ctypes.byref(exact), P, 64, *bwd_args(P)) == 2
