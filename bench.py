@@ -15,6 +15,7 @@ bracketed by a barrier and a device synchronize, max over ranks.  The working se
 from __future__ import annotations
 
 import argparse
+import copy
 import dataclasses
 import json
 import os
@@ -248,9 +249,52 @@ def run_reference(args, w):
 
 
 def run_train(args, w, fwd_only=False):
+    ws, rank, local = dist_setup()
+    line = measure_train(args, w, ws, rank, local, fwd_only)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_long(args):
+    """The long-context workload: B1 H16 T65536 d128, the training step (fwd + bwd) at every
+    gate chunk L in {32, 64, 128} with both content readouts.  One JSON line: the headline
+    fields are those of L = 64 with the boundary-state readout; `runs` holds all six."""
+    ws, rank, local = dist_setup()
+    runs, head = {}, None
+    for L in (32, 64, 128):
+        for mode in (0, 1):
+            w = I.long_context(L, mode)
+            if args.seq_len:
+                w = dataclasses.replace(w, T=args.seq_len, name=w.name.replace("_T65536_", f"_T{args.seq_len}_"))
+            sub = copy.copy(args)
+            sub.no_e2e = args.no_e2e or (L, mode) != (64, 0)   # end to end: the headline run only
+            sub.cpu_target_s = 6.0
+            line = measure_train(sub, w, ws, rank, local, False)
+            runs[f"L{L}_mc{mode}"] = {k: line[k] for k in ("value", "ms_per_step", "tensor_frac", "kernels_ms")}
+            runs[f"L{L}_mc{mode}"].update(hbm_frac=line["roofline"]["frac"], roofline_kernel=line["roofline"]["kernel"],
+                                          cpu_baseline=None if line["cpu_baseline"] is None
+                                          else line["cpu_baseline"]["value"])
+            if (L, mode) == (64, 0):
+                head = line
+    head["config"]["workload"] = head["config"]["workload"].replace("_L64_mc0", "")
+    head["config"]["runs_of"] = "gate chunk L in {32, 64, 128} x readout mc in {0, 1}; headline: L64 mc0"
+    head["runs"] = runs
+    head["gpu_launches"] = sum(launches_per_step(dataclasses.replace(w, L=int(k[1:k.index('_')]),
+                                                                     mc_mode=int(k[-1])), False) * args.steps
+                               for k in runs)
+    if rank == 0:
+        print(json.dumps(head), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def measure_train(args, w, ws, rank, local, fwd_only=False):
     import torch
     import chunk_gated_delta_b200 as carve
-    ws, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
@@ -351,7 +395,8 @@ def run_train(args, w, fwd_only=False):
         e2e = measure_e2e(args, host, dv_, step, stream, ws, w, {"o": fwd_out["o"]} if fwd_only else bwd_out)
     cpu = None
     if not args.no_cpu_baseline and rank == 0 and ws == 1 and not packed:
-        v, cores, sample = cpu_oracle_sample(w, d, dO, fwd_only=fwd_only)
+        v, cores, sample = cpu_oracle_sample(w, d, dO, target_s=getattr(args, "cpu_target_s", 12.0),
+                                             fwd_only=fwd_only)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
     line = {
         "metric": "fwd tokens/s per layer (B200, 16 heads, d=128)" if fwd_only else METRIC, "value": value,
@@ -372,11 +417,7 @@ def run_train(args, w, fwd_only=False):
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, fwd_only, args.decay) * args.steps,
         "clocks": clk.summary(),
     }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if ws > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    return line
 
 
 # Decode: per (b,h) and step, the fp32 state read and written (8 d^2 = 131,072 B at d = 128),
@@ -617,9 +658,10 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="carve", choices=["carve", "reference"])
-    ap.add_argument("--workload", default="train", choices=["train", "fwd", "decode", "exact", "deviation"],
+    ap.add_argument("--workload", default="train", choices=["train", "fwd", "decode", "exact", "deviation", "long"],
                     help="exact: the training step of the exact content-aware recurrence (chunk = 1); deviation: "
-                         "the chunk-aligned readout's output deviation from the exact recurrence")
+                         "the chunk-aligned readout's output deviation from the exact recurrence; long: the "
+                         "long-context training step (B1 H16 T65536) at L in {32, 64, 128} x both readouts")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
@@ -647,7 +689,12 @@ def main():
             raise SystemExit("--varlen applies to the train and fwd workloads")
         w = dataclasses.replace(w, B=1, T=w.B * w.T, name=w.name.replace(f"_B{w.B}_", "_varlen_").replace(
             f"_T{w.T}_", f"_{w.B * w.T}tok_"))
-    if args.workload == "deviation":
+    if args.workload == "long":
+        if args.impl == "reference":
+            run_reference(args, I.long_context(64, 0))
+        else:
+            run_long(args)
+    elif args.workload == "deviation":
         run_deviation(args, dataclasses.replace(w, io="fp32", name=w.name.replace("train_", "deviation_")))
     elif args.impl == "reference":
         run_reference(args, w)

@@ -61,8 +61,9 @@ def load():
     lib.carve_bwd_varlen.argtypes = [D, P, ctypes.c_int64] + [P] * 32
     lib.carve_check.argtypes = [P]
     lib.carve_selftest_timeout.argtypes = [ctypes.c_uint32, P]
+    lib.carve_selftest_stall.argtypes = [ctypes.c_uint32]
     for f in (lib.carve_fwd, lib.carve_bwd, lib.carve_fwd_varlen, lib.carve_bwd_varlen, lib.carve_step,
-              lib.carve_check, lib.carve_selftest_timeout):
+              lib.carve_check, lib.carve_selftest_timeout, lib.carve_selftest_stall):
         f.restype = ctypes.c_int
     _lib = lib
     return lib

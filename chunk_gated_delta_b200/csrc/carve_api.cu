@@ -2,6 +2,8 @@
 // kernel dispatch.  Nothing here allocates, frees or synchronises.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "../../include/carve.h"
 #include "carve_device.cuh"
 
@@ -61,6 +63,18 @@ carve_status check_packed(const carve_dims *d, long long total) {
     if (total < 0 || total > 0x7fffffffLL) return CARVE_ERR_INVALID_ARG;
     if (total * d->H * (d->dk > d->dv ? d->dk : d->dv) > (1LL << 40)) return CARVE_ERR_UNSUPPORTED;
     return CARVE_OK;
+}
+
+// Test hook of carve_selftest_stall: polls of the next tensor-core call's barrier waits, 0 when
+// unarmed.  Taken (and cleared) by the first carve_fwd / carve_bwd that launches a tensor-core
+// sweep.
+std::atomic<uint32_t> g_stall_polls{0};
+
+template <class Args>
+void set_wait(Args &a, bool tensor_core) {
+    const uint32_t p = tensor_core ? g_stall_polls.exchange(0) : 0u;
+    a.stall = p != 0;
+    a.wait_limit = p ? p : carve::kWaitLimit;
 }
 
 size_t n_chunks(const carve_dims *d) { return (size_t)((d->T + d->chunk - 1) / d->chunk); }
@@ -166,11 +180,13 @@ static carve_status fwd_impl(const carve_dims *d, const int32_t *cu, long long t
     if (exact(d)) {
         if (cu) return CARVE_ERR_UNSUPPORTED;   // packed sequences: chunked kernels only
         e = carve::launch_fwd_exact(d->dk, d->dv, d->io == CARVE_IO_BF16, a, cs);
-    } else if (saved != nullptr && tc_saved)
+    } else if (saved != nullptr && tc_saved) {
+        set_wait(a, true);
         e = carve::launch_fwd_tc(a, 32, cs);
-    else if (saved == nullptr && tc_fwd_chunk(d) > 0)
+    } else if (saved == nullptr && tc_fwd_chunk(d) > 0) {
+        set_wait(a, true);
         e = carve::launch_fwd_tc(a, tc_fwd_chunk(d), cs);
-    else
+    } else
         e = carve::launch_fwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, cs);
     return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
@@ -213,6 +229,7 @@ static carve_status bwd_impl(const carve_dims *d, const int32_t *cu, long long t
                                                        static_cast<cudaStream_t>(stream));
         return ex == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
     }
+    set_wait(a, tc);
     cudaError_t e = tc ? carve::launch_bwd_tc(a, dA, dB, static_cast<cudaStream_t>(stream))
                        : carve::launch_bwd_simt(d->dk, d->dv, d->io == CARVE_IO_BF16, a, dA, dB,
                                                 static_cast<cudaStream_t>(stream));
@@ -288,6 +305,12 @@ carve_status carve_check(void *stream) {
     const int t = carve::tc_fwd_take_timeout() | carve::tc_bwd_take_timeout() | carve::step_take_timeout();
     const int bad = carve::simt_take_bad_seqlens() | carve::tc_fwd_take_bad_seqlens() | carve::tc_bwd_take_bad_seqlens();
     return t ? CARVE_ERR_TIMEOUT : bad ? CARVE_ERR_INVALID_ARG : CARVE_OK;
+}
+
+carve_status carve_selftest_stall(uint32_t iterations) {
+    if (iterations < 1 || iterations > 1000000) return CARVE_ERR_INVALID_ARG;
+    g_stall_polls.store(iterations);
+    return CARVE_OK;
 }
 
 carve_status carve_selftest_timeout(uint32_t iterations, void *stream) {

@@ -94,6 +94,8 @@ struct FwdArgs {
     const int *cu_seqlens;  // [B+1] or null: B sequences packed along the token axis
     long long total;        // rows of the packed token tensors (with cu_seqlens)
     int B, H, T, R, L, mc_mode;
+    uint32_t wait_limit;    // polls of each bounded barrier wait (tensor-core kernels)
+    int stall;              // test hook: skip the first tile copy so that its wait gives up
 };
 
 struct BwdArgs {
@@ -109,7 +111,13 @@ struct BwdArgs {
     const int *cu_seqlens;  // [B+1] or null: B sequences packed along the token axis
     long long total;        // rows of the packed token tensors (with cu_seqlens)
     int B, H, T, R, L, mc_mode;
+    uint32_t wait_limit;    // polls of each bounded barrier wait (tensor-core kernels)
+    int stall;              // test hook: skip the first tile copy so that its wait gives up
 };
+
+// Polls of a bounded barrier wait in normal operation (each poll may suspend the thread for
+// a while, so this is of the order of a second: far beyond any copy that completes).
+constexpr uint32_t kWaitLimit = 1u << 26;
 
 // Tokens of sequence b: rows [toff, toff + Tn) of tensor batch bb.  Without cu_seqlens the
 // unit is batch element b with all T tokens; with it, the sequences are packed along the token

@@ -25,7 +25,16 @@
 // stored per gate chunk and added by a parallel pass after the sweep.
 // Terms that cancel pairwise in the reverse cumulative sum of dLam (a Gram entry's row and
 // column token; Kbar_s against the chunk's last token) are formed from the same rounded values
-// on both sides, so the cancellation stays exact to fp32 rounding.
+// on both sides, so the cancellation stays exact to fp32 rounding.  Two such pairs have no
+// dependence on Lam at all and are left out of dLam on both sides: the diagonal of Aqk
+// (q_t . k_t, decay factor 1; its fp32 value goes to dq and dk directly) and the Kbar term of
+// the chunk's last token (factor e^{Lam_C - Lam_C} = 1).  Under strong erasure the gradient of
+// log a is tiny (proportional to a) while those pairs are O(1), so their rounding would swamp
+// it.  For the same reason the off-diagonal Gram blocks' factor e^{Lam_m(1) - Lam_m(0)} is
+// never formed alone (it underflows fp32 under strong decay where the whole product does
+// not): the row block's part and the column block's part are applied separately.  Where the
+// retention floor binds, the gradient of log a is scaled to the exact recurrence's
+// (floor_scale) instead of being dropped.
 #include "carve_tc_common.cuh"
 
 namespace carve {
@@ -52,10 +61,12 @@ struct __align__(16) TcBwdSmem {
     __nv_bfloat16 tii[kBNB * 16 * 24];
     float akk_d[kBC * 17];
     float rfac[kBC * kLdF], dlam[kBC * kLdF];
-    float p7[kBNB * 128], r15[kBNB * 128], em[kBNB * 128], fm[kBNB * 128], cij[128];
+    float p7[kBNB * 128], r15[kBNB * 128], em[kBNB * 128], fm[kBNB * 128];
     float gam[128], wv[kBC], dwp[8 * kBC], s0ds[128], xp[8 * 128], htot[2 * kBNB * 128], pdd[2 * kBNB * 128];
     float bpart[kBNB * 128];
     float delta[128], ddelta[128], dzv[64], dmv[128], dox[128], qbar[128];
+    float daqd[kBC];   // diagonal of dAqk (kept out of the bf16 tile)
+    float fs0[128];    // floor_scale of the sequence's first token, per key channel (first chunk)
     float dwc, ddw;   // the write gate's content term of the gate chunk and its gradient
     uint64_t bar, bar_s0;
 };
@@ -173,7 +184,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         bulk_g2s(sm.s0b, states + (size_t)cc * 128 * kLdOp, 128u * kLdOp * 2u, &sm.bar_s0);
     };
     if (!VL || NCCn > 0) {
-        issue(NCCn - 1);
+        if (!a.stall) issue(NCCn - 1);
         issue_s0(NCCn - 1);
     }
     uint32_t phase = 0;
@@ -235,8 +246,18 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 *reinterpret_cast<uint32_t *>(sm.ds1b + v1 * kLdOp + col) = pack_bf16(ds[j][2], ds[j][3]);
             }
         }
-        if (!mbar_wait(&sm.bar, phase)) atomicOr(&g_tc_bwd_timeout, 1);
-        __syncthreads();
+        {   // a wait that gives up ends the sweep of the whole CTA: recorded, the copies in flight
+            // (this chunk's tiles and its start state) waited for once more, bounded, and left
+            const bool lost = !mbar_wait(&sm.bar, phase, a.wait_limit);
+            if (__syncthreads_or(lost)) {
+                if (tid == 0) {
+                    atomicOr(&g_tc_bwd_timeout, 1);
+                    mbar_wait(&sm.bar, phase, a.wait_limit);
+                    mbar_wait(&sm.bar_s0, phase, a.wait_limit);
+                }
+                return;
+            }
+        }
         if constexpr (VL) {
             if (nv < C) {   // rows past the sequence's end (another sequence's, or zero fill): cleared;
                             // the proxy fence after the Qt / Kt stores below orders these writes
@@ -330,6 +351,15 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             }
         }
         if (tid < C) sm.wv[tid] = (!VL || tid < nv) ? sigmoid_f(pw + sm.dwc) : 0.f;
+        if (cc == 0 && tid < 64) {   // token 0 of the sequence (these threads hold its gate logits)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float gx = e ? glr[0].y : glr[0].x, beta = (e ? bxr[0].y : bxr[0].x) + sm.delta[c0 + e];
+                const float D = DEC ? __expf(amp * softplus_fast(gx + tb[e], __expf(gx + tb[e]))) * (1.f + __expf(-beta))
+                                    : (1.f + __expf(gx)) * (1.f + __expf(-beta));
+                sm.fs0[c0 + e] = floor_scale(__fdividef(1.f, D), false);
+            }
+        }
         __syncthreads();
         if (tid < 128) {
             float dblk[NB];   // decay over each 16-token block
@@ -348,7 +378,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 sm.fm[i * 128 + tid] = sm.r15[i * 128 + tid] * F;
                 F *= dblk[i];
             }
-            sm.cij[tid] = sm.r15[tid] * sm.p7[128 + tid];   // e^{Lam_m(1) - Lam_m(0)}
         }
         // decayed operands Qt = Qm Em, Kt = Krm Em into the (now free) raw q / k tiles, swizzled:
         // items of 8 channels of one token row, each forming its block's decay prefix
@@ -379,10 +408,16 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             *reinterpret_cast<uint4 *>(dst + t * 128 + ((c8 ^ (t & 7)) << 3)) = y;
         }
         fence_proxy_async_smem();   // the next chunk's tile copy overwrites these
-        if (!mbar_wait(&sm.bar_s0, phase)) atomicOr(&g_tc_bwd_timeout, 2);
+        const bool lost_s0 = !mbar_wait(&sm.bar_s0, phase, a.wait_limit);
+        colsum_partial();   // for gamma * dgamma (discarded if the state copy did not arrive)
+        if (__syncthreads_or(lost_s0)) {   // the state copy is the only one in flight here
+            if (tid == 0) {
+                atomicOr(&g_tc_bwd_timeout, 2);
+                mbar_wait(&sm.bar_s0, phase, a.wait_limit);
+            }
+            return;
+        }
         phase ^= 1u;
-        colsum_partial();   // for gamma * dgamma
-        __syncthreads();
         if (tid < 128) {
             float x = 0.f;
 #pragma unroll
@@ -402,12 +437,16 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     uint32_t af[4], bfr[4];
                     load_a(af, rowop, kLdOp, 16 * i, 16 * ks, lane);
                     load_b_nk(bfr, sm.kcm, kLdOp, 16 * j, 16 * ks, lane);
-                    if (j < i) {
-                        const float *f = sm.cij + 16 * ks + 2 * c4;
-                        bfr[0] = scale_bf16x2(bfr[0], f[0], f[1]);
-                        bfr[1] = scale_bf16x2(bfr[1], f[8], f[9]);
-                        bfr[2] = scale_bf16x2(bfr[2], f[0], f[1]);
-                        bfr[3] = scale_bf16x2(bfr[3], f[8], f[9]);
+                    if (j < i) {   // e^{Lam_m(1) - Lam_m(0)} split: p7 of the row block, r15 of the column block
+                        const float *fp = sm.p7 + i * 128 + 16 * ks + 2 * c4, *fr = sm.r15 + j * 128 + 16 * ks + 2 * c4;
+                        af[0] = scale_bf16x2(af[0], fp[0], fp[1]);
+                        af[1] = scale_bf16x2(af[1], fp[0], fp[1]);
+                        af[2] = scale_bf16x2(af[2], fp[8], fp[9]);
+                        af[3] = scale_bf16x2(af[3], fp[8], fp[9]);
+                        bfr[0] = scale_bf16x2(bfr[0], fr[0], fr[1]);
+                        bfr[1] = scale_bf16x2(bfr[1], fr[8], fr[9]);
+                        bfr[2] = scale_bf16x2(bfr[2], fr[0], fr[1]);
+                        bfr[3] = scale_bf16x2(bfr[3], fr[8], fr[9]);
                     }
                     mma_bf16(acc[0], af, bfr[0], bfr[1]);
                     mma_bf16(acc[1], af, bfr[2], bfr[3]);
@@ -646,6 +685,18 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 mma_bf16(ds[2 * np + 1], ar, bk[2], bk[3]);
             }
         }
+        if (cc == 0) {   // dS0 = dP_0 Diag(a_0): where the floor binds at the first token, the exact
+                         // recurrence's a_0 (floor_scale); the content term is added after this
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int col = 8 * j + 2 * c4;
+                const float f0 = sm.fs0[col], f1 = sm.fs0[col + 1];
+                ds[j][0] *= f0;
+                ds[j][1] *= f1;
+                ds[j][2] *= f0;
+                ds[j][3] *= f1;
+            }
+        }
         __syncthreads();
         if (cc > 0) issue(cc - 1);   // q, k, v, dO and the Qt / Kt tiles of this chunk are read
         // ---- dAqk = dO U^T (s <= t), dAkk = -dR U^T (s < t): reductions over v, six 16x16 tiles
@@ -667,14 +718,17 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 for (int e = 0; e < 4; ++e) {
                     const int tr = 16 * i + g + ((e >> 1) << 3);
                     const int sc = 16 * j + 8 * nt + 2 * c4 + (e & 1);
-                    if (type == 0) sm.daqk[tr * kLdT + sc] = __float2bfloat16_rn(sc <= tr ? acc[nt][e] : 0.f);
+                    if (type == 0) {
+                        sm.daqk[tr * kLdT + sc] = __float2bfloat16_rn(sc < tr ? acc[nt][e] : 0.f);
+                        if (sc == tr) sm.daqd[tr] = acc[nt][e];
+                    }
                     else sm.dakk[tr * kLdT + sc] = __float2bfloat16_rn(sc < tr ? -acc[nt][e] : 0.f);
                 }
         }
         __syncthreads();
         // ---- per (token block, channel quarter): Gq, Gkr, Gkc, Gkb -> dq, dk, dLam
         // Paired terms that cancel in the reverse cumulative sum of dLam are built from the same
-        // rounded operands on both sides: the off-diagonal decay factor C is applied to fp32
+        // rounded operands on both sides: the off-diagonal decay factor is applied to fp32
         // products, never to one side's bf16 operand.
         {
             const int ib2 = warp >> 2, ch0 = 32 * (warp & 3);
@@ -760,19 +814,32 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                         mma_bf16(tc[2 * np2 + 1], ak, bk[2], bk[3]);
                     }
                 }
+                // the off-diagonal pair's factor e^{Lam_m(i) - Lam_m(j)} (i the later block) is
+                // applied in two parts, the one that bounds the operand inside the sum first: r15
+                // of block j with kcm, p7 of block i with qm / krm
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float c = offdiag ? sm.cij[ch0 + 8 * nt + 2 * c4 + (e & 1)] : 1.f;
-                        gq[nt][e] += c * tq[nt][e];
-                        gkr[nt][e] += c * tk[nt][e];
-                        gkc[nt][e] += c * tc[nt][e];
+                        const int c = ch0 + 8 * nt + 2 * c4 + (e & 1);
+                        if (!offdiag) {
+                            gq[nt][e] += tq[nt][e];
+                            gkr[nt][e] += tk[nt][e];
+                            gkc[nt][e] += tc[nt][e];
+                        } else if (row_side) {   // i = ib2, j = j2
+                            const float fr = sm.r15[j2 * 128 + c], fp = sm.p7[ib2 * 128 + c];
+                            gq[nt][e] += (tq[nt][e] * fr) * fp;
+                            gkr[nt][e] += (tk[nt][e] * fr) * fp;
+                        } else {                 // i = j2, j = ib2
+                            const float fp = sm.p7[j2 * 128 + c], fr = sm.r15[ib2 * 128 + c];
+                            gkc[nt][e] += (tc[nt][e] * fp) * fr;
+                        }
                     }
             }
             float bsum[4][2];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) bsum[nt][0] = bsum[nt][1] = 0.f;
+            const int tlast = nv - 1;   // the chunk's last live token: its Kbar factor is 1
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -784,18 +851,20 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.qm + t * kLdOp + ch);
                     const __nv_bfloat162 kr2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.krm + t * kLdOp + ch);
                     const __nv_bfloat162 kc2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.kcm + t * kLdOp + ch);
+                    const float dgd = sm.daqd[t];
+                    const bool tl = t == tlast;
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
                         const int e = 2 * hh + e2;
                         const float r = e2 ? r2.y : r2.x;
                         const float ri = __fdividef(1.f, r);
-                        const float Gq = gq[nt][e], Gkr = gkr[nt][e], Gkc = gkc[nt][e] + gkb[nt][e];
+                        const float Gq = gq[nt][e], Gkr = gkr[nt][e], Gkc = gkc[nt][e];
                         const float qmv = bf(e2 ? q2.y : q2.x), krv = bf(e2 ? kr2.y : kr2.x);
                         const float kcv = bf(e2 ? kc2.y : kc2.x);
-                        dqv[e2] = r * Gq;
-                        dkv[e2] = r * Gkr + ri * Gkc;
-                        dlv[e2] = qmv * Gq + krv * Gkr - kcv * Gkc;
-                        bsum[nt][e2] += kcv * gkb[nt][e];     // Kbar_t dKbar_t
+                        dqv[e2] = r * (Gq + dgd * kcv);
+                        dkv[e2] = r * Gkr + ri * (Gkc + gkb[nt][e] + dgd * qmv);
+                        dlv[e2] = qmv * Gq + krv * Gkr - kcv * (tl ? Gkc : Gkc + gkb[nt][e]);
+                        if (!tl) bsum[nt][e2] += kcv * gkb[nt][e];     // Kbar_t dKbar_t
                     }
                     *reinterpret_cast<float2 *>(sm.dlam + t * kLdF + ch) = make_float2(dlv[0], dlv[1]);
                     const size_t gi = base_bh + (size_t)(t0 + t) * tstride + ch;
@@ -883,20 +952,20 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 for (int e = 0; e < 2; ++e) {
                     run[e] += e ? d2.y : d2.x;
                     if (t == 7) run[e] += xl[e];
-                    const float gx = e ? glr[t].y : glr[t].x, e2 = __expf(-((e ? bxr[t].y : bxr[t].x) + dl[e]));
+                    const float gx = e ? glr[t].y : glr[t].x, nb = -((e ? bxr[t].y : bxr[t].x) + dl[e]);   // nb = -beta
+                    const float e2 = __expf(nb);
                     if constexpr (DEC) {   // log g = -amp softplus(x), x = g_logit + tau: d/dx = -amp sigmoid(x)
                         const float x = gx + tb[e], e1 = __expf(x), sp = softplus_fast(x, e1);
-                        const bool floor = !(__fdividef(1.f, __expf(amp * sp) * (1.f + e2)) >= kAMin) || inert;
-                        dg[e] = floor ? 0.f : -amp * sigmoid_fast(x, e1) * run[e];
-                        db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
+                        const float dla = run[e] * floor_scale(__fdividef(1.f, __expf(amp * sp) * (1.f + e2)), inert);
+                        dg[e] = -amp * sigmoid_fast(x, e1) * dla;
+                        db[e] = sigmoid_fast(nb, e2) * dla;
                         dtp[e] += dg[e];
-                        dap += floor ? 0.f : run[e] * (-amp * sp);   // d A_dec = dlog a . log g
+                        dap += dla * (-amp * sp);   // d A_dec = dlog a . log g
                     } else {
                         const float e1 = __expf(gx);
-                        const float D = (1.f + e1) * (1.f + e2);
-                        const bool floor = !(__fdividef(1.f, D) >= kAMin) || inert;
-                        dg[e] = floor ? 0.f : -__fdividef(e1, 1.f + e1) * run[e];
-                        db[e] = floor ? 0.f : __fdividef(e2, 1.f + e2) * run[e];
+                        const float dla = run[e] * floor_scale(__fdividef(1.f, (1.f + e1) * (1.f + e2)), inert);
+                        dg[e] = -sigmoid_fast(gx, e1) * dla;
+                        db[e] = sigmoid_fast(nb, e2) * dla;
                     }
                     pdd[e] += db[e];
                 }
@@ -909,6 +978,14 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         if (cc > 0) {   // the gate logits were read for the last time in the scan above
             load_gates(cc - 1);
             load_w(cc - 1);
+        }
+        // the content path's factor A (this thread's slice A[h][part + 8x][tid / 8], rank <= 32),
+        // read from L2 now so that its latency overlaps the stores below
+        float apre[16];
+        if (gate_start) {
+            const int j = tid / 8, part = tid % 8;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) apre[x] = j < R ? a.A[((size_t)h * 128 + part + 8 * x) * R + j] : 0.f;
         }
         __syncthreads();
         if (tid < 128) {
@@ -927,12 +1004,18 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         __syncthreads();
         // ---- content path at the gate chunk's first token
         if (gate_start) {
-            for (int j0 = 0; j0 < R; j0 += 32) {   // dz = A^T dDelta, 8 threads per output
-                const int j = j0 + tid / 8, part = tid % 8;
-                float s = 0.f;
-                if (j < R)
+            float bpre[16];   // B[h][half + 2x][tid / 2], issued before dz so that it overlaps it
+            {
+                const int vv = tid >> 1, half = tid & 1;
 #pragma unroll
-                    for (int i = part; i < 128; i += 8) s += a.A[((size_t)h * 128 + i) * R + j] * sm.ddelta[i];
+                for (int x = 0; x < 16; ++x)
+                    bpre[x] = half + 2 * x < R ? a.Bm[((size_t)h * R + half + 2 * x) * 128 + vv] : 0.f;
+            }
+            {   // dz = A^T dDelta (+ Aw d(dw)), 8 threads per output
+                const int j = tid / 8, part = tid % 8;
+                float s = 0.f;
+#pragma unroll
+                for (int x = 0; x < 16; ++x) s += apre[x] * sm.ddelta[part + 8 * x];
                 s += __shfl_xor_sync(0xffffffffu, s, 4);
                 s += __shfl_xor_sync(0xffffffffu, s, 2);
                 s += __shfl_xor_sync(0xffffffffu, s, 1);
@@ -945,8 +1028,9 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             {   // dm = B^T dz, two threads per output
                 const int vv = tid >> 1, half = tid & 1;
                 float sacc = 0.f;
-#pragma unroll 8
-                for (int j = half; j < R; j += 2) sacc += a.Bm[((size_t)h * R + j) * 128 + vv] * sm.dzv[j];
+#pragma unroll
+                for (int x = 0; x < 16; ++x)
+                    if (half + 2 * x < R) sacc += bpre[x] * sm.dzv[half + 2 * x];
                 sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
                 if (half == 0) sm.dmv[vv] = sacc;
             }

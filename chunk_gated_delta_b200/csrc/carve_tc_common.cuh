@@ -22,6 +22,15 @@ __device__ __forceinline__ void retention(float g_logit, float beta, float &a, f
     inv_a = floor ? kInvAMin : D;
 }
 
+// Factor on the gradient of log a in the backward.  The kernels differentiate the floored
+// retention; where the floor binds (unfloored retention r < e^-10) the exact recurrence's
+// gradient of log a is r e^10 times that one: the gradient with respect to log a_t is a_t times
+// the product of the state before t with the gradient after the decay, and the floor moves
+// those two only by O(e^-10) relative.  Inert rows (past a packed sequence's end) have none.
+__device__ __forceinline__ float floor_scale(float r, bool inert) {
+    return inert ? 0.f : (r >= kAMin ? 1.f : r * kInvAMin);
+}
+
 // softplus(x) and sigmoid(x) from one fast exponential; beyond x = 15, log(1 + e^x) is x and
 // sigmoid(x) is 1 to fp32 rounding (and e^x may overflow), so both take those values there
 __device__ __forceinline__ float softplus_fast(float x, float e1) { return x > 15.f ? x : __logf(1.f + e1); }

@@ -14,7 +14,9 @@
 //              (m = middle of the token's 16-block) built from running products of a and 1/a,
 //              so every factor lies in [e^-80, e^80]; chunk-level factors (block products) carry
 //              the rest and are all <= 1
-//   Gram       Akk, Aqk: block (i,j) = rows_i . diag(e^{Lam_m(i) - Lam_m(j)}) . cols_j^T
+//   Gram       Akk, Aqk: block (i,j) = rows_i . diag(e^{Lam_m(i) - Lam_m(j)}) . cols_j^T, the factor
+//              split between the row operand (decay to block i's middle from block i's start)
+//              and the column operand (the rest), so that neither part underflows alone
 //   G          S0 [Kt; Qt]^T   (Kt = k e^{Lam}, Qt = q e^{Lam})            per warp, mma
 //   solve      X = Diag(w)(V - Kt S0^T);  U_i = (X_i - sum_j U_j M_ij^T) T_ii^T,  T_ii = (I + D A_ii)^-1
 //   output     O^T = S0 Qt^T + U^T Aqk^T                                  per warp, mma
@@ -40,19 +42,24 @@ struct __align__(16) TcFwdSmem {
     static constexpr int ST = NB == 2 ? 2 : 1;
     static constexpr bool GT = NB == 2;
     static constexpr int GSZ = GT ? C * 128 : 4;
+    // raw tiles by TMA; after the gate phase rq / rk of the stage hold the swizzled Qt / Kt
     __nv_bfloat16 rq[ST][C * 128], rk[ST][C * 128], rv[ST][C * 128];
     float rgl[ST][GSZ], rbx[ST][GSZ];
-    __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp], qt[C * kLdOp], kt[C * kLdOp];
+    // mid-block referenced operands; qm doubles as the output tile once the Gram has used it
+    __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp];
     __nv_bfloat16 aqk[C * LDA], mkk[C * LDA];
     __nv_bfloat16 tii[NB * 16 * 24];
     float akk_d[NB * 16 * 17];
     float p7[NB * 128], r15[NB * 128], fm[NB * 128], cij[NPAIR * 128];
-    float gam[128], wv[C], qbar[128], mvec[128], osum[128], mprev[128], zvec[64], delta[128];
-    float Ah[128 * kTcMaxRank], Bh[kTcMaxRank * 128];   // the head's low-rank factors
+    float gam[128], wv[C], qbar[128], osum[128], mprev[128];
+    float zp[8 * 32], dpart[2 * 128];   // content signal: per-warp parts of z, two parts of Delta
+    float AhT[kTcMaxRank * 128], BhT[128 * kTcMaxRank];   // the head's factors: A^T [j][k], B^T [v][j]
+    __nv_bfloat16 stile[GT ? 128 * kLdOp : 8];             // bf16 chunk-start state on its way out
     uint64_t bar[ST];
-    // the output tile is staged in qt once the S-GEMM has consumed it
-    __device__ __nv_bfloat16 *ost() { return qt; }
+    __device__ __nv_bfloat16 *ost() { return qm; }
 };
+// the dynamic shared-memory limit of one CTA on sm_100 (227 KB)
+static_assert(sizeof(TcFwdSmem<2>) <= 232448 && sizeof(TcFwdSmem<4>) <= 232448, "shared memory");
 
 struct TileMaps {
     CUtensorMap q, k, v, gl, bx;
@@ -80,6 +87,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     const size_t tstride = (size_t)H * 128;
     const size_t base_bh = ((size_t)bb * T + toff) * tstride + (size_t)h * 128;   // token 0 of this unit
     const int v0 = 16 * warp + g, v1 = v0 + 8;
+    const bool save = SM::GT && a.saved_states != nullptr;   // the bf16 chunk-start states for the backward
+    __nv_bfloat16 *states = save ? reinterpret_cast<__nv_bfloat16 *>(a.saved_states) : nullptr;
     // the decay's amplitude and the biases of this thread's gate channels 2 (tid & 63) + {0, 1}
     const float amp = DEC ? decay_amp(a.A_dec, h) : 1.f;
     const float tb0 = DEC ? decay_bias(a.tau, h, 2 * (tid & 63), 128) : 0.f;
@@ -107,9 +116,11 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         sm.mprev[tid] = a.m_prev_in ? a.m_prev_in[(size_t)u * 128 + tid] : 0.f;
         sm.osum[tid] = 0.f;
     }
-    for (int idx = tid; idx < 128 * R; idx += 256) {
-        sm.Ah[idx] = a.A[(size_t)h * 128 * R + idx];
-        sm.Bh[idx] = a.Bm[(size_t)h * R * 128 + idx];
+    for (int idx = tid; idx < 128 * kTcMaxRank; idx += 256) {   // zero beyond the rank
+        const int j = idx >> 7, k = idx & 127;                   // AhT[j][k] = A[h][k][j]
+        sm.AhT[idx] = j < R ? a.A[((size_t)h * 128 + k) * R + j] : 0.f;
+        const int v = idx / kTcMaxRank, j2 = idx % kTcMaxRank;   // BhT[v][j] = B[h][j][v]
+        sm.BhT[idx] = j2 < R ? a.Bm[((size_t)h * R + j2) * 128 + v] : 0.f;
     }
     __syncthreads();
 
@@ -140,7 +151,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             tma_prefetch_desc(&maps.bx);
         }
     }
-    if (!VL || NCCn > 0) {
+    if ((!VL || NCCn > 0) && !a.stall) {
         issue(0, 0);
         if (SM::ST == 1) issue(0, 1);
     }
@@ -182,7 +193,22 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 }
             }
         }
-        if (!mbar_wait(&sm.bar[st], (phase_bits >> st) & 1u)) atomicOr(&g_tc_timeout, 1);
+        if (first && a.mc_mode == 0 && a.saved_aux && tid < 128) {   // the mean q, prefetched
+            sm.qbar[tid] = pqb;
+            pqb = load_qbar(gc + 1);
+        }
+        if (save && tid == 0) bulk_wait_read<0>();   // the previous state copy has left stile
+        {   // a wait that gives up ends the sweep of the whole CTA: recorded, the copies of this
+            // stage (the only ones in flight here) waited for once more, bounded, and left
+            const bool lost = !mbar_wait(&sm.bar[st], (phase_bits >> st) & 1u, a.wait_limit);
+            if (__syncthreads_or(lost)) {
+                if (tid == 0) {
+                    atomicOr(&g_tc_timeout, 1);
+                    mbar_wait(&sm.bar[st], (phase_bits >> st) & 1u, a.wait_limit);
+                }
+                return;
+            }
+        }
         phase_bits ^= 1u << st;
         if (SM::ST == 2 && cc + 1 < NCCn) issue(cc + 1, 0);   // the other stage is free since last chunk
         if constexpr (VL) {
@@ -200,22 +226,21 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         const float wcur = wnext;
         if (tid < C && cc + 1 < NCCn && (!VL || t0 + C + tid < Tn))
             wnext = a.w_logit[((size_t)bb * T + toff + t0 + C + tid) * H + h];
-        if (a.saved_states) {   // bf16 copy of the chunk-start state, rows padded to 136
-            __nv_bfloat16 *stb = reinterpret_cast<__nv_bfloat16 *>(a.saved_states) + ((size_t)u * NCC + cc) * 128 * kLdOp;
+        if (save) {   // bf16 chunk-start state: this warp's 16 rows into the state tile (rows v, padded)
+            const int mi = lane >> 3, r = lane & 7;   // lane l addresses row r of matrix mi of each x4
+            const uint32_t base = smem_u32(sm.stile + (16 * warp + 8 * (mi & 1) + r) * kLdOp + 8 * (mi >> 1));
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int col = 8 * j + 2 * c4;
-                *reinterpret_cast<uint32_t *>(stb + v0 * kLdOp + col) = pack_bf16(s[j][0], s[j][1]);
-                *reinterpret_cast<uint32_t *>(stb + v1 * kLdOp + col) = pack_bf16(s[j][2], s[j][3]);
-            }
+            for (int q2 = 0; q2 < 8; ++q2)   // key columns 16 q2 .. 16 q2 + 15
+                stsm_x4(base + 32 * q2, pack_bf16(s[2 * q2][0], s[2 * q2][1]), pack_bf16(s[2 * q2][2], s[2 * q2][3]),
+                        pack_bf16(s[2 * q2 + 1][0], s[2 * q2 + 1][1]), pack_bf16(s[2 * q2 + 1][2], s[2 * q2 + 1][3]));
+            fence_proxy_async_smem();   // the bulk copy after the gate phase reads these
         }
-        // ---- content signal at a gate-chunk start
+        // ---- content signal at a gate-chunk start: m for this warp's rows, its part of z = B m,
+        //      then Delta = A z in two parts per key channel (summed by the gate phase)
         if (first) {
-            if (a.mc_mode == 0) {
-                if (tid < 128 && a.saved_aux) {   // written by the chunk-mean prologue, prefetched
-                    sm.qbar[tid] = pqb;
-                    pqb = load_qbar(gc + 1);
-                } else if (tid < 128) {
+            float *aux = a.saved_aux ? a.saved_aux + ((size_t)u * NG + gc) * (kTcAuxFixed + R) : nullptr;
+            if (a.mc_mode == 0 && !a.saved_aux) {   // mean q of the gate chunk, computed here
+                if (tid < 128) {
                     float acc = 0.f;
                     if (CPG == 1) {
                         for (int t = 0; t < C; ++t) acc += bf(sm.rq[st][t * 128 + tid]);
@@ -226,7 +251,10 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                     sm.qbar[tid] = acc / (float)n;
                 }
                 __syncthreads();
-                float p0 = 0.f, p1 = 0.f;
+            }
+            float p0, p1;   // m[v0], m[v1] (every lane of the row's quad after the reductions)
+            if (a.mc_mode == 0) {   // m = S_[c-1] qbar
+                p0 = p1 = 0.f;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int col = 8 * j + 2 * c4;
@@ -238,32 +266,50 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
                 p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
                 p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
-                if (c4 == 0) {
-                    sm.mvec[v0] = p0;
-                    sm.mvec[v1] = p1;
-                }
-            } else if (tid < 128) {
-                sm.mvec[tid] = sm.mprev[tid];
+            } else {                // m = mean output of the previous gate chunk
+                p0 = sm.mprev[v0];
+                p1 = sm.mprev[v1];
             }
-            __syncthreads();
-            content_signal<128, 128>(sm.Bh, sm.Ah, sm.mvec, sm.zvec, sm.delta, R);
+            if (aux && c4 == 0) {
+                aux[v0] = p0;
+                aux[v1] = p1;
+            }
+            {   // this warp's part of z: lane j over the warp's 16 rows
+                float zz = 0.f;
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const float ma = __shfl_sync(0xffffffffu, p0, 4 * r), mb = __shfl_sync(0xffffffffu, p1, 4 * r);
+                    zz += sm.BhT[(16 * warp + r) * kTcMaxRank + lane] * ma +
+                          sm.BhT[(16 * warp + 8 + r) * kTcMaxRank + lane] * mb;
+                }
+                sm.zp[warp * 32 + lane] = zz;
+            }
             if (tid < 128) sm.osum[tid] = 0.f;
+            __syncthreads();
+            float zj = 0.f;   // z_j, j = lane, in every warp (fixed order over the parts)
+#pragma unroll
+            for (int w2 = 0; w2 < 8; ++w2) zj += sm.zp[w2 * 32 + lane];
             {   // dw_c = Aw . z: the same projection of m_c biases the write gate (every warp forms
                 // it, so each write-gate thread holds it in a register for the whole gate chunk)
-                float x = (a.Aw && lane < R) ? a.Aw[(size_t)h * R + lane] * sm.zvec[lane] : 0.f;
+                float x = (a.Aw && lane < R) ? a.Aw[(size_t)h * R + lane] * zj : 0.f;
 #pragma unroll
                 for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
                 dwc = x;
             }
-            if (a.saved_aux) {
-                float *aux = a.saved_aux + ((size_t)u * NG + gc) * (kTcAuxFixed + R);
-                if (tid < 128) {
-                    aux[tid] = sm.mvec[tid];
-                    aux[128 + R + tid] = sm.delta[tid];
-                }
-                if (tid < R) aux[128 + tid] = sm.zvec[tid];
+            if (aux) {
+                if (warp == 0 && lane < R) aux[128 + lane] = zj;
                 if (tid == 0) aux[kTcAuxDw + R] = dwc;
             }
+            {   // Delta = A z: two parts of sixteen rank indices each, per key channel
+                const int part = tid >> 7, kk = tid & 127;
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    acc += sm.AhT[(16 * part + i) * 128 + kk] * __shfl_sync(0xffffffffu, zj, 16 * part + i);
+                sm.dpart[part * 128 + kk] = acc;
+            }
+            __syncthreads();
+            if (aux && tid < 128) aux[128 + R + tid] = sm.dpart[tid] + sm.dpart[128 + tid];
         }
         // ---- gates and mid-block referenced operands: per work item, two channels over half a
         //      16-token block, factors referenced to the block's token 7 (running products
@@ -272,7 +318,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         for (int x = 0; x < NP; ++x) {
             const int p = tid + 256 * x, cp = p & 63, hf = (p >> 6) & 1, i = p >> 7, c0 = 2 * cp;
             if (p < 128 * NB) {
-                const float dl0 = sm.delta[c0], dl1 = sm.delta[c0 + 1];
+                const float dl0 = sm.dpart[c0] + sm.dpart[128 + c0], dl1 = sm.dpart[c0 + 1] + sm.dpart[128 + c0 + 1];
                 float av[2][8], ia[2][8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
@@ -341,9 +387,13 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         }
         if (tid < C) sm.wv[tid] = (!VL || tid < nv) ? sigmoid_f(wcur + dwc) : 0.f;
         __syncthreads();
-        // ---- decayed operands Qt = Qm Em, Kt = Krm Em: one (channel, 16-token block) item per
-        //      thread, each forming its own prefix of block decays; chunk-level factors per
-        //      channel alongside
+        if (save && tid == 0) {   // the chunk-start state, written to stile above
+            bulk_s2g(states + ((size_t)u * NCC + cc) * 128 * kLdOp, sm.stile, 128u * kLdOp * 2u);
+            bulk_commit();
+        }
+        // ---- decayed operands Qt = Qm Em, Kt = Krm Em into the (now free) raw q / k tiles,
+        //      swizzled: one (channel, 16-token block) item per thread, each forming its own
+        //      prefix of block decays; chunk-level factors per channel alongside
 #pragma unroll
         for (int x = 0; x < NP; ++x) {
             const int p = tid + 256 * x, ch = p & 127, i = p >> 7;
@@ -354,8 +404,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int row = 16 * i + t;
-                    sm.qt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
-                    sm.kt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+                    sm.rq[st][swz128(row, ch)] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
+                    sm.rk[st][swz128(row, ch)] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
                 }
             }
         }
@@ -373,16 +423,20 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 sm.fm[i * 128 + tid] = sm.r15[i * 128 + tid] * F;
                 F *= dblk[i];
             }
+            // column factor of the Gram block pair (i, j < i): e^{Lam_m(i) - Lam_m(j)} = p7_i cij,
+            // cij = r15_j times the decay of the blocks between j and i; the two parts stay
+            // representable where their product would underflow
 #pragma unroll
             for (int i = 1; i < NB; ++i) {
-                float prod = 1.f;
+                float mid = 1.f;
 #pragma unroll
                 for (int j = i - 1; j >= 0; --j) {
-                    prod *= sm.r15[j * 128 + tid] * sm.p7[(j + 1) * 128 + tid];   // e^{Lam_m(j+1) - Lam_m(j)}
-                    sm.cij[pair_index(i, j) * 128 + tid] = prod;
+                    sm.cij[pair_index(i, j) * 128 + tid] = sm.r15[j * 128 + tid] * mid;
+                    mid *= dblk[j];
                 }
             }
         }
+        fence_proxy_async_smem();   // a later tile copy overwrites Qt / Kt
         __syncthreads();
         // ---- Gram blocks: the NB (NB + 1) / 2 blocks (i, j <= i) of each type dealt round-robin
         //      over the warps; T_ii after a diagonal Akk block, by the warp that formed it
@@ -402,8 +456,13 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                         uint32_t af[4], bfr[4];
                         load_a(af, rowop, kLdOp, 16 * i, 16 * ks, lane);
                         load_b_nk(bfr, sm.kcm, kLdOp, 16 * j, 16 * ks, lane);
-                        if (j < i) {
+                        if (j < i) {   // e^{Lam_m(i) - Lam_m(j)} = p7 of block i (rows) x cij (columns)
+                            const float *fp = sm.p7 + i * 128 + 16 * ks + 2 * c4;
                             const float *f = sm.cij + pair_index(i, j) * 128 + 16 * ks + 2 * c4;
+                            af[0] = scale_bf16x2(af[0], fp[0], fp[1]);
+                            af[1] = scale_bf16x2(af[1], fp[0], fp[1]);
+                            af[2] = scale_bf16x2(af[2], fp[8], fp[9]);
+                            af[3] = scale_bf16x2(af[3], fp[8], fp[9]);
                             bfr[0] = scale_bf16x2(bfr[0], f[0], f[1]);
                             bfr[1] = scale_bf16x2(bfr[1], f[8], f[9]);
                             bfr[2] = scale_bf16x2(bfr[2], f[0], f[1]);
@@ -453,7 +512,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 #pragma unroll
             for (int np = 0; np < 2 * NB; ++np) {
                 uint32_t bfr[4];
-                load_b_nk(bfr, np < NB ? sm.kt : sm.qt, kLdOp, 16 * (np % NB), 16 * ks, lane);
+                load_b_nk_swz(bfr, np < NB ? sm.rk[st] : sm.rq[st], 16 * (np % NB), 16 * ks, lane);
                 mma_bf16(ga[2 * np], af, bfr[0], bfr[1]);
                 mma_bf16(ga[2 * np + 1], af, bfr[2], bfr[3]);
             }
@@ -587,6 +646,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         }
     }
     if (a.m_prev_out && tid < 128) a.m_prev_out[(size_t)u * 128 + tid] = sm.mprev[tid];
+    if (save && tid == 0) bulk_wait<0>();   // the state copies are complete before the CTA ends
 }
 
 // Per (batch, gate chunk): mean of q over the gate chunk's tokens for every head, into the saved

@@ -25,11 +25,16 @@
  *
  * The library evaluates this chunk-parallel in WY form on the GPU (one triangular solve per
  * chunk shared by all value channels; CARVE blog section 2.3).  Every entry point is
- * stream-ordered on the caller's stream, allocates nothing, frees nothing and never
- * synchronises the device.  All pointers are DEVICE pointers unless stated otherwise; the
- * caller owns every buffer.  Arguments are validated on the host before any launch; a
- * rejected call launches nothing and returns a non-zero status.  Apart from
- * carve_bwd_noalloc (which shares one scratch array, see below), no entry point keeps
+ * stream-ordered on the caller's stream, allocates nothing and frees nothing.  None
+ * synchronises the device, with two exceptions: carve_check waits for its stream (that is
+ * its purpose) and then reads and clears the device status words with synchronous copies,
+ * and the first carve_bwd_noalloc call on each device looks up its scratch array's device
+ * address (which may load the module).  The first tensor-core launch of each kernel on a
+ * device also raises its shared-memory limit (a kernel attribute, no synchronisation).  All
+ * pointers are DEVICE pointers unless stated otherwise; the caller owns every buffer.
+ * Arguments are validated on the host before any launch; a rejected call launches nothing
+ * and returns a non-zero status.  Apart from carve_bwd_noalloc (which shares one scratch
+ * array) and the test hook carve_selftest_stall (a one-shot flag), no entry point keeps
  * mutable global state, so concurrent calls on different streams with disjoint buffers are
  * safe.
  *
@@ -244,6 +249,19 @@ carve_status carve_check(void *stream);
  * CARVE_ERR_TIMEOUT.  Nothing else is touched.  No counterpart in the pages.
  */
 carve_status carve_selftest_timeout(uint32_t iterations, void *stream);
+
+/*
+ * carve_selftest_stall -- test hook for the same path inside the tensor-core sweep kernels:
+ * arms a one-shot that the next carve_fwd or carve_bwd call running a tensor-core sweep (bf16,
+ * dk = dv = 128, rank <= 32) takes and clears.  That call skips the tile copy of its first
+ * compute chunk and bounds each of its barrier waits by `iterations` polls (1 to 1,000,000),
+ * so its first wait gives up in every CTA: the sweep records it, waits (bounded) for the
+ * copies it still has in flight and ends; the call's outputs are undefined and the next
+ * carve_check returns CARVE_ERR_TIMEOUT.  The one-shot is process-wide state (the one
+ * exception, with carve_bwd_noalloc, to "no mutable global state" above).  No counterpart in
+ * the pages.
+ */
+carve_status carve_selftest_stall(uint32_t iterations);
 
 #ifdef __cplusplus
 }

@@ -28,7 +28,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     assert declared_functions() == ["carve_bwd", "carve_bwd_noalloc", "carve_bwd_varlen", "carve_bwd_workspace_bytes",
                                     "carve_check", "carve_fwd", "carve_fwd_varlen", "carve_saved_bytes",
-                                    "carve_selftest_timeout", "carve_status_string", "carve_step"]
+                                    "carve_selftest_stall", "carve_selftest_timeout", "carve_status_string",
+                                    "carve_step"]
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -137,9 +138,11 @@ def test_null_and_misaligned_pointers_rejected(lib):
 
 
 def test_selftest_timeout_bounds_checked_on_host(lib):
-    """Out-of-range poll counts are rejected before any launch."""
+    """Out-of-range poll counts are rejected before any launch (and arm nothing)."""
     assert lib.carve_selftest_timeout(0, None) == 1
     assert lib.carve_selftest_timeout(1_000_001, None) == 1
+    assert lib.carve_selftest_stall(0) == 1
+    assert lib.carve_selftest_stall(1_000_001) == 1
 
 
 def test_varlen_arguments_checked_on_host(lib):
