@@ -979,14 +979,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             load_gates(cc - 1);
             load_w(cc - 1);
         }
-        // the content path's factor A (this thread's slice A[h][part + 8x][tid / 8], rank <= 32),
-        // read from L2 now so that its latency overlaps the stores below
-        float apre[16];
-        if (gate_start) {
-            const int j = tid / 8, part = tid % 8;
-#pragma unroll
-            for (int x = 0; x < 16; ++x) apre[x] = j < R ? a.A[((size_t)h * 128 + part + 8 * x) * R + j] : 0.f;
-        }
         __syncthreads();
         if (tid < 128) {
             float x = 0.f;
@@ -1004,7 +996,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         __syncthreads();
         // ---- content path at the gate chunk's first token
         if (gate_start) {
-            float bpre[16];   // B[h][half + 2x][tid / 2], issued before dz so that it overlaps it
+            float bpre[16];   // B[h][half + 2x][tid / 2] (rank <= 32), issued before dz so that it overlaps it
             {
                 const int vv = tid >> 1, half = tid & 1;
 #pragma unroll
@@ -1015,7 +1007,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 const int j = tid / 8, part = tid % 8;
                 float s = 0.f;
 #pragma unroll
-                for (int x = 0; x < 16; ++x) s += apre[x] * sm.ddelta[part + 8 * x];
+                for (int x = 0; x < 16; ++x)
+                    s += (j < R ? a.A[((size_t)h * 128 + part + 8 * x) * R + j] : 0.f) * sm.ddelta[part + 8 * x];
                 s += __shfl_xor_sync(0xffffffffu, s, 4);
                 s += __shfl_xor_sync(0xffffffffu, s, 2);
                 s += __shfl_xor_sync(0xffffffffu, s, 1);
