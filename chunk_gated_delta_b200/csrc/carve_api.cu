@@ -104,11 +104,11 @@ int tc_fwd_chunk(const carve_dims *d) {
 bool use_tc_bwd(const carve_dims *d) { return tc_shape(d) && d->T % 32 == 0; }
 
 // Bytes of the boundary states at the head of the `saved` buffer: fp32 states every 16 tokens
-// for the SIMT kernels; bf16 states every 32 tokens, rows padded to 136, for the tensor-core
+// for the SIMT kernels; bf16 states every 32 tokens (128 rows of 256 bytes) for the tensor-core
 // kernels.  The per-chunk content signals (fp32) follow.
 size_t saved_states_bytes(const carve_dims *d) {
     const size_t units = (size_t)d->B * d->H;
-    if (use_tc_bwd(d)) return units * (size_t)(d->T / 32) * 128 * 136 * 2;
+    if (use_tc_bwd(d)) return units * (size_t)(d->T / 32) * 128 * 128 * 2;
     return units * (size_t)(d->T / carve::kSub) * d->dv * d->dk * sizeof(float);
 }
 

@@ -66,26 +66,6 @@ __device__ __forceinline__ void load_a_t(uint32_t (&a)[4], const __nv_bfloat16 *
     ldsm_x4_t(a, smem_u32(base + k * ld + m));
 }
 
-__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
-}
-
-// B fragment of one n-tile (n0..n0+7) x 16 k from an [n][k] tile (k contiguous)
-__device__ __forceinline__ void load_b1_nk(uint32_t (&b)[2], const __nv_bfloat16 *base, int ld, int n0, int k0, int lane) {
-    const int n = n0 + (lane & 7), k = k0 + ((lane >> 3) & 1) * 8;
-    ldsm_x2(b, smem_u32(base + n * ld + k));
-}
-
-// B fragment of one n-tile x 16 k from a [k][n] tile (n contiguous), via the transposing load
-__device__ __forceinline__ void load_b1_kn(uint32_t (&b)[2], const __nv_bfloat16 *base, int ld, int n0, int k0, int lane) {
-    const int k = k0 + (lane & 7) + (((lane >> 3) & 1) << 3);
-    ldsm_x2_t(b, smem_u32(base + k * ld + n0));
-}
-
 // B fragments of two n-tiles (n0.., n0+8..) x 16 k from an [n][k] tile (k contiguous):
 // b[0], b[1] -> tile n0;  b[2], b[3] -> tile n0+8
 __device__ __forceinline__ void load_b_nk(uint32_t (&b)[4], const __nv_bfloat16 *base, int ld, int n0, int k0, int lane) {
@@ -99,31 +79,11 @@ __device__ __forceinline__ void load_b_kn(uint32_t (&b)[4], const __nv_bfloat16 
     ldsm_x4_t(b, smem_u32(base + k * ld + n));
 }
 
-// Transpose of the 8x8 bf16 matrix held one bf16x2 per lane in the fragment layout (lane l: row
-// l / 4, columns 2 (l % 4) and 2 (l % 4) + 1).
-__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-    return y;
-}
-
-// B fragment (16 k x 8 n) of the matrix whose C fragment (16 rows x 8 columns, fp32) is c: the
-// C tile's rows become the contraction index (bf16-rounded; two transposes, no shared memory).
-__device__ __forceinline__ void c_to_b(const float (&c)[4], uint32_t &b0, uint32_t &b1) {
-    b0 = movm_t(pack_bf16(c[0], c[1]));
-    b1 = movm_t(pack_bf16(c[2], c[3]));
-}
-
-// Four 8x8 bf16 matrices to shared memory; lane l gives the address of row l % 8 of matrix
-// l / 8 (of the stored layout).  .trans stores each matrix transposed.
+// Four 8x8 bf16 matrices to shared memory (the inverse of ldsm_x4): lane l gives the address of
+// row l % 8 of matrix l / 8; register i holds matrix i in the fragment layout above.
 __device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
     asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(r0), "r"(r1),
                  "r"(r2), "r"(r3)
-                 : "memory");
-}
-__device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
-    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(r0),
-                 "r"(r1), "r"(r2), "r"(r3)
                  : "memory");
 }
 
@@ -138,13 +98,6 @@ __device__ __forceinline__ int swz128(int r, int c) {   // element offset of (ro
 __device__ __forceinline__ void load_a_swz(uint32_t (&a)[4], const __nv_bfloat16 *base, int m0, int k0, int lane) {
     const int r = m0 + (lane & 15), k = k0 + (lane >> 4) * 8;
     ldsm_x4(a, smem_u32(base + swz128(r, k)));
-}
-
-// load_a_t on a swizzled [k][m] tile (A = X^T, X rows k0.., columns m0..)
-__device__ __forceinline__ void load_a_t_swz(uint32_t (&a)[4], const __nv_bfloat16 *base, int m0, int k0, int lane) {
-    const int mat = lane >> 3, r = lane & 7;
-    const int k = k0 + r + ((mat >> 1) << 3), m = m0 + ((mat & 1) << 3);
-    ldsm_x4_t(a, smem_u32(base + swz128(k, m)));
 }
 
 // load_b_nk on a swizzled [n][k] tile

@@ -55,7 +55,7 @@ struct __align__(16) TcBwdSmem {
     __nv_bfloat16 rq[kBC * 128], rk[kBC * 128], rv[kBC * 128], rdo[kBC * 128];
     __nv_bfloat16 dop[kBC * kLdOp];
     __nv_bfloat16 qm[kBC * kLdOp], krm[kBC * kLdOp], kcm[kBC * kLdOp];
-    __nv_bfloat16 s0b[128 * kLdOp], ds1b[128 * kLdOp];
+    __nv_bfloat16 s0b[128 * 128], ds1b[128 * kLdOp];   // s0b: the saved state as written (swizzled rows)
     __nv_bfloat16 ub[kBC * kLdOp], drb[kBC * kLdOp];
     __nv_bfloat16 aqk[kBC * kLdT], akk[kBC * kLdT], mkk[kBC * kLdT], daqk[kBC * kLdT], dakk[kBC * kLdT];
     __nv_bfloat16 tii[kBNB * 16 * 24];
@@ -94,8 +94,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     const size_t tstride = (size_t)H * 128;
     const size_t base_bh = ((size_t)bb * T + toff) * tstride + (size_t)h * 128;
     const int v0 = 16 * warp + g, v1 = v0 + 8;
-    // bf16 chunk-start states written by the forward, rows padded to kLdOp
-    const __nv_bfloat16 *states = reinterpret_cast<const __nv_bfloat16 *>(a.saved_states) + (size_t)u * NCC * 128 * kLdOp;
+    // bf16 chunk-start states written by the forward: 128 rows of 256 bytes, 16-byte chunks swizzled
+    const __nv_bfloat16 *states = reinterpret_cast<const __nv_bfloat16 *>(a.saved_states) + (size_t)u * NCC * 128 * 128;
     // workspace: per gate chunk dDelta (128) and dz (32) for the dA / dB reduction, then the
     // readout vectors of dq (128 per gate chunk)
     float *wsg = a.ws + (size_t)u * NG * kTcGradRec;
@@ -130,8 +130,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int col = 8 * j + 2 * c4;
-            const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + v0 * kLdOp + col);
-            const __nv_bfloat162 s1 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + v1 * kLdOp + col);
+            const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + swz128(v0, col));
+            const __nv_bfloat162 s1 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + swz128(v1, col));
             v[j][0] = ds[j][0] * bf(s0.x) + ds[j][2] * bf(s1.x);
             v[j][1] = ds[j][1] * bf(s0.y) + ds[j][3] * bf(s1.y);
         }
@@ -180,8 +180,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     };
     auto issue_s0 = [&](int cc) {
         if (tid != 0) return;
-        mbar_expect_tx(&sm.bar_s0, 128u * kLdOp * 2u);
-        bulk_g2s(sm.s0b, states + (size_t)cc * 128 * kLdOp, 128u * kLdOp * 2u, &sm.bar_s0);
+        mbar_expect_tx(&sm.bar_s0, 128u * 128u * 2u);
+        bulk_g2s(sm.s0b, states + (size_t)cc * 128 * 128, 128u * 128u * 2u, &sm.bar_s0);
     };
     if (!VL || NCCn > 0) {
         if (!a.stall) issue(NCCn - 1);
@@ -202,8 +202,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         }
     };
     if (!VL || NCCn > 0) load_gates(NCCn - 1);
-    // the saved record of the next gate chunk and the write logits of the next compute chunk,
-    // loaded one iteration ahead
+    // the saved record of the next gate chunk (loaded when the current one is taken) and the
+    // write logits of the next compute chunk (loaded one iteration ahead)
     float pd = 0.f, pq = 0.f, pw = 0.f, pdw = 0.f;
     auto load_aux = [&](int gc) {   // Delta, the mean q and the write-gate term of a gate chunk
         const float *aux = a.saved_aux + ((size_t)u * NG + gc) * (kTcAuxFixed + R);
@@ -237,14 +237,17 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 sm.dwc = pdw;
                 sm.ddw = 0.f;
             }
+            if (gc > 0) load_aux(gc - 1);   // the previous gate chunk's record, a gate chunk ahead
         }
-        {   // the carried gradient as a bf16 tile
+        {   // the carried gradient as a bf16 tile [v][k]: this warp's 16 rows (stmatrix; lane l
+            // addresses row l % 8 of matrix l / 8 of each x4: rows +0 / +8, columns +0 / +8)
+            const int mi = lane >> 3, r = lane & 7;
+            const uint32_t base = smem_u32(sm.ds1b + (16 * warp + 8 * (mi & 1) + r) * kLdOp + 8 * (mi >> 1));
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int col = 8 * j + 2 * c4;
-                *reinterpret_cast<uint32_t *>(sm.ds1b + v0 * kLdOp + col) = pack_bf16(ds[j][0], ds[j][1]);
-                *reinterpret_cast<uint32_t *>(sm.ds1b + v1 * kLdOp + col) = pack_bf16(ds[j][2], ds[j][3]);
-            }
+            for (int q2 = 0; q2 < 8; ++q2)   // key columns 16 q2 .. 16 q2 + 15
+                stsm_x4(base + 32 * q2, pack_bf16(ds[2 * q2][0], ds[2 * q2][1]), pack_bf16(ds[2 * q2][2], ds[2 * q2][3]),
+                        pack_bf16(ds[2 * q2 + 1][0], ds[2 * q2 + 1][1]),
+                        pack_bf16(ds[2 * q2 + 1][2], ds[2 * q2 + 1][3]));
         }
         {   // a wait that gives up ends the sweep of the whole CTA: recorded, the copies in flight
             // (this chunk's tiles and its start state) waited for once more, bounded, and left
@@ -485,7 +488,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             uint32_t af[4];
-            load_a(af, sm.s0b, kLdOp, 16 * warp, 16 * ks, lane);
+            load_a_swz(af, sm.s0b, 16 * warp, 16 * ks, lane);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bfr[4];
@@ -748,7 +751,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 for (int np2 = 0; np2 < 2; ++np2) {
                     const int n0 = ch0 + 16 * np2;
                     uint32_t bs[4], bd[4];
-                    load_b_kn(bs, sm.s0b, kLdOp, n0, 16 * ks, lane);
+                    load_b_kn_swz(bs, sm.s0b, n0, 16 * ks, lane);
                     load_b_kn(bd, sm.ds1b, kLdOp, n0, 16 * ks, lane);
                     mma_bf16(gq[2 * np2], ao, bs[0], bs[1]);
                     mma_bf16(gq[2 * np2 + 1], ao, bs[2], bs[3]);
@@ -1033,13 +1036,16 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 // chunk is added by the readout pass after this kernel (vector stored per gate chunk)
                 {
                     const int ch = tid & 127, half = tid >> 7;
-                    float sa[4] = {0.f, 0.f, 0.f, 0.f};
+                    int off[8];   // column of `ch` in a swizzled row r with r mod 8 = x
 #pragma unroll
-                    for (int r = 0; r < 64; r += 4)
+                    for (int x = 0; x < 8; ++x) off[x] = ((((ch >> 3) ^ x) << 3) | (ch & 7));
+                    float sa[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int x = 0; x < 4; ++x)
-                            sa[x] += bf(sm.s0b[(64 * half + r + x) * kLdOp + ch]) * sm.dmv[64 * half + r + x];
-                    sm.pdd[half * 128 + ch] = (sa[0] + sa[1]) + (sa[2] + sa[3]);
+                    for (int r = 0; r < 64; r += 8)
+#pragma unroll
+                        for (int x = 0; x < 8; ++x)
+                            sa[x] += bf(sm.s0b[(64 * half + r + x) * 128 + off[x]]) * sm.dmv[64 * half + r + x];
+                    sm.pdd[half * 128 + ch] = ((sa[0] + sa[1]) + (sa[2] + sa[3])) + ((sa[4] + sa[5]) + (sa[6] + sa[7]));
                 }
                 __syncthreads();
                 if (tid < 128) {
@@ -1064,7 +1070,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         __syncthreads();
         if (cc > 0) {
             if (!s0_early) issue_s0(cc - 1);
-            if (gate_start) load_aux((cc - 1) / CPG);   // chunk cc - 1 ends the previous gate chunk
         }
     }
     if (a.dS0) {

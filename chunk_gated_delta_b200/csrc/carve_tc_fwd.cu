@@ -21,9 +21,14 @@
 //   solve      X = Diag(w)(V - Kt S0^T);  U_i = (X_i - sum_j U_j M_ij^T) T_ii^T,  T_ii = (I + D A_ii)^-1
 //   output     O^T = S0 Qt^T + U^T Aqk^T                                  per warp, mma
 //   state      S = S Diag(gamma) + U^T Kbar,  Kbar = k e^{Lam_C - Lam}         per warp, mma
-// Raw q/k/v rows are prefetched into shared memory by the bulk-copy (TMA) engine while the
-// previous chunk computes.  The floor a >= e^-10 bounds the deviation from the exact
-// recurrence by e^-10 per step in channels that are being erased anyway.
+//   content   at a gate-chunk start, m for each warp's rows (S_[c-1] mean q, or the previous
+//              chunk's mean output), z = B m reduced over the warps, Delta = A z per key channel,
+//              from A^T and B^T staged in shared memory
+// Raw q/k/v rows (and, with 32-token chunks, the gate logits) are prefetched into shared memory
+// by the bulk-copy (TMA) engine while the previous chunk computes; the bf16 chunk-start state
+// saved for the backward is written into the stage's consumed gate tiles (stmatrix) and leaves
+// through one bulk copy.  The floor a >= e^-10 bounds the deviation from the exact recurrence
+// by e^-10 per step in channels that are being erased anyway.
 #include "carve_tc_common.cuh"
 
 namespace carve {
@@ -42,11 +47,12 @@ struct __align__(16) TcFwdSmem {
     static constexpr int ST = NB == 2 ? 2 : 1;
     static constexpr bool GT = NB == 2;
     static constexpr int GSZ = GT ? C * 128 : 4;
-    // raw tiles by TMA; after the gate phase rq / rk of the stage hold the swizzled Qt / Kt
+    // raw tiles by TMA; a stage's two gate-logit tiles (32 KB with 32-token chunks) carry the
+    // bf16 chunk-start state on its way out once the gate phase has read them
     __nv_bfloat16 rq[ST][C * 128], rk[ST][C * 128], rv[ST][C * 128];
-    float rgl[ST][GSZ], rbx[ST][GSZ];
+    float rgx[ST][2][GSZ];
     // mid-block referenced operands; qm doubles as the output tile once the Gram has used it
-    __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp];
+    __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp], qt[C * kLdOp], kt[C * kLdOp];
     __nv_bfloat16 aqk[C * LDA], mkk[C * LDA];
     __nv_bfloat16 tii[NB * 16 * 24];
     float akk_d[NB * 16 * 17];
@@ -54,12 +60,12 @@ struct __align__(16) TcFwdSmem {
     float gam[128], wv[C], qbar[128], osum[128], mprev[128];
     float zp[8 * 32], dpart[2 * 128];   // content signal: per-warp parts of z, two parts of Delta
     float AhT[kTcMaxRank * 128], BhT[128 * kTcMaxRank];   // the head's factors: A^T [j][k], B^T [v][j]
-    __nv_bfloat16 stile[GT ? 128 * kLdOp : 8];             // bf16 chunk-start state on its way out
     uint64_t bar[ST];
     __device__ __nv_bfloat16 *ost() { return qm; }
 };
 // the dynamic shared-memory limit of one CTA on sm_100 (227 KB)
 static_assert(sizeof(TcFwdSmem<2>) <= 232448 && sizeof(TcFwdSmem<4>) <= 232448, "shared memory");
+static_assert(sizeof(TcFwdSmem<2>::rgx[0]) == 128 * 128 * 2, "a stage's gate tiles hold one bf16 state");
 
 struct TileMaps {
     CUtensorMap q, k, v, gl, bx;
@@ -136,8 +142,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             tma_load_3d(sm.rq[st], &maps.q, 0, h, row, bar);
             tma_load_3d(sm.rk[st], &maps.k, 0, h, row, bar);
             if (SM::GT) {
-                tma_load_3d(sm.rgl[st], &maps.gl, 0, h, row, bar);
-                tma_load_3d(sm.rbx[st], &maps.bx, 0, h, row, bar);
+                tma_load_3d(sm.rgx[st][0], &maps.gl, 0, h, row, bar);
+                tma_load_3d(sm.rgx[st][1], &maps.bx, 0, h, row, bar);
             }
         }
         if (which == 1 || SM::ST == 2) tma_load_3d(sm.rv[st], &maps.v, 0, h, row, bar);
@@ -197,7 +203,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             sm.qbar[tid] = pqb;
             pqb = load_qbar(gc + 1);
         }
-        if (save && tid == 0) bulk_wait_read<0>();   // the previous state copy has left stile
+        if (save && tid == 0) bulk_wait_read<0>();   // the last state copy has left its stage before that
+                                                     // stage's next tile copy is issued below
         {   // a wait that gives up ends the sweep of the whole CTA: recorded, the copies of this
             // stage (the only ones in flight here) waited for once more, bounded, and left
             const bool lost = !mbar_wait(&sm.bar[st], (phase_bits >> st) & 1u, a.wait_limit);
@@ -226,15 +233,6 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         const float wcur = wnext;
         if (tid < C && cc + 1 < NCCn && (!VL || t0 + C + tid < Tn))
             wnext = a.w_logit[((size_t)bb * T + toff + t0 + C + tid) * H + h];
-        if (save) {   // bf16 chunk-start state: this warp's 16 rows into the state tile (rows v, padded)
-            const int mi = lane >> 3, r = lane & 7;   // lane l addresses row r of matrix mi of each x4
-            const uint32_t base = smem_u32(sm.stile + (16 * warp + 8 * (mi & 1) + r) * kLdOp + 8 * (mi >> 1));
-#pragma unroll
-            for (int q2 = 0; q2 < 8; ++q2)   // key columns 16 q2 .. 16 q2 + 15
-                stsm_x4(base + 32 * q2, pack_bf16(s[2 * q2][0], s[2 * q2][1]), pack_bf16(s[2 * q2][2], s[2 * q2][3]),
-                        pack_bf16(s[2 * q2 + 1][0], s[2 * q2 + 1][1]), pack_bf16(s[2 * q2 + 1][2], s[2 * q2 + 1][3]));
-            fence_proxy_async_smem();   // the bulk copy after the gate phase reads these
-        }
         // ---- content signal at a gate-chunk start: m for this warp's rows, its part of z = B m,
         //      then Delta = A z in two parts per key channel (summed by the gate phase)
         if (first) {
@@ -325,8 +323,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                     float2 gv, bv;
                     if (SM::GT) {
                         const int row = 16 * i + 8 * hf + t;
-                        gv = *reinterpret_cast<const float2 *>(&sm.rgl[st][row * 128 + c0]);
-                        bv = *reinterpret_cast<const float2 *>(&sm.rbx[st][row * 128 + c0]);
+                        gv = *reinterpret_cast<const float2 *>(&sm.rgx[st][0][row * 128 + c0]);
+                        bv = *reinterpret_cast<const float2 *>(&sm.rgx[st][1][row * 128 + c0]);
                     } else {
                         gv = glr[x][t];
                         bv = bxr[x][t];
@@ -387,13 +385,21 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         }
         if (tid < C) sm.wv[tid] = (!VL || tid < nv) ? sigmoid_f(wcur + dwc) : 0.f;
         __syncthreads();
-        if (save && tid == 0) {   // the chunk-start state, written to stile above
-            bulk_s2g(states + ((size_t)u * NCC + cc) * 128 * kLdOp, sm.stile, 128u * kLdOp * 2u);
-            bulk_commit();
+        __nv_bfloat16 *stile = reinterpret_cast<__nv_bfloat16 *>(sm.rgx[st]);
+        if (save) {   // bf16 chunk-start state into the stage's gate tiles (read above): this warp's
+                      // 16 rows, 256-byte rows with their 16-byte chunks swizzled
+            const int mi = lane >> 3, r = lane & 7;   // lane l addresses row r of matrix mi of each x4
+            const int row = 16 * warp + 8 * (mi & 1) + r;
+#pragma unroll
+            for (int q2 = 0; q2 < 8; ++q2)   // key columns 16 q2 .. 16 q2 + 15
+                stsm_x4(smem_u32(stile + swz128(row, 16 * q2 + 8 * (mi >> 1))), pack_bf16(s[2 * q2][0], s[2 * q2][1]),
+                        pack_bf16(s[2 * q2][2], s[2 * q2][3]), pack_bf16(s[2 * q2 + 1][0], s[2 * q2 + 1][1]),
+                        pack_bf16(s[2 * q2 + 1][2], s[2 * q2 + 1][3]));
+            fence_proxy_async_smem();   // read by the bulk copy below, overwritten by a later tile copy
         }
-        // ---- decayed operands Qt = Qm Em, Kt = Krm Em into the (now free) raw q / k tiles,
-        //      swizzled: one (channel, 16-token block) item per thread, each forming its own
-        //      prefix of block decays; chunk-level factors per channel alongside
+        // ---- decayed operands Qt = Qm Em, Kt = Krm Em: one (channel, 16-token block) item per
+        //      thread, each forming its own prefix of block decays; chunk-level factors per
+        //      channel alongside
 #pragma unroll
         for (int x = 0; x < NP; ++x) {
             const int p = tid + 256 * x, ch = p & 127, i = p >> 7;
@@ -404,8 +410,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int row = 16 * i + t;
-                    sm.rq[st][swz128(row, ch)] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
-                    sm.rk[st][swz128(row, ch)] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+                    sm.qt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
+                    sm.kt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
                 }
             }
         }
@@ -436,8 +442,11 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 }
             }
         }
-        fence_proxy_async_smem();   // a later tile copy overwrites Qt / Kt
         __syncthreads();
+        if (save && tid == 0) {   // the chunk-start state, written to the stage's gate tiles above
+            bulk_s2g(states + ((size_t)u * NCC + cc) * 128 * 128, stile, 128u * 128u * 2u);
+            bulk_commit();
+        }
         // ---- Gram blocks: the NB (NB + 1) / 2 blocks (i, j <= i) of each type dealt round-robin
         //      over the warps; T_ii after a diagonal Akk block, by the warp that formed it
         constexpr int NBLK = NB * (NB + 1) / 2;
@@ -512,7 +521,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 #pragma unroll
             for (int np = 0; np < 2 * NB; ++np) {
                 uint32_t bfr[4];
-                load_b_nk_swz(bfr, np < NB ? sm.rk[st] : sm.rq[st], 16 * (np % NB), 16 * ks, lane);
+                load_b_nk(bfr, np < NB ? sm.kt : sm.qt, kLdOp, 16 * (np % NB), 16 * ks, lane);
                 mma_bf16(ga[2 * np], af, bfr[0], bfr[1]);
                 mma_bf16(ga[2 * np + 1], af, bfr[2], bfr[3]);
             }
@@ -725,7 +734,8 @@ cudaError_t launch_tc_fwd_t(const FwdArgs &a, cudaStream_t st) {
 int tc_compute_chunk(int L) { return L == 32 ? 32 : (L == 64 || L == 128) ? 64 : 0; }
 
 // C = 32 or 64 tokens per compute chunk.  With a.saved_states set (32-token chunks), a bf16
-// copy of the state at every compute-chunk start ([T/32][128][136] per unit, rows padded) and
+// copy of the state at every compute-chunk start ([T/32][128][128] per unit, each row's 16-byte
+// chunks at positions c ^ (row & 7)) and
 // per gate chunk the record (m, z, Delta, mean q, dw) of kTcAuxFixed + R floats are written for the
 // backward.
 cudaError_t launch_fwd_tc(const FwdArgs &a, int C, cudaStream_t st) {
