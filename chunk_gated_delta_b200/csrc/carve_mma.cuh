@@ -86,6 +86,28 @@ __device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1,
                  "r"(r2), "r"(r3)
                  : "memory");
 }
+// The same with each matrix stored transposed: lane l addresses row l % 8 of the stored
+// (transposed) matrix l / 8.
+__device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
+// C fragments of a warp's 16 rows x (8 * nt2 * 2) columns, stored transposed into a row-major
+// [column][row] tile (ld elements per stored row) at stored columns m0 .. m0 + 15: tile j holds
+// columns 8j .. 8j + 7; two tiles per stmatrix
+template <int NT>
+__device__ __forceinline__ void store_frags_t(__nv_bfloat16 *base, int ld, int m0, const float (*y)[4], int lane) {
+    const int mi = lane >> 3, r = lane & 7;
+#pragma unroll
+    for (int p = 0; p < NT / 2; ++p) {
+        const int row = 8 * (2 * p + (mi >> 1)) + r;   // stored row = original column
+        stsm_x4_t(smem_u32(base + row * ld + m0 + 8 * (mi & 1)), pack_bf16(y[2 * p][0], y[2 * p][1]),
+                  pack_bf16(y[2 * p][2], y[2 * p][3]), pack_bf16(y[2 * p + 1][0], y[2 * p + 1][1]),
+                  pack_bf16(y[2 * p + 1][2], y[2 * p + 1][3]));
+    }
+}
 
 // ---- swizzled [rows][128] bf16 tiles (256-byte rows, no padding): the 16-byte chunk c of
 //      row r is stored at chunk c ^ (r & 7), so the eight rows of an 8x8 ldmatrix always hit

@@ -560,14 +560,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 mma_bf16(rr[2 * i], ua, bfr[0], bfr[1]);
                 mma_bf16(rr[2 * i + 1], ua, bfr[2], bfr[3]);
             }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int t = 8 * j + 2 * c4;
-            sm.ub[t * kLdOp + v0] = __float2bfloat16_rn(ga[j][0]);
-            sm.ub[(t + 1) * kLdOp + v0] = __float2bfloat16_rn(ga[j][1]);
-            sm.ub[t * kLdOp + v1] = __float2bfloat16_rn(ga[j][2]);
-            sm.ub[(t + 1) * kLdOp + v1] = __float2bfloat16_rn(ga[j][3]);
-        }
+        store_frags_t<4>(sm.ub, kLdOp, 16 * warp, ga, lane);   // U^T -> [t][v]
         // ---- dU^T = dO^T Aqk + dS1 Kbar^T
         float du[4][4];
 #pragma unroll
@@ -642,10 +635,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             dr[j][1] = w1 * du[j][1];
             dr[j][2] = w0 * du[j][2];
             dr[j][3] = w1 * du[j][3];
-            sm.drb[t * kLdOp + v0] = __float2bfloat16_rn(dr[j][0]);
-            sm.drb[(t + 1) * kLdOp + v0] = __float2bfloat16_rn(dr[j][1]);
-            sm.drb[t * kLdOp + v1] = __float2bfloat16_rn(dr[j][2]);
-            sm.drb[(t + 1) * kLdOp + v1] = __float2bfloat16_rn(dr[j][3]);
             float p0 = du[j][0] * rr[j][0] + du[j][2] * rr[j][2];
             float p1 = du[j][1] * rr[j][1] + du[j][3] * rr[j][3];
 #pragma unroll
@@ -658,6 +647,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 sm.dwp[warp * C + t + 1] = p1;
             }
         }
+        store_frags_t<4>(sm.drb, kLdOp, 16 * warp, dr, lane);   // dR^T -> [t][v]
         // ---- dS0 = dS1 Diag(gamma) + dO^T Qt - dR^T Kt
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -993,8 +983,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             const int t = idx >> 5, c = (idx & 31) * 4;
             const float *gsrc = sm.dlam + t * kLdF + c, *bsrc = sm.rfac + t * kLdF + c;
             const size_t gi = base_bh + (size_t)(t0 + t) * tstride + c;
-            *reinterpret_cast<float4 *>(a.dg_logit + gi) = make_float4(gsrc[0], gsrc[1], gsrc[2], gsrc[3]);
-            *reinterpret_cast<float4 *>(a.dbx + gi) = make_float4(bsrc[0], bsrc[1], bsrc[2], bsrc[3]);
+            *reinterpret_cast<float4 *>(a.dg_logit + gi) = *reinterpret_cast<const float4 *>(gsrc);
+            *reinterpret_cast<float4 *>(a.dbx + gi) = *reinterpret_cast<const float4 *>(bsrc);
         }
         __syncthreads();
         // ---- content path at the gate chunk's first token

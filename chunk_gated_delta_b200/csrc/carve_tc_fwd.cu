@@ -585,15 +585,11 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             float os0 = 0.f, os1 = 0.f;
 #pragma unroll
             for (int j = 0; j < 2 * NB; ++j) {
-                const int t = 8 * j + 2 * c4;
                 const float *y = ga[2 * NB + j];
-                sm.ost()[t * kLdOp + v0] = __float2bfloat16_rn(y[0]);
-                sm.ost()[(t + 1) * kLdOp + v0] = __float2bfloat16_rn(y[1]);
-                sm.ost()[t * kLdOp + v1] = __float2bfloat16_rn(y[2]);
-                sm.ost()[(t + 1) * kLdOp + v1] = __float2bfloat16_rn(y[3]);
                 os0 += y[0] + y[1];
                 os1 += y[2] + y[3];
             }
+            store_frags_t<2 * NB>(sm.ost(), kLdOp, 16 * warp, ga + 2 * NB, lane);   // O^T -> [t][v]
             os0 += __shfl_xor_sync(0xffffffffu, os0, 1);
             os0 += __shfl_xor_sync(0xffffffffu, os0, 2);
             os1 += __shfl_xor_sync(0xffffffffu, os1, 1);
