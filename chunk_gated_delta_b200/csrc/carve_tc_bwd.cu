@@ -68,8 +68,16 @@ struct __align__(16) TcBwdSmem {
     float daqd[kBC];   // diagonal of dAqk (kept out of the bf16 tile)
     float fs0[128];    // floor_scale of the sequence's first token, per key channel (first chunk)
     float dwc, ddw;   // the write gate's content term of the gate chunk and its gradient
-    uint64_t bar, bar_s0;
+    uint64_t bar, bar_s0, bar_ab;
 };
+
+// the dynamic shared-memory limit of one CTA on sm_100 (227 KB); the content path's factors
+// (2 x 128 x rank floats) fit in the dO and operand tiles, which are contiguous
+static_assert(sizeof(TcBwdSmem) <= 232448, "shared memory");
+static_assert(offsetof(TcBwdSmem, kcm) + sizeof(TcBwdSmem::kcm) - offsetof(TcBwdSmem, dop) >= 256 * kTcMaxRankBwd * 4 &&
+                  offsetof(TcBwdSmem, qm) == offsetof(TcBwdSmem, dop) + sizeof(TcBwdSmem::dop) &&
+                  offsetof(TcBwdSmem, kcm) == offsetof(TcBwdSmem, krm) + sizeof(TcBwdSmem::krm),
+              "A and B of the content path fit in dop .. kcm");
 
 __device__ int g_tc_bwd_timeout;
 __device__ int g_tc_bwd_bad_seqlens;   // set when a packed sequence's offsets are out of range
@@ -107,6 +115,12 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     const float amp = DEC ? decay_amp(a.A_dec, h) : 1.f;
     const float tb[2] = {DEC ? decay_bias(a.tau, h, c0, 128) : 0.f, DEC ? decay_bias(a.tau, h, c0 + 1, 128) : 0.f};
     float dtp[2] = {0.f, 0.f}, dap = 0.f;
+    // the content path's factors A [128][R] and B [R][128] of this head, brought in by a bulk copy
+    // at each gate chunk's first token into the dO and operand tiles (contiguous, 34,816 bytes,
+    // all consumed by then); lane j's write-gate factor
+    float *abuf = reinterpret_cast<float *>(sm.dop);
+    const float awj = (a.Aw && lane < R) ? a.Aw[(size_t)h * R + lane] : 0.f;
+    uint32_t ab_phase = 0;
 
     float ds[16][4];
 #pragma unroll
@@ -163,6 +177,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     if (tid == 0) {
         mbar_init(&sm.bar, 1);
         mbar_init(&sm.bar_s0, 1);
+        mbar_init(&sm.bar_ab, 1);
         fence_mbar_init();
     }
     if (tid < 128) {
@@ -881,6 +896,11 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         // with the boundary-state readout: the next chunk's state can come in now
         const bool s0_early = !(gate_start && a.mc_mode == 0);
         if (cc > 0 && s0_early) issue_s0(cc - 1);
+        if (gate_start && tid == 0) {
+            mbar_expect_tx(&sm.bar_ab, 256u * R * 4u);
+            bulk_g2s(abuf, a.A + (size_t)h * 128 * R, 128u * R * 4u, &sm.bar_ab);
+            bulk_g2s(abuf + 128 * R, a.Bm + (size_t)h * R * 128, 128u * R * 4u, &sm.bar_ab);
+        }
         // ---- reverse cumulative sum of dLam within the chunk, gate gradients.  Half-block
         //      totals first (the chunk's last-token term xl joins the last half), then each
         //      thread scans its 8 tokens from the total of everything after them.
@@ -989,34 +1009,38 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
         __syncthreads();
         // ---- content path at the gate chunk's first token
         if (gate_start) {
-            float bpre[16];   // B[h][half + 2x][tid / 2] (rank <= 32), issued before dz so that it overlaps it
-            {
-                const int vv = tid >> 1, half = tid & 1;
+            const float *As = abuf, *Bs = abuf + 128 * R;
+            const bool lost_ab = !mbar_wait(&sm.bar_ab, ab_phase, a.wait_limit);
+            if (warp == 0) {   // dz = A^T dDelta (+ Aw d(dw)): lane j over the 128 key channels
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (lane < R)
+#pragma unroll 8
+                    for (int i = 0; i < 128; i += 4)
 #pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    bpre[x] = half + 2 * x < R ? a.Bm[((size_t)h * R + half + 2 * x) * 128 + vv] : 0.f;
+                        for (int x = 0; x < 4; ++x) s4[x] += As[(i + x) * R + lane] * sm.ddelta[i + x];
+                if (lane < R) sm.dzv[lane] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + awj * sm.ddw;
             }
-            {   // dz = A^T dDelta (+ Aw d(dw)), 8 threads per output
-                const int j = tid / 8, part = tid % 8;
-                float s = 0.f;
-#pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    s += (j < R ? a.A[((size_t)h * 128 + part + 8 * x) * R + j] : 0.f) * sm.ddelta[part + 8 * x];
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                if (j < R && part == 0) sm.dzv[j] = s + (a.Aw ? a.Aw[(size_t)h * R + j] * sm.ddw : 0.f);
+            if (__syncthreads_or(lost_ab)) {   // the factor copy did not arrive: end the sweep; the
+                                               // copies that may still be in flight are waited for
+                if (tid == 0) {
+                    atomicOr(&g_tc_bwd_timeout, 4);
+                    mbar_wait(&sm.bar_ab, ab_phase, a.wait_limit);
+                    if (cc > 0) {
+                        mbar_wait(&sm.bar, phase, a.wait_limit);
+                        if (s0_early) mbar_wait(&sm.bar_s0, phase, a.wait_limit);
+                    }
+                }
+                return;
             }
-            __syncthreads();
+            ab_phase ^= 1u;
             if (tid < 128) wsg[(size_t)gc * kTcGradRec + tid] = sm.ddelta[tid];
             if (tid < R) wsg[(size_t)gc * kTcGradRec + 128 + tid] = sm.dzv[tid];
             if (tid == 0) wsg[(size_t)gc * kTcGradRec + kTcGradDw] = sm.ddw;
             {   // dm = B^T dz, two threads per output
                 const int vv = tid >> 1, half = tid & 1;
                 float sacc = 0.f;
-#pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    if (half + 2 * x < R) sacc += bpre[x] * sm.dzv[half + 2 * x];
+#pragma unroll 8
+                for (int j = half; j < R; j += 2) sacc += Bs[j * 128 + vv] * sm.dzv[j];
                 sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
                 if (half == 0) sm.dmv[vv] = sacc;
             }
