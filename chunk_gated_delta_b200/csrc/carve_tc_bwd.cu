@@ -74,6 +74,11 @@ struct __align__(16) TcBwdSmem {
 // the dynamic shared-memory limit of one CTA on sm_100 (227 KB); the content path's factors
 // (2 x 128 x rank floats) fit in the dO and operand tiles, which are contiguous
 static_assert(sizeof(TcBwdSmem) <= 232448, "shared memory");
+// rows of d g_logit / dbx (staged in dlam / rfac) and dv (drb) leave by 1-D bulk copies
+static_assert(offsetof(TcBwdSmem, dlam) % 16 == 0 && offsetof(TcBwdSmem, rfac) % 16 == 0 &&
+                  offsetof(TcBwdSmem, drb) % 16 == 0 && (kLdF * 4) % 16 == 0 && (kLdOp * 2) % 16 == 0,
+              "bulk-store sources on 16-byte boundaries");
+static_assert(offsetof(TcBwdSmem, dmv) % 16 == 0, "dm read as float4");
 static_assert(offsetof(TcBwdSmem, kcm) + sizeof(TcBwdSmem::kcm) - offsetof(TcBwdSmem, dop) >= 256 * kTcMaxRankBwd * 4 &&
                   offsetof(TcBwdSmem, qm) == offsetof(TcBwdSmem, dop) + sizeof(TcBwdSmem::dop) &&
                   offsetof(TcBwdSmem, kcm) == offsetof(TcBwdSmem, krm) + sizeof(TcBwdSmem::krm),
@@ -264,6 +269,9 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                         pack_bf16(ds[2 * q2 + 1][0], ds[2 * q2 + 1][1]),
                         pack_bf16(ds[2 * q2 + 1][2], ds[2 * q2 + 1][3]));
         }
+        // the previous chunk's gradient rows have left dlam / rfac / drb before the barrier below
+        // (those tiles are written again in this chunk)
+        if (lane < 4) bulk_wait_read<0>();
         {   // a wait that gives up ends the sweep of the whole CTA: recorded, the copies in flight
             // (this chunk's tiles and its start state) waited for once more, bounded, and left
             const bool lost = !mbar_wait(&sm.bar, phase, a.wait_limit);
@@ -273,6 +281,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     mbar_wait(&sm.bar, phase, a.wait_limit);
                     mbar_wait(&sm.bar_s0, phase, a.wait_limit);
                 }
+                if (lane < 4) bulk_wait<0>();
                 return;
             }
         }
@@ -433,6 +442,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 atomicOr(&g_tc_bwd_timeout, 2);
                 mbar_wait(&sm.bar_s0, phase, a.wait_limit);
             }
+            if (lane < 4) bulk_wait<0>();
             return;
         }
         phase ^= 1u;
@@ -936,11 +946,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
             if (tid == 0) sm.ddw += x;
         }
-        for (int idx = tid; idx < nv * 16; idx += 256) {   // dv = dR
-            const int t = idx >> 4, part = idx & 15;
-            *reinterpret_cast<uint4 *>(dv + base_bh + (size_t)(t0 + t) * tstride + part * 8) =
-                *reinterpret_cast<const uint4 *>(sm.drb + t * kLdOp + part * 8);
-        }
         __syncthreads();
         {
             float run[2] = {0.f, 0.f};
@@ -967,18 +972,21 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                     if (t == 7) run[e] += xl[e];
                     const float gx = e ? glr[t].y : glr[t].x, nb = -((e ? bxr[t].y : bxr[t].x) + dl[e]);   // nb = -beta
                     const float e2 = __expf(nb);
+                    // the unfloored retention and both sigmoids from the reciprocals 1 / (1 + e^x)
+                    const float rb = __fdividef(1.f, 1.f + e2), sb = nb > 15.f ? 1.f : e2 * rb;   // sigmoid(-beta)
                     if constexpr (DEC) {   // log g = -amp softplus(x), x = g_logit + tau: d/dx = -amp sigmoid(x)
                         const float x = gx + tb[e], e1 = __expf(x), sp = softplus_fast(x, e1);
-                        const float dla = run[e] * floor_scale(__fdividef(1.f, __expf(amp * sp) * (1.f + e2)), inert);
-                        dg[e] = -amp * sigmoid_fast(x, e1) * dla;
-                        db[e] = sigmoid_fast(nb, e2) * dla;
+                        const float ra = __fdividef(1.f, 1.f + e1);
+                        const float dla = run[e] * floor_scale(__expf(-amp * sp) * rb, inert);
+                        dg[e] = -amp * (x > 15.f ? 1.f : e1 * ra) * dla;
+                        db[e] = sb * dla;
                         dtp[e] += dg[e];
                         dap += dla * (-amp * sp);   // d A_dec = dlog a . log g
                     } else {
-                        const float e1 = __expf(gx);
-                        const float dla = run[e] * floor_scale(__fdividef(1.f, (1.f + e1) * (1.f + e2)), inert);
-                        dg[e] = -sigmoid_fast(gx, e1) * dla;
-                        db[e] = sigmoid_fast(nb, e2) * dla;
+                        const float e1 = __expf(gx), ra = __fdividef(1.f, 1.f + e1);
+                        const float dla = run[e] * floor_scale(ra * rb, inert);
+                        dg[e] = -(gx > 15.f ? 1.f : e1 * ra) * dla;
+                        db[e] = sb * dla;
                     }
                     pdd[e] += db[e];
                 }
@@ -992,33 +1000,35 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             load_gates(cc - 1);
             load_w(cc - 1);
         }
+        fence_proxy_async_smem();   // dg / db (and dR, written earlier) are read by bulk copies next
         __syncthreads();
+        if (lane < 4) {   // d g_logit, dbx and dv of token 4 warp + lane: one bulk copy per row
+            const int t = 4 * warp + lane;
+            if (!VL || t < nv) {
+                const size_t gi = base_bh + (size_t)(t0 + t) * tstride;
+                bulk_s2g(a.dg_logit + gi, sm.dlam + t * kLdF, 128u * 4u);
+                bulk_s2g(a.dbx + gi, sm.rfac + t * kLdF, 128u * 4u);
+                bulk_s2g(dv + gi, sm.drb + t * kLdOp, 128u * 2u);
+            }
+            bulk_commit();
+        }
         if (tid < 128) {
             float x = 0.f;
 #pragma unroll
             for (int h2 = 0; h2 < 2 * NB; ++h2) x += sm.pdd[h2 * 128 + tid];
             sm.ddelta[tid] += x;
         }
-        for (int idx = tid; idx < nv * 32; idx += 256) {   // d g_logit, dbx: four channels per store
-            const int t = idx >> 5, c = (idx & 31) * 4;
-            const float *gsrc = sm.dlam + t * kLdF + c, *bsrc = sm.rfac + t * kLdF + c;
-            const size_t gi = base_bh + (size_t)(t0 + t) * tstride + c;
-            *reinterpret_cast<float4 *>(a.dg_logit + gi) = *reinterpret_cast<const float4 *>(gsrc);
-            *reinterpret_cast<float4 *>(a.dbx + gi) = *reinterpret_cast<const float4 *>(bsrc);
-        }
-        __syncthreads();
-        // ---- content path at the gate chunk's first token
+        // ---- content path at the gate chunk's first token (the other chunks need no barrier
+        //      here: nothing read below this point is written before the next chunk's first one)
         if (gate_start) {
+            __syncthreads();
             const float *As = abuf, *Bs = abuf + 128 * R;
             const bool lost_ab = !mbar_wait(&sm.bar_ab, ab_phase, a.wait_limit);
-            if (warp == 0) {   // dz = A^T dDelta (+ Aw d(dw)): lane j over the 128 key channels
-                float s4[4] = {0.f, 0.f, 0.f, 0.f};
-                if (lane < R)
-#pragma unroll 8
-                    for (int i = 0; i < 128; i += 4)
+            if (lane < R) {   // dz = A^T dDelta: lane j, key channels warp + 8 i, partial per warp
+                float s2[2] = {0.f, 0.f};
 #pragma unroll
-                        for (int x = 0; x < 4; ++x) s4[x] += As[(i + x) * R + lane] * sm.ddelta[i + x];
-                if (lane < R) sm.dzv[lane] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + awj * sm.ddw;
+                for (int i = 0; i < 16; ++i) s2[i & 1] += As[(warp + 8 * i) * R + lane] * sm.ddelta[warp + 8 * i];
+                sm.xp[warp * 32 + lane] = s2[0] + s2[1];
             }
             if (__syncthreads_or(lost_ab)) {   // the factor copy did not arrive: end the sweep; the
                                                // copies that may still be in flight are waited for
@@ -1030,12 +1040,20 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                         if (s0_early) mbar_wait(&sm.bar_s0, phase, a.wait_limit);
                     }
                 }
+                if (lane < 4) bulk_wait<0>();
                 return;
             }
             ab_phase ^= 1u;
+            if (tid < R) {   // the eight partials (+ Aw d(dw))
+                float z = awj * sm.ddw;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) z += sm.xp[w * 32 + tid];
+                sm.dzv[tid] = z;
+                wsg[(size_t)gc * kTcGradRec + 128 + tid] = z;
+            }
             if (tid < 128) wsg[(size_t)gc * kTcGradRec + tid] = sm.ddelta[tid];
-            if (tid < R) wsg[(size_t)gc * kTcGradRec + 128 + tid] = sm.dzv[tid];
             if (tid == 0) wsg[(size_t)gc * kTcGradRec + kTcGradDw] = sm.ddw;
+            __syncthreads();
             {   // dm = B^T dz, two threads per output
                 const int vv = tid >> 1, half = tid & 1;
                 float sacc = 0.f;
@@ -1048,22 +1066,34 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
             if (a.mc_mode == 0) {
                 // m = S0 qbar:  dS0 += dm qbar^T here;  dq_t += S0^T dm / n for every t of the gate
                 // chunk is added by the readout pass after this kernel (vector stored per gate chunk)
-                {
-                    const int ch = tid & 127, half = tid >> 7;
-                    int off[8];   // column of `ch` in a swizzled row r with r mod 8 = x
+                {   // S0^T dm: channel pair 2 cp, 2 cp + 1 over rows 32 rq .. 32 rq + 31
+                    const int cpr = tid & 63, rq = tid >> 6;
+                    int off[8];   // the pair's column in a swizzled row r with r mod 8 = x
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) off[x] = ((((ch >> 3) ^ x) << 3) | (ch & 7));
-                    float sa[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    for (int x = 0; x < 8; ++x) off[x] = ((((cpr >> 2) ^ x) << 3) | ((2 * cpr) & 7));
+                    float sa[4][2] = {};
 #pragma unroll
-                    for (int r = 0; r < 64; r += 8)
+                    for (int r = 0; r < 32; r += 8)
 #pragma unroll
-                        for (int x = 0; x < 8; ++x)
-                            sa[x] += bf(sm.s0b[(64 * half + r + x) * 128 + off[x]]) * sm.dmv[64 * half + r + x];
-                    sm.pdd[half * 128 + ch] = ((sa[0] + sa[1]) + (sa[2] + sa[3])) + ((sa[4] + sa[5]) + (sa[6] + sa[7]));
+                        for (int x4 = 0; x4 < 2; ++x4) {
+                            const float4 m4 = *reinterpret_cast<const float4 *>(sm.dmv + 32 * rq + r + 4 * x4);
+                            const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                            for (int y = 0; y < 4; ++y) {
+                                const int x = 4 * x4 + y;
+                                const __nv_bfloat162 s2 =
+                                    *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + (32 * rq + r + x) * 128 + off[x]);
+                                sa[y][0] += bf(s2.x) * mv[y];
+                                sa[y][1] += bf(s2.y) * mv[y];
+                            }
+                        }
+                    *reinterpret_cast<float2 *>(sm.pdd + rq * 128 + 2 * cpr) =
+                        make_float2((sa[0][0] + sa[1][0]) + (sa[2][0] + sa[3][0]), (sa[0][1] + sa[1][1]) + (sa[2][1] + sa[3][1]));
                 }
                 __syncthreads();
                 if (tid < 128) {
-                    wsv[(size_t)gc * 128 + tid] = (sm.pdd[tid] + sm.pdd[128 + tid]) / (float)n;
+                    wsv[(size_t)gc * 128 + tid] =
+                        ((sm.pdd[tid] + sm.pdd[128 + tid]) + (sm.pdd[256 + tid] + sm.pdd[384 + tid])) / (float)n;
                     sm.dox[tid] = 0.f;
                 }
                 const float m0 = sm.dmv[v0], m1 = sm.dmv[v1];
@@ -1080,12 +1110,11 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 sm.dox[tid] = gc > 0 ? sm.dmv[tid] / (float)L : 0.f;
                 if (gc == 0 && a.dm_prev_in) a.dm_prev_in[(size_t)u * 128 + tid] = sm.dmv[tid];
             }
-        }
-        __syncthreads();
-        if (cc > 0) {
-            if (!s0_early) issue_s0(cc - 1);
+            __syncthreads();
+            if (cc > 0 && !s0_early) issue_s0(cc - 1);
         }
     }
+    if (lane < 4) bulk_wait<0>();   // the last gradient rows are written before the CTA ends
     if (a.dS0) {
         float *D = a.dS0 + (size_t)u * 128 * 128;
 #pragma unroll

@@ -31,10 +31,9 @@ __device__ __forceinline__ float floor_scale(float r, bool inert) {
     return inert ? 0.f : (r >= kAMin ? 1.f : r * kInvAMin);
 }
 
-// softplus(x) and sigmoid(x) from one fast exponential; beyond x = 15, log(1 + e^x) is x and
-// sigmoid(x) is 1 to fp32 rounding (and e^x may overflow), so both take those values there
+// softplus(x) from one fast exponential e1 = e^x; beyond x = 15, log(1 + e^x) is x to fp32
+// rounding (and e^x may overflow), so it takes that value there (sigmoid(x) likewise takes 1)
 __device__ __forceinline__ float softplus_fast(float x, float e1) { return x > 15.f ? x : __logf(1.f + e1); }
-__device__ __forceinline__ float sigmoid_fast(float x, float e1) { return x > 15.f ? 1.f : __fdividef(e1, 1.f + e1); }
 
 // The same with the decay's amplitude and bias: 1 / g = e^{amp softplus(x)}, x = g_logit + tau
 // (the product form above is its amp = 1, tau = 0 case, evaluated with fewer operations).
