@@ -36,6 +36,7 @@
 // retention floor binds, the gradient of log a is scaled to the exact recurrence's
 // (floor_scale) instead of being dropped.
 #include "carve_tc_common.cuh"
+#include "carve_umma.cuh"
 
 namespace carve {
 
@@ -55,7 +56,7 @@ struct __align__(16) TcBwdSmem {
     __nv_bfloat16 rq[kBC * 128], rk[kBC * 128], rv[kBC * 128], rdo[kBC * 128];
     __nv_bfloat16 dop[kBC * kLdOp];
     __nv_bfloat16 qm[kBC * kLdOp], krm[kBC * kLdOp], kcm[kBC * kLdOp];
-    __nv_bfloat16 s0b[128 * 128], ds1b[128 * kLdOp];   // s0b: the saved state as written (swizzled rows)
+    __nv_bfloat16 s0b[128 * 128], ds1b[128 * kLdOp];   // s0b: the saved state as written (tensor-core layout)
     __nv_bfloat16 ub[kBC * kLdOp], drb[kBC * kLdOp];
     __nv_bfloat16 aqk[kBC * kLdT], akk[kBC * kLdT], mkk[kBC * kLdT], daqk[kBC * kLdT], dakk[kBC * kLdT];
     __nv_bfloat16 tii[kBNB * 16 * 24];
@@ -107,7 +108,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
     const size_t tstride = (size_t)H * 128;
     const size_t base_bh = ((size_t)bb * T + toff) * tstride + (size_t)h * 128;
     const int v0 = 16 * warp + g, v1 = v0 + 8;
-    // bf16 chunk-start states written by the forward: 128 rows of 256 bytes, 16-byte chunks swizzled
+    // bf16 chunk-start states written by the forward: 128 rows in the tensor core's 128-byte-swizzle
+    // operand layout (two 64-column halves of 128-byte rows)
     const __nv_bfloat16 *states = reinterpret_cast<const __nv_bfloat16 *>(a.saved_states) + (size_t)u * NCC * 128 * 128;
     // workspace: per gate chunk dDelta (128) and dz (32) for the dA / dB reduction, then the
     // readout vectors of dq (128 per gate chunk)
@@ -149,8 +151,8 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int col = 8 * j + 2 * c4;
-            const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + swz128(v0, col));
-            const __nv_bfloat162 s1 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + swz128(v1, col));
+            const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + umma_off(v0, col, 128));
+            const __nv_bfloat162 s1 = *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + umma_off(v1, col, 128));
             v[j][0] = ds[j][0] * bf(s0.x) + ds[j][2] * bf(s1.x);
             v[j][1] = ds[j][1] * bf(s0.y) + ds[j][3] * bf(s1.y);
         }
@@ -513,7 +515,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             uint32_t af[4];
-            load_a_swz(af, sm.s0b, 16 * warp, 16 * ks, lane);
+            load_a_um(af, sm.s0b, 128, 16 * warp, 16 * ks, lane);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bfr[4];
@@ -766,7 +768,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 for (int np2 = 0; np2 < 2; ++np2) {
                     const int n0 = ch0 + 16 * np2;
                     uint32_t bs[4], bd[4];
-                    load_b_kn_swz(bs, sm.s0b, n0, 16 * ks, lane);
+                    load_b_kn_um(bs, sm.s0b, 128, n0, 16 * ks, lane);
                     load_b_kn(bd, sm.ds1b, kLdOp, n0, 16 * ks, lane);
                     mma_bf16(gq[2 * np2], ao, bs[0], bs[1]);
                     mma_bf16(gq[2 * np2 + 1], ao, bs[2], bs[3]);
@@ -1068,9 +1070,6 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                 // chunk is added by the readout pass after this kernel (vector stored per gate chunk)
                 {   // S0^T dm: channel pair 2 cp, 2 cp + 1 over rows 32 rq .. 32 rq + 31
                     const int cpr = tid & 63, rq = tid >> 6;
-                    int off[8];   // the pair's column in a swizzled row r with r mod 8 = x
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) off[x] = ((((cpr >> 2) ^ x) << 3) | ((2 * cpr) & 7));
                     float sa[4][2] = {};
 #pragma unroll
                     for (int r = 0; r < 32; r += 8)
@@ -1082,7 +1081,7 @@ __global__ void __launch_bounds__(256, 1) tc_bwd_kernel(BwdArgs a, const __grid_
                             for (int y = 0; y < 4; ++y) {
                                 const int x = 4 * x4 + y;
                                 const __nv_bfloat162 s2 =
-                                    *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + (32 * rq + r + x) * 128 + off[x]);
+                                    *reinterpret_cast<const __nv_bfloat162 *>(sm.s0b + umma_off(32 * rq + r + x, 2 * cpr, 128));
                                 sa[y][0] += bf(s2.x) * mv[y];
                                 sa[y][1] += bf(s2.y) * mv[y];
                             }

@@ -30,6 +30,7 @@
 // through one bulk copy.  The floor a >= e^-10 bounds the deviation from the exact recurrence
 // by e^-10 per step in channels that are being erased anyway.
 #include "carve_tc_common.cuh"
+#include "carve_umma.cuh"
 
 namespace carve {
 
@@ -47,12 +48,18 @@ struct __align__(16) TcFwdSmem {
     static constexpr int ST = NB == 2 ? 2 : 1;
     static constexpr bool GT = NB == 2;
     static constexpr int GSZ = GT ? C * 128 : 4;
+    // 32-token chunks: G = S0 [Kt; Qt]^T on the 5th-generation tensor core (one M = 128, N = 64,
+    // K = 128 product per chunk, accumulator in TMEM), both operands in the tensor core's
+    // 128-byte-swizzle layout
+    static constexpr bool UM = NB == 2;
     // raw tiles by TMA; a stage's two gate-logit tiles (32 KB with 32-token chunks) carry the
-    // bf16 chunk-start state on its way out once the gate phase has read them
+    // bf16 chunk-start state (the A operand of G, and the state saved for the backward) once
+    // the gate phase has read them
     __nv_bfloat16 rq[ST][C * 128], rk[ST][C * 128], rv[ST][C * 128];
     float rgx[ST][2][GSZ];
+    __nv_bfloat16 ktq[UM ? 2 * C * 128 : 8];   // [Kt; Qt]: the B operand of G
     // mid-block referenced operands; qm doubles as the output tile once the Gram has used it
-    __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp], qt[C * kLdOp], kt[C * kLdOp];
+    __nv_bfloat16 qm[C * kLdOp], krm[C * kLdOp], kcm[C * kLdOp], qt[UM ? 8 : C * kLdOp], kt[UM ? 8 : C * kLdOp];
     __nv_bfloat16 aqk[C * LDA], mkk[C * LDA];
     __nv_bfloat16 tii[NB * 16 * 24];
     float akk_d[NB * 16 * 17];
@@ -61,11 +68,21 @@ struct __align__(16) TcFwdSmem {
     float zp[8 * 32], dpart[2 * 128];   // content signal: per-warp parts of z, two parts of Delta
     float AhT[kTcMaxRank * 128], BhT[128 * kTcMaxRank];   // the head's factors: A^T [j][k], B^T [v][j]
     uint64_t bar[ST];
+    uint64_t mma_bar;   // completion of G on the tensor core
+    uint32_t tmem;      // TMEM base address of G's accumulator (64 columns)
     __device__ __nv_bfloat16 *ost() { return qm; }
 };
 // the dynamic shared-memory limit of one CTA on sm_100 (227 KB)
 static_assert(sizeof(TcFwdSmem<2>) <= 232448 && sizeof(TcFwdSmem<4>) <= 232448, "shared memory");
 static_assert(sizeof(TcFwdSmem<2>::rgx[0]) == 128 * 128 * 2, "a stage's gate tiles hold one bf16 state");
+// tensor-core operands start on 1024-byte boundaries (the dynamic shared memory base is checked
+// at run time)
+static_assert(offsetof(TcFwdSmem<2>, rgx) % 1024 == 0 && sizeof(TcFwdSmem<2>::rgx[0]) % 1024 == 0 &&
+                  offsetof(TcFwdSmem<2>, ktq) % 1024 == 0,
+              "tensor-core operand alignment");
+static_assert(offsetof(TcFwdSmem<2>, p7) % 16 == 0 && offsetof(TcFwdSmem<2>, r15) % 16 == 0 &&
+                  offsetof(TcFwdSmem<2>, qm) % 16 == 0 && offsetof(TcFwdSmem<2>, krm) % 16 == 0,
+              "decay factors and operands read as 16-byte vectors");
 
 struct TileMaps {
     CUtensorMap q, k, v, gl, bx;
@@ -92,7 +109,10 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
     const size_t tstride = (size_t)H * 128;
     const size_t base_bh = ((size_t)bb * T + toff) * tstride + (size_t)h * 128;   // token 0 of this unit
-    const int v0 = 16 * warp + g, v1 = v0 + 8;
+    // this warp's 16 state rows: with the tensor-core G, the rows whose TMEM lanes the warp may
+    // read (lane quarter warp % 4, half warp / 4)
+    const int vb = SM::UM ? 32 * (warp & 3) + 16 * (warp >> 2) : 16 * warp;
+    const int v0 = vb + g, v1 = v0 + 8;
     const bool save = SM::GT && a.saved_states != nullptr;   // the bf16 chunk-start states for the backward
     __nv_bfloat16 *states = save ? reinterpret_cast<__nv_bfloat16 *>(a.saved_states) : nullptr;
     // the decay's amplitude and the biases of this thread's gate channels 2 (tid & 63) + {0, 1}
@@ -114,7 +134,16 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
         }
     }
+    if (SM::UM && (smem_u32(smraw) & 1023u)) {   // operand layout needs a 1024-byte aligned base
+        if (tid == 0) atomicOr(&g_tc_timeout, 4);
+        return;
+    }
+    if (SM::UM && warp == 0) {
+        tmem_alloc(&sm.tmem, 64);
+        tc_fence_before_sync();
+    }
     if (tid == 0) {
+        if (SM::UM) mbar_init(&sm.mma_bar, 1);
         for (int i = 0; i < SM::ST; ++i) mbar_init(&sm.bar[i], 1);
         fence_mbar_init();
     }
@@ -129,6 +158,11 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         sm.BhT[idx] = j2 < R ? a.Bm[((size_t)h * R + j2) * 128 + v] : 0.f;
     }
     __syncthreads();
+    uint32_t tmem = 0, mma_phase = 0;   // G's accumulator; parity of the G product to wait for
+    if (SM::UM) {
+        tc_fence_after_sync();
+        tmem = sm.tmem;
+    }
 
     // Input tiles of chunk cc by TMA (one tensor copy per tile) into stage cc % ST.  With two
     // stages everything is issued at once, one chunk ahead; with one stage q/k (which = 0,
@@ -213,6 +247,10 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                     atomicOr(&g_tc_timeout, 1);
                     mbar_wait(&sm.bar[st], (phase_bits >> st) & 1u, a.wait_limit);
                 }
+                if (SM::UM && warp == 0) {   // no product is in flight at a chunk's start
+                    tc_fence_after_sync();
+                    tmem_dealloc(tmem, 64);
+                }
                 return;
             }
         }
@@ -277,8 +315,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
 #pragma unroll
                 for (int r = 0; r < 8; ++r) {
                     const float ma = __shfl_sync(0xffffffffu, p0, 4 * r), mb = __shfl_sync(0xffffffffu, p1, 4 * r);
-                    zz += sm.BhT[(16 * warp + r) * kTcMaxRank + lane] * ma +
-                          sm.BhT[(16 * warp + 8 + r) * kTcMaxRank + lane] * mb;
+                    zz += sm.BhT[(vb + r) * kTcMaxRank + lane] * ma + sm.BhT[(vb + 8 + r) * kTcMaxRank + lane] * mb;
                 }
                 sm.zp[warp * 32 + lane] = zz;
             }
@@ -386,32 +423,53 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         if (tid < C) sm.wv[tid] = (!VL || tid < nv) ? sigmoid_f(wcur + dwc) : 0.f;
         __syncthreads();
         __nv_bfloat16 *stile = reinterpret_cast<__nv_bfloat16 *>(sm.rgx[st]);
-        if (save) {   // bf16 chunk-start state into the stage's gate tiles (read above): this warp's
-                      // 16 rows, 256-byte rows with their 16-byte chunks swizzled
+        if (SM::UM) {   // bf16 chunk-start state into the stage's gate tiles (read above): this warp's
+                        // 16 rows, in the tensor core's operand layout (the A operand of G, and the
+                        // state saved for the backward)
             const int mi = lane >> 3, r = lane & 7;   // lane l addresses row r of matrix mi of each x4
-            const int row = 16 * warp + 8 * (mi & 1) + r;
+            const int row = vb + 8 * (mi & 1) + r;
 #pragma unroll
             for (int q2 = 0; q2 < 8; ++q2)   // key columns 16 q2 .. 16 q2 + 15
-                stsm_x4(smem_u32(stile + swz128(row, 16 * q2 + 8 * (mi >> 1))), pack_bf16(s[2 * q2][0], s[2 * q2][1]),
+                stsm_x4(smem_u32(stile + umma_off(row, 16 * q2 + 8 * (mi >> 1), 128)), pack_bf16(s[2 * q2][0], s[2 * q2][1]),
                         pack_bf16(s[2 * q2][2], s[2 * q2][3]), pack_bf16(s[2 * q2 + 1][0], s[2 * q2 + 1][1]),
                         pack_bf16(s[2 * q2 + 1][2], s[2 * q2 + 1][3]));
-            fence_proxy_async_smem();   // read by the bulk copy below, overwritten by a later tile copy
         }
-        // ---- decayed operands Qt = Qm Em, Kt = Krm Em: one (channel, 16-token block) item per
-        //      thread, each forming its own prefix of block decays; chunk-level factors per
-        //      channel alongside
+        // ---- decayed operands Qt = Qm Em, Kt = Krm Em (chunk-level factors per channel alongside)
+        if constexpr (SM::UM) {   // into [Kt; Qt] (rows 0 .. C-1: Kt, C .. 2C-1: Qt): one (channel,
+                                  // 16-token block) item per thread; a row's chunk position in the
+                                  // operand layout depends on the token index mod 8 alone
+            const int ch = tid & 127, i = tid >> 7, cc = (ch >> 3) & 7;
+            float E = 1.f;
+            for (int j = 0; j < i; ++j) E *= sm.p7[j * 128 + ch] * sm.r15[j * 128 + ch];
+            const float em = E * sm.p7[i * 128 + ch];
+            __nv_bfloat16 kv[16], qv[16];   // all loads first (the stores below go through a pointer)
 #pragma unroll
-        for (int x = 0; x < NP; ++x) {
-            const int p = tid + 256 * x, ch = p & 127, i = p >> 7;
-            if (p < 128 * NB) {
-                float E = 1.f;
-                for (int j = 0; j < i; ++j) E *= sm.p7[j * 128 + ch] * sm.r15[j * 128 + ch];
-                const float em = E * sm.p7[i * 128 + ch];
+            for (int t = 0; t < 16; ++t) {
+                const int row = 16 * i + t;
+                kv[t] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+                qv[t] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
+            }
+            __nv_bfloat16 *kb = sm.ktq + (ch >> 6) * (2 * C * 64) + 16 * i * 64 + (ch & 7);
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int row = 16 * i + t;
-                    sm.qt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
-                    sm.kt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+            for (int t = 0; t < 16; ++t) {
+                const int o = t * 64 + ((cc ^ (t & 7)) << 3);
+                kb[o] = kv[t];
+                kb[o + C * 64] = qv[t];
+            }
+        } else {   // one (channel, 16-token block) item per thread
+#pragma unroll
+            for (int x = 0; x < NP; ++x) {
+                const int p = tid + 256 * x, ch = p & 127, i = p >> 7;
+                if (p < 128 * NB) {
+                    float E = 1.f;
+                    for (int j = 0; j < i; ++j) E *= sm.p7[j * 128 + ch] * sm.r15[j * 128 + ch];
+                    const float em = E * sm.p7[i * 128 + ch];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        const int row = 16 * i + t;
+                        sm.qt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.qm[row * kLdOp + ch]) * em);
+                        sm.kt[row * kLdOp + ch] = __float2bfloat16_rn(bf(sm.krm[row * kLdOp + ch]) * em);
+                    }
                 }
             }
         }
@@ -442,7 +500,23 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 }
             }
         }
+        if (SM::UM) fence_proxy_async_smem();   // the state and [Kt; Qt] tiles are read by the tensor
+                                                // core and the state copy below
         __syncthreads();
+        if (SM::UM && tid == 224) {   // G = S0 [Kt; Qt]^T, issued by warp 7 (no Gram block): eight
+                                      // K = 16 slices, each half of the 128-byte-swizzled rows
+                                      // holding four of them
+            tc_fence_after_sync();
+            const uint32_t a0 = smem_u32(stile), b0 = smem_u32(sm.ktq);
+            constexpr uint32_t idesc = umma_idesc_bf16(128, 2 * C);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t off = (uint32_t)(ks & 3) * 32u;
+                umma_bf16(tmem, umma_desc(a0 + (uint32_t)(ks >> 2) * (128u * 128u) + off),
+                          umma_desc(b0 + (uint32_t)(ks >> 2) * (2u * C * 128u) + off), idesc, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.mma_bar);
+        }
         if (save && tid == 0) {   // the chunk-start state, written to the stage's gate tiles above
             bulk_s2g(states + ((size_t)u * NCC + cc) * 128 * 128, stile, 128u * 128u * 2u);
             bulk_commit();
@@ -509,24 +583,45 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
         }
         // ---- G = S0 [Kt; Qt]^T  (rows v of this warp)
         float ga[4 * NB][4];
-#pragma unroll
-        for (int j = 0; j < 4 * NB; ++j) ga[j][0] = ga[j][1] = ga[j][2] = ga[j][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            uint32_t af[4];
-            af[0] = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
-            af[1] = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
-            af[2] = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-            af[3] = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
-#pragma unroll
-            for (int np = 0; np < 2 * NB; ++np) {
-                uint32_t bfr[4];
-                load_b_nk(bfr, np < NB ? sm.kt : sm.qt, kLdOp, 16 * (np % NB), 16 * ks, lane);
-                mma_bf16(ga[2 * np], af, bfr[0], bfr[1]);
-                mma_bf16(ga[2 * np + 1], af, bfr[2], bfr[3]);
+        if constexpr (SM::UM) {   // from the tensor core: wait for the product, load this warp's rows
+            const bool lost = __any_sync(0xffffffffu, !mbar_wait(&sm.mma_bar, mma_phase, a.wait_limit));
+            mma_phase ^= 1u;
+            tc_fence_after_sync();
+            if (!lost) tmem_ld_frags8(tmem + ((uint32_t)vb << 16), ga);
+            tc_fence_before_sync();
+            if (__syncthreads_or(lost)) {   // the product did not complete: recorded, waited for once
+                                            // more (bounded), TMEM freed, the sweep left
+                if (tid == 0) {
+                    atomicOr(&g_tc_timeout, 2);
+                    mbar_wait(&sm.mma_bar, mma_phase ^ 1u, a.wait_limit);
+                    if (save) bulk_wait<0>();
+                }
+                if (warp == 0) {
+                    tc_fence_after_sync();
+                    tmem_dealloc(tmem, 64);
+                }
+                return;
             }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4 * NB; ++j) ga[j][0] = ga[j][1] = ga[j][2] = ga[j][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t af[4];
+                af[0] = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
+                af[1] = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
+                af[2] = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+                af[3] = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+                for (int np = 0; np < 2 * NB; ++np) {
+                    uint32_t bfr[4];
+                    load_b_nk(bfr, np < NB ? sm.kt : sm.qt, kLdOp, 16 * (np % NB), 16 * ks, lane);
+                    mma_bf16(ga[2 * np], af, bfr[0], bfr[1]);
+                    mma_bf16(ga[2 * np + 1], af, bfr[2], bfr[3]);
+                }
+            }
+            __syncthreads();
         }
-        __syncthreads();
         if (SM::ST == 1 && cc + 1 < NCCn) issue(cc + 1, 0);
         // ---- X = Diag(w)(V - Kt S0^T), as X^T (rows v, cols t)
 #pragma unroll
@@ -589,7 +684,7 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                 os0 += y[0] + y[1];
                 os1 += y[2] + y[3];
             }
-            store_frags_t<2 * NB>(sm.ost(), kLdOp, 16 * warp, ga + 2 * NB, lane);   // O^T -> [t][v]
+            store_frags_t<2 * NB>(sm.ost(), kLdOp, vb, ga + 2 * NB, lane);   // O^T -> [t][v]
             os0 += __shfl_xor_sync(0xffffffffu, os0, 1);
             os0 += __shfl_xor_sync(0xffffffffu, os0, 2);
             os1 += __shfl_xor_sync(0xffffffffu, os1, 1);
@@ -652,6 +747,10 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     }
     if (a.m_prev_out && tid < 128) a.m_prev_out[(size_t)u * 128 + tid] = sm.mprev[tid];
     if (save && tid == 0) bulk_wait<0>();   // the state copies are complete before the CTA ends
+    if (SM::UM && warp == 0) {   // every warp's last load of G came before the last chunk's barriers
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 64);
+    }
 }
 
 // Per (batch, gate chunk): mean of q over the gate chunk's tokens for every head, into the saved
