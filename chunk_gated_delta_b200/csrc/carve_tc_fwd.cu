@@ -2,9 +2,11 @@
 //
 // One CTA (8 warps) per (batch, head) unit sweeps the sequence in compute chunks of
 // C = 16*NB tokens (C = min(chunk, 64); a 128-token gate chunk is two compute chunks sharing
-// one content signal).  Warp w owns state rows v in [16w, 16w+16): its 16x128 slice of the
-// fp32 state lives in registers as mma accumulator fragments for the whole sweep, so the
-// state never round-trips through memory except when it is saved for the backward.
+// one content signal).  Each warp owns 16 state rows (rows [16w, 16w+16) with 64-token chunks;
+// with 32-token chunks rows 32 (w % 4) + 16 (w / 4) + [0, 16), the TMEM lanes the warp may
+// read): its 16x128 slice of the fp32 state lives in registers as mma accumulator fragments for
+// the whole sweep, so the state never round-trips through memory except when it is saved for
+// the backward (and, as a bf16 tile, read by the tensor core).
 //
 // Per compute chunk (CARVE blog section 2.3: one WY solve shared by all value channels):
 //   gates      a_t = 1 / ((1 + e^{g_logit})(1 + e^{-(bx + Delta)})) (with the decay amplitude and
@@ -17,7 +19,10 @@
 //   Gram       Akk, Aqk: block (i,j) = rows_i . diag(e^{Lam_m(i) - Lam_m(j)}) . cols_j^T, the factor
 //              split between the row operand (decay to block i's middle from block i's start)
 //              and the column operand (the rest), so that neither part underflows alone
-//   G          S0 [Kt; Qt]^T   (Kt = k e^{Lam}, Qt = q e^{Lam})            per warp, mma
+//   G          S0 [Kt; Qt]^T   (Kt = k e^{Lam}, Qt = q e^{Lam}); 32-token chunks: one tcgen05
+//              MMA (M = 128, N = 64, K = 128) from the bf16 state tile and [Kt; Qt] in shared
+//              memory, accumulator in TMEM, read back by each warp as mma fragments;
+//              64-token chunks: per warp, mma
 //   solve      X = Diag(w)(V - Kt S0^T);  U_i = (X_i - sum_j U_j M_ij^T) T_ii^T,  T_ii = (I + D A_ii)^-1
 //   output     O^T = S0 Qt^T + U^T Aqk^T                                  per warp, mma
 //   state      S = S Diag(gamma) + U^T Kbar,  Kbar = k e^{Lam_C - Lam}         per warp, mma
