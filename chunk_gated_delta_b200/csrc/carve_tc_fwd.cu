@@ -172,8 +172,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
     // Input tiles of chunk cc by TMA (one tensor copy per tile) into stage cc % ST.  With two
     // stages everything is issued at once, one chunk ahead; with one stage q/k (which = 0,
     // arming the barrier) go out mid-chunk and v (which = 1) at the end of the previous chunk.
-    auto issue = [&](int cc, int which) {
-        if (tid != 0) return;
+    auto issue = [&](int cc, int which, int by = 0) {   // by: the issuing thread
+        if (tid != by) return;
         const int row = bb * T + toff + cc * C, st = cc % SM::ST;
         uint64_t *bar = &sm.bar[st];
         if (which == 0) {
@@ -260,7 +260,6 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             }
         }
         phase_bits ^= 1u << st;
-        if (SM::ST == 2 && cc + 1 < NCCn) issue(cc + 1, 0);   // the other stage is free since last chunk
         if constexpr (VL) {
             if (nv < C) {   // rows past the sequence's end (another sequence's, or zero fill): cleared
                 for (int idx = tid; idx < (C - nv) * 16; idx += 256) {
@@ -522,6 +521,10 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
             }
             umma_commit(&sm.mma_bar);
         }
+        // the other stage's tiles were last read in the previous chunk (its state copy has been
+        // waited for before this chunk's first barrier): the next chunk's tiles go there, issued
+        // by warp 6, which has no Gram block to form next
+        if (SM::ST == 2 && cc + 1 < NCCn) issue(cc + 1, 0, 192);
         if (save && tid == 0) {   // the chunk-start state, written to the stage's gate tiles above
             bulk_s2g(states + ((size_t)u * NCC + cc) * 128 * 128, stile, 128u * 128u * 2u);
             bulk_commit();
@@ -600,6 +603,8 @@ __global__ void __launch_bounds__(256, 1) tc_fwd_kernel(FwdArgs a, const __grid_
                     atomicOr(&g_tc_timeout, 2);
                     mbar_wait(&sm.mma_bar, mma_phase ^ 1u, a.wait_limit);
                     if (save) bulk_wait<0>();
+                    if (SM::ST == 2 && cc + 1 < NCCn)   // the next chunk's tiles, issued above
+                        mbar_wait(&sm.bar[(cc + 1) % SM::ST], (phase_bits >> ((cc + 1) % SM::ST)) & 1u, a.wait_limit);
                 }
                 if (warp == 0) {
                     tc_fence_after_sync();
