@@ -388,6 +388,9 @@ def measure_train(args, w, ws, rank, local, fwd_only=False):
     achieved = dbytes / (dms * 1e-3) / 1e9
     flops = (fwd_flops(dd, L, w.R) + (0 if fwd_only else bwd_flops(dd, L, w.R))) * th * ws
     tensor_frac = flops / (ms * 1e-3) / (peaks["bf16"] * 1e12 * ws)
+    kflops = {"carve_fwd": fwd_flops(dd, L, w.R) * th}
+    if not fwd_only:
+        kflops["carve_bwd"] = bwd_flops(dd, L, w.R) * th
     traffic = None if (opt or packed) else load_traffic(w.name, dom)
 
     e2e = None
@@ -414,6 +417,7 @@ def measure_train(args, w, ws, rank, local, fwd_only=False):
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm"], "traffic": traffic, "peak_source": peaks["source"]},
         "kernels_ms": {"carve_fwd": fwd_ms, "carve_bwd": bwd_ms},
+        "per_kernel": kernel_rooflines(kern, kflops, peaks),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, fwd_only, args.decay) * args.steps,
         "clocks": clk.summary(),
     }
@@ -573,6 +577,19 @@ def run_deviation(args, w):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def kernel_rooflines(kern, flops, peaks):
+    """Per ABI call: its CUDA-event time, algorithmic HBM rate and bf16 tensor rate, each with its
+    fraction of the peak.  kern: call -> (ms, algorithmic bytes); flops: call -> FLOPs."""
+    out = {}
+    for k, (kms, kbytes) in kern.items():
+        sec = kms * 1e-3
+        gbs = kbytes / sec / 1e9
+        tfs = flops[k] / sec / 1e12
+        out[k] = {"ms": kms, "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm"], "tflops": tfs,
+                  "tensor_frac": tfs / peaks["bf16"]}
+    return out
 
 
 def load_traffic(workload, call):

@@ -42,3 +42,16 @@ def test_algorithmic_bytes_per_token_head():
     # forward: q, k, v, o (bf16) + gates (fp32) = 2052 B, plus the saved state 4 d^2 / L
     assert bench.fwd_bytes(128, 64) == 2052 + 4 * 128 * 128 / 64
     assert bench.bwd_bytes(128, 64) == 3848 + 4 * 128 * 128 / 64
+
+
+def test_kernel_rooflines():
+    """Per-call rates: bytes and FLOPs over the call's own time, against the peaks."""
+    peaks = {"hbm": 6650.0, "bf16": 1590.0}
+    kern = {"carve_fwd": (0.5, 1.0e9), "carve_bwd": (2.0, 4.0e9)}
+    flops = {"carve_fwd": 2.0e11, "carve_bwd": 1.0e12}
+    r = bench.kernel_rooflines(kern, flops, peaks)
+    assert set(r) == {"carve_fwd", "carve_bwd"}
+    assert abs(r["carve_fwd"]["hbm_gbs"] - 2000.0) < 1e-9 and abs(r["carve_bwd"]["hbm_gbs"] - 2000.0) < 1e-9
+    assert abs(r["carve_fwd"]["tflops"] - 400.0) < 1e-9 and abs(r["carve_bwd"]["tflops"] - 500.0) < 1e-9
+    assert abs(r["carve_bwd"]["hbm_frac"] - 2000.0 / 6650.0) < 1e-12
+    assert abs(r["carve_fwd"]["tensor_frac"] - 400.0 / 1590.0) < 1e-12
