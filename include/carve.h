@@ -233,12 +233,14 @@ carve_status carve_step(const carve_dims *d, const void *q, const void *k, const
  * carve_check -- blocks the host until the work queued on `stream` has finished, then
  * reports what the device saw: CARVE_ERR_CUDA if the stream reports an error,
  * CARVE_ERR_TIMEOUT if a bounded device-side wait of a carve kernel (a shared-memory
- * barrier waiting for a bulk copy) gave up since the previous carve_check,
- * CARVE_ERR_INVALID_ARG if a varlen call met out-of-range sequence offsets, else CARVE_OK.
- * The device status words are cleared by the call.  A kernel whose wait gives up records
- * it, stops its sweep, waits (again bounded) for its own copies in flight and returns, so
- * the CUDA context stays usable; the outputs of that call are undefined.  The pages have
- * no counterpart to this entry point.
+ * barrier waiting for a bulk copy or a tensor-core product) gave up since the previous
+ * carve_check (the tensor-core forward also reports it, without computing anything, if its
+ * dynamic shared memory were not 1024-byte aligned; never observed), CARVE_ERR_INVALID_ARG
+ * if a varlen call met out-of-range sequence offsets, else CARVE_OK.  The device status words
+ * are cleared by the call.  A kernel whose wait gives up records it, stops its sweep, waits
+ * (again bounded) for its own copies and products in flight, frees the tensor memory it
+ * holds and returns, so the CUDA context stays usable; the outputs of that call are
+ * undefined.  The pages have no counterpart to this entry point.
  */
 carve_status carve_check(void *stream);
 
