@@ -15,7 +15,7 @@
 namespace carve {
 
 // element offset of (row r, column c) in a [rows][128] bf16 tile of the layout above
-__device__ __forceinline__ int umma_off(int r, int c, int rows) {
+__host__ __device__ __forceinline__ int umma_off(int r, int c, int rows) {
     return (c >> 6) * (rows * 64) + r * 64 + ((((c >> 3) & 7) ^ (r & 7)) << 3) + (c & 7);
 }
 
